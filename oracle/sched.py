@@ -1,0 +1,228 @@
+"""Reference block allocator and scheduling step — TEST INFRASTRUCTURE ONLY.
+
+Written from "vLLM 推理加速原理详解：大模型服务吞吐量为何能提升 10 倍":
+
+* section "PagedAttention：把操作系统的虚拟内存搬进 GPU": the cache is cut into
+  fixed-size physical blocks; each sequence's block table maps its logical
+  blocks to physical ones; blocks are taken on demand as tokens are produced
+  (no reservation for the maximum length); every block has the same size,
+  so any free block serves any request; several logical blocks (prefix or
+  beam sharing) may map to one physical block.
+* section "连续批处理：别再等最慢的那个请求了" — the scheduling loop printed
+  there: (1) drop finished requests and free their blocks, (2) read the
+  number of free blocks, (3) while requests wait and the free count is above
+  MIN_BLOCKS, pop the first waiting request and, if the block manager can
+  allocate it, allocate and move it to the running set, (4) decode the
+  running set.
+
+Readings where the page leaves a step open (each also listed in the design doc):
+
+* sharing implies a reference count per physical block; a block returns to
+  the free list when its count reaches zero;
+* the free list is FIFO: allocation takes from the head, freeing appends to
+  the tail in block-table order (deterministic, so two implementations can be
+  compared exactly);
+* writing into a block whose count is above one first copies it
+  (copy-on-write) into a fresh block, which replaces it in the writer's table;
+* in step (3) the printed loop pops a request before testing it and never
+  puts it back; the reading taken keeps FIFO order instead: a head request
+  that cannot be allocated stays at the head and admission stops; the free
+  count is re-read after each admission; admission also stops at
+  ``max_num_seqs`` running sequences (the page's ``max_num_seqs`` setting);
+* MIN_BLOCKS defaults to the number of running sequences: one block per
+  running sequence is kept in reserve for this iteration's appended token.  A
+  waiting request is admitted only if its prompt's blocks fit in the free
+  blocks while that reserve (counting the request itself) stays free, so the
+  appends of step (4) never run out of blocks;
+* step (4) appends one token slot to every running sequence (admitted ones
+  included) before the decode.
+"""
+
+from __future__ import annotations
+
+from collections import deque
+
+
+class OracleOOM(Exception):
+    """No free block for a required allocation."""
+
+
+class OracleStateError(Exception):
+    """Unknown or duplicate sequence, or a block freed twice."""
+
+
+def blocks_for(num_tokens: int, block_size: int) -> int:
+    return -(-num_tokens // block_size)
+
+
+class BlockManager:
+    def __init__(self, num_blocks: int, block_size: int, initial_free_order=None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise ValueError("num_blocks and block_size must be positive")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        order = list(range(num_blocks)) if initial_free_order is None else [int(b) for b in initial_free_order]
+        if sorted(order) != list(range(num_blocks)):
+            raise ValueError("initial free order must be a permutation of the blocks")
+        self.free_list = deque(order)
+        self.refcount = [0] * num_blocks
+        self.tables: dict[int, list[int]] = {}
+        self.tokens: dict[int, int] = {}
+        self.num_cow = 0
+        self.num_alloc = 0
+        self.num_freed = 0
+
+    # verbs named on the page
+    def get_num_free_blocks(self) -> int:
+        return len(self.free_list)
+
+    def can_allocate(self, num_tokens: int) -> bool:
+        return blocks_for(num_tokens, self.block_size) <= len(self.free_list)
+
+    def _take(self) -> int:
+        if not self.free_list:
+            raise OracleOOM("no free block")
+        b = self.free_list.popleft()
+        assert self.refcount[b] == 0
+        self.refcount[b] = 1
+        self.num_alloc += 1
+        return b
+
+    def allocate(self, seq_id: int, num_tokens: int) -> None:
+        if seq_id in self.tables:
+            raise OracleStateError(f"sequence {seq_id} already exists")
+        if num_tokens < 0:
+            raise ValueError("negative token count")
+        need = blocks_for(num_tokens, self.block_size)
+        if need > len(self.free_list):
+            raise OracleOOM("not enough free blocks")
+        self.tables[seq_id] = [self._take() for _ in range(need)]
+        self.tokens[seq_id] = num_tokens
+
+    def free(self, seq_id: int) -> None:
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        for b in self.tables.pop(seq_id):
+            if self.refcount[b] <= 0:
+                raise OracleStateError(f"block {b} freed twice")
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                self.free_list.append(b)
+                self.num_freed += 1
+        del self.tokens[seq_id]
+
+    # sharing and growth
+    def fork(self, parent: int, child: int) -> None:
+        if parent not in self.tables:
+            raise OracleStateError(f"sequence {parent} is unknown")
+        if child in self.tables:
+            raise OracleStateError(f"sequence {child} already exists")
+        self.tables[child] = list(self.tables[parent])
+        self.tokens[child] = self.tokens[parent]
+        for b in self.tables[child]:
+            self.refcount[b] += 1
+
+    def append_slot(self, seq_id: int):
+        """Reserve the slot of the sequence's next token.
+
+        Returns (slot, cow_src, cow_dst); cow_* are -1 unless the last block
+        was shared and had to be copied first.  slot = block * block_size +
+        offset."""
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        table = self.tables[seq_id]
+        pos = self.tokens[seq_id]
+        cow_src = cow_dst = -1
+        if pos % self.block_size == 0:
+            table.append(self._take())
+        else:
+            last = table[-1]
+            if self.refcount[last] > 1:
+                new = self._take()
+                self.refcount[last] -= 1
+                table[-1] = new
+                cow_src, cow_dst = last, new
+                self.num_cow += 1
+        self.tokens[seq_id] = pos + 1
+        slot = table[pos // self.block_size] * self.block_size + pos % self.block_size
+        return slot, cow_src, cow_dst
+
+    def block_table(self, seq_id: int) -> list[int]:
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        return list(self.tables[seq_id])
+
+    def snapshot(self):
+        return list(self.free_list), list(self.refcount)
+
+
+class Scheduler:
+    """One scheduling iteration per :meth:`step`, in the page's order."""
+
+    def __init__(self, bm: BlockManager, max_num_seqs: int, min_blocks: int | None = None):
+        self.bm = bm
+        self.max_num_seqs = max_num_seqs
+        self.min_blocks = min_blocks  # None: number of running sequences
+        self.waiting: deque[tuple[int, int]] = deque()
+        self.running: list[int] = []
+
+    def add_request(self, seq_id: int, prompt_len: int) -> None:
+        self.waiting.append((seq_id, prompt_len))
+
+    def adopt(self, seq_id: int) -> None:
+        """Put a sequence that already holds blocks (e.g. a fork) in the running set."""
+        if seq_id not in self.bm.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        self.running.append(seq_id)
+
+    def _min_blocks(self) -> int:
+        return len(self.running) if self.min_blocks is None else self.min_blocks
+
+    def step(self, finished_ids):
+        # (1) remove finished requests and return their blocks
+        finished = set(int(x) for x in finished_ids)
+        for sid in finished:
+            if sid not in self.running:
+                raise OracleStateError(f"sequence {sid} is not running")
+        self.running = [r for r in self.running if r not in finished]
+        for sid in finished_ids:
+            self.bm.free(int(sid))
+        # (2) free block count
+        free_blocks = self.bm.get_num_free_blocks()
+        # (3) admit waiting requests, first come first served
+        admitted = []
+        prompt_slots = []
+        while (self.waiting and free_blocks > self._min_blocks()
+               and len(self.running) < self.max_num_seqs):
+            sid, plen = self.waiting[0]
+            reserve = self._min_blocks() + (1 if self.min_blocks is None else 0)
+            if not (self.bm.can_allocate(plen)
+                    and blocks_for(plen, self.bm.block_size) + reserve <= free_blocks):
+                break
+            self.waiting.popleft()
+            self.bm.allocate(sid, plen)
+            self.running.append(sid)
+            admitted.append(sid)
+            table = self.bm.tables[sid]
+            bs = self.bm.block_size
+            prompt_slots.extend(table[t // bs] * bs + t % bs for t in range(plen))
+            free_blocks = self.bm.get_num_free_blocks()
+        # (4) one new token slot per running sequence, then decode
+        decode_slots, cow = [], []
+        for sid in self.running:
+            slot, cs, cd = self.bm.append_slot(sid)
+            decode_slots.append(slot)
+            if cs >= 0:
+                cow.append((cs, cd))
+        return {
+            "running": list(self.running),
+            "block_tables": [self.bm.block_table(s) for s in self.running],
+            "context_lens": [self.bm.tokens[s] for s in self.running],
+            "slot_mapping": prompt_slots + decode_slots,
+            "cow_pairs": cow,
+            "admitted": admitted,
+        }
+
+    def stats(self):
+        used = self.bm.num_blocks - self.bm.get_num_free_blocks()
+        return len(self.running), len(self.waiting), used, self.bm.num_blocks
