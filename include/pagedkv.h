@@ -1,0 +1,285 @@
+/*
+ * pagedkv — paged KV cache and PagedAttention decode for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every entry point returns an int status (KV_OK or a negative
+ * KV_ERR_* code); kv_last_error() gives a message for the calling thread's
+ * last failure.  GPU entry points only enqueue work on the caller's stream
+ * and never synchronise (except kv_get_device_error).  The library never
+ * allocates device memory: the caller owns every device buffer and passes
+ * raw pointers.  Host handles (kv_pool, kv_alloc, kv_sched) are owned by the
+ * library between their create and destroy calls and are not thread-safe.
+ *
+ * The method follows the page "vLLM 推理加速原理详解：大模型服务吞吐量为何能
+ * 提升 10 倍" (fudengji.cn), cited below by section:
+ *   [PA]   "PagedAttention：把操作系统的虚拟内存搬进 GPU" — the KV cache is cut
+ *          into fixed-size physical blocks; a per-sequence block table maps
+ *          logically contiguous blocks to physically scattered ones; blocks
+ *          are taken on demand; several logical blocks may share one physical
+ *          block; the attention kernel reads K/V from the non-contiguous
+ *          blocks.
+ *   [CB]   "连续批处理：别再等最慢的那个请求了" — after every decode iteration,
+ *          free the finished requests' blocks, read the free-block count,
+ *          admit waiting requests first come first served while blocks allow
+ *          (free_blocks > MIN_BLOCKS and can_allocate), then decode the
+ *          running set.
+ *   [PIT]  "vLLM 也不是银弹：真实部署中的坑" — FP8 KV cache as the remedy for
+ *          long-context memory pressure; the whole cache is one preallocated
+ *          pool.
+ *   [MON]  "从零开始：vLLM 部署的实战建议", step four — running / waiting
+ *          request counts and cache usage as the metrics to watch.
+ *
+ * Pool layout (the pages leave it open; this library fixes it): for each
+ * layer, K and V are separate device arrays, each
+ *     [num_blocks][kv_heads][block_size][head_dim]
+ * elements, row-major, so one (block, kv head) tile of block_size x head_dim
+ * elements is contiguous.  A token slot is block * block_size + offset.  For
+ * FP8 pools each layer also has K and V scale arrays [num_blocks][kv_heads]
+ * of fp32: the stored E4M3 code times its (block, head) scale is the value.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* kv_stream_t;
+
+/* Element types.  KV_F32 is valid only as an attention output type. */
+typedef enum { KV_F16 = 0, KV_BF16 = 1, KV_FP8_E4M3 = 2, KV_F32 = 3 } kv_dtype;
+
+enum {
+  KV_OK = 0,
+  KV_ERR_ARG = -1,     /* invalid argument; nothing was enqueued */
+  KV_ERR_OOM = -2,     /* the allocator has too few free blocks */
+  KV_ERR_STATE = -3,   /* unknown / duplicate sequence, double free, unbound layer */
+  KV_ERR_BOUNDS = -4,  /* device-reported: block id, slot or length out of range */
+  KV_ERR_CUDA = -5,    /* a CUDA runtime / driver call failed */
+  KV_ERR_TIMEOUT = -6  /* device-reported: a pipeline wait gave up (bounded spin) */
+};
+
+typedef struct kv_pool kv_pool;
+typedef struct kv_alloc kv_alloc;
+typedef struct kv_sched kv_sched;
+
+/* Message for the calling thread's most recent failure ("" if none). */
+const char* kv_last_error(void);
+/* ABI version, currently 1. */
+int kv_version(void);
+
+/* ------------------------------------------------------------------ pool */
+
+/* Describe a preallocated pool ([PA], [PIT]): num_layers layers of
+ * num_blocks physical blocks of block_size token slots for kv_heads heads of
+ * head_dim elements of `dtype` (KV_F16, KV_BF16 or KV_FP8_E4M3).
+ * Supported: block_size a multiple of 16 up to 256; head_dim 64 or 128;
+ * num_blocks >= 1; 1 <= kv_heads; 1 <= num_layers <= 4096.  Host only; no
+ * device work.  *out is owned by the caller until kv_pool_destroy.
+ * Errors: KV_ERR_ARG for an unsupported geometry. */
+int kv_pool_create(int block_size, int num_blocks, int kv_heads, int head_dim,
+                   kv_dtype dtype, int num_layers, kv_pool** out);
+
+/* Bytes the caller must allocate per layer for K (and the same again for
+ * V), and for each FP8 scale array (0 for 16-bit pools).  Either pointer may
+ * be NULL. */
+int kv_pool_bytes(const kv_pool* pool, size_t* kv_bytes_per_layer,
+                  size_t* scale_bytes_per_layer);
+
+/* Attach caller-owned device memory to `layer`: k_base and v_base of
+ * kv_bytes_per_layer bytes each, 16-byte aligned; k_scale and v_scale
+ * [num_blocks][kv_heads] fp32 for FP8 pools (NULL otherwise).  Builds the
+ * layer's TMA descriptors, so it needs a working CUDA driver; the pointers
+ * must belong to the device that later launches use.  Rebinding replaces the
+ * old pointers.  Errors: KV_ERR_ARG (bad layer, NULL or misaligned pointer,
+ * scales missing for FP8), KV_ERR_CUDA (descriptor creation failed). */
+int kv_pool_bind(kv_pool* pool, int layer, void* k_base, void* v_base, float* k_scale,
+                 float* v_scale);
+
+/* Decode launch configuration.  partition_tokens: context-partition length
+ * for split decode, 0 for automatic, else a multiple of 16 in [16, 4096];
+ * contexts longer than one partition are split into partitions whose
+ * partial results are merged by a log-sum-exp reduce (see
+ * paged_attention_decode).  stages: shared-memory pipeline depth per warp,
+ * 0 for automatic, else 2..4.  Host only. */
+int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages);
+
+int kv_pool_destroy(kv_pool* pool);
+
+/* ------------------------------------------------------------ cache write */
+
+/* Scatter new tokens' K and V into their slots ([PA]: blocks grow on demand,
+ * each new token goes to the slot its sequence's table assigns).
+ *   k_new, v_new   device [num_tokens][kv_heads][head_dim] of src_dtype
+ *                  (KV_F16 or KV_BF16); for 16-bit pools src_dtype must be
+ *                  the pool dtype and the bits are copied unchanged.
+ *   slot_mapping   device int64 [num_tokens]; token t goes to block
+ *                  slot / block_size, offset slot % block_size; slot < 0
+ *                  skips the token.
+ *   k_inv_scale, v_inv_scale   FP8 pools only: device fp32
+ *                  [num_blocks][kv_heads]; each value is widened to fp32,
+ *                  multiplied in fp32 by inv_scale[block][head], rounded to
+ *                  E4M3 to nearest even and saturated to +-448 (NaN stays
+ *                  NaN).  NULL for 16-bit pools.
+ * Slots must be distinct (two tokens into one slot race).  A slot beyond the
+ * pool is skipped and reported as KV_ERR_BOUNDS by kv_get_device_error.
+ * num_tokens == 0 enqueues nothing.  Errors: KV_ERR_ARG, KV_ERR_STATE
+ * (layer not bound), KV_ERR_CUDA (launch failed). */
+int paged_kv_write(const kv_pool* pool, int layer, const void* k_new, const void* v_new,
+                   kv_dtype src_dtype, const int64_t* slot_mapping, int num_tokens,
+                   const float* k_inv_scale, const float* v_inv_scale, kv_stream_t stream);
+
+/* ------------------------------------------------------------- block copy */
+
+/* Copy-on-write support for shared blocks ([PA]: several logical blocks may
+ * map to one physical block; a sequence that writes into a shared block
+ * first gets a private copy).  pairs: device int32 [num_pairs][2] of
+ * (src, dst) physical block ids.  For every bound layer, K and V (and the
+ * FP8 scales) of block src are copied to block dst.  Pairs run in parallel:
+ * every dst must be distinct and must not be any pair's src.  An id outside
+ * the pool skips that pair and is reported as KV_ERR_BOUNDS by
+ * kv_get_device_error.  num_pairs == 0 enqueues nothing.  Errors:
+ * KV_ERR_ARG, KV_ERR_STATE (a layer not bound), KV_ERR_CUDA. */
+int block_copy(const kv_pool* pool, const int32_t* pairs, int num_pairs, kv_stream_t stream);
+
+/* -------------------------------------------------------- decode attention */
+
+/* Scratch bytes paged_attention_decode needs for these sizes (0 when no
+ * context is split).  Same partition policy as the decode call. */
+size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
+                                       int max_context_len);
+
+/* PagedAttention decode ([PA]): for every sequence s and query head h,
+ *     out[s][h] = sum_t softmax_t(scale * q[s][h] . K_t) V_t
+ * over the sequence's tokens t < context_lens[s], where token t is read at
+ * block block_tables[s][t / block_size], offset t % block_size, kv head
+ * h / (num_q_heads / kv_heads) (consecutive query heads share a kv head).
+ * Softmax and accumulation run in fp32 with a running max and sum.
+ *   q             device [batch][num_q_heads][head_dim] of q_dtype; for
+ *                 16-bit pools q_dtype must be the pool dtype; FP8 pools
+ *                 take KV_F16 or KV_BF16 queries.
+ *   num_q_heads   a multiple of kv_heads with num_q_heads / kv_heads <= 8.
+ *   block_tables  device int32 [batch][max_blocks_per_seq]; entries past
+ *                 ceil(context_len / block_size) are not read.
+ *   context_lens  device int32 [batch]; 0 gives an all-zero output row.
+ *   max_context_len  host upper bound on every context_lens entry; it sizes
+ *                 the launch.  A length above it, above
+ *                 max_blocks_per_seq * block_size, or negative is clamped
+ *                 and reported as KV_ERR_BOUNDS by kv_get_device_error, as is
+ *                 a block id outside the pool (that block is skipped).
+ *   out           device [batch][num_q_heads][head_dim] of out_dtype
+ *                 (q_dtype or KV_F32).
+ *   workspace     device scratch of workspace_bytes >=
+ *                 paged_attention_workspace_bytes(...), 16-byte aligned;
+ *                 may be NULL when that is 0.  Contexts longer than one
+ *                 partition are split: each partition writes its unnormalised
+ *                 output, running max and sum there, and a second kernel
+ *                 merges them by log-sum-exp.
+ * batch == 0 enqueues nothing.  Errors: KV_ERR_ARG, KV_ERR_STATE (layer not
+ * bound), KV_ERR_CUDA. */
+int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
+                           int num_q_heads, const int32_t* block_tables,
+                           int max_blocks_per_seq, const int32_t* context_lens, int batch,
+                           int max_context_len, float scale, void* out, kv_dtype out_dtype,
+                           void* workspace, size_t workspace_bytes, kv_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the current device's error word:
+ * *err = KV_OK, KV_ERR_BOUNDS or KV_ERR_TIMEOUT (the first error any kernel
+ * of this library recorded since the last call).  Errors: KV_ERR_CUDA. */
+int kv_get_device_error(kv_stream_t stream, int* err);
+
+/* ------------------------------------------------------ block allocator */
+
+/* Refcounted free-list allocator of physical blocks ([PA]: blocks on demand,
+ * any free block serves any request, shared blocks).  Deterministic: the free
+ * list is FIFO (take from the head, freed blocks go to the tail in block-table
+ * order); initial_free_order (a permutation of 0..num_blocks-1, or NULL for
+ * ascending) sets its starting order.  Host only. */
+int kv_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                    kv_alloc** out);
+/* Number of free blocks ([CB] get_num_free_blocks). */
+int kv_alloc_num_free(const kv_alloc* a, int* n);
+/* *yes = 1 iff ceil(num_tokens / block_size) blocks are free ([CB] can_allocate). */
+int kv_alloc_can_allocate(const kv_alloc* a, int num_tokens, int* yes);
+/* New sequence holding ceil(num_tokens / block_size) fresh blocks ([CB]
+ * allocate).  KV_ERR_STATE if seq_id exists, KV_ERR_OOM if too few blocks
+ * (nothing changes). */
+int kv_alloc_allocate(kv_alloc* a, int64_t seq_id, int num_tokens);
+/* Reserve the slot of the sequence's next token: a new block when its token
+ * count is a multiple of block_size; otherwise, if its last block is shared
+ * (refcount > 1), a copy-on-write: a fresh block replaces it in this table
+ * and (*cow_src, *cow_dst) name the copy the caller must run with block_copy
+ * before writing.  cow_* are -1 when no copy is needed.  KV_ERR_OOM if a
+ * block is needed and none is free (nothing changes). */
+int kv_alloc_append_slot(kv_alloc* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                         int32_t* cow_dst);
+/* child shares every block of parent (refcount + 1 each) and its length. */
+int kv_alloc_fork(kv_alloc* a, int64_t parent, int64_t child);
+/* Drop the sequence ([CB] free(block_table)): each of its blocks loses one
+ * reference and returns to the free list at zero. */
+int kv_alloc_free(kv_alloc* a, int64_t seq_id);
+/* Copy the block table (at most cap entries) into out; *n = its length. */
+int kv_alloc_block_table(const kv_alloc* a, int64_t seq_id, int32_t* out, int cap, int* n);
+int kv_alloc_num_tokens(const kv_alloc* a, int64_t seq_id, int* n);
+int kv_alloc_refcount(const kv_alloc* a, int32_t block, int* rc);
+/* Free list in order (n_free entries) and all num_blocks refcounts; either
+ * array may be NULL. */
+int kv_alloc_snapshot(const kv_alloc* a, int32_t* free_list, int* n_free, int32_t* refcounts);
+/* Lifetime counters: blocks taken, blocks returned, copy-on-write copies. */
+int kv_alloc_counters(const kv_alloc* a, int64_t* allocated, int64_t* freed, int64_t* cow);
+int kv_alloc_destroy(kv_alloc* a);
+
+/* --------------------------------------------------------- scheduling step */
+
+/* Continuous-batching scheduler over an allocator ([CB]).  max_num_seqs caps
+ * the running set; min_blocks is MIN_BLOCKS of the loop, or < 0 for "the
+ * number of running sequences" (one block per running sequence kept in
+ * reserve for its appended token; a request is admitted only if its prompt
+ * blocks fit with that reserve, counting itself, still free).  The allocator
+ * must outlive the scheduler. */
+int kv_sched_create(kv_alloc* a, int max_num_seqs, int min_blocks, kv_sched** out);
+/* Queue a request (FIFO) whose prompt has prompt_len tokens. */
+int kv_sched_add_request(kv_sched* s, int64_t seq_id, int prompt_len);
+/* Put a sequence that already holds blocks (e.g. a fork) in the running set. */
+int kv_sched_adopt(kv_sched* s, int64_t seq_id);
+
+typedef struct {
+  int batch;        /* running sequences after the step */
+  int num_tokens;   /* slots to write: admitted prompts' tokens, then one per running seq */
+  int num_cow;      /* copy-on-write pairs to run before the write */
+  int num_admitted; /* requests moved from waiting to running */
+  int max_blocks;   /* longest block table among the running sequences */
+} kv_step_info;
+
+/* One iteration in the page's order ([CB]): (1) the finished sequences
+ * (each must be running) leave the running set and are freed; (2) read the
+ * free count; (3) while requests wait, free > MIN_BLOCKS and fewer than
+ * max_num_seqs run, the head request is admitted if its prompt fits (else it
+ * stays at the head and admission stops); (4) one slot is appended for every
+ * running sequence.  Outputs are kept until the next step; read them with
+ * kv_sched_outputs.  KV_ERR_STATE (bad finished id) changes nothing;
+ * KV_ERR_OOM means the appends of (4) would run out of blocks: (1)-(3) are
+ * applied, no slot is appended. */
+int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_step_info* info);
+/* Copy the last step's outputs to host arrays sized from kv_step_info (any
+ * may be NULL): running_ids[batch]; block_tables[batch][table_width]
+ * (table_width >= max_blocks, padded with -1); context_lens[batch] (tokens
+ * after the append); slot_mapping[num_tokens]; cow_pairs[num_cow][2];
+ * admitted_ids[num_admitted]. */
+int kv_sched_outputs(const kv_sched* s, int64_t* running_ids, int32_t* block_tables,
+                     int table_width, int32_t* context_lens, int64_t* slot_mapping,
+                     int32_t* cow_pairs, int64_t* admitted_ids);
+/* [MON]: running and waiting request counts, used and total blocks
+ * (cache usage = used / total). */
+int kv_sched_stats(const kv_sched* s, int* running, int* waiting, int* used_blocks,
+                   int* total_blocks);
+int kv_sched_destroy(kv_sched* s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

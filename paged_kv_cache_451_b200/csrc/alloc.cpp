@@ -1,0 +1,450 @@
+// Refcounted free-list block allocator and continuous-batching step.
+//
+// Block rules: "vLLM 推理加速原理详解：大模型服务吞吐量为何能提升 10 倍",
+// section "PagedAttention：把操作系统的虚拟内存搬进 GPU" — fixed-size physical
+// blocks taken on demand, a per-sequence block table, any free block serves
+// any request, several logical blocks may share one physical block.
+// Scheduling loop: same page, section "连续批处理：别再等最慢的那个请求了" —
+// free finished requests, read the free count, admit waiting requests first
+// come first served while free_blocks > MIN_BLOCKS and can_allocate, then
+// decode the running set.
+//
+// Policies the page leaves open, fixed here so runs are reproducible:
+// FIFO free list (take from the head, return to the tail in table order);
+// copy-on-write when appending into a block whose refcount is above one;
+// head-of-line admission (a request that does not fit stays first and
+// admission stops); MIN_BLOCKS defaults to the running count and a request
+// is admitted only if its prompt blocks fit with that reserve (counting the
+// request) left free, so the appends of the step cannot run out.
+
+#include <cstdint>
+#include <cstring>
+#include <deque>
+#include <new>
+#include <string>
+#include <unordered_map>
+#include <unordered_set>
+#include <vector>
+
+#include "host_common.h"
+
+namespace pagedkv {
+
+namespace {
+thread_local std::string g_msg;
+}
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_msg = buf;
+  return code;
+}
+
+int ok() {
+  g_msg.clear();
+  return KV_OK;
+}
+
+const char* last_error() { return g_msg.c_str(); }
+
+}  // namespace pagedkv
+
+using pagedkv::fail;
+using pagedkv::ok;
+
+struct SeqState {
+  std::vector<int32_t> blocks;
+  int64_t tokens = 0;
+};
+
+struct kv_alloc {
+  int num_blocks = 0;
+  int block_size = 0;
+  std::deque<int32_t> free_list;
+  std::vector<int32_t> refcount;
+  std::unordered_map<int64_t, SeqState> seqs;
+  int64_t n_alloc = 0, n_freed = 0, n_cow = 0;
+
+  int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
+
+  int32_t take() {
+    int32_t b = free_list.front();
+    free_list.pop_front();
+    refcount[b] = 1;
+    ++n_alloc;
+    return b;
+  }
+
+  void release(int32_t b) {
+    if (--refcount[b] == 0) {
+      free_list.push_back(b);
+      ++n_freed;
+    }
+  }
+
+  // Blocks one append to `s` needs: 1 for a new block or a copy, else 0.
+  bool append_needs_block(const SeqState& s) const {
+    if (s.tokens % block_size == 0) return true;
+    return refcount[s.blocks.back()] > 1;
+  }
+
+  int append(SeqState& s, int64_t* slot, int32_t* cs, int32_t* cd) {
+    int64_t pos = s.tokens;
+    *cs = -1;
+    *cd = -1;
+    if (pos % block_size == 0) {
+      if (free_list.empty()) return KV_ERR_OOM;
+      s.blocks.push_back(take());
+    } else {
+      int32_t last = s.blocks.back();
+      if (refcount[last] > 1) {
+        if (free_list.empty()) return KV_ERR_OOM;
+        int32_t fresh = take();
+        --refcount[last];
+        s.blocks.back() = fresh;
+        *cs = last;
+        *cd = fresh;
+        ++n_cow;
+      }
+    }
+    s.tokens = pos + 1;
+    *slot = (int64_t)s.blocks[pos / block_size] * block_size + pos % block_size;
+    return KV_OK;
+  }
+};
+
+extern "C" {
+
+const char* kv_last_error(void) { return pagedkv::last_error(); }
+int kv_version(void) { return 1; }
+
+int kv_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                    kv_alloc** out) {
+  if (!out) return fail(KV_ERR_ARG, "out is NULL");
+  if (num_blocks <= 0 || block_size <= 0)
+    return fail(KV_ERR_ARG, "num_blocks (%d) and block_size (%d) must be positive", num_blocks,
+                block_size);
+  kv_alloc* a = new (std::nothrow) kv_alloc();
+  if (!a) return fail(KV_ERR_OOM, "host allocation failed");
+  a->num_blocks = num_blocks;
+  a->block_size = block_size;
+  a->refcount.assign(num_blocks, 0);
+  if (initial_free_order) {
+    std::vector<char> seen(num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+      int32_t b = initial_free_order[i];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete a;
+        return fail(KV_ERR_ARG, "initial_free_order is not a permutation of 0..%d", num_blocks - 1);
+      }
+      seen[b] = 1;
+      a->free_list.push_back(b);
+    }
+  } else {
+    for (int i = 0; i < num_blocks; ++i) a->free_list.push_back(i);
+  }
+  *out = a;
+  return ok();
+}
+
+int kv_alloc_destroy(kv_alloc* a) {
+  delete a;
+  return ok();
+}
+
+int kv_alloc_num_free(const kv_alloc* a, int* n) {
+  if (!a || !n) return fail(KV_ERR_ARG, "NULL argument");
+  *n = (int)a->free_list.size();
+  return ok();
+}
+
+int kv_alloc_can_allocate(const kv_alloc* a, int num_tokens, int* yes) {
+  if (!a || !yes || num_tokens < 0) return fail(KV_ERR_ARG, "bad argument");
+  *yes = a->blocks_for(num_tokens) <= (int64_t)a->free_list.size();
+  return ok();
+}
+
+int kv_alloc_allocate(kv_alloc* a, int64_t seq_id, int num_tokens) {
+  if (!a || num_tokens < 0) return fail(KV_ERR_ARG, "bad argument");
+  if (a->seqs.count(seq_id)) return fail(KV_ERR_STATE, "sequence %lld already exists", (long long)seq_id);
+  int64_t need = a->blocks_for(num_tokens);
+  if (need > (int64_t)a->free_list.size())
+    return fail(KV_ERR_OOM, "need %lld blocks, %zu free", (long long)need, a->free_list.size());
+  SeqState s;
+  s.blocks.reserve(need);
+  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(a->take());
+  s.tokens = num_tokens;
+  a->seqs.emplace(seq_id, std::move(s));
+  return ok();
+}
+
+int kv_alloc_append_slot(kv_alloc* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                         int32_t* cow_dst) {
+  if (!a || !slot || !cow_src || !cow_dst) return fail(KV_ERR_ARG, "NULL argument");
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  int rc = a->append(it->second, slot, cow_src, cow_dst);
+  if (rc != KV_OK) return fail(rc, "no free block for sequence %lld", (long long)seq_id);
+  return ok();
+}
+
+int kv_alloc_fork(kv_alloc* a, int64_t parent, int64_t child) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  auto it = a->seqs.find(parent);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)parent);
+  if (a->seqs.count(child)) return fail(KV_ERR_STATE, "sequence %lld already exists", (long long)child);
+  SeqState s = it->second;
+  for (int32_t b : s.blocks) ++a->refcount[b];
+  a->seqs.emplace(child, std::move(s));
+  return ok();
+}
+
+int kv_alloc_free(kv_alloc* a, int64_t seq_id) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  for (int32_t b : it->second.blocks) a->release(b);
+  a->seqs.erase(it);
+  return ok();
+}
+
+int kv_alloc_block_table(const kv_alloc* a, int64_t seq_id, int32_t* out, int cap, int* n) {
+  if (!a || !n || cap < 0 || (cap > 0 && !out)) return fail(KV_ERR_ARG, "bad argument");
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  const auto& b = it->second.blocks;
+  *n = (int)b.size();
+  for (int i = 0; i < cap && i < (int)b.size(); ++i) out[i] = b[i];
+  return ok();
+}
+
+int kv_alloc_num_tokens(const kv_alloc* a, int64_t seq_id, int* n) {
+  if (!a || !n) return fail(KV_ERR_ARG, "NULL argument");
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  *n = (int)it->second.tokens;
+  return ok();
+}
+
+int kv_alloc_refcount(const kv_alloc* a, int32_t block, int* rc) {
+  if (!a || !rc || block < 0 || block >= a->num_blocks) return fail(KV_ERR_ARG, "bad argument");
+  *rc = a->refcount[block];
+  return ok();
+}
+
+int kv_alloc_snapshot(const kv_alloc* a, int32_t* free_list, int* n_free, int32_t* refcounts) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  if (n_free) *n_free = (int)a->free_list.size();
+  if (free_list) {
+    int i = 0;
+    for (int32_t b : a->free_list) free_list[i++] = b;
+  }
+  if (refcounts) std::memcpy(refcounts, a->refcount.data(), sizeof(int32_t) * a->num_blocks);
+  return ok();
+}
+
+int kv_alloc_counters(const kv_alloc* a, int64_t* allocated, int64_t* freed, int64_t* cow) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  if (allocated) *allocated = a->n_alloc;
+  if (freed) *freed = a->n_freed;
+  if (cow) *cow = a->n_cow;
+  return ok();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ scheduler
+
+struct Request {
+  int64_t id;
+  int prompt_len;
+};
+
+struct kv_sched {
+  kv_alloc* a = nullptr;
+  int max_num_seqs = 0;
+  int min_blocks = -1;
+  std::deque<Request> waiting;
+  std::vector<int64_t> running;
+  // outputs of the last step
+  std::vector<int64_t> out_running;
+  std::vector<std::vector<int32_t>> out_tables;
+  std::vector<int32_t> out_lens;
+  std::vector<int64_t> out_slots;
+  std::vector<int32_t> out_cow;
+  std::vector<int64_t> out_admitted;
+
+  int min_blocks_now() const { return min_blocks < 0 ? (int)running.size() : min_blocks; }
+};
+
+extern "C" {
+
+int kv_sched_create(kv_alloc* a, int max_num_seqs, int min_blocks, kv_sched** out) {
+  if (!a || !out || max_num_seqs <= 0) return fail(KV_ERR_ARG, "bad argument");
+  kv_sched* s = new (std::nothrow) kv_sched();
+  if (!s) return fail(KV_ERR_OOM, "host allocation failed");
+  s->a = a;
+  s->max_num_seqs = max_num_seqs;
+  s->min_blocks = min_blocks;
+  *out = s;
+  return ok();
+}
+
+int kv_sched_destroy(kv_sched* s) {
+  delete s;
+  return ok();
+}
+
+int kv_sched_add_request(kv_sched* s, int64_t seq_id, int prompt_len) {
+  if (!s || prompt_len < 0) return fail(KV_ERR_ARG, "bad argument");
+  s->waiting.push_back({seq_id, prompt_len});
+  return ok();
+}
+
+int kv_sched_adopt(kv_sched* s, int64_t seq_id) {
+  if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
+  if (!s->a->seqs.count(seq_id)) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  for (int64_t r : s->running)
+    if (r == seq_id) return fail(KV_ERR_STATE, "sequence %lld is already running", (long long)seq_id);
+  s->running.push_back(seq_id);
+  return ok();
+}
+
+int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_step_info* info) {
+  if (!s || !info || n_finished < 0 || (n_finished > 0 && !finished_ids))
+    return fail(KV_ERR_ARG, "bad argument");
+  kv_alloc* a = s->a;
+  // validate before changing anything
+  std::unordered_set<int64_t> fin;
+  std::unordered_set<int64_t> run(s->running.begin(), s->running.end());
+  for (int i = 0; i < n_finished; ++i) {
+    if (!run.count(finished_ids[i]))
+      return fail(KV_ERR_STATE, "finished sequence %lld is not running", (long long)finished_ids[i]);
+    if (!fin.insert(finished_ids[i]).second)
+      return fail(KV_ERR_STATE, "sequence %lld finished twice", (long long)finished_ids[i]);
+  }
+  s->out_running.clear();
+  s->out_tables.clear();
+  s->out_lens.clear();
+  s->out_slots.clear();
+  s->out_cow.clear();
+  s->out_admitted.clear();
+
+  // (1) drop finished requests, return their blocks
+  std::vector<int64_t> keep;
+  keep.reserve(s->running.size());
+  for (int64_t r : s->running)
+    if (!fin.count(r)) keep.push_back(r);
+  s->running.swap(keep);
+  for (int i = 0; i < n_finished; ++i) kv_alloc_free(a, finished_ids[i]);
+
+  // (2) free block count
+  int64_t free_blocks = (int64_t)a->free_list.size();
+
+  // (3) admit first come first served
+  std::vector<int64_t> prompt_slots;
+  while (!s->waiting.empty() && free_blocks > s->min_blocks_now() &&
+         (int)s->running.size() < s->max_num_seqs) {
+    const Request req = s->waiting.front();
+    int64_t need = a->blocks_for(req.prompt_len);
+    int64_t reserve = s->min_blocks_now() + (s->min_blocks < 0 ? 1 : 0);
+    if (need > free_blocks || need + reserve > free_blocks) break;
+    if (a->seqs.count(req.id)) return fail(KV_ERR_STATE, "sequence %lld already exists", (long long)req.id);
+    s->waiting.pop_front();
+    kv_alloc_allocate(a, req.id, req.prompt_len);
+    s->running.push_back(req.id);
+    s->out_admitted.push_back(req.id);
+    const SeqState& st = a->seqs[req.id];
+    for (int t = 0; t < req.prompt_len; ++t)
+      prompt_slots.push_back((int64_t)st.blocks[t / a->block_size] * a->block_size + t % a->block_size);
+    free_blocks = (int64_t)a->free_list.size();
+  }
+
+  // (4) one slot per running sequence; check the whole batch fits first
+  {
+    int64_t need = 0;
+    std::unordered_map<int32_t, int64_t> shared_appenders;
+    for (int64_t r : s->running) {
+      const SeqState& st = a->seqs[r];
+      if (st.tokens % a->block_size == 0) {
+        ++need;
+      } else if (a->refcount[st.blocks.back()] > 1) {
+        ++shared_appenders[st.blocks.back()];
+      }
+    }
+    for (auto& kv : shared_appenders) {
+      int64_t copies = a->refcount[kv.first] - 1;
+      need += kv.second < copies ? kv.second : copies;
+    }
+    if (need > (int64_t)a->free_list.size()) {
+      info->batch = (int)s->running.size();
+      info->num_tokens = info->num_cow = 0;
+      info->num_admitted = (int)s->out_admitted.size();
+      info->max_blocks = 0;
+      return fail(KV_ERR_OOM, "appends need %lld blocks, %zu free", (long long)need,
+                  a->free_list.size());
+    }
+  }
+  s->out_slots = prompt_slots;
+  int max_blocks = 0;
+  for (int64_t r : s->running) {
+    SeqState& st = a->seqs[r];
+    int64_t slot;
+    int32_t cs, cd;
+    a->append(st, &slot, &cs, &cd);
+    s->out_slots.push_back(slot);
+    if (cs >= 0) {
+      s->out_cow.push_back(cs);
+      s->out_cow.push_back(cd);
+    }
+    s->out_running.push_back(r);
+    s->out_tables.push_back(st.blocks);
+    s->out_lens.push_back((int32_t)st.tokens);
+    if ((int)st.blocks.size() > max_blocks) max_blocks = (int)st.blocks.size();
+  }
+  info->batch = (int)s->running.size();
+  info->num_tokens = (int)s->out_slots.size();
+  info->num_cow = (int)s->out_cow.size() / 2;
+  info->num_admitted = (int)s->out_admitted.size();
+  info->max_blocks = max_blocks;
+  return ok();
+}
+
+int kv_sched_outputs(const kv_sched* s, int64_t* running_ids, int32_t* block_tables,
+                     int table_width, int32_t* context_lens, int64_t* slot_mapping,
+                     int32_t* cow_pairs, int64_t* admitted_ids) {
+  if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
+  if (block_tables) {
+    for (const auto& t : s->out_tables)
+      if ((int)t.size() > table_width)
+        return fail(KV_ERR_ARG, "table_width %d < longest table %zu", table_width, t.size());
+    for (size_t i = 0; i < s->out_tables.size(); ++i) {
+      int32_t* row = block_tables + i * (size_t)table_width;
+      const auto& t = s->out_tables[i];
+      for (int j = 0; j < table_width; ++j) row[j] = j < (int)t.size() ? t[j] : -1;
+    }
+  }
+  if (running_ids) std::memcpy(running_ids, s->out_running.data(), sizeof(int64_t) * s->out_running.size());
+  if (context_lens) std::memcpy(context_lens, s->out_lens.data(), sizeof(int32_t) * s->out_lens.size());
+  if (slot_mapping) std::memcpy(slot_mapping, s->out_slots.data(), sizeof(int64_t) * s->out_slots.size());
+  if (cow_pairs) std::memcpy(cow_pairs, s->out_cow.data(), sizeof(int32_t) * s->out_cow.size());
+  if (admitted_ids)
+    std::memcpy(admitted_ids, s->out_admitted.data(), sizeof(int64_t) * s->out_admitted.size());
+  return ok();
+}
+
+int kv_sched_stats(const kv_sched* s, int* running, int* waiting, int* used_blocks,
+                   int* total_blocks) {
+  if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
+  if (running) *running = (int)s->running.size();
+  if (waiting) *waiting = (int)s->waiting.size();
+  if (used_blocks) *used_blocks = s->a->num_blocks - (int)s->a->free_list.size();
+  if (total_blocks) *total_blocks = s->a->num_blocks;
+  return ok();
+}
+
+}  // extern "C"

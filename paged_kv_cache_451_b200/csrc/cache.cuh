@@ -1,0 +1,121 @@
+// Slot-mapped cache write and copy-on-write block copy.
+//
+// "vLLM 推理加速原理详解：大模型服务吞吐量为何能提升 10 倍", section
+// "PagedAttention：把操作系统的虚拟内存搬进 GPU": a sequence's cache grows a
+// block at a time as tokens arrive, and several logical blocks may map to
+// one physical block.  The write puts each new token's K/V row in the slot
+// its block table assigns; the copy gives a writer its own copy of a shared
+// block.  FP8 (section "vLLM 也不是银弹：真实部署中的坑") quantises on write.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "device_common.cuh"
+#include "ptx.cuh"
+
+namespace pagedkv {
+
+struct WriteParams {
+  const uint8_t* k_new;  // [T][kv_heads][D] 16-bit elements
+  const uint8_t* v_new;
+  const int64_t* slots;  // [T]
+  uint8_t* k;            // pool [num_blocks][kv_heads][block_size][D]
+  uint8_t* v;
+  const float* k_inv;    // FP8: [num_blocks][kv_heads]
+  const float* v_inv;
+  int64_t rows;          // T * kv_heads
+  int kv_heads;
+  int head_dim;
+  int block_size;
+  int num_blocks;
+  int src_bf16;
+};
+
+// One thread per 8 elements of one (token, head) row.  16-bit pools copy
+// 16 bytes; FP8 pools widen to fp32, multiply by the (block, head) inverse
+// scale in fp32 and round to E4M3 (nearest even, saturating).
+template <bool kFp8>
+__global__ void __launch_bounds__(256) kv_write_kernel(const WriteParams p) {
+  const int tpr = p.head_dim / 8;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gid / tpr;
+  const int part = (int)(gid - row * tpr);
+  if (row >= p.rows) return;
+  const int64_t t = row / p.kv_heads;
+  const int h = (int)(row - t * p.kv_heads);
+  const int64_t slot = p.slots[t];
+  if (slot < 0) return;
+  const int64_t blk = slot / p.block_size;
+  const int off = (int)(slot - blk * p.block_size);
+  if (blk >= p.num_blocks) {
+    record_error(KV_ERR_BOUNDS);
+    return;
+  }
+  const int64_t src = (row * p.head_dim + part * 8) * 2;
+  const int64_t dst_elem = ((blk * p.kv_heads + h) * p.block_size + off) * (int64_t)p.head_dim + part * 8;
+  const uint4 kx = *reinterpret_cast<const uint4*>(p.k_new + src);
+  const uint4 vx = *reinterpret_cast<const uint4*>(p.v_new + src);
+  if constexpr (!kFp8) {
+    *reinterpret_cast<uint4*>(p.k + dst_elem * 2) = kx;
+    *reinterpret_cast<uint4*>(p.v + dst_elem * 2) = vx;
+  } else {
+    const float ki = p.k_inv[blk * p.kv_heads + h];
+    const float vi = p.v_inv[blk * p.kv_heads + h];
+    auto quant = [&](const uint4& x, float inv) {
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint32_t q[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float a = bits_to_float(w[2 * j] & 0xffff, p.src_bf16) * inv;
+        const float b = bits_to_float(w[2 * j] >> 16, p.src_bf16) * inv;
+        const float c = bits_to_float(w[2 * j + 1] & 0xffff, p.src_bf16) * inv;
+        const float d = bits_to_float(w[2 * j + 1] >> 16, p.src_bf16) * inv;
+        q[j] = (uint32_t)f32x2_to_e4m3x2(a, b) | ((uint32_t)f32x2_to_e4m3x2(c, d) << 16);
+      }
+      return make_uint2(q[0], q[1]);
+    };
+    *reinterpret_cast<uint2*>(p.k + dst_elem) = quant(kx, ki);
+    *reinterpret_cast<uint2*>(p.v + dst_elem) = quant(vx, vi);
+  }
+}
+
+constexpr int kCopyLayers = 64;  // layers per block_copy launch
+
+struct CopyParams {
+  const int32_t* pairs;  // [num_pairs][2] (src, dst)
+  int num_pairs;
+  int num_blocks;
+  int kv_heads;
+  int64_t block_bytes;   // kv_heads * block_size * D * elem bytes (a multiple of 16)
+  void* k[kCopyLayers];
+  void* v[kCopyLayers];
+  float* ks[kCopyLayers];
+  float* vs[kCopyLayers];
+};
+
+// grid = (num_pairs, layers in this launch, 2 for K and V)
+__global__ void __launch_bounds__(256) block_copy_kernel(const CopyParams p) {
+  const int pi = blockIdx.x;
+  const int layer = blockIdx.y;
+  const bool is_v = blockIdx.z == 1;
+  const int32_t src = p.pairs[2 * pi];
+  const int32_t dst = p.pairs[2 * pi + 1];
+  if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+    if (threadIdx.x == 0) record_error(KV_ERR_BOUNDS);
+    return;
+  }
+  if (src == dst) return;
+  uint8_t* base = static_cast<uint8_t*>(is_v ? p.v[layer] : p.k[layer]);
+  const uint4* s = reinterpret_cast<const uint4*>(base + (int64_t)src * p.block_bytes);
+  uint4* d = reinterpret_cast<uint4*>(base + (int64_t)dst * p.block_bytes);
+  const int64_t n16 = p.block_bytes / 16;
+  for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) d[i] = s[i];
+  float* sc = is_v ? p.vs[layer] : p.ks[layer];
+  if (sc != nullptr)
+    for (int h = threadIdx.x; h < p.kv_heads; h += blockDim.x)
+      sc[(int64_t)dst * p.kv_heads + h] = sc[(int64_t)src * p.kv_heads + h];
+}
+
+}  // namespace pagedkv

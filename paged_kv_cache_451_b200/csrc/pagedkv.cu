@@ -1,0 +1,405 @@
+// C ABI of the GPU path: pool descriptors, TMA descriptors, launches.
+// All device code lives in this one translation unit (kernels in the .cuh
+// files) so every kernel shares one device error word.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "cache.cuh"
+#include "decode.cuh"
+#include "device_common.cuh"
+#include "host_common.h"
+#include "pool.h"
+
+using pagedkv::fail;
+using pagedkv::ok;
+
+namespace pagedkv {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kMaxLayers = 4096;
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultPartition = 512;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D view of one layer's K (or V) array: x = head_dim elements, y = kv_heads
+// * block_size rows, z = num_blocks; box = (up to 128 bytes of a row) x 16
+// rows x 1 block, with the swizzle matching the box row width.
+int make_map(const kv_pool* pool, void* base, CUtensorMap* map) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (no CUDA driver?)");
+  const int eb = elem_bytes(pool->dtype);
+  const int rowb = pool->head_dim * eb;
+  const int boxb = std::min(rowb, 128);
+  cuuint64_t dims[3] = {(cuuint64_t)pool->head_dim, (cuuint64_t)pool->kv_heads * pool->block_size,
+                        (cuuint64_t)pool->num_blocks};
+  cuuint64_t strides[2] = {(cuuint64_t)rowb, (cuuint64_t)rowb * pool->kv_heads * pool->block_size};
+  cuuint32_t box[3] = {(cuuint32_t)(boxb / eb), (cuuint32_t)kChunk, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 3,
+                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   boxb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return KV_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(KV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// cudaFuncSetAttribute once per (kernel instance, device).
+template <class K>
+int ensure_smem(K kernel, int bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const uint64_t bit = 1ull << (dev % kMaxDevices);
+  if (done.load(std::memory_order_acquire) & bit) return KV_OK;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return KV_OK;
+}
+
+int partition_tokens(const kv_pool* pool, int max_context_len) {
+  if (pool->partition_tokens > 0) return pool->partition_tokens;
+  (void)max_context_len;
+  return kDefaultPartition;
+}
+
+int num_parts_for(const kv_pool* pool, int max_context_len) {
+  const int pt = partition_tokens(pool, max_context_len);
+  return std::max(1, (max_context_len + pt - 1) / pt);
+}
+
+int stages_for(const kv_pool* pool) {
+  if (pool->stages > 0) return pool->stages;
+  return pool->dtype == KV_FP8_E4M3 ? 4 : 3;
+}
+
+template <int KV, int D, int STAGES>
+int launch_decode_t(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cudaStream_t stream) {
+  using Shape = DecodeShape<KV, D, kWarps, STAGES>;
+  auto kernel = paged_decode_kernel<KV, D, kWarps, STAGES>;
+  int rc = ensure_smem(kernel, Shape::SMEM_BYTES);
+  if (rc != KV_OK) return rc;
+  kernel<<<grid, kWarps * 32, Shape::SMEM_BYTES, stream>>>(p, lb.k_map, lb.v_map);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
+  return KV_OK;
+}
+
+template <int KV, int D>
+int launch_decode_d(int stages, const DecodeParams& p, const LayerBinding& lb, dim3 grid,
+                    cudaStream_t stream) {
+  switch (stages) {
+    case 2: return launch_decode_t<KV, D, 2>(p, lb, grid, stream);
+    case 3: return launch_decode_t<KV, D, 3>(p, lb, grid, stream);
+    case 4: return launch_decode_t<KV, D, 4>(p, lb, grid, stream);
+    default: return fail(KV_ERR_ARG, "unsupported stage count %d", stages);
+  }
+}
+
+template <int KV>
+int launch_decode_kv(int head_dim, int stages, const DecodeParams& p, const LayerBinding& lb,
+                     dim3 grid, cudaStream_t stream) {
+  if (head_dim == 64) return launch_decode_d<KV, 64>(stages, p, lb, grid, stream);
+  return launch_decode_d<KV, 128>(stages, p, lb, grid, stream);
+}
+
+bool valid_q_dtype(kv_dtype pool, kv_dtype q) {
+  if (pool == KV_FP8_E4M3) return q == KV_F16 || q == KV_BF16;
+  return q == pool;
+}
+
+int out_kind(kv_dtype t) { return t == KV_F32 ? OUT_F32 : (t == KV_BF16 ? OUT_BF16 : OUT_F16); }
+
+}  // namespace
+}  // namespace pagedkv
+
+using namespace pagedkv;
+
+extern "C" {
+
+int kv_pool_create(int block_size, int num_blocks, int kv_heads, int head_dim, kv_dtype dtype,
+                   int num_layers, kv_pool** out) {
+  if (!out) return fail(KV_ERR_ARG, "out is NULL");
+  if (block_size < 16 || block_size > 256 || block_size % 16 != 0)
+    return fail(KV_ERR_ARG, "block_size %d must be a multiple of 16 in [16, 256]", block_size);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(KV_ERR_ARG, "head_dim %d unsupported (64 or 128)", head_dim);
+  if (dtype != KV_F16 && dtype != KV_BF16 && dtype != KV_FP8_E4M3)
+    return fail(KV_ERR_ARG, "pool dtype %d unsupported", (int)dtype);
+  if (num_blocks <= 0 || kv_heads <= 0 || num_layers <= 0 || num_layers > kMaxLayers)
+    return fail(KV_ERR_ARG, "bad geometry: num_blocks %d kv_heads %d num_layers %d", num_blocks,
+                kv_heads, num_layers);
+  if ((int64_t)kv_heads * block_size > (1ll << 31))
+    return fail(KV_ERR_ARG, "kv_heads * block_size too large");
+  kv_pool* p = new (std::nothrow) kv_pool();
+  if (!p) return fail(KV_ERR_OOM, "host allocation failed");
+  p->block_size = block_size;
+  p->num_blocks = num_blocks;
+  p->kv_heads = kv_heads;
+  p->head_dim = head_dim;
+  p->dtype = dtype;
+  p->num_layers = num_layers;
+  p->layers.resize(num_layers);
+  *out = p;
+  return ok();
+}
+
+int kv_pool_bytes(const kv_pool* pool, size_t* kv_bytes_per_layer, size_t* scale_bytes_per_layer) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (kv_bytes_per_layer) *kv_bytes_per_layer = pool->layer_bytes();
+  if (scale_bytes_per_layer) *scale_bytes_per_layer = pool->scale_bytes();
+  return ok();
+}
+
+int kv_pool_bind(kv_pool* pool, int layer, void* k_base, void* v_base, float* k_scale,
+                 float* v_scale) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (layer < 0 || layer >= pool->num_layers)
+    return fail(KV_ERR_ARG, "layer %d out of range [0, %d)", layer, pool->num_layers);
+  if (!k_base || !v_base) return fail(KV_ERR_ARG, "K/V base is NULL");
+  if (((uintptr_t)k_base | (uintptr_t)v_base) & 15)
+    return fail(KV_ERR_ARG, "K/V base must be 16-byte aligned");
+  const bool fp8 = pool->dtype == KV_FP8_E4M3;
+  if (fp8 && (!k_scale || !v_scale)) return fail(KV_ERR_ARG, "FP8 pools need K and V scales");
+  if (!fp8 && (k_scale || v_scale)) return fail(KV_ERR_ARG, "scales are only for FP8 pools");
+  LayerBinding lb;
+  int rc = make_map(pool, k_base, &lb.k_map);
+  if (rc != KV_OK) return rc;
+  rc = make_map(pool, v_base, &lb.v_map);
+  if (rc != KV_OK) return rc;
+  lb.k = k_base;
+  lb.v = v_base;
+  lb.k_scale = k_scale;
+  lb.v_scale = v_scale;
+  lb.bound = true;
+  pool->layers[layer] = lb;
+  return ok();
+}
+
+int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (partition_tokens != 0 &&
+      (partition_tokens < kChunk || partition_tokens > kChunk * kMaxPartChunks ||
+       partition_tokens % kChunk != 0))
+    return fail(KV_ERR_ARG, "partition_tokens %d must be 0 or a multiple of 16 in [16, %d]",
+                partition_tokens, kChunk * kMaxPartChunks);
+  if (stages != 0 && (stages < 2 || stages > 4))
+    return fail(KV_ERR_ARG, "stages %d must be 0 or 2..4", stages);
+  pool->partition_tokens = partition_tokens;
+  pool->stages = stages;
+  return ok();
+}
+
+int kv_pool_destroy(kv_pool* pool) {
+  delete pool;
+  return ok();
+}
+
+int paged_kv_write(const kv_pool* pool, int layer, const void* k_new, const void* v_new,
+                   kv_dtype src_dtype, const int64_t* slot_mapping, int num_tokens,
+                   const float* k_inv_scale, const float* v_inv_scale, kv_stream_t stream) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (layer < 0 || layer >= pool->num_layers) return fail(KV_ERR_ARG, "layer %d out of range", layer);
+  if (num_tokens < 0) return fail(KV_ERR_ARG, "num_tokens < 0");
+  const LayerBinding& lb = pool->layers[layer];
+  if (!lb.bound) return fail(KV_ERR_STATE, "layer %d is not bound", layer);
+  const bool fp8 = pool->dtype == KV_FP8_E4M3;
+  if (!valid_q_dtype(pool->dtype, src_dtype))
+    return fail(KV_ERR_ARG, "source dtype %d does not fit pool dtype %d", (int)src_dtype,
+                (int)pool->dtype);
+  if (fp8 && (!k_inv_scale || !v_inv_scale)) return fail(KV_ERR_ARG, "FP8 writes need inverse scales");
+  if (num_tokens == 0) return ok();
+  if (!k_new || !v_new || !slot_mapping) return fail(KV_ERR_ARG, "NULL input");
+  if (((uintptr_t)k_new | (uintptr_t)v_new) & 15) return fail(KV_ERR_ARG, "k_new/v_new must be 16-byte aligned");
+  WriteParams p;
+  p.k_new = static_cast<const uint8_t*>(k_new);
+  p.v_new = static_cast<const uint8_t*>(v_new);
+  p.slots = slot_mapping;
+  p.k = static_cast<uint8_t*>(lb.k);
+  p.v = static_cast<uint8_t*>(lb.v);
+  p.k_inv = k_inv_scale;
+  p.v_inv = v_inv_scale;
+  p.rows = (int64_t)num_tokens * pool->kv_heads;
+  p.kv_heads = pool->kv_heads;
+  p.head_dim = pool->head_dim;
+  p.block_size = pool->block_size;
+  p.num_blocks = pool->num_blocks;
+  p.src_bf16 = src_dtype == KV_BF16;
+  const int64_t threads = p.rows * (pool->head_dim / 8);
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > 0x7fffffff) return fail(KV_ERR_ARG, "too many tokens");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (fp8)
+    kv_write_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(p);
+  else
+    kv_write_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kv_write_kernel launch");
+  return ok();
+}
+
+int block_copy(const kv_pool* pool, const int32_t* pairs, int num_pairs, kv_stream_t stream) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (num_pairs < 0 || num_pairs > 0x7fffffff / 2) return fail(KV_ERR_ARG, "bad num_pairs");
+  if (num_pairs == 0) return ok();
+  if (!pairs) return fail(KV_ERR_ARG, "pairs is NULL");
+  for (int l = 0; l < pool->num_layers; ++l)
+    if (!pool->layers[l].bound) return fail(KV_ERR_STATE, "layer %d is not bound", l);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int l0 = 0; l0 < pool->num_layers; l0 += kCopyLayers) {
+    const int nl = std::min(kCopyLayers, pool->num_layers - l0);
+    CopyParams p;
+    std::memset(&p, 0, sizeof p);
+    p.pairs = pairs;
+    p.num_pairs = num_pairs;
+    p.num_blocks = pool->num_blocks;
+    p.kv_heads = pool->kv_heads;
+    p.block_bytes = (int64_t)pool->block_bytes();
+    for (int i = 0; i < nl; ++i) {
+      const LayerBinding& lb = pool->layers[l0 + i];
+      p.k[i] = lb.k;
+      p.v[i] = lb.v;
+      p.ks[i] = lb.k_scale;
+      p.vs[i] = lb.v_scale;
+    }
+    block_copy_kernel<<<dim3(num_pairs, nl, 2), 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "block_copy_kernel launch");
+  }
+  return ok();
+}
+
+size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
+                                       int max_context_len) {
+  if (!pool || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
+  const int np = num_parts_for(pool, max_context_len);
+  if (np <= 1) return 0;
+  return (size_t)batch * num_q_heads * np * (pool->head_dim + 2) * sizeof(float);
+}
+
+int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
+                           int num_q_heads, const int32_t* block_tables, int max_blocks_per_seq,
+                           const int32_t* context_lens, int batch, int max_context_len,
+                           float scale, void* out, kv_dtype out_dtype, void* workspace,
+                           size_t workspace_bytes, kv_stream_t stream) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (layer < 0 || layer >= pool->num_layers) return fail(KV_ERR_ARG, "layer %d out of range", layer);
+  const LayerBinding& lb = pool->layers[layer];
+  if (!lb.bound) return fail(KV_ERR_STATE, "layer %d is not bound", layer);
+  if (batch < 0 || max_context_len < 0 || max_blocks_per_seq < 0)
+    return fail(KV_ERR_ARG, "negative size");
+  if (batch > 65535) return fail(KV_ERR_ARG, "batch %d above 65535", batch);
+  if (num_q_heads <= 0 || num_q_heads % pool->kv_heads != 0 ||
+      num_q_heads / pool->kv_heads > kMaxGroup)
+    return fail(KV_ERR_ARG, "num_q_heads %d must be a multiple of kv_heads %d, at most %dx",
+                num_q_heads, pool->kv_heads, kMaxGroup);
+  if (pool->kv_heads > 65535) return fail(KV_ERR_ARG, "kv_heads above 65535");
+  if (!valid_q_dtype(pool->dtype, q_dtype))
+    return fail(KV_ERR_ARG, "q dtype %d does not fit pool dtype %d", (int)q_dtype, (int)pool->dtype);
+  if (out_dtype != q_dtype && out_dtype != KV_F32)
+    return fail(KV_ERR_ARG, "out dtype must be the q dtype or KV_F32");
+  if (!std::isfinite(scale)) return fail(KV_ERR_ARG, "scale is not finite");
+  if (batch == 0) return ok();
+  if (!q || !block_tables || !context_lens || !out) return fail(KV_ERR_ARG, "NULL input");
+  if ((uintptr_t)q & 7) return fail(KV_ERR_ARG, "q must be 8-byte aligned");
+  if ((int64_t)max_blocks_per_seq * pool->block_size < max_context_len)
+    return fail(KV_ERR_ARG, "max_blocks_per_seq %d cannot hold max_context_len %d",
+                max_blocks_per_seq, max_context_len);
+  const int pt = partition_tokens(pool, max_context_len);
+  const int np = num_parts_for(pool, max_context_len);
+  if (np > 65535) return fail(KV_ERR_ARG, "too many partitions");
+  const size_t need = paged_attention_workspace_bytes(pool, batch, num_q_heads, max_context_len);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(KV_ERR_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if (need > 0 && ((uintptr_t)workspace & 15)) return fail(KV_ERR_ARG, "workspace must be 16-byte aligned");
+
+  DecodeParams p;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.k_scale = lb.k_scale;
+  p.v_scale = lb.v_scale;
+  p.out = out;
+  float* ws = static_cast<float*>(workspace);
+  p.part_o = need ? ws : nullptr;
+  p.part_ml = need ? ws + (size_t)batch * num_q_heads * np * pool->head_dim : nullptr;
+  p.q_bf16 = q_dtype == KV_BF16;
+  p.out_kind = out_kind(out_dtype);
+  p.num_q_heads = num_q_heads;
+  p.group = num_q_heads / pool->kv_heads;
+  p.kv_heads = pool->kv_heads;
+  p.block_size = pool->block_size;
+  p.num_blocks = pool->num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.part_chunks = pt / kChunk;
+  p.num_parts = np;
+  p.ctx_cap = (int)std::min<int64_t>((int64_t)max_blocks_per_seq * pool->block_size, max_context_len);
+  p.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(np, pool->kv_heads, batch);
+  const int stages = stages_for(pool);
+  int rc;
+  switch (pool->dtype) {
+    case KV_F16: rc = launch_decode_kv<KV_KIND_F16>(pool->head_dim, stages, p, lb, grid, s); break;
+    case KV_BF16: rc = launch_decode_kv<KV_KIND_BF16>(pool->head_dim, stages, p, lb, grid, s); break;
+    default: rc = launch_decode_kv<KV_KIND_E4M3>(pool->head_dim, stages, p, lb, grid, s); break;
+  }
+  if (rc != KV_OK) return rc;
+  if (np > 1) {
+    const int64_t rows = (int64_t)batch * num_q_heads;
+    const int blocks = (int)((rows + 7) / 8);
+    lse_reduce_kernel<<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, context_lens, out, p.out_kind,
+                                             num_q_heads, pool->head_dim, np, pt, p.ctx_cap, batch);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
+  }
+  return ok();
+}
+
+int kv_get_device_error(kv_stream_t stream, int* err) {
+  if (!err) return fail(KV_ERR_ARG, "err is NULL");
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int h = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  *err = h;
+  return ok();
+}
+
+}  // extern "C"
