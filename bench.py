@@ -1,0 +1,519 @@
+"""Benchmark of the paged-decode hot path on B200.
+
+One step = the cache write of the step's new tokens (paged_kv_write) and one
+PagedAttention decode over every sequence (paged_attention_decode, with its
+split-K reduce when contexts are split), all through the C ABI, on inputs
+resident in HBM.  Default workload: one Llama-2-13B-shaped layer (40 MHA
+heads, head_dim 128, fp16, block 16, batch 64, context lengths uniform in
+[128, 2048]).
+
+Prints one JSON line (rank 0).  ``value`` is achieved GB/s of algorithmic
+bytes (K/V read + q read + output write + the step's cache-write bytes) over
+the device-timed step, summed over ranks; ``--impl reference`` times the CPU
+oracle on the same workload instead.
+
+Multi-GPU: ``torchrun --nproc-per-node N bench.py --gpus N``: every rank runs
+an independent replica (decode shards by sequence with no exchange), time is
+the max over ranks, ``value`` the bytes of all ranks over that time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: achieved KV-read GB/s (% of HBM peak); decode seqs/s"
+FALLBACK_HBM_GBS = 6650.0
+DTYPE_NAME = {0: "f16", 1: "bf16", 2: "e4m3"}
+ELEM = {0: 2, 1: 2, 2: 1}
+
+
+# ------------------------------------------------------------------ helpers
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_451_b200", "csrc")
+    for f in ("decode.cuh", "ptx.cuh", "pagedkv.cu"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload):
+    """DRAM bytes per decode launch from a committed ncu capture, if it was
+    taken on the current decode source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f).get(workload)
+    except Exception:  # noqa: BLE001
+        return None
+    if not rec or rec.get("source_hash") != decode_source_hash():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls NVML (the library nvidia-smi reads) for SM clock and throttle
+    reasons while the timed region runs.  Read-only."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples, self.reasons = [], 0
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:  # noqa: BLE001
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.ok = True
+        except Exception:  # noqa: BLE001
+            pass
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                self.reasons |= self.get_reasons(self.h)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples), "source": "nvml"}
+
+
+# --------------------------------------------------------------- workloads
+
+class Case:
+    """Device-resident inputs of one workload replica."""
+
+    def __init__(self, name, rank, torch, pk, W):
+        from workloads import (WORKLOADS, blocks_needed, context_lens, device_normal_bits,
+                               device_pool, pool_blocks, scattered_tables, rng_for)
+        w = WORKLOADS[name]
+        self.w, self.torch, self.pk = w, torch, pk
+        self.lens = context_lens(w)
+        nb = pool_blocks(w, self.lens)
+        self.nb = nb
+        rng = np.random.default_rng([w.seed, 1000 + rank])
+        self.tables = scattered_tables(rng, self.lens, w.block_size, nb)
+        dev = torch.device("cuda")
+        seed = w.seed * 7919 + rank
+        self.L = w.num_layers
+        self.k, self.v, self.ks, self.vs = [], [], [], []
+        self.pool = pk.kv_pool_create(w.block_size, nb, w.kv_heads, w.head_dim, w.kv_fmt, self.L)
+        for layer in range(self.L):
+            k, v, ks, vs = device_pool(w, nb, dev, seed=seed + 13 * layer)
+            self.k.append(k)
+            self.v.append(v)
+            self.ks.append(ks)
+            self.vs.append(vs)
+            pk.kv_pool_bind(self.pool, layer, k, v, ks, vs)
+        B, Hq, Hkv, D = w.batch, w.num_q_heads, w.kv_heads, w.head_dim
+        self.q = [device_normal_bits((B, Hq, D), w.q_fmt, dev, seed + 1 + 17 * l) for l in range(self.L)]
+        self.kn = [device_normal_bits((B, Hkv, D), w.q_fmt, dev, seed + 2 + 17 * l) for l in range(self.L)]
+        self.vn = [device_normal_bits((B, Hkv, D), w.q_fmt, dev, seed + 3 + 17 * l) for l in range(self.L)]
+        # the step writes each sequence's last token (position len-1)
+        pos = self.lens.astype(np.int64) - 1
+        self.slots_h = (self.tables[np.arange(B), pos // w.block_size].astype(np.int64) * w.block_size
+                        + pos % w.block_size)
+        self.slots = torch.from_numpy(self.slots_h).to(dev)
+        self.tables_d = torch.from_numpy(self.tables).to(dev)
+        self.lens_d = torch.from_numpy(self.lens).to(dev)
+        self.inv = None
+        if w.kv_fmt == 2:
+            self.inv = [(1.0 / self.ks[l], 1.0 / self.vs[l]) for l in range(self.L)]
+        self.max_ctx = int(self.lens.max())
+        out_dt = torch.float16 if w.q_fmt == 0 else torch.bfloat16
+        self.out = [torch.empty((B, Hq, D), dtype=out_dt, device=dev) for _ in range(self.L)]
+        self.ws_bytes = pk.paged_attention_workspace_bytes(self.pool, B, Hq, self.max_ctx)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.split = self.ws_bytes > 0
+        e_kv, e_q = ELEM[w.kv_fmt], ELEM[w.q_fmt]
+        blocks_touched = int(blocks_needed(self.lens, w.block_size).sum())
+        self.decode_bytes = self.L * (int(self.lens.astype(np.int64).sum()) * Hkv * D * 2 * e_kv
+                                      + B * Hq * D * (e_q + e_q)
+                                      + (2 * 4 * blocks_touched * Hkv if w.kv_fmt == 2 else 0))
+        self.write_bytes = self.L * B * Hkv * D * 2 * (e_q + e_kv)
+        self.step_bytes = self.decode_bytes + self.write_bytes
+        self.launches_per_step = self.L * (2 + (1 if self.split else 0))
+
+    def write(self, layer, kn=None, vn=None, slots=None):
+        w, pk = self.w, self.pk
+        inv = self.inv[layer] if self.inv else (None, None)
+        pk.paged_kv_write(self.pool, layer, self.kn[layer] if kn is None else kn,
+                          self.vn[layer] if vn is None else vn, w.q_fmt,
+                          self.slots if slots is None else slots, w.batch, inv[0], inv[1])
+
+    def decode(self, layer, q=None, tables=None, lens=None, out=None):
+        w, pk = self.w, self.pk
+        pk.paged_attention_decode(self.pool, layer, self.q[layer] if q is None else q, w.q_fmt,
+                                  w.num_q_heads, self.tables_d if tables is None else tables,
+                                  self.tables.shape[1], self.lens_d if lens is None else lens, w.batch,
+                                  self.max_ctx, w.scale, self.out[layer] if out is None else out,
+                                  w.q_fmt, self.ws, self.ws_bytes)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import paged_kv_cache_451_b200 as pk
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    case = Case(args.workload, rank, torch, pk, args)
+    if args.partition or args.stages:
+        pk.kv_pool_set_decode_config(case.pool, args.partition, args.stages)
+        case.ws_bytes = pk.paged_attention_workspace_bytes(case.pool, case.w.batch, case.w.num_q_heads, case.max_ctx)
+        case.ws = torch.empty(max(case.ws_bytes, 16), dtype=torch.uint8, device="cuda")
+        case.split = case.ws_bytes > 0
+        case.launches_per_step = case.L * (2 + (1 if case.split else 0))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step(ev_write=None, ev_dec=None):
+        for layer in range(case.L):
+            case.write(layer)
+            if ev_write is not None:
+                ev_write[layer].record(stream)
+            case.decode(layer)
+            if ev_dec is not None:
+                ev_dec[layer].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error during warm-up")
+
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    evw = [[torch.cuda.Event(enable_timing=True) for _ in range(case.L)] for _ in range(K)]
+    evd = [[torch.cuda.Event(enable_timing=True) for _ in range(case.L)] for _ in range(K)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev0[i].record(stream)
+            step(evw[i], evd[i])
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    step_ms = [ev0[i].elapsed_time(evd[i][-1]) for i in range(K)]
+    dec_ms = []
+    for i in range(K):
+        for layer in range(case.L):
+            dec_ms.append(evw[i][layer].elapsed_time(evd[i][layer]))
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    dec_bytes_per_launch = case.decode_bytes / case.L
+
+    # end to end through the C ABI with host buffers (pinned), copies timed
+    e2e = run_e2e(case, torch, pk, flush, stream, K, args.warmup)
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error during timing")
+
+    peak, peak_kind = hbm_peak()
+    value = world * case.step_bytes / (ms_per_step * 1e-3) / 1e9
+    achieved = dec_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
+    w = case.w
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": DTYPE_NAME[w.kv_fmt],
+        "data": "synthetic (seeded N(0,1) q/K/V drawn on device; seeded lengths and scattered block placement)",
+        "config": {
+            "workload": describe(w, case),
+            "global_batch": w.batch * world,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed between steps (256 MiB write)",
+            "split_k": bool(case.split),
+        },
+        "seqs_per_s": round(world * w.batch / (ms_per_step * 1e-3), 1),
+        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
+        "hbm_peak_gbs": peak,
+        "hbm_peak_kind": peak_kind,
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "paged_attention_decode (decode kernel" + (" + LSE reduce)" if case.split else ")"),
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": committed_traffic(args.workload),
+            "algorithmic_bytes_per_launch": dec_bytes_per_launch,
+            "launch_ms": round(dec_avg_ms, 5),
+            "peak_note": f"{peak_kind} copy bandwidth",
+        },
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": case.launches_per_step * K,
+    }
+    if dist:
+        dist.barrier()
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, torch, target_s=args.cpu_seconds)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def describe(w, case=None):
+    names = {
+        "tiny": "tiny: 1 layer, 4 seqs ctx {2,18,34,101}, 4 MHA heads, head_dim 64, block 16, fp16",
+        "llama13b": "Llama-2-13B-shaped layer: 40 MHA heads, head_dim 128, block 16, fp16, batch 64, ctx U[128,2048]",
+        "kv_example": "KV-size example: 32 layers x 32 heads x head_dim 128, bf16, block 16, batch 32, ctx 2048",
+        "gqa_trace": "GQA 64/8 heads, head_dim 128, bf16, block 16, batch 256, lognormal ctx (median 1024, cap 8192)",
+        "fp8_long": "long-context FP8: 32 MHA heads, head_dim 128, E4M3 cache + per-(block,head) scales, bf16 q, batch 8, ctx 16384",
+    }
+    s = names[w.name]
+    if case is not None:
+        s += f"; pool {case.nb} blocks; sum ctx {int(case.lens.sum())}"
+    return s
+
+
+def run_e2e(case, torch, pk, flush, stream, K, W):
+    """Same step, inputs from pinned host memory: H2D of q, new K/V, slots,
+    tables and lengths, then the write and decode, then D2H of the output."""
+    w = case.w
+    hq = [t.cpu().pin_memory() for t in case.q]
+    hk = [t.cpu().pin_memory() for t in case.kn]
+    hv = [t.cpu().pin_memory() for t in case.vn]
+    hs = torch.from_numpy(case.slots_h).pin_memory()
+    ht = torch.from_numpy(case.tables).pin_memory()
+    hl = torch.from_numpy(case.lens).pin_memory()
+    hout = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in case.out]
+    dq = [torch.empty_like(t) for t in case.q]
+    dk = [torch.empty_like(t) for t in case.kn]
+    dv = [torch.empty_like(t) for t in case.vn]
+    ds, dt, dl = torch.empty_like(case.slots), torch.empty_like(case.tables_d), torch.empty_like(case.lens_d)
+    h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv) + sum(
+        t.numel() * t.element_size() for t in (hs, ht, hl))
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+
+    def step():
+        ds.copy_(hs, non_blocking=True)
+        dt.copy_(ht, non_blocking=True)
+        dl.copy_(hl, non_blocking=True)
+        for layer in range(case.L):
+            dq[layer].copy_(hq[layer], non_blocking=True)
+            dk[layer].copy_(hk[layer], non_blocking=True)
+            dv[layer].copy_(hv[layer], non_blocking=True)
+            case.write(layer, dk[layer], dv[layer], ds)
+            case.decode(layer, dq[layer], dt, dl)
+            hout[layer].copy_(case.out[layer], non_blocking=True)
+
+    for _ in range(W):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        a[i].record(stream)
+        step()
+        b[i].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a[i].elapsed_time(b[i]) for i in range(K)) / K
+    return {"value": round(case.step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------- CPU oracle legs
+
+def oracle_sample(case_like, seqs, layer=0):
+    """Host inputs of the sampled sequences (their blocks, remapped tables)."""
+    import torch
+    w = case_like.w
+    bs = w.block_size
+    used, sub = [], np.full((len(seqs), case_like.tables.shape[1]), -1, np.int32)
+    for i, s in enumerate(seqs):
+        for j in range(-(-int(case_like.lens[s]) // bs)):
+            sub[i, j] = len(used)
+            used.append(int(case_like.tables[s, j]))
+    idx = torch.tensor(used, dtype=torch.long, device=case_like.k[layer].device)
+    raw = np.uint8 if w.kv_fmt == 2 else np.uint16
+    kh = case_like.k[layer].index_select(0, idx).cpu().numpy().view(raw)
+    vh = case_like.v[layer].index_select(0, idx).cpu().numpy().view(raw)
+    ks = vs = None
+    if w.kv_fmt == 2:
+        ks = case_like.ks[layer].index_select(0, idx).cpu().numpy()
+        vs = case_like.vs[layer].index_select(0, idx).cpu().numpy()
+    q = case_like.q[layer].cpu().numpy().view(np.uint16)[list(seqs)]
+    return kh, vh, ks, vs, q, sub, case_like.lens[list(seqs)].astype(np.int32)
+
+
+def cpu_baseline(case, torch, target_s=15.0, steps=1):
+    """The oracle, as it stands, on a bounded sample of the same workload."""
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    w = case.w
+    order = list(range(w.batch))
+    # calibrate on one sequence, then size the sample to ~target_s
+    t0 = time.perf_counter()
+    args = oracle_sample(case, order[:1])
+    oracle.paged_decode(args[0], args[1], w.kv_fmt, args[4], w.q_fmt, args[5], args[6], w.scale,
+                        w.block_size, args[2], args[3])
+    one = max(time.perf_counter() - t0, 1e-3)
+    n = int(min(w.batch, max(1, target_s / one / max(1, case.L))))
+    seqs = order[:n]
+    total_s, total_bytes, passes = 0.0, 0, 0
+    samples = [oracle_sample(case, seqs, layer) for layer in range(case.L)] if case.L == 1 else None
+    # repeat the sample until about target_s of CPU work (at least `steps` passes)
+    while passes < steps or total_s < 0.5 * target_s:
+        for layer in range(case.L):
+            kh, vh, ks, vs, q, sub, lens = samples[0] if samples else oracle_sample(case, seqs, layer)
+            t0 = time.perf_counter()
+            oracle.paged_decode(kh, vh, w.kv_fmt, q, w.q_fmt, sub, lens, w.scale, w.block_size, ks, vs)
+            total_s += time.perf_counter() - t0
+            total_bytes += (int(lens.astype(np.int64).sum()) * w.kv_heads * w.head_dim * 2 * ELEM[w.kv_fmt]
+                            + n * w.num_q_heads * w.head_dim * 2 * ELEM[w.q_fmt])
+        passes += 1
+        if n < w.batch:
+            break
+    steps = passes
+    return {"value": round(total_bytes / total_s / 1e9, 4), "unit": "GB/s",
+            "seqs_per_s": round(steps * n / total_s, 3), "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {w.batch} sequences x {case.L} layer(s), decode only, fp64 C oracle "
+                      f"(OpenMP over (sequence, head)); {total_s:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle timed on the host cores, each step a
+    bounded sample of the same workload."""
+    import torch
+    if rank != 0:
+        return None
+    torch.cuda.set_device(0)
+    import paged_kv_cache_451_b200 as pk
+    case = Case(args.workload, 0, torch, pk, args)
+    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(case, torch, target_s=per_step)
+    res = cpu_baseline(case, torch, target_s=per_step * args.steps, steps=1)
+    w = case.w
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": res["value"],
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": None,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": describe(w, case), "global_batch": w.batch},
+        "seqs_per_s": res["seqs_per_s"],
+        "cpu_baseline": res,
+        "e2e": {"value": res["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama13b",
+                    choices=["tiny", "llama13b", "kv_example", "fp8_long"])
+    ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
+    ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_ours(args, rank, world, local_rank)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -100,11 +100,14 @@ int kv_pool_bind(kv_pool* pool, int layer, void* k_base, void* v_base, float* k_
                  float* v_scale);
 
 /* Decode launch configuration.  partition_tokens: context-partition length
- * for split decode, 0 for automatic, else a multiple of 16 in [16, 4096];
- * contexts longer than one partition are split into partitions whose
- * partial results are merged by a log-sum-exp reduce (see
- * paged_attention_decode).  stages: shared-memory pipeline depth per warp,
- * 0 for automatic, else 2..4.  Host only. */
+ * for split decode, else a multiple of 16 in [16, 4096]; contexts longer
+ * than one partition are split into partitions whose partial results are
+ * merged by a log-sum-exp reduce (see paged_attention_decode).  0 chooses
+ * automatically: no split while batch * kv_heads gives about eight waves of
+ * resident CTAs (and max_context_len <= 4096), else just enough partitions
+ * of at least 256 tokens to reach that.  stages: shared-memory pipeline
+ * depth per warp, 0 for automatic (about 24 KB of K/V in flight per warp),
+ * else 2, 3, 4, 6 or 8.  Host only. */
 int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages);
 
 int kv_pool_destroy(kv_pool* pool);

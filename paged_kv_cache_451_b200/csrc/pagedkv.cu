@@ -27,7 +27,6 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kMaxLayers = 4096;
 constexpr int kMaxDevices = 64;
-constexpr int kDefaultPartition = 512;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -74,10 +73,10 @@ int cuda_fail(cudaError_t e, const char* what) {
   return fail(KV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// cudaFuncSetAttribute once per (kernel instance, device).
+// cudaFuncSetAttribute once per (kernel, device); `done` must be a flag word
+// owned by that kernel alone.
 template <class K>
-int ensure_smem(K kernel, int bytes) {
-  static std::atomic<uint64_t> done{0};
+int ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -89,27 +88,76 @@ int ensure_smem(K kernel, int bytes) {
   return KV_OK;
 }
 
-int partition_tokens(const kv_pool* pool, int max_context_len) {
-  if (pool->partition_tokens > 0) return pool->partition_tokens;
-  (void)max_context_len;
-  return kDefaultPartition;
-}
-
-int num_parts_for(const kv_pool* pool, int max_context_len) {
-  const int pt = partition_tokens(pool, max_context_len);
-  return std::max(1, (max_context_len + pt - 1) / pt);
-}
-
 int stages_for(const kv_pool* pool) {
   if (pool->stages > 0) return pool->stages;
-  return pool->dtype == KV_FP8_E4M3 ? 4 : 3;
+  // about 24 KB of K/V in flight per warp: 3 stages of 8 KB (16-bit, D 128),
+  // 6 of 4 KB (FP8 D 128 or 16-bit D 64), 8 of 2 KB (FP8 D 64)
+  const int stage_bytes = 2 * kChunk * pool->head_dim * elem_bytes(pool->dtype);
+  return stage_bytes >= 8192 ? 3 : (stage_bytes >= 4096 ? 6 : 8);
+}
+
+template <int KV, int D>
+int smem_bytes_d(int stages) {
+  switch (stages) {
+    case 2: return DecodeShape<KV, D, kWarps, 2>::SMEM_BYTES;
+    case 3: return DecodeShape<KV, D, kWarps, 3>::SMEM_BYTES;
+    case 4: return DecodeShape<KV, D, kWarps, 4>::SMEM_BYTES;
+    case 6: return DecodeShape<KV, D, kWarps, 6>::SMEM_BYTES;
+    default: return DecodeShape<KV, D, kWarps, 8>::SMEM_BYTES;
+  }
+}
+
+int smem_bytes(const kv_pool* pool, int stages) {
+  const bool d64 = pool->head_dim == 64;
+  switch (pool->dtype) {
+    case KV_FP8_E4M3: return d64 ? smem_bytes_d<KV_KIND_E4M3, 64>(stages) : smem_bytes_d<KV_KIND_E4M3, 128>(stages);
+    default: return d64 ? smem_bytes_d<KV_KIND_F16, 64>(stages) : smem_bytes_d<KV_KIND_F16, 128>(stages);
+  }
+}
+
+// Resident decode CTAs the current device holds at once.
+int decode_slots(const kv_pool* pool) {
+  static std::atomic<int> sm_count[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  int sms = sm_count[dev % kMaxDevices].load(std::memory_order_relaxed);
+  if (sms == 0) {
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+    sm_count[dev % kMaxDevices].store(sms, std::memory_order_relaxed);
+  }
+  const int per_sm = std::max(1, (227 * 1024) / smem_bytes(pool, stages_for(pool)));
+  return sms * per_sm;
+}
+
+// Partition length in tokens.  Automatic: keep each (sequence, kv head) in
+// one CTA when there are enough of them for about eight waves of resident
+// CTAs; otherwise split the longest context into just enough partitions to
+// reach that, and always keep partitions within kMaxPartChunks chunks.
+int partition_tokens(const kv_pool* pool, int batch, int max_context_len) {
+  if (pool->partition_tokens > 0) return pool->partition_tokens;
+  const int ctx = std::max(max_context_len, 1);
+  const int64_t units = std::max<int64_t>(1, (int64_t)batch * pool->kv_heads);
+  const int64_t want = 8ll * decode_slots(pool);
+  int64_t np = std::max<int64_t>((ctx + kChunk * kMaxPartChunks - 1) / (kChunk * kMaxPartChunks),
+                                 (want + units - 1) / units);
+  np = std::min<int64_t>(np, (ctx + 255) / 256);  // partitions of at least 256 tokens
+  np = std::max<int64_t>(np, 1);
+  const int64_t per = (ctx + np - 1) / np;
+  return (int)std::min<int64_t>(kChunk * kMaxPartChunks, (per + kChunk - 1) / kChunk * kChunk);
+}
+
+int num_parts_for(const kv_pool* pool, int batch, int max_context_len) {
+  const int pt = partition_tokens(pool, batch, max_context_len);
+  return std::max(1, (max_context_len + pt - 1) / pt);
 }
 
 template <int KV, int D, int STAGES>
 int launch_decode_t(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cudaStream_t stream) {
   using Shape = DecodeShape<KV, D, kWarps, STAGES>;
   auto kernel = paged_decode_kernel<KV, D, kWarps, STAGES>;
-  int rc = ensure_smem(kernel, Shape::SMEM_BYTES);
+  static std::atomic<uint64_t> done{0};  // one flag word per instantiation
+  int rc = ensure_smem(kernel, Shape::SMEM_BYTES, done);
   if (rc != KV_OK) return rc;
   kernel<<<grid, kWarps * 32, Shape::SMEM_BYTES, stream>>>(p, lb.k_map, lb.v_map);
   cudaError_t e = cudaGetLastError();
@@ -124,6 +172,8 @@ int launch_decode_d(int stages, const DecodeParams& p, const LayerBinding& lb, d
     case 2: return launch_decode_t<KV, D, 2>(p, lb, grid, stream);
     case 3: return launch_decode_t<KV, D, 3>(p, lb, grid, stream);
     case 4: return launch_decode_t<KV, D, 4>(p, lb, grid, stream);
+    case 6: return launch_decode_t<KV, D, 6>(p, lb, grid, stream);
+    case 8: return launch_decode_t<KV, D, 8>(p, lb, grid, stream);
     default: return fail(KV_ERR_ARG, "unsupported stage count %d", stages);
   }
 }
@@ -215,8 +265,8 @@ int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages) {
        partition_tokens % kChunk != 0))
     return fail(KV_ERR_ARG, "partition_tokens %d must be 0 or a multiple of 16 in [16, %d]",
                 partition_tokens, kChunk * kMaxPartChunks);
-  if (stages != 0 && (stages < 2 || stages > 4))
-    return fail(KV_ERR_ARG, "stages %d must be 0 or 2..4", stages);
+  if (stages != 0 && stages != 2 && stages != 3 && stages != 4 && stages != 6 && stages != 8)
+    return fail(KV_ERR_ARG, "stages %d must be 0, 2, 3, 4, 6 or 8", stages);
   pool->partition_tokens = partition_tokens;
   pool->stages = stages;
   return ok();
@@ -304,7 +354,7 @@ int block_copy(const kv_pool* pool, const int32_t* pairs, int num_pairs, kv_stre
 size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
                                        int max_context_len) {
   if (!pool || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
-  const int np = num_parts_for(pool, max_context_len);
+  const int np = num_parts_for(pool, batch, max_context_len);
   if (np <= 1) return 0;
   return (size_t)batch * num_q_heads * np * (pool->head_dim + 2) * sizeof(float);
 }
@@ -337,8 +387,8 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   if ((int64_t)max_blocks_per_seq * pool->block_size < max_context_len)
     return fail(KV_ERR_ARG, "max_blocks_per_seq %d cannot hold max_context_len %d",
                 max_blocks_per_seq, max_context_len);
-  const int pt = partition_tokens(pool, max_context_len);
-  const int np = num_parts_for(pool, max_context_len);
+  const int pt = partition_tokens(pool, batch, max_context_len);
+  const int np = num_parts_for(pool, batch, max_context_len);
   if (np > 65535) return fail(KV_ERR_ARG, "too many partitions");
   const size_t need = paged_attention_workspace_bytes(pool, batch, num_q_heads, max_context_len);
   if (need > 0 && (!workspace || workspace_bytes < need))

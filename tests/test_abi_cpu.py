@@ -62,11 +62,15 @@ def test_pool_bytes_and_workspace_sizes():
     pool = pk.kv_pool_create(16, 100, 8, 128, pk.KV_BF16, 2)
     kvb, sb = pk.kv_pool_bytes(pool)
     assert kvb == 100 * 8 * 16 * 128 * 2 and sb == 0
-    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 512) == 0
-    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 513) == 4 * 64 * 2 * 130 * 4
+    # automatic policy: many (sequence, kv head) units -> one partition each
+    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 4096) == 0
+    # few units -> split into partitions of at least 256 tokens
+    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 512) == 4 * 64 * 2 * 130 * 4
+    pk.kv_pool_set_decode_config(pool, 4096, 0)
+    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 4096) == 0
     pk.kv_pool_set_decode_config(pool, 256, 2)
     assert pk.paged_attention_workspace_bytes(pool, 4, 64, 513) == 4 * 64 * 3 * 130 * 4
-    for bad in ((8, 0), (4112, 0), (100, 0), (0, 5), (0, 1)):
+    for bad in ((8, 0), (4112, 0), (100, 0), (0, 5), (0, 1), (0, 7)):
         with pytest.raises(pk.KVError):
             pk.kv_pool_set_decode_config(pool, *bad)
     pk.kv_pool_destroy(pool)
