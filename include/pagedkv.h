@@ -189,6 +189,40 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
                            int max_context_len, float scale, void* out, kv_dtype out_dtype,
                            void* workspace, size_t workspace_bytes, kv_stream_t stream);
 
+/* Largest scratch paged_attention_decode_noalloc can use (16 MiB). */
+#define KV_NOALLOC_WORKSPACE_BYTES (16u << 20)
+
+/* The same decode as paged_attention_decode, for callers that cannot
+ * allocate device memory: a C host program or plugin that only receives the
+ * pool and the tensors it is handed, code whose whole memory budget is
+ * already given to the KV pool, or a hot path that must not call cudaMalloc
+ * because it can synchronise the device.  Instead of a caller-provided
+ * workspace, the split-K partials go to one scratch array that the library
+ * defines in device memory at file scope, KV_NOALLOC_WORKSPACE_BYTES long;
+ * every GPU that loads the library holds it until the process exits.  This
+ * entry point allocates nothing and has no counterpart on the pages; it is an
+ * interface convenience only.
+ *   Arguments are those of paged_attention_decode without the workspace.
+ *   Sizes whose paged_attention_workspace_bytes(...) exceeds
+ *   KV_NOALLOC_WORKSPACE_BYTES are rejected with KV_ERR_ARG (use
+ *   paged_attention_decode with your own workspace, or a partition setting
+ *   that needs fewer partials).
+ *   The first call on a device looks up the scratch array's device address
+ *   (once per device, with that device current); make that first call before
+ *   any stream capture.
+ *   All calls share the one array, which keeps whatever the last call wrote;
+ *   nothing in it has to start at zero, because every partial a call reads
+ *   was written earlier in that same call.  Calls whose kernels can overlap
+ *   on the GPU (other streams, other host threads) race on the array and
+ *   must be serialised by the caller.
+ * Errors: as paged_attention_decode, plus KV_ERR_CUDA if the scratch address
+ * lookup fails. */
+int paged_attention_decode_noalloc(const kv_pool* pool, int layer, const void* q,
+                                   kv_dtype q_dtype, int num_q_heads,
+                                   const int32_t* block_tables, int max_blocks_per_seq,
+                                   const int32_t* context_lens, int batch, int max_context_len,
+                                   float scale, void* out, kv_dtype out_dtype, kv_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the current device's error word:
  * *err = KV_OK, KV_ERR_BOUNDS or KV_ERR_TIMEOUT (the first error any kernel
  * of this library recorded since the last call).  Errors: KV_ERR_CUDA. */

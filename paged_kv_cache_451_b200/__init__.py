@@ -68,6 +68,9 @@ _SIGS = {
     "paged_attention_decode": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int,
                                        c_void_p, c_int, c_int, c_float, c_void_p, c_int, c_void_p,
                                        c_size_t, c_void_p]),
+    "paged_attention_decode_noalloc": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p,
+                                               c_int, c_void_p, c_int, c_int, c_float, c_void_p,
+                                               c_int, c_void_p]),
     "kv_get_device_error": (c_int, [c_void_p, P(c_int)]),
     "kv_alloc_create": (c_int, [c_int, c_int, c_void_p, P(c_void_p)]),
     "kv_alloc_num_free": (c_int, [c_void_p, P(c_int)]),
@@ -189,6 +192,18 @@ def paged_attention_decode(pool, layer, q, q_dtype, num_q_heads, block_tables, m
                                        _ptr(block_tables), max_blocks_per_seq, _ptr(context_lens),
                                        batch, max_context_len, float(scale), _ptr(out), out_dtype,
                                        _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+KV_NOALLOC_WORKSPACE_BYTES = 16 << 20
+
+
+def paged_attention_decode_noalloc(pool, layer, q, q_dtype, num_q_heads, block_tables,
+                                   max_blocks_per_seq, context_lens, batch, max_context_len, scale,
+                                   out, out_dtype, stream=None):
+    _check(_lib.paged_attention_decode_noalloc(pool, layer, _ptr(q), q_dtype, num_q_heads,
+                                               _ptr(block_tables), max_blocks_per_seq,
+                                               _ptr(context_lens), batch, max_context_len,
+                                               float(scale), _ptr(out), out_dtype, _stream(stream)))
 
 
 def kv_get_device_error(stream=None) -> int:

@@ -439,6 +439,66 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   return ok();
 }
 
+}  // extern "C"
+
+// Scratch for paged_attention_decode_noalloc: split-K partials of the calls
+// that cannot allocate.  Shared by every such call on a device.
+static __device__ __align__(256) float g_noalloc_scratch[KV_NOALLOC_WORKSPACE_BYTES / sizeof(float)];
+
+namespace pagedkv {
+namespace {
+
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (host code cannot use the symbol itself as a device address).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= kMaxDevices) return fail(KV_ERR_ARG, "device %d beyond %d devices", dev, kMaxDevices);
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+      g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return KV_OK;
+}
+
+}  // namespace
+}  // namespace pagedkv
+
+extern "C" {
+
+int paged_attention_decode_noalloc(const kv_pool* pool, int layer, const void* q,
+                                   kv_dtype q_dtype, int num_q_heads,
+                                   const int32_t* block_tables, int max_blocks_per_seq,
+                                   const int32_t* context_lens, int batch, int max_context_len,
+                                   float scale, void* out, kv_dtype out_dtype, kv_stream_t stream) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  const size_t need = paged_attention_workspace_bytes(pool, batch, num_q_heads, max_context_len);
+  if (need > KV_NOALLOC_WORKSPACE_BYTES)
+    return fail(KV_ERR_ARG,
+                "these sizes need %zu bytes of split-K scratch, above the %u-byte static scratch; "
+                "call paged_attention_decode with a workspace instead",
+                need, (unsigned)KV_NOALLOC_WORKSPACE_BYTES);
+  void* scratch = nullptr;
+  if (need > 0) {
+    int rc = noalloc_scratch(&scratch);
+    if (rc != KV_OK) return rc;
+  }
+  return paged_attention_decode(pool, layer, q, q_dtype, num_q_heads, block_tables,
+                                max_blocks_per_seq, context_lens, batch, max_context_len, scale, out,
+                                out_dtype, scratch, need > 0 ? KV_NOALLOC_WORKSPACE_BYTES : 0, stream);
+}
+
 int kv_get_device_error(kv_stream_t stream, int* err) {
   if (!err) return fail(KV_ERR_ARG, "err is NULL");
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
