@@ -219,8 +219,8 @@ def run_ours(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     case = Case(args.workload, rank, torch, pk, args)
-    if args.partition or args.stages:
-        pk.kv_pool_set_decode_config(case.pool, args.partition, args.stages)
+    if args.partition or args.stages or args.warps:
+        pk.kv_pool_set_decode_config(case.pool, args.partition, args.stages, args.warps)
         case.ws_bytes = pk.paged_attention_workspace_bytes(case.pool, case.w.batch, case.w.num_q_heads, case.max_ctx)
         case.ws = torch.empty(max(case.ws_bytes, 16), dtype=torch.uint8, device="cuda")
         case.split = case.ws_bytes > 0
@@ -330,6 +330,111 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
         dist.destroy_process_group()
     return line
+
+
+def unique_and_logical_tokens(tables, lens, block_size):
+    """Token slots the decode reads: counted once per physical block (unique,
+    what DRAM must deliver when shared blocks hit in L2) and once per
+    sequence (logical)."""
+    best = {}
+    logical = 0
+    for row, n in zip(tables, lens):
+        n = int(n)
+        logical += n
+        for j in range(-(-n // block_size)):
+            b = int(row[j])
+            best[b] = max(best.get(b, 0), min(block_size, n - j * block_size))
+    return sum(best.values()), logical
+
+
+def run_trace(args, rank, world, local_rank):
+    """The GQA continuous-batching trace: one step = one trace iteration."""
+    import torch
+    import paged_kv_cache_451_b200 as pk
+    from workloads import WORKLOADS, gqa_trace_plan
+    from workloads.gqa_trace import GqaTrace
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = WORKLOADS["gqa_trace"]
+    plan = gqa_trace_plan(w)
+    tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    iters = w.extra["iters"]
+    W = min(args.warmup, iters - 1)
+    K = max(1, min(args.steps, iters - W))
+    e = w.extra
+    hq, hkv, d = w.num_q_heads, w.kv_heads, w.head_dim
+    for it in range(W):
+        flush.zero_()
+        tr.iteration(it, out_dtype=w.q_fmt)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    uniq_b = logi_b = other_b = 0
+    launches = 0
+    host_s = sched_s = 0.0
+
+    def gate_and_start(i):
+        # keep the GPU busy (~1 ms device sleep) while the host enqueues the
+        # iteration, so the timed interval is the fed-GPU time of the step
+        torch.cuda._sleep(2_000_000)
+        starts[i].record(stream)
+
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.zero_()
+            t0 = time.perf_counter()
+            fin, arr, pl, q, kn, vn, out = tr.iteration(W + i, out_dtype=w.q_fmt,
+                                                        before_launch=lambda: gate_and_start(i),
+                                                        after_launch=lambda: ends[i].record(stream))
+            host_s += time.perf_counter() - t0
+            sched_s += tr.last_schedule_s
+            info = pl["info"]
+            u, l = unique_and_logical_tokens(pl["block_tables"], pl["context_lens"], w.block_size)
+            per_tok = hkv * d * 2 * 2
+            uniq_b += u * per_tok
+            logi_b += l * per_tok
+            other_b += (info.batch * hq * d * 4 + info.num_tokens * hkv * d * 2 * 4
+                        + info.num_cow * hkv * w.block_size * d * 2 * 2 * 2)
+            launches += 2 + (1 if info.num_cow else 0) + (
+                1 if pk.paged_attention_workspace_bytes(tr.pool, info.batch, hq, int(pl["context_lens"].max())) else 0)
+        torch.cuda.synchronize()
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error during the trace")
+    total_ms = sum(starts[i].elapsed_time(ends[i]) for i in range(K))
+    if dist:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    ms = total_ms / K
+    peak, peak_kind = hbm_peak()
+    value = world * (uniq_b + other_b) / (total_ms * 1e-3) / 1e9
+    logical = world * (logi_b + other_b) / (total_ms * 1e-3) / 1e9
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded lognormal lengths, shared prefix, Poisson arrivals; q/K/V drawn on device)",
+        "config": {"workload": describe(w), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between iterations (256 MiB write)",
+                   "step": "one trace iteration: native scheduler step, metadata upload, copy-on-write block copies, cache write, decode"},
+        "logical_gbs": round(logical, 2),
+        "unique_bytes_per_step": int((uniq_b + other_b) / K), "logical_bytes_per_step": int((logi_b + other_b) / K),
+        "host_scheduler_ms_per_step": round(1e3 * sched_s / K, 3),
+        "host_iteration_ms_per_step": round(1e3 * host_s / K, 3),
+        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2), "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
+        "clocks": clk.summary(), "gpu_launches": launches,
+    }
 
 
 def describe(w, case=None):
@@ -496,9 +601,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama13b",
-                    choices=["tiny", "llama13b", "kv_example", "fp8_long"])
+                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long"])
     ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")
+    ap.add_argument("--warps", type=int, default=0, help="warps per decode CTA (0: auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -509,6 +615,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         line = run_reference(args, rank, world)
+    elif args.workload == "gqa_trace":
+        line = run_trace(args, rank, world, local_rank)
     else:
         line = run_ours(args, rank, world, local_rank)
     if rank == 0 and line is not None:

@@ -76,7 +76,7 @@ int kv_version(void);
 /* Describe a preallocated pool ([PA], [PIT]): num_layers layers of
  * num_blocks physical blocks of block_size token slots for kv_heads heads of
  * head_dim elements of `dtype` (KV_F16, KV_BF16 or KV_FP8_E4M3).
- * Supported: block_size a multiple of 16 up to 256; head_dim 64 or 128;
+ * Supported: block_size 16, 32, 64, 128 or 256; head_dim 64 or 128;
  * num_blocks >= 1; 1 <= kv_heads; 1 <= num_layers <= 4096.  Host only; no
  * device work.  *out is owned by the caller until kv_pool_destroy.
  * Errors: KV_ERR_ARG for an unsupported geometry. */
@@ -100,15 +100,18 @@ int kv_pool_bind(kv_pool* pool, int layer, void* k_base, void* v_base, float* k_
                  float* v_scale);
 
 /* Decode launch configuration.  partition_tokens: context-partition length
- * for split decode, else a multiple of 16 in [16, 4096]; contexts longer
+ * for split decode, else a multiple of 16 in [16, 16384]; contexts longer
  * than one partition are split into partitions whose partial results are
  * merged by a log-sum-exp reduce (see paged_attention_decode).  0 chooses
- * automatically: no split while batch * kv_heads gives about eight waves of
- * resident CTAs (and max_context_len <= 4096), else just enough partitions
- * of at least 256 tokens to reach that.  stages: shared-memory pipeline
- * depth per warp, 0 for automatic (about 24 KB of K/V in flight per warp),
- * else 2, 3, 4, 6 or 8.  Host only. */
-int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages);
+ * automatically: partitions of at most 2048 tokens, and more of them (down
+ * to 512 tokens) while batch * kv_heads * partitions is under three waves of
+ * resident CTAs.  stages: shared-memory pipeline
+ * depth per warp, 0 for automatic, else 2, 3, 4, 6 or 8; warps: warps per
+ * CTA, 0 for automatic, else 4 or 8.  Automatic: 4 warps x 3 stages for
+ * 8 KB and 4 KB stages (16-bit or FP8 with head_dim 128, 16-bit with 64),
+ * 4 x 6 for 2 KB stages.  A shape whose shared memory exceeds 227 KB per CTA is rejected
+ * with KV_ERR_ARG.  Host only. */
+int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages, int warps);
 
 int kv_pool_destroy(kv_pool* pool);
 
@@ -179,8 +182,9 @@ size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q
  *                 paged_attention_workspace_bytes(...), 16-byte aligned;
  *                 may be NULL when that is 0.  Contexts longer than one
  *                 partition are split: each partition writes its unnormalised
- *                 output, running max and sum there, and a second kernel
- *                 merges them by log-sum-exp.
+ *                 output and its running maxima and sum there
+ *                 (head_dim + 4 floats per (sequence, head, partition)), and
+ *                 a second kernel merges them by log-sum-exp.
  * batch == 0 enqueues nothing.  Errors: KV_ERR_ARG, KV_ERR_STATE (layer not
  * bound), KV_ERR_CUDA. */
 int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,

@@ -194,33 +194,30 @@ def kv_write(k_pool, v_pool, kv_fmt, k_new, v_new, src_fmt, slot_mapping, block_
              k_inv_scale=None, v_inv_scale=None):
     """Host mirror of the slot-mapped cache write, in place on raw pools.
 
-    Token t's row k_new[t][h] goes to physical block slot // block_size at
-    offset slot % block_size (kv head h); a negative slot is skipped.  For a
-    16-bit pool the bits are copied unchanged (the source format must equal
-    the pool's).  For an FP8 pool each source value is widened to fp32 and
-    multiplied in fp32 by inv_scale[block][h], then rounded to E4M3 (nearest
-    even, saturating).  Raises IndexError for a block outside the pool.
+    Token t's rows new[t][h] (every kv head h) go to physical block
+    slot // block_size at offset slot % block_size; a negative slot is
+    skipped.  For a 16-bit pool the bits are copied unchanged (the source
+    format must equal the pool's).  For an FP8 pool each source value is
+    widened to fp32 and multiplied in fp32 by inv_scale[block][h], then
+    rounded to E4M3 (nearest even, saturating).  Slots are assumed distinct.
+    Raises IndexError for a block outside the pool.
     """
     nb, hkv, bs, d = k_pool.shape
     assert bs == block_size
-    slots = np.asarray(slot_mapping, dtype=np.int64)
+    slots = np.asarray(slot_mapping, dtype=np.int64).reshape(-1)
+    keep = np.nonzero(slots >= 0)[0]
+    blk, off = slots[keep] // block_size, slots[keep] % block_size
+    if blk.size and blk.max() >= nb:
+        raise IndexError("a slot is outside the pool")
     for pool, new, inv in ((k_pool, k_new, k_inv_scale), (v_pool, v_new, v_inv_scale)):
-        for t in range(slots.shape[0]):
-            slot = int(slots[t])
-            if slot < 0:
-                continue
-            blk, off = slot // block_size, slot % block_size
-            if blk >= nb:
-                raise IndexError(f"slot {slot} is outside the pool")
-            for h in range(hkv):
-                row = new[t, h]
-                if kv_fmt == E4M3:
-                    x = decode(row, src_fmt).astype(np.float32)
-                    y = (x * np.float32(inv[blk, h])).astype(np.float32)
-                    pool[blk, h, off, :] = e4m3_encode(y)
-                else:
-                    assert src_fmt == kv_fmt
-                    pool[blk, h, off, :] = row
+        rows = np.asarray(new)[keep]  # [n][hkv][d] raw source storage
+        if kv_fmt == E4M3:
+            x = decode(rows, src_fmt).astype(np.float32)  # exact: 16-bit values fit fp32
+            y = (x * np.asarray(inv, np.float32)[blk][:, :, None]).astype(np.float32)
+            pool[blk, :, off, :] = e4m3_encode(y)
+        else:
+            assert src_fmt == kv_fmt
+            pool[blk, :, off, :] = rows
 
 
 def block_copy(pools, pairs):

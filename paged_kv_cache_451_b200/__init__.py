@@ -59,7 +59,7 @@ _SIGS = {
     "kv_pool_create": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, P(c_void_p)]),
     "kv_pool_bytes": (c_int, [c_void_p, P(c_size_t), P(c_size_t)]),
     "kv_pool_bind": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
-    "kv_pool_set_decode_config": (c_int, [c_void_p, c_int, c_int]),
+    "kv_pool_set_decode_config": (c_int, [c_void_p, c_int, c_int, c_int]),
     "kv_pool_destroy": (c_int, [c_void_p]),
     "paged_kv_write": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_int,
                                c_void_p, c_void_p, c_void_p]),
@@ -160,8 +160,8 @@ def kv_pool_bind(pool, layer, k_base, v_base, k_scale=None, v_scale=None):
     _check(_lib.kv_pool_bind(pool, layer, _ptr(k_base), _ptr(v_base), _ptr(k_scale), _ptr(v_scale)))
 
 
-def kv_pool_set_decode_config(pool, partition_tokens=0, stages=0):
-    _check(_lib.kv_pool_set_decode_config(pool, partition_tokens, stages))
+def kv_pool_set_decode_config(pool, partition_tokens=0, stages=0, warps=0):
+    _check(_lib.kv_pool_set_decode_config(pool, partition_tokens, stages, warps))
 
 
 def kv_pool_destroy(pool):

@@ -26,12 +26,16 @@
 //                                            product keeps ~16 significant bits
 //                                            of P; O = rows 0..7 + rows 8..15.
 // FP8 (E4M3) pools are decoded to f16 in registers (exact); the queries are
-// scaled by a power of two per head so they fit f16 without losing bits, and
-// the per-(block, head) scales multiply the logits (K) and the probabilities
-// (V, relative to the partition's largest V scale so P stays in [0, 1]).
+// scaled by a power of two per head so they fit f16 without losing bits; the
+// K scale of each (block, head) multiplies its logits.  The V scale enters
+// the weights of P.V: besides the running max m_z of the logits (which
+// normalises the softmax sum l) a second running max m_w of logit +
+// log2|V scale| normalises the weights fed to the MMA, so the dominant terms
+// of the output always sit near 1 in f16, whatever the spread of V scales;
+// the output is (O / l) * 2^(m_w - m_z).
 //
 // A context longer than one partition is split: each partition writes its
-// unnormalised output, max and sum, and lse_reduce_kernel merges them.
+// unnormalised output and (m_z, l, m_w), and lse_reduce_kernel merges them.
 #pragma once
 
 #include <cuda.h>
@@ -45,7 +49,7 @@
 namespace pagedkv {
 
 constexpr int kChunk = 16;           // tokens per MMA tile
-constexpr int kMaxPartChunks = 256;  // at most 4096 tokens per partition
+constexpr int kMaxPartChunks = 1024;  // at most 16384 tokens per partition
 constexpr int kMaxGroup = 8;         // query heads per kv head in one CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -60,13 +64,14 @@ struct DecodeParams {
   const float* v_scale;
   void* out;                    // [batch][num_q_heads][D]
   float* part_o;                // split: [batch][num_q_heads][num_parts][D]
-  float* part_ml;               // split: [batch][num_q_heads][num_parts][2]
+  float* part_ml;               // split: [batch][num_q_heads][num_parts][4] = m_z, l, m_w, 0
   int q_bf16;
   int out_kind;
   int num_q_heads;
   int group;                    // num_q_heads / kv_heads, <= 8
   int kv_heads;
   int block_size;
+  int cpb_shift;                // log2(block_size / 16)
   int num_blocks;
   int max_blocks;
   int ctx_cap;                  // min(max_blocks * block_size, max_context_len)
@@ -101,10 +106,12 @@ struct DecodeShape {
   static constexpr int BUF_BYTES = STAGES_BYTES > MERGE_BYTES ? STAGES_BYTES : MERGE_BYTES;
   static constexpr int BAR_OFF = BUF_BYTES;
   static constexpr int BLK_OFF = BAR_OFF + WARPS * STAGES * 8;
+  static constexpr int SCALE_ENTRIES = kFp8 ? kMaxPartChunks : 0;  // FP8 scale tables only
   static constexpr int KSC_OFF = BLK_OFF + kMaxPartChunks * 4;
-  static constexpr int VSC_OFF = KSC_OFF + kMaxPartChunks * 4;
-  static constexpr int ML_OFF = VSC_OFF + kMaxPartChunks * 4;
-  static constexpr int SMEM_BYTES = ML_OFF + WARPS * kMaxGroup * 8 + 1024;  // + alignment slack
+  static constexpr int VSC_OFF = KSC_OFF + SCALE_ENTRIES * 4;
+  static constexpr int VSG_OFF = VSC_OFF + SCALE_ENTRIES * 4;
+  static constexpr int ML_OFF = VSG_OFF + SCALE_ENTRIES * 4;
+  static constexpr int SMEM_BYTES = ML_OFF + WARPS * kMaxGroup * 16 + 1024;  // + alignment slack
   static_assert(BOXB == 128 || BOXB == 64, "row bytes must be 64 or a multiple of 128");
 };
 
@@ -118,7 +125,7 @@ __device__ __forceinline__ uint32_t tile_off(int row, int chunk16) {
 }
 
 template <int KV, int D, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32)
+__global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1)
 paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap) {
   using S = DecodeShape<KV, D, WARPS, STAGES>;
@@ -139,7 +146,7 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   const int kvh = blockIdx.y;
   const int seq = blockIdx.z;
   const int bs = p.block_size;
-  const int cpb = bs / kChunk;
+  const int cpb_shift = p.cpb_shift;  // log2(block_size / 16)
 
   int n = p.context_lens[seq];
   if (n < 0 || n > p.ctx_cap) {
@@ -156,7 +163,8 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   const uint32_t bars = sbase + S::BAR_OFF;
   int32_t* blk_ids = reinterpret_cast<int32_t*>(smem + S::BLK_OFF);
   float* ksc = reinterpret_cast<float*>(smem + S::KSC_OFF);
-  float* vsc = reinterpret_cast<float*>(smem + S::VSC_OFF);
+  float* vsc = reinterpret_cast<float*>(smem + S::VSC_OFF);  // log2 |V scale|
+  float* vsg = reinterpret_cast<float*>(smem + S::VSG_OFF);  // sign of the V scale
   float* mls = reinterpret_cast<float*>(smem + S::ML_OFF);
 
   if (threadIdx.x == 0) {
@@ -165,7 +173,7 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   }
   for (int i = threadIdx.x; i < nchunks; i += WARPS * 32) {
     const int c = c0 + i;
-    int32_t b = p.block_tables[(int64_t)seq * p.max_blocks + c / cpb];
+    int32_t b = p.block_tables[(int64_t)seq * p.max_blocks + (c >> cpb_shift)];
     if (b < 0 || b >= p.num_blocks) {
       record_error(KV_ERR_BOUNDS);
       b = -1;
@@ -178,7 +186,8 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
         sv = p.v_scale[(int64_t)b * p.kv_heads + kvh];
       }
       ksc[i] = sk;
-      vsc[i] = sv;
+      vsc[i] = sv != 0.f ? lg2(fabsf(sv)) : -INFINITY;
+      vsg[i] = sv < 0.f ? -1.f : 1.f;
     }
   }
   if (lane == 0) {
@@ -232,16 +241,6 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
     }
   }
 
-  float v_ref = 1.f, v_ref_inv = 1.f;
-  if constexpr (kFp8) {
-    float mx = 0.f;
-    for (int i = lane; i < nchunks; i += 32) mx = fmaxf(mx, fabsf(vsc[i]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    v_ref = mx;
-    v_ref_inv = mx > 0.f ? 1.f / mx : 0.f;
-  }
-
   // ---- per-warp pipeline over chunks i = warp, warp + WARPS, ...
   const int my_n = nchunks > warp ? (nchunks - warp + WARPS - 1) / WARPS : 0;
   const uint32_t wstage = sbase + warp * STAGES * S::STAGEB;
@@ -256,7 +255,7 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       mbar_arrive(bar);  // complete the phase without data; the chunk is skipped
       return;
     }
-    const int y = kvh * bs + ((c0 + i) % cpb) * kChunk;
+    const int y = kvh * bs + ((c0 + i) & ((1 << cpb_shift) - 1)) * kChunk;
     const uint32_t kd = wstage + st * S::STAGEB;
     mbar_arrive_expect_tx(bar, S::STAGEB);
 #pragma unroll
@@ -271,8 +270,9 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   }
   __syncwarp();
 
-  float m_run = -INFINITY;
-  float l_run = 0.f;
+  float m_run = -INFINITY;   // running max of the logits (log2 domain)
+  float l_run = 0.f;         // running softmax sum, relative to m_run
+  float mw_run = -INFINITY;  // FP8: running max of logit + log2|V scale|
   float o[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
@@ -293,16 +293,18 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       const uint32_t kb = wstage + st * S::STAGEB;
       const uint32_t vb = kb + S::TILEB;
 
-      // S = Q . K^T: s[0] tokens 0..7, s[1] tokens 8..15
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // S = Q . K^T: tile 0 = tokens 0..7, tile 1 = tokens 8..15.  Even and odd
+      // k-steps accumulate separately (four independent MMA chains) and are
+      // summed afterwards, halving the dependent-MMA latency per chunk.
+      float sa[2][2][4] = {};
       if constexpr (!kFp8) {
         const int row = (lane & 7) + ((lane >> 4) << 3);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t b0, b1, b2, b3;
           ldsm_x4(kb + tile_off<S>(row, ks * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-          mma_16816<kBf16Mma>(s[0], qa[ks][0], qa[ks][0], qa[ks][1], qa[ks][1], b0, b1);
-          mma_16816<kBf16Mma>(s[1], qa[ks][0], qa[ks][0], qa[ks][1], qa[ks][1], b2, b3);
+          mma_16816<kBf16Mma>(sa[ks & 1][0], qa[ks][0], qa[ks][0], qa[ks][1], qa[ks][1], b0, b1);
+          mma_16816<kBf16Mma>(sa[ks & 1][1], qa[ks][0], qa[ks][0], qa[ks][1], qa[ks][1], b2, b3);
         }
       } else {
         const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
@@ -311,21 +313,24 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
           uint32_t r0, r1, r2, r3;
           ldsm_x4(kb + tile_off<S>(row, kp * 2 + (lane >> 4)), r0, r1, r2, r3);
           const int k0 = 2 * kp, k1 = 2 * kp + 1;
-          mma_16816<false>(s[0], qa[k0][0], qa[k0][0], qa[k0][1], qa[k0][1],
-                           e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r0 >> 16));
-          mma_16816<false>(s[1], qa[k0][0], qa[k0][0], qa[k0][1], qa[k0][1],
-                           e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r1 >> 16));
-          mma_16816<false>(s[0], qa[k1][0], qa[k1][0], qa[k1][1], qa[k1][1],
-                           e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r2 >> 16));
-          mma_16816<false>(s[1], qa[k1][0], qa[k1][0], qa[k1][1], qa[k1][1],
-                           e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r3 >> 16));
+          uint32_t f0l, f0h, f1l, f1h, f2l, f2h, f3l, f3h;
+          e4m3x4_to_f16x4(r0, f0l, f0h);
+          e4m3x4_to_f16x4(r1, f1l, f1h);
+          e4m3x4_to_f16x4(r2, f2l, f2h);
+          e4m3x4_to_f16x4(r3, f3l, f3h);
+          mma_16816<false>(sa[0][0], qa[k0][0], qa[k0][0], qa[k0][1], qa[k0][1], f0l, f0h);
+          mma_16816<false>(sa[0][1], qa[k0][0], qa[k0][0], qa[k0][1], qa[k0][1], f1l, f1h);
+          mma_16816<false>(sa[1][0], qa[k1][0], qa[k1][0], qa[k1][1], qa[k1][1], f2l, f2h);
+          mma_16816<false>(sa[1][1], qa[k1][0], qa[k1][0], qa[k1][1], qa[k1][1], f3l, f3h);
         }
       }
+      const float s00 = sa[0][0][0] + sa[1][0][0], s01 = sa[0][0][1] + sa[1][0][1];
+      const float s10 = sa[0][1][0] + sa[1][1][0], s11 = sa[0][1][1] + sa[1][1][1];
 
       // online softmax (log2 domain) over this lane's 4 tokens of row gq
       float zs = zrow;
       if constexpr (kFp8) zs *= ksc[i];
-      float z[4] = {s[0][0] * zs, s[0][1] * zs, s[1][0] * zs, s[1][1] * zs};
+      float z[4] = {s00 * zs, s01 * zs, s10 * zs, s11 * zs};
       if (vt < kChunk) {
         if (2 * cq >= vt) z[0] = -INFINITY;
         if (2 * cq + 1 >= vt) z[1] = -INFINITY;
@@ -342,19 +347,26 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       for (int e = 0; e < 4; ++e) pr[e] = ex2(z[e] - m_new);
       l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
       m_run = m_new;
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      float alpha_o = alpha;  // rescale of O
+      if constexpr (kFp8) {
+        // weights pr * 2^(lw + m_new - mw_new) = 2^(z + lw - mw_new) <= 1
+        const float lw = vsc[i];
+        const float mw_new = fmaxf(mw_run, mx + lw);
+        const bool none = mw_new == -INFINITY;
+        alpha_o = none ? 1.f : ex2(mw_run - mw_new);
+        const float c = none ? 0.f : ex2(lw + m_new - mw_new) * vsg[i];
+        mw_run = mw_new;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] *= c;
+      }
+      if (__any_sync(0xffffffffu, alpha_o != 1.f)) {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          o[t][0] *= alpha;
-          o[t][1] *= alpha;
-          o[t][2] *= alpha;
-          o[t][3] *= alpha;
+          o[t][0] *= alpha_o;
+          o[t][1] *= alpha_o;
+          o[t][2] *= alpha_o;
+          o[t][3] *= alpha_o;
         }
-      }
-      if constexpr (kFp8) {
-        const float w = vsc[i] * v_ref_inv;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) pr[e] *= w;
       }
       // P as A fragment: rows 0..7 the 16-bit values, rows 8..15 the residuals
       uint32_t pa0, pa1, pa2, pa3;
@@ -434,8 +446,10 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       row[d1] = o[t][1] + o[t][3];
     }
     if (cq == 0) {
-      mls[(warp * kMaxGroup + gq) * 2 + 0] = m_run;
-      mls[(warp * kMaxGroup + gq) * 2 + 1] = l_run;
+      float* ml = mls + (warp * kMaxGroup + gq) * 4;
+      ml[0] = m_run;
+      ml[1] = l_run;
+      ml[2] = kFp8 ? mw_run : m_run;
     }
   }
   __syncthreads();
@@ -444,38 +458,44 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   for (int idx = threadIdx.x; idx < p.group * D; idx += WARPS * 32) {
     const int g = idx / D;
     const int d = idx - g * D;
-    float M = -INFINITY;
+    float Mz = -INFINITY, Mw = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, mls[(w * kMaxGroup + g) * 2]);
-    float O = 0.f, L = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < WARPS; ++w) {
-        const float mw = mls[(w * kMaxGroup + g) * 2];
-        const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
-        O += f * obuf[(w * kMaxGroup + g) * D + d];
-        L += f * mls[(w * kMaxGroup + g) * 2 + 1];
-      }
+    for (int w = 0; w < WARPS; ++w) {
+      Mz = fmaxf(Mz, mls[(w * kMaxGroup + g) * 4 + 0]);
+      Mw = fmaxf(Mw, mls[(w * kMaxGroup + g) * 4 + 2]);
     }
-    if constexpr (kFp8) O *= v_ref;
+    float O = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      const float* ml = mls + (w * kMaxGroup + g) * 4;
+      if (ml[0] != -INFINITY) L += ml[1] * ex2(ml[0] - Mz);
+      if (ml[2] != -INFINITY) O += obuf[(w * kMaxGroup + g) * D + d] * ex2(ml[2] - Mw);
+    }
     const int h = kvh * p.group + g;
     const int64_t sh = (int64_t)seq * p.num_q_heads + h;
     if (!split) {
-      store_out(p.out, p.out_kind, sh * D + d, L > 0.f ? O / L : 0.f);
+      float r = 0.f;
+      if (L > 0.f && Mw != -INFINITY) r = kFp8 ? (O / L) * ex2(Mw - Mz) : O / L;
+      store_out(p.out, p.out_kind, sh * D + d, r);
     } else {
       const int64_t pi = sh * p.num_parts + part;
       p.part_o[pi * D + d] = O;
       if (d == 0) {
-        p.part_ml[pi * 2 + 0] = M;
-        p.part_ml[pi * 2 + 1] = L;
+        p.part_ml[pi * 4 + 0] = Mz;
+        p.part_ml[pi * 4 + 1] = L;
+        p.part_ml[pi * 4 + 2] = Mw;
+        p.part_ml[pi * 4 + 3] = 0.f;
       }
     }
   }
 }
 
-// Merge of split partials: for each (sequence, query head),
-//   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  out = sum_p o_p 2^(m_p - M) / L
-// (m in the log2 domain).  One warp per (sequence, head).
+// Merge of split partials: for each (sequence, query head), with partition p
+// holding (o_p, m_z,p, l_p, m_w,p) in the log2 domain,
+//   Mz = max m_z,p,  L = sum l_p 2^(m_z,p - Mz),
+//   Mw = max m_w,p,  O = sum o_p 2^(m_w,p - Mw),   out = (O / L) 2^(Mw - Mz).
+// (For 16-bit caches m_w = m_z.)  One warp per (sequence, head); head_dim is
+// 64 or 128.
 __global__ void __launch_bounds__(256)
 lse_reduce_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                   const int32_t* __restrict__ context_lens, void* out, int out_kind,
@@ -488,32 +508,58 @@ lse_reduce_kernel(const float* __restrict__ part_o, const float* __restrict__ pa
   int n = context_lens[seq];
   n = n < 0 ? 0 : (n > ctx_cap ? ctx_cap : n);
   const int np = max(1, (n + part_tokens - 1) / part_tokens);
-  const float* ml = part_ml + idx * num_parts * 2;
-  float M = -INFINITY;
-  for (int q = lane; q < np; q += 32) M = fmaxf(M, ml[2 * q]);
+  const float4* ml = reinterpret_cast<const float4*>(part_ml) + idx * num_parts;
+  float Mz = -INFINITY, Mw = -INFINITY;
+  for (int q = lane; q < np; q += 32) {
+    const float4 v = ml[q];
+    Mz = fmaxf(Mz, v.x);
+    Mw = fmaxf(Mw, v.z);
+  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  for (int o = 16; o > 0; o >>= 1) {
+    Mz = fmaxf(Mz, __shfl_xor_sync(0xffffffffu, Mz, o));
+    Mw = fmaxf(Mw, __shfl_xor_sync(0xffffffffu, Mw, o));
+  }
   float L = 0.f;
-  if (M != -INFINITY) {
-    for (int q = lane; q < np; q += 32) {
-      const float mq = ml[2 * q];
-      if (mq != -INFINITY) L += ml[2 * q + 1] * ex2(mq - M);
-    }
+  for (int q = lane; q < np; q += 32) {
+    const float4 v = ml[q];
+    if (v.x != -INFINITY) L += v.y * ex2(v.x - Mz);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  const float* po = part_o + idx * num_parts * head_dim;
-  for (int d = lane; d < head_dim; d += 32) {
-    float acc = 0.f;
-    if (M != -INFINITY) {
-      for (int q = 0; q < np; ++q) {
-        const float mq = ml[2 * q];
-        if (mq != -INFINITY) acc += po[(int64_t)q * head_dim + d] * ex2(mq - M);
+  const bool empty = !(L > 0.f) || Mw == -INFINITY;
+  const float scale = empty ? 0.f : ex2(Mw - Mz) / L;
+  // each lane owns head_dim / 32 consecutive dims; partition weights are
+  // computed once per 32 partitions and broadcast
+  const int per = head_dim / 32;  // 2 or 4
+  const float* po = part_o + idx * num_parts * head_dim + lane * per;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (!empty) {
+    for (int q0 = 0; q0 < np; q0 += 32) {
+      float wq = 0.f;
+      if (q0 + lane < np) {
+        const float mq = ml[q0 + lane].z;
+        wq = mq == -INFINITY ? 0.f : ex2(mq - Mw);
+      }
+      const int nq = min(32, np - q0);
+      for (int j = 0; j < nq; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, wq, j);
+        const float* src = po + (int64_t)(q0 + j) * head_dim;
+        if (per == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          acc[0] += wj * v.x;
+          acc[1] += wj * v.y;
+          acc[2] += wj * v.z;
+          acc[3] += wj * v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(src);
+          acc[0] += wj * v.x;
+          acc[1] += wj * v.y;
+        }
       }
     }
-    store_out(out, out_kind, idx * head_dim + d, acc * inv);
   }
+  for (int k = 0; k < per; ++k) store_out(out, out_kind, idx * head_dim + lane * per + k, acc[k] * scale);
 }
 
 }  // namespace pagedkv

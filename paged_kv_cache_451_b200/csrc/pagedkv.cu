@@ -24,9 +24,9 @@ using pagedkv::ok;
 namespace pagedkv {
 namespace {
 
-constexpr int kWarps = 4;
 constexpr int kMaxLayers = 4096;
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSmemPerCta = 227 * 1024;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -70,6 +70,7 @@ int make_map(const kv_pool* pool, void* base, CUtensorMap* map) {
 }
 
 int cuda_fail(cudaError_t e, const char* what) {
+  (void)cudaGetLastError();  // do not leave this error pending for the next check
   return fail(KV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
@@ -88,32 +89,55 @@ int ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done) {
   return KV_OK;
 }
 
-int stages_for(const kv_pool* pool) {
-  if (pool->stages > 0) return pool->stages;
-  // about 24 KB of K/V in flight per warp: 3 stages of 8 KB (16-bit, D 128),
-  // 6 of 4 KB (FP8 D 128 or 16-bit D 64), 8 of 2 KB (FP8 D 64)
-  const int stage_bytes = 2 * kChunk * pool->head_dim * elem_bytes(pool->dtype);
-  return stage_bytes >= 8192 ? 3 : (stage_bytes >= 4096 ? 6 : 8);
+// Pipeline shape: warps per CTA and stages per warp.  4 warps of 3 stages of
+// 8 KB (16-bit, D 128: two CTAs per SM); 3 stages of 4 KB (FP8 D 128, 16-bit
+// D 64: three CTAs per SM, the register limit); 6 stages of 2 KB.  Measured
+// on B200: more warps per CTA or deeper rings were slower for every format.
+struct PipeShape {
+  int warps;
+  int stages;
+};
+
+PipeShape pipe_for(kv_dtype dtype, int head_dim, int stages, int warps) {
+  const int stage_bytes = 2 * kChunk * head_dim * elem_bytes(dtype);
+  PipeShape ps;
+  if (stage_bytes >= 8192) ps = {4, 3};
+  else if (stage_bytes >= 4096) ps = {4, 3};
+  else ps = {4, 6};
+  if (warps > 0) ps.warps = warps;
+  if (stages > 0) ps.stages = stages;
+  return ps;
+}
+
+PipeShape pipe_for(const kv_pool* pool) {
+  return pipe_for(pool->dtype, pool->head_dim, pool->stages, pool->warps);
+}
+
+template <int KV, int D, int W>
+int smem_bytes_w(int stages) {
+  switch (stages) {
+    case 2: return DecodeShape<KV, D, W, 2>::SMEM_BYTES;
+    case 3: return DecodeShape<KV, D, W, 3>::SMEM_BYTES;
+    case 4: return DecodeShape<KV, D, W, 4>::SMEM_BYTES;
+    case 6: return DecodeShape<KV, D, W, 6>::SMEM_BYTES;
+    default: return DecodeShape<KV, D, W, 8>::SMEM_BYTES;
+  }
 }
 
 template <int KV, int D>
-int smem_bytes_d(int stages) {
-  switch (stages) {
-    case 2: return DecodeShape<KV, D, kWarps, 2>::SMEM_BYTES;
-    case 3: return DecodeShape<KV, D, kWarps, 3>::SMEM_BYTES;
-    case 4: return DecodeShape<KV, D, kWarps, 4>::SMEM_BYTES;
-    case 6: return DecodeShape<KV, D, kWarps, 6>::SMEM_BYTES;
-    default: return DecodeShape<KV, D, kWarps, 8>::SMEM_BYTES;
+int smem_bytes_d(PipeShape ps) {
+  return ps.warps == 8 ? smem_bytes_w<KV, D, 8>(ps.stages) : smem_bytes_w<KV, D, 4>(ps.stages);
+}
+
+int smem_bytes(kv_dtype dtype, int head_dim, PipeShape ps) {
+  const bool d64 = head_dim == 64;
+  switch (dtype) {
+    case KV_FP8_E4M3: return d64 ? smem_bytes_d<KV_KIND_E4M3, 64>(ps) : smem_bytes_d<KV_KIND_E4M3, 128>(ps);
+    default: return d64 ? smem_bytes_d<KV_KIND_F16, 64>(ps) : smem_bytes_d<KV_KIND_F16, 128>(ps);
   }
 }
 
-int smem_bytes(const kv_pool* pool, int stages) {
-  const bool d64 = pool->head_dim == 64;
-  switch (pool->dtype) {
-    case KV_FP8_E4M3: return d64 ? smem_bytes_d<KV_KIND_E4M3, 64>(stages) : smem_bytes_d<KV_KIND_E4M3, 128>(stages);
-    default: return d64 ? smem_bytes_d<KV_KIND_F16, 64>(stages) : smem_bytes_d<KV_KIND_F16, 128>(stages);
-  }
-}
+int decode_occupancy(const kv_pool* pool);  // defined with the launchers below
 
 // Resident decode CTAs the current device holds at once.
 int decode_slots(const kv_pool* pool) {
@@ -122,27 +146,35 @@ int decode_slots(const kv_pool* pool) {
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   int sms = sm_count[dev % kMaxDevices].load(std::memory_order_relaxed);
   if (sms == 0) {
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+      (void)cudaGetLastError();
       sms = 148;
+    }
     sm_count[dev % kMaxDevices].store(sms, std::memory_order_relaxed);
   }
-  const int per_sm = std::max(1, (227 * 1024) / smem_bytes(pool, stages_for(pool)));
-  return sms * per_sm;
+  return sms * decode_occupancy(pool);
 }
 
-// Partition length in tokens.  Automatic: keep each (sequence, kv head) in
-// one CTA when there are enough of them for about eight waves of resident
-// CTAs; otherwise split the longest context into just enough partitions to
-// reach that, and always keep partitions within kMaxPartChunks chunks.
+// Partition length in tokens.  Automatic: contexts are cut into partitions
+// of at most kAutoPartition tokens; if that leaves fewer than kWaves waves of
+// resident CTAs, into more (down to kMinPartition tokens) until it does not.
+// Measured on B200: one partition per 2K-token context is best for uniform
+// 16-bit contexts (the 32-layer example), ~2K-token partitions for the
+// 16K-token FP8 contexts.
+constexpr int kWaves = 3;
+constexpr int kAutoPartition = 2048;
+constexpr int kMinPartition = 512;
+
 int partition_tokens(const kv_pool* pool, int batch, int max_context_len) {
   if (pool->partition_tokens > 0) return pool->partition_tokens;
   const int ctx = std::max(max_context_len, 1);
   const int64_t units = std::max<int64_t>(1, (int64_t)batch * pool->kv_heads);
-  const int64_t want = 8ll * decode_slots(pool);
-  int64_t np = std::max<int64_t>((ctx + kChunk * kMaxPartChunks - 1) / (kChunk * kMaxPartChunks),
-                                 (want + units - 1) / units);
-  np = std::min<int64_t>(np, (ctx + 255) / 256);  // partitions of at least 256 tokens
-  np = std::max<int64_t>(np, 1);
+  const int64_t want = (int64_t)kWaves * decode_slots(pool);
+  int64_t np = (ctx + kAutoPartition - 1) / kAutoPartition;
+  if (units * np < want) {
+    np = std::max<int64_t>(np, (want + units - 1) / units);
+    np = std::min<int64_t>(np, std::max<int64_t>(1, (ctx + kMinPartition - 1) / kMinPartition));
+  }
   const int64_t per = (ctx + np - 1) / np;
   return (int)std::min<int64_t>(kChunk * kMaxPartChunks, (per + kChunk - 1) / kChunk * kChunk);
 }
@@ -152,37 +184,89 @@ int num_parts_for(const kv_pool* pool, int batch, int max_context_len) {
   return std::max(1, (max_context_len + pt - 1) / pt);
 }
 
-template <int KV, int D, int STAGES>
+// Resident CTAs per SM of one decode instantiation on the current device
+// (occupancy API; registers and shared memory both count).
+template <int KV, int D, int W, int STAGES>
+int decode_occupancy() {
+  using Shape = DecodeShape<KV, D, W, STAGES>;
+  auto kernel = paged_decode_kernel<KV, D, W, STAGES>;
+  static std::atomic<int> cached[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  int v = cached[dev % kMaxDevices].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Shape::SMEM_BYTES) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, W * 32, Shape::SMEM_BYTES) !=
+          cudaSuccess ||
+      v <= 0) {
+    (void)cudaGetLastError();
+    v = std::max(1, kMaxSmemPerCta / Shape::SMEM_BYTES);  // no device: shared-memory bound
+  }
+  cached[dev % kMaxDevices].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+template <int KV, int D, int W>
+int occupancy_w(int stages) {
+  switch (stages) {
+    case 2: return decode_occupancy<KV, D, W, 2>();
+    case 3: return decode_occupancy<KV, D, W, 3>();
+    case 4: return decode_occupancy<KV, D, W, 4>();
+    case 6: return decode_occupancy<KV, D, W, 6>();
+    default: return decode_occupancy<KV, D, W, 8>();
+  }
+}
+
+template <int KV, int D>
+int occupancy_d(PipeShape ps) {
+  return ps.warps == 8 ? occupancy_w<KV, D, 8>(ps.stages) : occupancy_w<KV, D, 4>(ps.stages);
+}
+
+int decode_occupancy(const kv_pool* pool) {
+  const PipeShape ps = pipe_for(pool);
+  const bool d64 = pool->head_dim == 64;
+  switch (pool->dtype) {
+    case KV_FP8_E4M3: return d64 ? occupancy_d<KV_KIND_E4M3, 64>(ps) : occupancy_d<KV_KIND_E4M3, 128>(ps);
+    case KV_BF16: return d64 ? occupancy_d<KV_KIND_BF16, 64>(ps) : occupancy_d<KV_KIND_BF16, 128>(ps);
+    default: return d64 ? occupancy_d<KV_KIND_F16, 64>(ps) : occupancy_d<KV_KIND_F16, 128>(ps);
+  }
+}
+
+template <int KV, int D, int W, int STAGES>
 int launch_decode_t(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cudaStream_t stream) {
-  using Shape = DecodeShape<KV, D, kWarps, STAGES>;
-  auto kernel = paged_decode_kernel<KV, D, kWarps, STAGES>;
+  using Shape = DecodeShape<KV, D, W, STAGES>;
+  auto kernel = paged_decode_kernel<KV, D, W, STAGES>;
   static std::atomic<uint64_t> done{0};  // one flag word per instantiation
   int rc = ensure_smem(kernel, Shape::SMEM_BYTES, done);
   if (rc != KV_OK) return rc;
-  kernel<<<grid, kWarps * 32, Shape::SMEM_BYTES, stream>>>(p, lb.k_map, lb.v_map);
+  kernel<<<grid, W * 32, Shape::SMEM_BYTES, stream>>>(p, lb.k_map, lb.v_map);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
   return KV_OK;
 }
 
-template <int KV, int D>
-int launch_decode_d(int stages, const DecodeParams& p, const LayerBinding& lb, dim3 grid,
+template <int KV, int D, int W>
+int launch_decode_w(int stages, const DecodeParams& p, const LayerBinding& lb, dim3 grid,
                     cudaStream_t stream) {
   switch (stages) {
-    case 2: return launch_decode_t<KV, D, 2>(p, lb, grid, stream);
-    case 3: return launch_decode_t<KV, D, 3>(p, lb, grid, stream);
-    case 4: return launch_decode_t<KV, D, 4>(p, lb, grid, stream);
-    case 6: return launch_decode_t<KV, D, 6>(p, lb, grid, stream);
-    case 8: return launch_decode_t<KV, D, 8>(p, lb, grid, stream);
+    case 2: return launch_decode_t<KV, D, W, 2>(p, lb, grid, stream);
+    case 3: return launch_decode_t<KV, D, W, 3>(p, lb, grid, stream);
+    case 4: return launch_decode_t<KV, D, W, 4>(p, lb, grid, stream);
+    case 6: return launch_decode_t<KV, D, W, 6>(p, lb, grid, stream);
+    case 8: return launch_decode_t<KV, D, W, 8>(p, lb, grid, stream);
     default: return fail(KV_ERR_ARG, "unsupported stage count %d", stages);
   }
 }
 
 template <int KV>
-int launch_decode_kv(int head_dim, int stages, const DecodeParams& p, const LayerBinding& lb,
+int launch_decode_kv(int head_dim, PipeShape ps, const DecodeParams& p, const LayerBinding& lb,
                      dim3 grid, cudaStream_t stream) {
-  if (head_dim == 64) return launch_decode_d<KV, 64>(stages, p, lb, grid, stream);
-  return launch_decode_d<KV, 128>(stages, p, lb, grid, stream);
+  if (head_dim == 64)
+    return ps.warps == 8 ? launch_decode_w<KV, 64, 8>(ps.stages, p, lb, grid, stream)
+                         : launch_decode_w<KV, 64, 4>(ps.stages, p, lb, grid, stream);
+  return ps.warps == 8 ? launch_decode_w<KV, 128, 8>(ps.stages, p, lb, grid, stream)
+                       : launch_decode_w<KV, 128, 4>(ps.stages, p, lb, grid, stream);
 }
 
 bool valid_q_dtype(kv_dtype pool, kv_dtype q) {
@@ -202,8 +286,9 @@ extern "C" {
 int kv_pool_create(int block_size, int num_blocks, int kv_heads, int head_dim, kv_dtype dtype,
                    int num_layers, kv_pool** out) {
   if (!out) return fail(KV_ERR_ARG, "out is NULL");
-  if (block_size < 16 || block_size > 256 || block_size % 16 != 0)
-    return fail(KV_ERR_ARG, "block_size %d must be a multiple of 16 in [16, 256]", block_size);
+  if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128 &&
+      block_size != 256)
+    return fail(KV_ERR_ARG, "block_size %d must be 16, 32, 64, 128 or 256", block_size);
   if (head_dim != 64 && head_dim != 128)
     return fail(KV_ERR_ARG, "head_dim %d unsupported (64 or 128)", head_dim);
   if (dtype != KV_F16 && dtype != KV_BF16 && dtype != KV_FP8_E4M3)
@@ -258,7 +343,7 @@ int kv_pool_bind(kv_pool* pool, int layer, void* k_base, void* v_base, float* k_
   return ok();
 }
 
-int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages) {
+int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages, int warps) {
   if (!pool) return fail(KV_ERR_ARG, "NULL pool");
   if (partition_tokens != 0 &&
       (partition_tokens < kChunk || partition_tokens > kChunk * kMaxPartChunks ||
@@ -267,8 +352,16 @@ int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages) {
                 partition_tokens, kChunk * kMaxPartChunks);
   if (stages != 0 && stages != 2 && stages != 3 && stages != 4 && stages != 6 && stages != 8)
     return fail(KV_ERR_ARG, "stages %d must be 0, 2, 3, 4, 6 or 8", stages);
+  if (warps != 0 && warps != 4 && warps != 8)
+    return fail(KV_ERR_ARG, "warps %d must be 0, 4 or 8", warps);
+  const PipeShape ps = pipe_for(pool->dtype, pool->head_dim, stages, warps);
+  const int need = smem_bytes(pool->dtype, pool->head_dim, ps);
+  if (need > kMaxSmemPerCta)
+    return fail(KV_ERR_ARG, "%d warps x %d stages need %d bytes of shared memory per CTA, above %d",
+                ps.warps, ps.stages, need, kMaxSmemPerCta);
   pool->partition_tokens = partition_tokens;
   pool->stages = stages;
+  pool->warps = warps;
   return ok();
 }
 
@@ -356,7 +449,7 @@ size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q
   if (!pool || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
   const int np = num_parts_for(pool, batch, max_context_len);
   if (np <= 1) return 0;
-  return (size_t)batch * num_q_heads * np * (pool->head_dim + 2) * sizeof(float);
+  return (size_t)batch * num_q_heads * np * (pool->head_dim + 4) * sizeof(float);
 }
 
 int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
@@ -411,6 +504,8 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   p.group = num_q_heads / pool->kv_heads;
   p.kv_heads = pool->kv_heads;
   p.block_size = pool->block_size;
+  p.cpb_shift = 0;
+  while ((kChunk << p.cpb_shift) < pool->block_size) ++p.cpb_shift;
   p.num_blocks = pool->num_blocks;
   p.max_blocks = max_blocks_per_seq;
   p.part_chunks = pt / kChunk;
@@ -420,12 +515,12 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(np, pool->kv_heads, batch);
-  const int stages = stages_for(pool);
+  const PipeShape ps = pipe_for(pool);
   int rc;
   switch (pool->dtype) {
-    case KV_F16: rc = launch_decode_kv<KV_KIND_F16>(pool->head_dim, stages, p, lb, grid, s); break;
-    case KV_BF16: rc = launch_decode_kv<KV_KIND_BF16>(pool->head_dim, stages, p, lb, grid, s); break;
-    default: rc = launch_decode_kv<KV_KIND_E4M3>(pool->head_dim, stages, p, lb, grid, s); break;
+    case KV_F16: rc = launch_decode_kv<KV_KIND_F16>(pool->head_dim, ps, p, lb, grid, s); break;
+    case KV_BF16: rc = launch_decode_kv<KV_KIND_BF16>(pool->head_dim, ps, p, lb, grid, s); break;
+    default: rc = launch_decode_kv<KV_KIND_E4M3>(pool->head_dim, ps, p, lb, grid, s); break;
   }
   if (rc != KV_OK) return rc;
   if (np > 1) {

@@ -33,6 +33,7 @@ struct kv_pool {
   kv_dtype dtype = KV_F16;
   int partition_tokens = 0;  // 0: automatic
   int stages = 0;            // 0: automatic
+  int warps = 0;             // 0: automatic
   std::vector<pagedkv::LayerBinding> layers;
 
   size_t tile_bytes() const { return (size_t)block_size * head_dim * pagedkv::elem_bytes(dtype); }

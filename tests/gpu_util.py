@@ -34,11 +34,11 @@ class DevicePool:
     """A pool handle plus the device tensors bound to it."""
 
     def __init__(self, num_blocks, kv_heads, head_dim, block_size, fmt, num_layers=1,
-                 k=None, v=None, k_scale=None, v_scale=None, partition=0, stages=0):
+                 k=None, v=None, k_scale=None, v_scale=None, partition=0, stages=0, warps=0):
         self.fmt, self.num_blocks, self.kv_heads = fmt, num_blocks, kv_heads
         self.head_dim, self.block_size, self.num_layers = head_dim, block_size, num_layers
         self.h = pk.kv_pool_create(block_size, num_blocks, kv_heads, head_dim, fmt, num_layers)
-        pk.kv_pool_set_decode_config(self.h, partition, stages)
+        pk.kv_pool_set_decode_config(self.h, partition, stages, warps)
         shape = (num_blocks, kv_heads, block_size, head_dim)
         self.k, self.v, self.ks, self.vs = [], [], [], []
         for layer in range(num_layers):
@@ -54,8 +54,8 @@ class DevicePool:
             self.vs.append(vst)
             pk.kv_pool_bind(self.h, layer, kt, vt, kst, vst)
 
-    def set_config(self, partition=0, stages=0):
-        pk.kv_pool_set_decode_config(self.h, partition, stages)
+    def set_config(self, partition=0, stages=0, warps=0):
+        pk.kv_pool_set_decode_config(self.h, partition, stages, warps)
 
     def __del__(self):
         try:

@@ -48,6 +48,7 @@ def test_version_and_error_string():
     (16, 0, 1, 128, pk.KV_F16, 1),      # no blocks
     (16, 4, 1, 96, pk.KV_F16, 1),       # head_dim
     (24, 4, 1, 128, pk.KV_F16, 1),      # block size not a multiple of 16
+    (48, 4, 1, 128, pk.KV_F16, 1),      # block size not a power of two
     (16, 4, 1, 128, pk.KV_F32, 1),      # pool dtype
     (16, 4, 0, 128, pk.KV_BF16, 1),     # kv heads
     (16, 4, 1, 128, pk.KV_BF16, 0),     # layers
@@ -62,15 +63,17 @@ def test_pool_bytes_and_workspace_sizes():
     pool = pk.kv_pool_create(16, 100, 8, 128, pk.KV_BF16, 2)
     kvb, sb = pk.kv_pool_bytes(pool)
     assert kvb == 100 * 8 * 16 * 128 * 2 and sb == 0
-    # automatic policy: many (sequence, kv head) units -> one partition each
-    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 4096) == 0
-    # few units -> split into partitions of at least 256 tokens
-    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 512) == 4 * 64 * 2 * 130 * 4
-    pk.kv_pool_set_decode_config(pool, 4096, 0)
+    # automatic policy: partitions of at most 2048 tokens ...
+    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 2048) == 0
+    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 4096) == 512 * 64 * 2 * 132 * 4
+    # ... and more, down to 512 tokens, when there are few (sequence, kv head) units
+    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 1024) == 4 * 64 * 2 * 132 * 4
+    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 512) == 0
+    pk.kv_pool_set_decode_config(pool, 4096, 0, 0)
     assert pk.paged_attention_workspace_bytes(pool, 4, 64, 4096) == 0
-    pk.kv_pool_set_decode_config(pool, 256, 2)
-    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 513) == 4 * 64 * 3 * 130 * 4
-    for bad in ((8, 0), (4112, 0), (100, 0), (0, 5), (0, 1), (0, 7)):
+    pk.kv_pool_set_decode_config(pool, 256, 2, 4)
+    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 513) == 4 * 64 * 3 * 132 * 4
+    for bad in ((8, 0, 0), (16400, 0, 0), (100, 0, 0), (0, 5, 0), (0, 1, 0), (0, 7, 0), (0, 0, 6), (0, 4, 8)):
         with pytest.raises(pk.KVError):
             pk.kv_pool_set_decode_config(pool, *bad)
     pk.kv_pool_destroy(pool)

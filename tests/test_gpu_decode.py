@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 
 
 def run_case(kv_fmt, q_fmt, d, bs, hq, hkv, lens, partition=0, stages=0, seed=0, spare=5,
-             out_fmt=F32, scale=None):
+             out_fmt=F32, scale=None, warps=0):
     rng = np.random.default_rng(seed)
     lens = np.asarray(lens, np.int32)
     nb = int(sum(-(-max(int(n), 1) // bs) for n in lens)) + spare
@@ -35,7 +35,8 @@ def run_case(kv_fmt, q_fmt, d, bs, hq, hkv, lens, partition=0, stages=0, seed=0,
     q = normal_bits(rng, (len(lens), hq, d), q_fmt)
     pool = DevicePool(nb, hkv, d, bs, kv_fmt, k=[dev(kh)], v=[dev(vh)],
                       k_scale=None if ks is None else [dev(ks)],
-                      v_scale=None if vs is None else [dev(vs)], partition=partition, stages=stages)
+                      v_scale=None if vs is None else [dev(vs)], partition=partition, stages=stages,
+                      warps=warps)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     max_ctx = int(lens.max()) if len(lens) else 0
     out = decode(pool, dev(q), q_fmt, hq, dev(tables), dev(lens), max_ctx, scale, out_fmt)
@@ -58,11 +59,27 @@ def test_decode_matches_oracle_across_formats_and_groups(kv_fmt, q_fmt, d, hq, h
 
 @pytest.mark.parametrize("partition", [16, 48, 512, 4096])
 @pytest.mark.parametrize("stages", [2, 3, 4, 6, 8])
-def test_split_and_pipeline_depths_match_oracle(partition, stages):
+@pytest.mark.parametrize("warps", [4, 8])
+def test_split_and_pipeline_depths_match_oracle(partition, stages, warps):
+    if stages * warps >= 32:  # 8 KB stages: more than 227 KB of shared memory per CTA
+        pool = DevicePool(4, 1, 128, 16, BF16)
+        with pytest.raises(pk.KVError) as e:
+            pool.set_config(partition, stages, warps)
+        assert e.value.code == pk.KV_ERR_ARG
+        return
     lens = [1, 16, 47, 511, 512, 513, 1000, 1537, 0, 3]
-    out, ref = run_case(BF16, BF16, 128, 16, 8, 1, lens, partition=partition, stages=stages, seed=partition + stages)
+    out, ref = run_case(BF16, BF16, 128, 16, 8, 1, lens, partition=partition, stages=stages,
+                        warps=warps, seed=partition + stages + warps)
     assert max_abs(out.cpu().numpy(), ref) <= TOL[BF16]
     assert np.all(out[8].cpu().numpy() == 0)  # empty context
+
+
+@pytest.mark.parametrize("stages,warps", [(6, 4), (8, 4), (3, 8), (4, 8), (6, 8)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_pipeline_shapes(stages, warps, d):
+    out, ref = run_case(E4M3, BF16, d, 16, 8, 2, [1, 300, 2000, 17], partition=512, stages=stages,
+                        warps=warps, seed=stages + warps + d)
+    assert max_abs(out.cpu().numpy(), ref) <= TOL[E4M3]
 
 
 @pytest.mark.parametrize("bs", [16, 32, 64])
@@ -82,9 +99,11 @@ def test_fp8_long_context_split():
     assert max_abs(out.cpu().numpy(), ref) <= TOL[E4M3]
 
 
-def test_fp8_extreme_scales_and_peaked_softmax():
-    """Per-block V scales spanning 2^-30 .. 2^20 and logits with a dominant
-    token still match (the kernel normalises V scales per partition)."""
+@pytest.mark.parametrize("partition", [0, 64, 256])
+def test_fp8_extreme_scales_and_peaked_softmax(partition):
+    """Per-block V scales spanning 2^-30 .. 2^20 with a large logit scale
+    (peaked softmax) still match: the weights fed to the MMA are normalised
+    by their own running maximum, not by the largest V scale."""
     rng = np.random.default_rng(9)
     nb, hkv, bs, d = 64, 2, 16, 128
     kh, vh = e4m3_codes(rng, (nb, hkv, bs, d)), e4m3_codes(rng, (nb, hkv, bs, d))
@@ -93,7 +112,8 @@ def test_fp8_extreme_scales_and_peaked_softmax():
     lens = np.array([300, 17, 520], np.int32)
     tables = scattered_tables(rng, lens, bs, nb)
     q = normal_bits(rng, (3, 4, d), BF16)
-    pool = DevicePool(nb, hkv, d, bs, E4M3, k=[dev(kh)], v=[dev(vh)], k_scale=[dev(ks)], v_scale=[dev(vs)])
+    pool = DevicePool(nb, hkv, d, bs, E4M3, k=[dev(kh)], v=[dev(vh)], k_scale=[dev(ks)], v_scale=[dev(vs)],
+                      partition=partition)
     out = decode(pool, dev(q), BF16, 4, dev(tables), dev(lens), 520, 3.0).cpu().numpy()
     ref = oracle.paged_decode(kh, vh, E4M3, q, BF16, tables, lens, 3.0, bs, ks, vs)
     rel = np.abs(out - ref) / (np.abs(ref).max(axis=-1, keepdims=True) + 1e-30)
