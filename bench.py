@@ -135,6 +135,21 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples), "source": "nvml"}
 
 
+def max_over_ranks(value, dist, device):
+    """Max of a per-rank scalar over all ranks (timing plumbing only)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(bytes_per_rank, world, max_ms):
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_rank / (max_ms * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------- workloads
 
 class Case:
@@ -264,11 +279,7 @@ def run_ours(args, rank, world, local_rank):
     for i in range(K):
         for layer in range(case.L):
             dec_ms.append(evw[i][layer].elapsed_time(evd[i][layer]))
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / K
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     dec_bytes_per_launch = case.decode_bytes / case.L
@@ -279,7 +290,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device error during timing")
 
     peak, peak_kind = hbm_peak()
-    value = world * case.step_bytes / (ms_per_step * 1e-3) / 1e9
+    value = job_value(case.step_bytes, world, ms_per_step)
     achieved = dec_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     w = case.w
     line = {
@@ -409,11 +420,8 @@ def run_trace(args, rank, world, local_rank):
         torch.cuda.synchronize()
     if pk.kv_get_device_error() != pk.KV_OK:
         raise RuntimeError("device error during the trace")
-    total_ms = sum(starts[i].elapsed_time(ends[i]) for i in range(K))
+    total_ms = max_over_ranks(sum(starts[i].elapsed_time(ends[i]) for i in range(K)), dist, "cuda")
     if dist:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
         dist.destroy_process_group()
     ms = total_ms / K

@@ -227,6 +227,14 @@ int paged_attention_decode_noalloc(const kv_pool* pool, int layer, const void* q
                                    const int32_t* context_lens, int batch, int max_context_len,
                                    float scale, void* out, kv_dtype out_dtype, kv_stream_t stream);
 
+/* Self-test of the device-side failure path: enqueues one warp that waits,
+ * with the same bounded wait the decode pipeline uses, on a barrier that
+ * nothing completes.  After limit_ns nanoseconds (at most 10 s) the wait
+ * gives up and the kernel records KV_ERR_TIMEOUT, which the next
+ * kv_get_device_error returns; nothing is left in flight and the context
+ * stays usable.  For tests and health checks. */
+int kv_selftest_wait_timeout(uint64_t limit_ns, kv_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the current device's error word:
  * *err = KV_OK, KV_ERR_BOUNDS or KV_ERR_TIMEOUT (the first error any kernel
  * of this library recorded since the last call).  Errors: KV_ERR_CUDA. */

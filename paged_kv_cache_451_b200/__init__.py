@@ -71,6 +71,7 @@ _SIGS = {
     "paged_attention_decode_noalloc": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p,
                                                c_int, c_void_p, c_int, c_int, c_float, c_void_p,
                                                c_int, c_void_p]),
+    "kv_selftest_wait_timeout": (c_int, [ctypes.c_uint64, c_void_p]),
     "kv_get_device_error": (c_int, [c_void_p, P(c_int)]),
     "kv_alloc_create": (c_int, [c_int, c_int, c_void_p, P(c_void_p)]),
     "kv_alloc_num_free": (c_int, [c_void_p, P(c_int)]),
@@ -204,6 +205,10 @@ def paged_attention_decode_noalloc(pool, layer, q, q_dtype, num_q_heads, block_t
                                                _ptr(block_tables), max_blocks_per_seq,
                                                _ptr(context_lens), batch, max_context_len,
                                                float(scale), _ptr(out), out_dtype, _stream(stream)))
+
+
+def kv_selftest_wait_timeout(limit_ns, stream=None):
+    _check(_lib.kv_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def kv_get_device_error(stream=None) -> int:

@@ -118,4 +118,22 @@ __global__ void __launch_bounds__(256) block_copy_kernel(const CopyParams p) {
       sc[(int64_t)dst * p.kv_heads + h] = sc[(int64_t)src * p.kv_heads + h];
 }
 
+// Self-test of the bounded-wait error path used by the decode pipeline: one
+// warp waits on an mbarrier whose phase can never complete (a transaction
+// count that no copy will satisfy).  After limit_ns the wait gives up, the
+// kernel records KV_ERR_TIMEOUT and returns; nothing is in flight.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_arrive_expect_tx(b, 16);  // 16 bytes that never arrive
+  __syncwarp();
+  const bool ok = mbar_wait_bounded(b, 0, limit_ns);
+  if (!__all_sync(0xffffffffu, ok) && threadIdx.x == 0) record_error(KV_ERR_TIMEOUT);
+}
+
 }  // namespace pagedkv

@@ -19,7 +19,8 @@
 //   S[16 x 16]  = Q[16 x D] . K_chunk^T      rows 0..7: the query heads of this
 //                                            kv head (GQA group, zero-padded),
 //                                            rows 8..15: a copy of rows 0..7
-//   online softmax over S in the log2 domain (fp32)
+//   online softmax over S in the log2 domain (fp32), with a lazily moved
+//                                            reference max per row
 //   O[16 x D]  += P[16 x 16] . V_chunk       rows 0..7 carry the 16-bit value of
 //                                            the probabilities, rows 8..15 the
 //                                            16-bit rounding residual, so the
@@ -52,6 +53,11 @@ constexpr int kChunk = 16;           // tokens per MMA tile
 constexpr int kMaxPartChunks = 1024;  // at most 16384 tokens per partition
 constexpr int kMaxGroup = 8;         // query heads per kv head in one CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// A row's reference max is only moved (and its output rescaled) when the
+// chunk max exceeds it by more than this many binades; in between the
+// probabilities are exp2(z - m) <= 2^kLazyLog2, exact in the 16-bit hi/lo
+// split and harmless to the fp32 sums.
+constexpr float kLazyLog2 = 8.f;
 
 enum KvKind { KV_KIND_F16 = 0, KV_KIND_BF16 = 1, KV_KIND_E4M3 = 2 };
 enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_F32 = 3 };
@@ -340,26 +346,30 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       float mx = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_run, mx);
-      const float alpha = ex2(m_run - m_new);
+      const bool grow = mx > m_run + kLazyLog2;  // always true on a row's first chunk
+      const float m_new = grow ? mx : m_run;
+      const float alpha = grow ? ex2(m_run - m_new) : 1.f;
       float pr[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) pr[e] = ex2(z[e] - m_new);
       l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
       m_run = m_new;
       float alpha_o = alpha;  // rescale of O
+      bool grow_o = grow;
       if constexpr (kFp8) {
-        // weights pr * 2^(lw + m_new - mw_new) = 2^(z + lw - mw_new) <= 1
+        // weights pr * 2^(lw + m_new - mw_new) = 2^(z + lw - mw_new) <= 2^kLazyLog2
         const float lw = vsc[i];
-        const float mw_new = fmaxf(mw_run, mx + lw);
+        const bool grow_w = mx + lw > mw_run + kLazyLog2;
+        const float mw_new = grow_w ? mx + lw : mw_run;
         const bool none = mw_new == -INFINITY;
-        alpha_o = none ? 1.f : ex2(mw_run - mw_new);
+        alpha_o = (grow_w && !none) ? ex2(mw_run - mw_new) : 1.f;
+        grow_o = grow_w;
         const float c = none ? 0.f : ex2(lw + m_new - mw_new) * vsg[i];
         mw_run = mw_new;
 #pragma unroll
         for (int e = 0; e < 4; ++e) pr[e] *= c;
       }
-      if (__any_sync(0xffffffffu, alpha_o != 1.f)) {
+      if (__any_sync(0xffffffffu, grow_o)) {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
           o[t][0] *= alpha_o;

@@ -594,6 +594,15 @@ int paged_attention_decode_noalloc(const kv_pool* pool, int layer, const void* q
                                 out_dtype, scratch, need > 0 ? KV_NOALLOC_WORKSPACE_BYTES : 0, stream);
 }
 
+int kv_selftest_wait_timeout(uint64_t limit_ns, kv_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull)
+    return fail(KV_ERR_ARG, "limit_ns must be in (0, 10 s]");
+  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait_timeout_selftest_kernel launch");
+  return ok();
+}
+
 int kv_get_device_error(kv_stream_t stream, int* err) {
   if (!err) return fail(KV_ERR_ARG, "err is NULL");
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

@@ -98,6 +98,8 @@ def test_gpu_entries_reject_bad_arguments_before_launch():
         pk.block_copy(pool, 16, -1, stream=0)
     assert e.value.code == pk.KV_ERR_ARG
     with pytest.raises(pk.KVError):
+        pk.kv_selftest_wait_timeout(0, stream=0)
+    with pytest.raises(pk.KVError):
         pk.kv_pool_bind(pool, 0, 0, 0)
     with pytest.raises(pk.KVError):
         pk.kv_pool_bind(pool, 0, 24, 32)  # misaligned

@@ -170,3 +170,16 @@ def test_zero_batch_and_all_empty_contexts():
     assert np.all(out.cpu().numpy() == 0) and np.all(ref == 0)
     pool = DevicePool(4, 1, 64, 16, F16)
     pk.paged_attention_decode(pool.h, 0, 0, F16, 1, 0, 1, 0, 0, 16, 0.1, 0, F16)  # batch 0: no-op
+
+
+def test_bounded_wait_times_out_with_an_error_and_the_context_survives():
+    """A pipeline wait that can never complete gives up after its limit and
+    reports KV_ERR_TIMEOUT; the next decode on the same context is fine."""
+    import time
+    pk.kv_get_device_error()
+    t0 = time.perf_counter()
+    pk.kv_selftest_wait_timeout(50_000_000)  # 50 ms
+    assert pk.kv_get_device_error() == pk.KV_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    out, ref = run_case(F16, F16, 64, 16, 2, 2, [5, 40], seed=3)
+    assert max_abs(out.cpu().numpy(), ref) <= TOL[F16]
