@@ -188,6 +188,10 @@ class Case:
         self.slots = torch.from_numpy(self.slots_h).to(dev)
         self.tables_d = torch.from_numpy(self.tables).to(dev)
         self.lens_d = torch.from_numpy(self.lens).to(dev)
+        # the caller's scheduling order (placement only): long contexts first
+        from paged_kv_cache_451_b200.serving import schedule_order
+        self.order_h = schedule_order(self.lens, getattr(W, "order", None) or "longest")
+        self.order_d = torch.from_numpy(self.order_h).to(dev)
         self.inv = None
         if w.kv_fmt == 2:
             self.inv = [(1.0 / self.ks[l], 1.0 / self.vs[l]) for l in range(self.L)]
@@ -213,13 +217,14 @@ class Case:
                           self.vn[layer] if vn is None else vn, w.q_fmt,
                           self.slots if slots is None else slots, w.batch, inv[0], inv[1])
 
-    def decode(self, layer, q=None, tables=None, lens=None, out=None):
+    def decode(self, layer, q=None, tables=None, lens=None, out=None, order=None):
         w, pk = self.w, self.pk
         pk.paged_attention_decode(self.pool, layer, self.q[layer] if q is None else q, w.q_fmt,
                                   w.num_q_heads, self.tables_d if tables is None else tables,
                                   self.tables.shape[1], self.lens_d if lens is None else lens, w.batch,
                                   self.max_ctx, w.scale, self.out[layer] if out is None else out,
-                                  w.q_fmt, self.ws, self.ws_bytes)
+                                  w.q_fmt, self.ws, self.ws_bytes,
+                                  seq_order=self.order_d if order is None else order)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -312,6 +317,7 @@ def run_ours(args, rank, world, local_rank):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed between steps (256 MiB write)",
             "split_k": bool(case.split),
+            "order": args.order or "longest",
         },
         "seqs_per_s": round(world * w.batch / (ms_per_step * 1e-3), 1),
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
@@ -373,7 +379,8 @@ def run_trace(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = WORKLOADS["gqa_trace"]
     plan = gqa_trace_plan(w)
-    tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps))
+    tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
+                  order_policy=args.order or "batch")
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     iters = w.extra["iters"]
@@ -469,25 +476,28 @@ def run_e2e(case, torch, pk, flush, stream, K, W):
     hs = torch.from_numpy(case.slots_h).pin_memory()
     ht = torch.from_numpy(case.tables).pin_memory()
     hl = torch.from_numpy(case.lens).pin_memory()
+    ho = torch.from_numpy(case.order_h).pin_memory()
     hout = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in case.out]
     dq = [torch.empty_like(t) for t in case.q]
     dk = [torch.empty_like(t) for t in case.kn]
     dv = [torch.empty_like(t) for t in case.vn]
     ds, dt, dl = torch.empty_like(case.slots), torch.empty_like(case.tables_d), torch.empty_like(case.lens_d)
+    do = torch.empty_like(case.order_d)
     h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv) + sum(
-        t.numel() * t.element_size() for t in (hs, ht, hl))
+        t.numel() * t.element_size() for t in (hs, ht, hl, ho))
     d2h = sum(t.numel() * t.element_size() for t in hout)
 
     def step():
         ds.copy_(hs, non_blocking=True)
         dt.copy_(ht, non_blocking=True)
         dl.copy_(hl, non_blocking=True)
+        do.copy_(ho, non_blocking=True)
         for layer in range(case.L):
             dq[layer].copy_(hq[layer], non_blocking=True)
             dk[layer].copy_(hk[layer], non_blocking=True)
             dv[layer].copy_(hv[layer], non_blocking=True)
             case.write(layer, dk[layer], dv[layer], ds)
-            case.decode(layer, dq[layer], dt, dl)
+            case.decode(layer, dq[layer], dt, dl, order=do)
             hout[layer].copy_(case.out[layer], non_blocking=True)
 
     for _ in range(W):
@@ -613,6 +623,9 @@ def main():
     ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")
     ap.add_argument("--warps", type=int, default=0, help="warps per decode CTA (0: auto)")
+    ap.add_argument("--order", default=None, choices=["long_first", "longest", "batch"],
+                    help="decode scheduling order (default: longest first for one decode step, "
+                         "batch order for the continuous-batching trace)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

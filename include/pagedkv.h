@@ -185,13 +185,20 @@ size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q
  *                 output and its running maxima and sum there
  *                 (head_dim + 4 floats per (sequence, head, partition)), and
  *                 a second kernel merges them by log-sum-exp.
+ *   seq_order     NULL, or device int32 [batch]: a permutation of 0..batch-1
+ *                 giving the order in which sequences are scheduled onto the
+ *                 GPU; outputs are unaffected.  Longest context first keeps
+ *                 long sequences from starting last (a tail of idle SMs).
+ *                 An entry outside [0, batch) is skipped and reported as
+ *                 KV_ERR_BOUNDS.
  * batch == 0 enqueues nothing.  Errors: KV_ERR_ARG, KV_ERR_STATE (layer not
  * bound), KV_ERR_CUDA. */
 int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
                            int num_q_heads, const int32_t* block_tables,
                            int max_blocks_per_seq, const int32_t* context_lens, int batch,
                            int max_context_len, float scale, void* out, kv_dtype out_dtype,
-                           void* workspace, size_t workspace_bytes, kv_stream_t stream);
+                           void* workspace, size_t workspace_bytes, const int32_t* seq_order,
+                           kv_stream_t stream);
 
 /* Largest scratch paged_attention_decode_noalloc can use (16 MiB). */
 #define KV_NOALLOC_WORKSPACE_BYTES (16u << 20)
@@ -206,7 +213,8 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
  * every GPU that loads the library holds it until the process exits.  This
  * entry point allocates nothing and has no counterpart on the pages; it is an
  * interface convenience only.
- *   Arguments are those of paged_attention_decode without the workspace.
+ *   Arguments are those of paged_attention_decode without the workspace
+ *   (and with sequences scheduled in batch order).
  *   Sizes whose paged_attention_workspace_bytes(...) exceeds
  *   KV_NOALLOC_WORKSPACE_BYTES are rejected with KV_ERR_ARG (use
  *   paged_attention_decode with your own workspace, or a partition setting

@@ -67,7 +67,7 @@ _SIGS = {
     "paged_attention_workspace_bytes": (c_size_t, [c_void_p, c_int, c_int, c_int]),
     "paged_attention_decode": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int,
                                        c_void_p, c_int, c_int, c_float, c_void_p, c_int, c_void_p,
-                                       c_size_t, c_void_p]),
+                                       c_size_t, c_void_p, c_void_p]),
     "paged_attention_decode_noalloc": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p,
                                                c_int, c_void_p, c_int, c_int, c_float, c_void_p,
                                                c_int, c_void_p]),
@@ -188,11 +188,12 @@ def paged_attention_workspace_bytes(pool, batch, num_q_heads, max_context_len) -
 
 def paged_attention_decode(pool, layer, q, q_dtype, num_q_heads, block_tables, max_blocks_per_seq,
                            context_lens, batch, max_context_len, scale, out, out_dtype,
-                           workspace=None, workspace_bytes=0, stream=None):
+                           workspace=None, workspace_bytes=0, stream=None, seq_order=None):
     _check(_lib.paged_attention_decode(pool, layer, _ptr(q), q_dtype, num_q_heads,
                                        _ptr(block_tables), max_blocks_per_seq, _ptr(context_lens),
                                        batch, max_context_len, float(scale), _ptr(out), out_dtype,
-                                       _ptr(workspace), int(workspace_bytes), _stream(stream)))
+                                       _ptr(workspace), int(workspace_bytes), _ptr(seq_order),
+                                       _stream(stream)))
 
 
 KV_NOALLOC_WORKSPACE_BYTES = 16 << 20

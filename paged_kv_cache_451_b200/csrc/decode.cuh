@@ -15,17 +15,18 @@
 // own pipeline (lane 0 issues the copies for the chunk STAGES ahead) and keeps
 // its own running max / sum / output; warps are merged once at the end.
 //
-// Math per chunk (m16n8k16 tensor-core MMA, fp32 accumulate):
-//   S[16 x 16]  = Q[16 x D] . K_chunk^T      rows 0..7: the query heads of this
-//                                            kv head (GQA group, zero-padded),
-//                                            rows 8..15: a copy of rows 0..7
-//   online softmax over S in the log2 domain (fp32), with a lazily moved
-//                                            reference max per row
-//   O[16 x D]  += P[16 x 16] . V_chunk       rows 0..7 carry the 16-bit value of
-//                                            the probabilities, rows 8..15 the
-//                                            16-bit rounding residual, so the
-//                                            product keeps ~16 significant bits
-//                                            of P; O = rows 0..7 + rows 8..15.
+// Math per chunk, in transposed form (m16n8k16 tensor-core MMA, fp32
+// accumulate), so that K and V tiles from ldmatrix are A operands as they are
+// and the query group is a plain B operand:
+//   S^T[16 tokens x 8 heads]  = K_chunk[16 x D] . Q^T[D x 8]   (heads of this kv
+//                               head's GQA group, zero-padded to 8)
+//   online softmax over each head (column) in the log2 domain (fp32), with a
+//   lazily moved reference max per head
+//   P^T (16 tokens x 8 heads) is split into a 16-bit value and its 16-bit
+//   rounding residual (~16 significant bits together) and transposed into B
+//   fragments with movmatrix
+//   O^T[D x 8] += V^T[D x 16 tokens] . P^T, once for the value and once for the
+//   residual.
 // FP8 (E4M3) pools are decoded to f16 in registers (exact); the queries are
 // scaled by a power of two per head so they fit f16 without losing bits; the
 // K scale of each (block, head) multiplies its logits.  The V scale enters
@@ -43,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "device_common.cuh"
 #include "ptx.cuh"
@@ -66,6 +68,7 @@ struct DecodeParams {
   const void* q;                // [batch][num_q_heads][D] f16 / bf16
   const int32_t* block_tables;  // [batch][max_blocks]
   const int32_t* context_lens;  // [batch]
+  const int32_t* seq_order;     // NULL or [batch]: sequence of grid row z
   const float* k_scale;         // FP8: [num_blocks][kv_heads]
   const float* v_scale;
   void* out;                    // [batch][num_q_heads][D]
@@ -137,7 +140,7 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   using S = DecodeShape<KV, D, WARPS, STAGES>;
   constexpr bool kFp8 = S::kFp8;
   constexpr bool kBf16Mma = KV == KV_KIND_BF16;
-  constexpr int NT = D / 8;   // 8-column tiles of the output
+  constexpr int MT = D / 16;  // 16-row tiles of the transposed output O^T
   constexpr int KS = D / 16;  // 16-deep k-steps of q.K
 
   extern __shared__ uint8_t smem_raw[];
@@ -150,7 +153,14 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
 
   const int part = blockIdx.x;
   const int kvh = blockIdx.y;
-  const int seq = blockIdx.z;
+  int seq = blockIdx.z;
+  if (p.seq_order != nullptr) {
+    seq = p.seq_order[blockIdx.z];
+    if (seq < 0 || seq >= (int)gridDim.z) {
+      if (part == 0 && kvh == 0 && threadIdx.x == 0) record_error(KV_ERR_BOUNDS);
+      return;  // uniform over the CTA
+    }
+  }
   const int bs = p.block_size;
   const int cpb_shift = p.cpb_shift;  // log2(block_size / 16)
 
@@ -202,9 +212,11 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   }
   __syncthreads();
 
-  // ---- queries of this kv head's group as MMA A fragments (rows 8..15 = rows 0..7)
-  uint32_t qa[KS][2];
-  float zrow;
+  // ---- queries of this kv head's group as MMA B fragments: lane (gq, cq)
+  // holds head gq's values at MMA k = 2cq, 2cq+1 (qb[ks][0]) and 2cq+8, 2cq+9
+  // (qb[ks][1]); heads beyond the group are zero.
+  uint32_t qb[KS][2];
+  float zrow;  // logit scale of head gq (log2 units)
   {
     const bool valid = gq < p.group;
     const int64_t qrow = ((int64_t)seq * p.num_q_heads + kvh * p.group + (valid ? gq : 0)) * D;
@@ -212,8 +224,8 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
     if constexpr (!kFp8) {
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        qa[ks][0] = valid ? *reinterpret_cast<const uint32_t*>(qh + ks * 16 + 2 * cq) : 0u;
-        qa[ks][1] = valid ? *reinterpret_cast<const uint32_t*>(qh + ks * 16 + 8 + 2 * cq) : 0u;
+        qb[ks][0] = valid ? *reinterpret_cast<const uint32_t*>(qh + ks * 16 + 2 * cq) : 0u;
+        qb[ks][1] = valid ? *reinterpret_cast<const uint32_t*>(qh + ks * 16 + 8 + 2 * cq) : 0u;
       }
       zrow = p.scale_log2;
     } else {
@@ -240,21 +252,23 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       const float mult = __uint_as_float((uint32_t)(e + 127) << 23);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        qa[ks][0] = pack2<false>(v[ks][0] * mult, v[ks][1] * mult);
-        qa[ks][1] = pack2<false>(v[ks][2] * mult, v[ks][3] * mult);
+        qb[ks][0] = pack2<false>(v[ks][0] * mult, v[ks][1] * mult);
+        qb[ks][1] = pack2<false>(v[ks][2] * mult, v[ks][3] * mult);
       }
       zrow = p.scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23);
     }
   }
+  // this lane's S^T columns are heads 2cq and 2cq + 1
+  const float zs_a = __shfl_sync(0xffffffffu, zrow, (2 * cq) * 4);
+  const float zs_b = __shfl_sync(0xffffffffu, zrow, (2 * cq + 1) * 4);
 
   // ---- per-warp pipeline over chunks i = warp, warp + WARPS, ...
   const int my_n = nchunks > warp ? (nchunks - warp + WARPS - 1) / WARPS : 0;
   const uint32_t wstage = sbase + warp * STAGES * S::STAGEB;
   const uint32_t wbar = bars + warp * STAGES * 8;
 
-  auto issue = [&](int li) {
+  auto issue = [&](int li, int st) {
     const int i = warp + li * WARPS;
-    const int st = li % STAGES;
     const uint32_t bar = wbar + st * 8;
     const int32_t b = blk_ids[i];
     if (b < 0) {
@@ -272,22 +286,41 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   };
 
   if (lane == 0) {
-    for (int li = 0; li < STAGES && li < my_n; ++li) issue(li);
+    for (int li = 0; li < STAGES && li < my_n; ++li) issue(li, li);
   }
   __syncwarp();
 
-  float m_run = -INFINITY;   // running max of the logits (log2 domain)
-  float l_run = 0.f;         // running softmax sum, relative to m_run
-  float mw_run = -INFINITY;  // FP8: running max of logit + log2|V scale|
-  float o[NT][4];
+  // Per-lane running state for its two heads (a = 2cq, b = 2cq + 1).
+  float m_a = -INFINITY, m_b = -INFINITY;    // reference max of the logits (log2)
+  float l_a = 0.f, l_b = 0.f;                // this lane's share of the softmax sums
+  float mw_a = -INFINITY, mw_b = -INFINITY;  // FP8: reference max of logit + log2|V scale|
+  // O^T accumulators: tile t covers 16 output dims (rows) x 8 heads (columns)
+  float o[MT][4];
 #pragma unroll
-  for (int t = 0; t < NT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+  for (int t = 0; t < MT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+
+  // ldmatrix row (token) and 16-byte column chunk of this lane
+  const int krow = (lane & 7) + (((lane >> 3) & 1) << 3);  // K: m0 tok 0-7, m1 tok 8-15, ...
+  const int kcol = lane >> 4;
+  const int vrow = kFp8 ? krow : (lane & 7) + ((lane >> 4) << 3);
+  const int vcol = kFp8 ? (lane >> 4) : ((lane >> 3) & 1);
+  // Swizzled byte offsets of this lane's ldmatrix rows.  Column chunk
+  // 2j + col of a tile sits in box (2j + col) / CPR; within a box the swizzle
+  // XOR depends only on the lane's row, so the offsets repeat every CPR / 2
+  // steps up to a whole-box (compile-time) displacement.
+  constexpr int NOFF = S::CPR / 2;
+  uint32_t koff[NOFF], voff[NOFF];
+#pragma unroll
+  for (int j = 0; j < NOFF; ++j) {
+    koff[j] = tile_off<S>(krow, 2 * j + kcol);
+    voff[j] = tile_off<S>(vrow, 2 * j + vcol);
+  }
 
   int li = 0;
+  int st = 0;           // stage of chunk li
+  uint32_t parity = 0;  // barrier phase parity of chunk li
   bool failed = false;
   for (; li < my_n; ++li) {
-    const int st = li % STAGES;
-    const uint32_t parity = (li / STAGES) & 1;
     const bool ready = mbar_wait_bounded(wbar + st * 8, parity, kWaitLimitNs);
     if (!__all_sync(0xffffffffu, ready)) {
       failed = true;
@@ -299,132 +332,163 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       const uint32_t kb = wstage + st * S::STAGEB;
       const uint32_t vb = kb + S::TILEB;
 
-      // S = Q . K^T: tile 0 = tokens 0..7, tile 1 = tokens 8..15.  Even and odd
-      // k-steps accumulate separately (four independent MMA chains) and are
-      // summed afterwards, halving the dependent-MMA latency per chunk.
-      float sa[2][2][4] = {};
+      // S^T = K . Q^T (16 tokens x 8 heads); even / odd k-steps accumulate
+      // separately: lane (gq, cq) gets tokens gq, gq+8 of heads 2cq, 2cq+1
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       if constexpr (!kFp8) {
-        const int row = (lane & 7) + ((lane >> 4) << 3);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kb + tile_off<S>(row, ks * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-          mma_16816<kBf16Mma>(sa[ks & 1][0], qa[ks][0], qa[ks][0], qa[ks][1], qa[ks][1], b0, b1);
-          mma_16816<kBf16Mma>(sa[ks & 1][1], qa[ks][0], qa[ks][0], qa[ks][1], qa[ks][1], b2, b3);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kb + koff[ks % NOFF] + (ks / NOFF) * (kChunk * S::BOXB), a0, a1, a2, a3);
+          mma_16816<kBf16Mma>(sacc[ks & 1], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
         }
       } else {
-        const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
         for (int kp = 0; kp < KS / 2; ++kp) {
           uint32_t r0, r1, r2, r3;
-          ldsm_x4(kb + tile_off<S>(row, kp * 2 + (lane >> 4)), r0, r1, r2, r3);
-          const int k0 = 2 * kp, k1 = 2 * kp + 1;
+          ldsm_x4(kb + koff[kp % NOFF] + (kp / NOFF) * (kChunk * S::BOXB), r0, r1, r2, r3);
           uint32_t f0l, f0h, f1l, f1h, f2l, f2h, f3l, f3h;
           e4m3x4_to_f16x4(r0, f0l, f0h);
           e4m3x4_to_f16x4(r1, f1l, f1h);
           e4m3x4_to_f16x4(r2, f2l, f2h);
           e4m3x4_to_f16x4(r3, f3l, f3h);
-          mma_16816<false>(sa[0][0], qa[k0][0], qa[k0][0], qa[k0][1], qa[k0][1], f0l, f0h);
-          mma_16816<false>(sa[0][1], qa[k0][0], qa[k0][0], qa[k0][1], qa[k0][1], f1l, f1h);
-          mma_16816<false>(sa[1][0], qa[k1][0], qa[k1][0], qa[k1][1], qa[k1][1], f2l, f2h);
-          mma_16816<false>(sa[1][1], qa[k1][0], qa[k1][0], qa[k1][1], qa[k1][1], f3l, f3h);
+          mma_16816<false>(sacc[0], f0l, f1l, f0h, f1h, qb[2 * kp][0], qb[2 * kp][1]);
+          mma_16816<false>(sacc[1], f2l, f3l, f2h, f3h, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
         }
       }
-      const float s00 = sa[0][0][0] + sa[1][0][0], s01 = sa[0][0][1] + sa[1][0][1];
-      const float s10 = sa[0][1][0] + sa[1][1][0], s11 = sa[0][1][1] + sa[1][1][1];
 
-      // online softmax (log2 domain) over this lane's 4 tokens of row gq
-      float zs = zrow;
-      if constexpr (kFp8) zs *= ksc[i];
-      float z[4] = {s00 * zs, s01 * zs, s10 * zs, s11 * zs};
-      if (vt < kChunk) {
-        if (2 * cq >= vt) z[0] = -INFINITY;
-        if (2 * cq + 1 >= vt) z[1] = -INFINITY;
-        if (8 + 2 * cq >= vt) z[2] = -INFINITY;
-        if (9 + 2 * cq >= vt) z[3] = -INFINITY;
-      }
-      float mx = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const bool grow = mx > m_run + kLazyLog2;  // always true on a row's first chunk
-      const float m_new = grow ? mx : m_run;
-      const float alpha = grow ? ex2(m_run - m_new) : 1.f;
-      float pr[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) pr[e] = ex2(z[e] - m_new);
-      l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-      m_run = m_new;
-      float alpha_o = alpha;  // rescale of O
-      bool grow_o = grow;
+      // online softmax (log2 domain) for heads a, b over this lane's tokens
+      float zsa = zs_a, zsb = zs_b;
       if constexpr (kFp8) {
-        // weights pr * 2^(lw + m_new - mw_new) = 2^(z + lw - mw_new) <= 2^kLazyLog2
-        const float lw = vsc[i];
-        const bool grow_w = mx + lw > mw_run + kLazyLog2;
-        const float mw_new = grow_w ? mx + lw : mw_run;
-        const bool none = mw_new == -INFINITY;
-        alpha_o = (grow_w && !none) ? ex2(mw_run - mw_new) : 1.f;
-        grow_o = grow_w;
-        const float c = none ? 0.f : ex2(lw + m_new - mw_new) * vsg[i];
-        mw_run = mw_new;
+        zsa *= ksc[i];
+        zsb *= ksc[i];
+      }
+      float z[4] = {(sacc[0][0] + sacc[1][0]) * zsa, (sacc[0][1] + sacc[1][1]) * zsb,
+                    (sacc[0][2] + sacc[1][2]) * zsa, (sacc[0][3] + sacc[1][3]) * zsb};
+      if (vt < kChunk) {
+        if (gq >= vt) z[0] = z[1] = -INFINITY;
+        if (gq + 8 >= vt) z[2] = z[3] = -INFINITY;
+      }
+      // A head's max over the chunk is only needed when some value exceeds its
+      // reference max by more than 2^kLazyLog2 (the first chunk, rarely later);
+      // if no lane's own max does, no head max does, so all lanes agree.
+      float mxa = fmaxf(z[0], z[2]), mxb = fmaxf(z[1], z[3]);
+      float lw = 0.f;  // FP8: log2 |V scale| of this chunk
+      if constexpr (kFp8) lw = vsc[i];
+      bool need = mxa > m_a + kLazyLog2 || mxb > m_b + kLazyLog2;
+      if constexpr (kFp8)
+        need = need || mxa + lw > mw_a + kLazyLog2 || mxb + lw > mw_b + kLazyLog2;
+      if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pr[e] *= c;
+        for (int off = 4; off < 32; off <<= 1) {
+          mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, off));
+          mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, off));
+        }
+      }
+      const bool grow_a = mxa > m_a + kLazyLog2, grow_b = mxb > m_b + kLazyLog2;
+      const float ma = grow_a ? mxa : m_a, mb = grow_b ? mxb : m_b;
+      const float alpha_a = grow_a ? ex2(m_a - ma) : 1.f;
+      const float alpha_b = grow_b ? ex2(m_b - mb) : 1.f;
+      float pr[4] = {ex2(z[0] - ma), ex2(z[1] - mb), ex2(z[2] - ma), ex2(z[3] - mb)};
+      l_a = l_a * alpha_a + (pr[0] + pr[2]);
+      l_b = l_b * alpha_b + (pr[1] + pr[3]);
+      m_a = ma;
+      m_b = mb;
+      float ao_a = alpha_a, ao_b = alpha_b;  // rescale of O's columns a, b
+      bool grow_o = grow_a || grow_b;
+      if constexpr (kFp8) {
+        // weights pr * 2^(lw + m - mw) = 2^(z + lw - mw) <= 2^kLazyLog2
+        const bool gwa = mxa + lw > mw_a + kLazyLog2, gwb = mxb + lw > mw_b + kLazyLog2;
+        const float nwa = gwa ? mxa + lw : mw_a, nwb = gwb ? mxb + lw : mw_b;
+        ao_a = (gwa && nwa != -INFINITY) ? ex2(mw_a - nwa) : 1.f;
+        ao_b = (gwb && nwb != -INFINITY) ? ex2(mw_b - nwb) : 1.f;
+        grow_o = gwa || gwb;
+        const float ca = nwa == -INFINITY ? 0.f : ex2(lw + ma - nwa) * vsg[i];
+        const float cb = nwb == -INFINITY ? 0.f : ex2(lw + mb - nwb) * vsg[i];
+        mw_a = nwa;
+        mw_b = nwb;
+        pr[0] *= ca;
+        pr[2] *= ca;
+        pr[1] *= cb;
+        pr[3] *= cb;
       }
       if (__any_sync(0xffffffffu, grow_o)) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          o[t][0] *= alpha_o;
-          o[t][1] *= alpha_o;
-          o[t][2] *= alpha_o;
-          o[t][3] *= alpha_o;
+        for (int t = 0; t < MT; ++t) {
+          o[t][0] *= ao_a;
+          o[t][1] *= ao_b;
+          o[t][2] *= ao_a;
+          o[t][3] *= ao_b;
         }
       }
-      // P as A fragment: rows 0..7 the 16-bit values, rows 8..15 the residuals
-      uint32_t pa0, pa1, pa2, pa3;
-      split2<kBf16Mma>(pr[0], pr[1], pa0, pa1);
-      split2<kBf16Mma>(pr[2], pr[3], pa2, pa3);
 
-      // O += P . V
-      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;  // token masks for b0 / b1 registers
-      if (vt < kChunk) {
-        mlo = (2 * cq < vt ? 0x0000ffffu : 0u) | (2 * cq + 1 < vt ? 0xffff0000u : 0u);
-        mhi = (8 + 2 * cq < vt ? 0x0000ffffu : 0u) | (9 + 2 * cq < vt ? 0xffff0000u : 0u);
-      }
-      const int vrow = (lane & 7) + (((lane >> 3) & 1) << 3);
-      if constexpr (!kFp8) {
+      // P^T as B fragments: P (tokens x heads) in 16-bit value + residual
+      // halves, transposed so lane (g, c) holds tokens 2c, 2c+1 of head g
+      uint32_t h0, l0, h1, l1;
+      split2<kBf16Mma>(pr[0], pr[1], h0, l0);  // token gq, heads a, b
+      split2<kBf16Mma>(pr[2], pr[3], h1, l1);  // token gq + 8
+      const uint32_t bh0 = movmatrix_t(h0), bh1 = movmatrix_t(h1);
+      const uint32_t bl0 = movmatrix_t(l0), bl1 = movmatrix_t(l1);
+
+      // O^T += V^T . P^T.  The last chunk of a context zeroes the V values of
+      // its tokens >= vt (stale slots may hold any bits, and 0 * NaN is NaN);
+      // full chunks skip the masking.
+      auto pv = [&](uint32_t mlo, uint32_t mhi, auto masked) {
+        constexpr bool kMask = decltype(masked)::value;
+        if constexpr (!kFp8) {
 #pragma unroll
-        for (int jp = 0; jp < NT / 2; ++jp) {
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4_t(vb + tile_off<S>(vrow, jp * 2 + (lane >> 4)), r0, r1, r2, r3);
-          mma_16816<kBf16Mma>(o[2 * jp], pa0, pa1, pa2, pa3, r0 & mlo, r1 & mhi);
-          mma_16816<kBf16Mma>(o[2 * jp + 1], pa0, pa1, pa2, pa3, r2 & mlo, r3 & mhi);
+          for (int t = 0; t < MT; ++t) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vb + voff[t % NOFF] + (t / NOFF) * (kChunk * S::BOXB), a0, a1, a2, a3);
+            if constexpr (kMask) {
+              a0 &= mlo;
+              a1 &= mlo;
+              a2 &= mhi;
+              a3 &= mhi;
+            }
+            mma_16816<kBf16Mma>(o[t], a0, a1, a2, a3, bh0, bh1);
+            mma_16816<kBf16Mma>(o[t], a0, a1, a2, a3, bl0, bl1);
+          }
+        } else {
+#pragma unroll
+          for (int cp = 0; cp < MT / 2; ++cp) {
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_t(vb + voff[cp % NOFF] + (cp / NOFF) * (kChunk * S::BOXB), r0, r1, r2, r3);
+            if constexpr (kMask) {
+              r0 &= mlo;
+              r1 &= mhi;
+              r2 &= mlo;
+              r3 &= mhi;
+            }
+            // bytes of r: [tok 2c][d0], [tok 2c][d0+1], [tok 2c+1][d0], [tok 2c+1][d0+1],
+            // d0 = 16 * chunk + 2g; tile rows 0..7 take the even dims, 8..15 the odd
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t lo = h ? r2 : r0, hi = h ? r3 : r1;
+              const uint32_t a0 = e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0020));
+              const uint32_t a1 = e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0031));
+              const uint32_t a2 = e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0020));
+              const uint32_t a3 = e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0031));
+              mma_16816<false>(o[2 * cp + h], a0, a1, a2, a3, bh0, bh1);
+              mma_16816<false>(o[2 * cp + h], a0, a1, a2, a3, bl0, bl1);
+            }
+          }
         }
+      };
+      if (vt == kChunk) {
+        pv(0u, 0u, std::false_type{});
       } else {
-#pragma unroll
-        for (int jp = 0; jp < NT / 4; ++jp) {
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4_t(vb + tile_off<S>(vrow, jp * 2 + (lane >> 4)), r0, r1, r2, r3);
-          r0 &= mlo;
-          r1 &= mhi;
-          r2 &= mlo;
-          r3 &= mhi;
-          // bytes of r: [tok 2c][d0], [tok 2c][d0+1], [tok 2c+1][d0], [tok 2c+1][d0+1]
-          mma_16816<false>(o[4 * jp + 0], pa0, pa1, pa2, pa3,
-                           e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0020)),
-                           e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0020)));
-          mma_16816<false>(o[4 * jp + 1], pa0, pa1, pa2, pa3,
-                           e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0031)),
-                           e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0031)));
-          mma_16816<false>(o[4 * jp + 2], pa0, pa1, pa2, pa3,
-                           e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0020)),
-                           e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0020)));
-          mma_16816<false>(o[4 * jp + 3], pa0, pa1, pa2, pa3,
-                           e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0031)),
-                           e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0031)));
-        }
+        const uint32_t mlo = (2 * cq < vt ? 0x0000ffffu : 0u) | (2 * cq + 1 < vt ? 0xffff0000u : 0u);
+        const uint32_t mhi = (8 + 2 * cq < vt ? 0x0000ffffu : 0u) | (9 + 2 * cq < vt ? 0xffff0000u : 0u);
+        pv(mlo, mhi, std::true_type{});
       }
     }
     __syncwarp();
-    if (lane == 0 && li + STAGES < my_n) issue(li + STAGES);
+    if (lane == 0 && li + STAGES < my_n) issue(li + STAGES, st);
+    if (++st == STAGES) {
+      st = 0;
+      parity ^= 1u;
+    }
   }
 
   if (failed) {
@@ -436,30 +500,45 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   }
 
   // ---- merge the warps
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {  // sum over the 8 lanes of heads a, b
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
+  }
   __syncthreads();  // every warp is done with its stages: reuse them for the merge
   float* obuf = reinterpret_cast<float*>(smem);  // [WARPS][kMaxGroup][D]
-  if (gq < p.group) {
-    float* row = obuf + (warp * kMaxGroup + gq) * D;
+  const int ha = 2 * cq, hb = 2 * cq + 1;
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      int d0, d1;
-      if constexpr (!kFp8) {
-        d0 = 8 * t + 2 * cq;
-        d1 = d0 + 1;
-      } else {
-        d0 = 16 * (t >> 1) + 4 * cq + (t & 1);
-        d1 = d0 + 2;
-      }
-      row[d0] = o[t][0] + o[t][2];
-      row[d1] = o[t][1] + o[t][3];
+  for (int t = 0; t < MT; ++t) {
+    int d0, d1;  // output dims of accumulator rows gq and gq + 8
+    if constexpr (!kFp8) {
+      d0 = 16 * t + gq;
+      d1 = d0 + 8;
+    } else {
+      d0 = 16 * t + 2 * gq;
+      d1 = d0 + 1;
     }
-    if (cq == 0) {
-      float* ml = mls + (warp * kMaxGroup + gq) * 4;
-      ml[0] = m_run;
-      ml[1] = l_run;
-      ml[2] = kFp8 ? mw_run : m_run;
+    if (ha < p.group) {
+      obuf[(warp * kMaxGroup + ha) * D + d0] = o[t][0];
+      obuf[(warp * kMaxGroup + ha) * D + d1] = o[t][2];
+    }
+    if (hb < p.group) {
+      obuf[(warp * kMaxGroup + hb) * D + d0] = o[t][1];
+      obuf[(warp * kMaxGroup + hb) * D + d1] = o[t][3];
+    }
+  }
+  if (gq == 0) {
+    if (ha < p.group) {
+      float* ml = mls + (warp * kMaxGroup + ha) * 4;
+      ml[0] = m_a;
+      ml[1] = l_a;
+      ml[2] = kFp8 ? mw_a : m_a;
+    }
+    if (hb < p.group) {
+      float* ml = mls + (warp * kMaxGroup + hb) * 4;
+      ml[0] = m_b;
+      ml[1] = l_b;
+      ml[2] = kFp8 ? mw_b : m_b;
     }
   }
   __syncthreads();

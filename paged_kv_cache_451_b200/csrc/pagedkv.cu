@@ -456,7 +456,7 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
                            int num_q_heads, const int32_t* block_tables, int max_blocks_per_seq,
                            const int32_t* context_lens, int batch, int max_context_len,
                            float scale, void* out, kv_dtype out_dtype, void* workspace,
-                           size_t workspace_bytes, kv_stream_t stream) {
+                           size_t workspace_bytes, const int32_t* seq_order, kv_stream_t stream) {
   if (!pool) return fail(KV_ERR_ARG, "NULL pool");
   if (layer < 0 || layer >= pool->num_layers) return fail(KV_ERR_ARG, "layer %d out of range", layer);
   const LayerBinding& lb = pool->layers[layer];
@@ -492,6 +492,7 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   p.q = q;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
+  p.seq_order = seq_order;
   p.k_scale = lb.k_scale;
   p.v_scale = lb.v_scale;
   p.out = out;
@@ -591,7 +592,8 @@ int paged_attention_decode_noalloc(const kv_pool* pool, int layer, const void* q
   }
   return paged_attention_decode(pool, layer, q, q_dtype, num_q_heads, block_tables,
                                 max_blocks_per_seq, context_lens, batch, max_context_len, scale, out,
-                                out_dtype, scratch, need > 0 ? KV_NOALLOC_WORKSPACE_BYTES : 0, stream);
+                                out_dtype, scratch, need > 0 ? KV_NOALLOC_WORKSPACE_BYTES : 0, nullptr,
+                                stream);
 }
 
 int kv_selftest_wait_timeout(uint64_t limit_ns, kv_stream_t stream) {

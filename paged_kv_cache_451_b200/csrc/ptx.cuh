@@ -101,6 +101,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+// Transpose an 8x8 matrix of 16-bit elements held in the standard fragment
+// layout (lane 4g+c holds row g, columns 2c and 2c+1).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------ MMA
 
 // D += A(16x16, row) * B(16x8, col), fp32 accumulate.  kBf16 selects bf16

@@ -183,3 +183,36 @@ def test_bounded_wait_times_out_with_an_error_and_the_context_survives():
     assert time.perf_counter() - t0 < 5.0
     out, ref = run_case(F16, F16, 64, 16, 2, 2, [5, 40], seed=3)
     assert max_abs(out.cpu().numpy(), ref) <= TOL[F16]
+
+
+def test_scheduling_order_does_not_change_outputs():
+    """Any permutation in seq_order gives bit-identical outputs; an entry
+    outside the batch is reported and skipped."""
+    rng = np.random.default_rng(12)
+    lens = np.array([700, 3, 129, 2049, 0, 16, 1500], np.int32)
+    hq, hkv, d, bs = 8, 2, 128, 16
+    nb = int(sum(-(-max(int(n), 1) // bs) for n in lens)) + 4
+    kh, vh = normal_bits(rng, (nb, hkv, bs, d), BF16), normal_bits(rng, (nb, hkv, bs, d), BF16)
+    tables = scattered_tables(rng, np.maximum(lens, 1), bs, nb)
+    q = normal_bits(rng, (len(lens), hq, d), BF16)
+    for part in (0, 256):
+        pool = DevicePool(nb, hkv, d, bs, BF16, k=[dev(kh)], v=[dev(vh)], partition=part)
+        b, width, max_ctx = len(lens), tables.shape[1], int(lens.max())
+        wsb = pk.paged_attention_workspace_bytes(pool.h, b, hq, max_ctx)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        outs = []
+        for order in (None, np.argsort(-lens, kind="stable"), rng.permutation(b)):
+            out = torch.full((b, hq, d), float("nan"), device="cuda")
+            pk.paged_attention_decode(pool.h, 0, dev(q), BF16, hq, dev(tables), width, dev(lens), b, max_ctx,
+                                      0.09, out, pk.KV_F32, ws, wsb,
+                                      seq_order=None if order is None else dev(order.astype(np.int32)))
+            outs.append(out.cpu().numpy())
+        assert pk.kv_get_device_error() == pk.KV_OK
+        assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+        ref = oracle.paged_decode(kh, vh, BF16, q, BF16, tables, lens, 0.09, bs)
+        assert max_abs(outs[0], ref) <= TOL[BF16]
+    bad = np.array([0, 1, 2, 3, 4, 5, 7], np.int32)
+    out = torch.zeros((len(lens), hq, d), device="cuda")
+    pk.paged_attention_decode(pool.h, 0, dev(q), BF16, hq, dev(tables), tables.shape[1], dev(lens), len(lens),
+                              int(lens.max()), 0.09, out, pk.KV_F32, ws, wsb, seq_order=dev(bad))
+    assert pk.kv_get_device_error() == pk.KV_ERR_BOUNDS
