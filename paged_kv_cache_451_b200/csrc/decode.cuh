@@ -37,7 +37,8 @@
 // the output is (O / l) * 2^(m_w - m_z).
 //
 // A context longer than one partition is split: each partition writes its
-// unnormalised output and (m_z, l, m_w), and lse_reduce_kernel merges them.
+// unnormalised output and (m_z, l, m_w), and lse_reduce_kernel merges them;
+// a context within one partition is written normalised by its only CTA.
 #pragma once
 
 #include <cuda.h>
@@ -543,7 +544,9 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   }
   __syncthreads();
 
-  const bool split = p.num_parts > 1;
+  // a context that fits one partition is finished here even in split mode;
+  // the reduce kernel skips it
+  const bool split = p.num_parts > 1 && total_chunks > p.part_chunks;
   for (int idx = threadIdx.x; idx < p.group * D; idx += WARPS * 32) {
     const int g = idx / D;
     const int d = idx - g * D;
@@ -597,6 +600,7 @@ lse_reduce_kernel(const float* __restrict__ part_o, const float* __restrict__ pa
   int n = context_lens[seq];
   n = n < 0 ? 0 : (n > ctx_cap ? ctx_cap : n);
   const int np = max(1, (n + part_tokens - 1) / part_tokens);
+  if (np == 1) return;  // written by the decode kernel directly
   const float4* ml = reinterpret_cast<const float4*>(part_ml) + idx * num_parts;
   float Mz = -INFINITY, Mw = -INFINITY;
   for (int q = lane; q < np; q += 32) {

@@ -156,23 +156,26 @@ int decode_slots(const kv_pool* pool) {
 }
 
 // Partition length in tokens.  Automatic: contexts are cut into partitions
-// of at most kAutoPartition tokens; if that leaves fewer than kWaves waves of
-// resident CTAs, into more (down to kMinPartition tokens) until it does not.
-// Measured on B200: one partition per 2K-token context is best for uniform
-// 16-bit contexts (the 32-layer example), ~2K-token partitions for the
-// 16K-token FP8 contexts.
-constexpr int kWaves = 3;
-constexpr int kAutoPartition = 2048;
+// of at most kAutoPartition tokens.  If the (sequence, kv head) units then
+// give fewer than kWavesKeep waves of resident CTAs, contexts are split
+// further, into enough partitions (of at least kMinPartition tokens) for
+// kWavesSplit waves.  Measured on B200: unsplit 2K-token contexts with 1024
+// units (32-layer example, 3.5 waves), 4K-token partitions for a 256-sequence
+// lognormal batch (few long contexts; the others skip the reduce), 1-2K-token
+// partitions for 8 x 16K-token FP8 contexts (256 units).
+constexpr int kWavesKeep = 3;
+constexpr int kWavesSplit = 8;
+constexpr int kAutoPartition = 4096;
 constexpr int kMinPartition = 512;
 
 int partition_tokens(const kv_pool* pool, int batch, int max_context_len) {
   if (pool->partition_tokens > 0) return pool->partition_tokens;
   const int ctx = std::max(max_context_len, 1);
   const int64_t units = std::max<int64_t>(1, (int64_t)batch * pool->kv_heads);
-  const int64_t want = (int64_t)kWaves * decode_slots(pool);
+  const int64_t slots = decode_slots(pool);
   int64_t np = (ctx + kAutoPartition - 1) / kAutoPartition;
-  if (units * np < want) {
-    np = std::max<int64_t>(np, (want + units - 1) / units);
+  if (units < (int64_t)kWavesKeep * slots) {
+    np = std::max<int64_t>(np, (kWavesSplit * slots + units - 1) / units);
     np = std::min<int64_t>(np, std::max<int64_t>(1, (ctx + kMinPartition - 1) / kMinPartition));
   }
   const int64_t per = (ctx + np - 1) / np;

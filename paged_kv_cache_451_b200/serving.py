@@ -7,8 +7,8 @@ the order of the scheduling loop on "vLLM æŽ¨ç†åŠ é€ŸåŽŸç†è¯¦è§£ï¼šå¤§æ¨¡åž‹æœ
 1. ``kv_sched_step`` (native, host): free the finished sequences, admit
    waiting requests first come first served, append one slot per running
    sequence (copy-on-write pairs where a shared block is written);
-2. upload the step's metadata (block tables, context lengths, slots, copy
-   pairs) from pinned host buffers with one async copy each;
+2. upload the step's metadata (block tables, context lengths, slots,
+   scheduling order, copy pairs) with one async copy from a pinned buffer;
 3. ``block_copy`` for the copy-on-write pairs;
 4. ``paged_kv_write`` of the step's new tokens (admitted prompts, then one
    token per running sequence);
@@ -49,6 +49,13 @@ def schedule_order(context_lens, policy="long_first"):
 
 
 class DecodeLoop:
+    """Runs the iteration above on one device.  The step's metadata (slots,
+    block tables, context lengths, scheduling order, copy pairs) is packed
+    into one pinned buffer and uploaded with one copy on a side stream, into
+    one of two device buffers, so the upload of the next step overlaps the
+    kernels of the current one; events keep each buffer alive until the
+    kernels that read it have run."""
+
     def __init__(self, pool, sched, *, num_q_heads, kv_heads, head_dim, block_size, q_dtype,
                  scale, max_batch, max_blocks, max_tokens, max_context, device="cuda",
                  order_policy="batch"):
@@ -58,22 +65,18 @@ class DecodeLoop:
         self.hq, self.hkv, self.d, self.bs = num_q_heads, kv_heads, head_dim, block_size
         self.q_dtype, self.scale = q_dtype, scale
         self.max_batch, self.max_blocks, self.max_tokens = max_batch, max_blocks, max_tokens
-        pin = dict(pin_memory=True)
-        self.h_tables = torch.empty(max_batch * max_blocks, dtype=torch.int32, **pin)
-        self.h_lens = torch.empty(max_batch, dtype=torch.int32, **pin)
-        self.h_slots = torch.empty(max_tokens, dtype=torch.int64, **pin)
-        self.h_cow = torch.empty(2 * max_batch, dtype=torch.int32, **pin)
-        self.h_order = torch.empty(max_batch, dtype=torch.int32, **pin)
-        self.d_tables = torch.empty(max_batch * max_blocks, dtype=torch.int32, device=device)
-        self.d_lens = torch.empty(max_batch, dtype=torch.int32, device=device)
-        self.d_slots = torch.empty(max_tokens, dtype=torch.int64, device=device)
-        self.d_cow = torch.empty(2 * max_batch, dtype=torch.int32, device=device)
-        self.d_order = torch.empty(max_batch, dtype=torch.int32, device=device)
+        self.order_policy = order_policy
+        cap = 8 * max_tokens + 4 * (max_batch * max_blocks + 4 * max_batch)
+        self.cap = (cap + 255) // 256 * 256
+        self.h_buf = [torch.empty(self.cap, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        self.d_buf = [torch.empty(self.cap, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.copy_ev = [None, None]  # upload into buffer k finished
+        self.done_ev = [None, None]  # kernels reading buffer k finished
+        self.side = torch.cuda.Stream(device=device)
+        self.it = 0
         ws = paged_attention_workspace_bytes(pool, max_batch, num_q_heads, max_context)
         self.ws_cap = max(ws, 16)
         self.d_ws = torch.empty(self.ws_cap, dtype=torch.uint8, device=device)
-        self.copy_done = None
-        self.order_policy = order_policy
 
     def schedule(self, finished_ids):
         """Native scheduler step; returns the step's host outputs."""
@@ -84,40 +87,69 @@ class DecodeLoop:
         out["info"] = info
         return out
 
+    @staticmethod
+    def _layout(b, t, c, width):
+        off, lay = 0, {}
+        for name, n, size in (("slots", t, 8), ("tables", b * width, 4), ("lens", b, 4),
+                              ("order", b, 4), ("cow", 2 * c, 4)):
+            lay[name] = (off, n)
+            off += (n * size + 15) // 16 * 16
+        return lay, off
+
     def launch(self, plan, k_new, v_new, q, out, k_inv=None, v_inv=None, out_dtype=None,
                layer=0, stream=None):
         """Upload the plan's metadata and enqueue copy, write and decode."""
         torch = self.torch
         info = plan["info"]
-        b, t, c = info.batch, info.num_tokens, info.num_cow
-        if self.copy_done is not None:  # pinned buffers are reused: previous uploads must be done
-            self.copy_done.synchronize()
-        self.h_tables[: b * self.max_blocks].numpy()[:] = plan["block_tables"].reshape(-1)
-        self.h_lens[:b].numpy()[:] = plan["context_lens"]
-        self.h_order[:b].numpy()[:] = schedule_order(plan["context_lens"], self.order_policy)
-        self.h_slots[:t].numpy()[:] = plan["slot_mapping"]
-        if c:
-            self.h_cow[: 2 * c].numpy()[:] = plan["cow_pairs"].reshape(-1)
-        self.d_tables[: b * self.max_blocks].copy_(self.h_tables[: b * self.max_blocks], non_blocking=True)
-        self.d_lens[:b].copy_(self.h_lens[:b], non_blocking=True)
-        self.d_order[:b].copy_(self.h_order[:b], non_blocking=True)
-        self.d_slots[:t].copy_(self.h_slots[:t], non_blocking=True)
-        if c:
-            self.d_cow[: 2 * c].copy_(self.h_cow[: 2 * c], non_blocking=True)
-        self.copy_done = torch.cuda.Event()
-        self.copy_done.record()
+        b, t, c, w = info.batch, info.num_tokens, info.num_cow, self.max_blocks
+        k = self.it % 2
+        self.it += 1
+        lay, nbytes = self._layout(b, t, c, w)
+        if nbytes > self.cap:
+            raise RuntimeError("step metadata exceeds the loop's buffers")
+        if self.copy_ev[k] is not None:  # the pinned buffer is reused: its last upload must be done
+            self.copy_ev[k].synchronize()
+        hb = self.h_buf[k].numpy()
+
+        def put(name, arr, dtype):
+            off, n = lay[name]
+            if n:
+                hb[off:off + n * np.dtype(dtype).itemsize].view(dtype)[:] = np.asarray(arr, dtype).reshape(-1)
+
+        put("slots", plan["slot_mapping"], np.int64)
+        put("tables", plan["block_tables"], np.int32)
+        put("lens", plan["context_lens"], np.int32)
+        put("order", schedule_order(plan["context_lens"], self.order_policy), np.int32)
+        put("cow", plan["cow_pairs"], np.int32)
+        main = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(self.side):
+            if self.done_ev[k] is not None:  # the device buffer is reused after its readers ran
+                self.side.wait_event(self.done_ev[k])
+            self.d_buf[k][:nbytes].copy_(self.h_buf[k][:nbytes], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(self.side)
+            self.copy_ev[k] = ev
+        main.wait_event(ev)
+
+        def dview(name, dtype):
+            off, n = lay[name]
+            return self.d_buf[k][off:off + n * (8 if dtype == torch.int64 else 4)].view(dtype)
+
         max_ctx = int(plan["context_lens"].max()) if b else 0
         if c:
-            block_copy(self.pool, self.d_cow, c, stream)
+            block_copy(self.pool, dview("cow", torch.int32), c, main)
         if t:
-            paged_kv_write(self.pool, layer, k_new, v_new, self.q_dtype, self.d_slots, t, k_inv, v_inv,
-                           stream)
+            paged_kv_write(self.pool, layer, k_new, v_new, self.q_dtype, dview("slots", torch.int64), t,
+                           k_inv, v_inv, main)
         if b:
             need = paged_attention_workspace_bytes(self.pool, b, self.hq, max_ctx)
             if need > self.ws_cap:
                 raise RuntimeError("decode workspace too small")
-            paged_attention_decode(self.pool, layer, q, self.q_dtype, self.hq, self.d_tables,
-                                   self.max_blocks, self.d_lens, b, max_ctx, self.scale, out,
-                                   KV_F32 if out_dtype is None else out_dtype, self.d_ws, need, stream,
-                                   seq_order=self.d_order)
+            paged_attention_decode(self.pool, layer, q, self.q_dtype, self.hq, dview("tables", torch.int32),
+                                   w, dview("lens", torch.int32), b, max_ctx, self.scale, out,
+                                   KV_F32 if out_dtype is None else out_dtype, self.d_ws, need, main,
+                                   seq_order=dview("order", torch.int32))
+        done = torch.cuda.Event()
+        done.record(main)
+        self.done_ev[k] = done
         return max_ctx

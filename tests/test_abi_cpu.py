@@ -63,9 +63,9 @@ def test_pool_bytes_and_workspace_sizes():
     pool = pk.kv_pool_create(16, 100, 8, 128, pk.KV_BF16, 2)
     kvb, sb = pk.kv_pool_bytes(pool)
     assert kvb == 100 * 8 * 16 * 128 * 2 and sb == 0
-    # automatic policy: partitions of at most 2048 tokens ...
-    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 2048) == 0
-    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 4096) == 512 * 64 * 2 * 132 * 4
+    # automatic policy: partitions of at most 4096 tokens ...
+    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 4096) == 0
+    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 8192) == 512 * 64 * 2 * 132 * 4
     # ... and more, down to 512 tokens, when there are few (sequence, kv head) units
     assert pk.paged_attention_workspace_bytes(pool, 4, 64, 1024) == 4 * 64 * 2 * 132 * 4
     assert pk.paged_attention_workspace_bytes(pool, 4, 64, 512) == 0
