@@ -81,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_paged_decode.argtypes = dec + [c_p]
         L.oracle_paged_decode_partials.restype = c_i
         L.oracle_paged_decode_partials.argtypes = dec + [c_i, c_i, c_p, c_p, c_p]
+        L.oracle_paged_prefill.restype = c_i
+        L.oracle_paged_prefill.argtypes = [c_p, c_p, c_i, c_p, c_p, c_i, c_i, c_i, c_i, c_p, c_i, c_i,
+                                           c_p, c_p, c_i, c_p, c_i, c_d, c_i, c_p]
         L.oracle_lse_merge.restype = None
         L.oracle_lse_merge.argtypes = [c_i64, c_i, c_i, c_p, c_p, c_p, c_p]
         _lib = L
@@ -147,6 +150,38 @@ def paged_decode(k_pool, v_pool, kv_fmt, q, q_fmt, block_tables, context_lens,
                                    _ptr(cl), b, float(scale), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_paged_decode failed: {rc}")
+    return out
+
+
+def paged_prefill(k_pool, v_pool, kv_fmt, q, q_fmt, cu_q, block_tables, context_lens,
+                  scale, block_size, k_scale=None, v_scale=None, window=0):
+    """fp64 multi-token (causal) attention over a paged pool.
+
+    Sequence s has its last ``cu_q[s+1] - cu_q[s]`` cached tokens as new
+    query tokens; new token i sits at position p = n - q_len + i and attends
+    to positions max(0, p - window + 1) .. p (0 .. p when ``window`` is 0).
+    q: raw storage [cu_q[-1]][num_q_heads][head_dim]; returns float64 of the
+    same shape.  Raises ValueError on a bad block id or q_len > context.
+    """
+    k_pool = _c(k_pool, STORAGE[kv_fmt])
+    v_pool = _c(v_pool, STORAGE[kv_fmt])
+    q = _c(q, STORAGE[q_fmt])
+    cu = _c(cu_q, np.int32)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    ks = _c(k_scale, np.float32)
+    vs = _c(v_scale, np.float32)
+    nb, hkv, bs, d = k_pool.shape
+    assert bs == block_size
+    rows, hq, d2 = q.shape
+    b = cl.shape[0]
+    assert d2 == d and hq % hkv == 0 and cu.shape[0] == b + 1 and int(cu[-1]) == rows
+    out = np.zeros((rows, hq, d), dtype=np.float64)
+    rc = lib().oracle_paged_prefill(_ptr(k_pool), _ptr(v_pool), kv_fmt, _ptr(ks), _ptr(vs), nb, hkv,
+                                    bs, d, _ptr(q), q_fmt, hq, _ptr(cu), _ptr(bt), bt.shape[1],
+                                    _ptr(cl), b, float(scale), int(window), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_prefill failed: {rc}")
     return out
 
 

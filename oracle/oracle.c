@@ -352,3 +352,92 @@ void oracle_lse_merge(int64_t rows, int num_parts, int head_dim, const double* o
     for (int d = 0; d < head_dim; ++d) o[d] /= l;
   }
 }
+
+/* ------------------------------------------------ multi-token attention */
+
+/* Query element d of head h in packed row `row` of a [rows][num_q_heads]
+ * [head_dim] array (multi-token layout: one row per new token). */
+static double qrow_val(const oracle_decode_args* a, int64_t row, int h, int d) {
+  int64_t idx = (row * a->num_q_heads + h) * a->head_dim + d;
+  if (a->q_dtype == OR_F16) return oracle_f16_to_double(((const uint16_t*)a->q)[idx]);
+  if (a->q_dtype == OR_BF16) return oracle_bf16_to_double(((const uint16_t*)a->q)[idx]);
+  return (double)((const float*)a->q)[idx];
+}
+
+/* Multi-token attention over the paged cache: the step that processes a
+ * prompt (or a chunk of one, or several drafted tokens) before decoding
+ * continues ([PA] plus the time-to-first-token discussion of the same page's
+ * "连续批处理" section; the pages describe no kernel for it).  Reading taken:
+ * sequence s holds n = context_lens[s] tokens in the cache, the last
+ * q_len = cu_q[s+1] - cu_q[s] of which are its new tokens (already written);
+ * new token i sits at position p = n - q_len + i and attends to the cached
+ * positions t with lo <= t <= p (causal), where lo = 0 without a window and
+ * lo = max(0, p - window + 1) with a sliding window of `window` tokens (the
+ * long-context remedy named in the pitfalls section).  q and out are
+ * [cu_q[batch]][num_q_heads][head_dim]; row cu_q[s] + i belongs to token i
+ * of s.  Returns 0, -1 (bad block id), -2 (OOM), -3 (q_len > n, q_len < 0,
+ * or a negative window). */
+static int prefill_one(const oracle_decode_args* a, const int32_t* cu_q, int window, int s,
+                       int h, double* out) {
+  int D = a->head_dim;
+  int g = a->num_q_heads / a->kv_heads;
+  int n = a->context_lens[s];
+  int q_len = cu_q[s + 1] - cu_q[s];
+  if (q_len < 0 || q_len > n || window < 0) return -3;
+  if (q_len == 0) return 0;
+  double* K = (double*)malloc(sizeof(double) * (size_t)n * D);
+  double* V = (double*)malloc(sizeof(double) * (size_t)n * D);
+  double* z = (double*)malloc(sizeof(double) * (size_t)n);
+  int rc = 0;
+  if (!K || !V || !z) { rc = -2; goto done; }
+  if (gather(a, a->k_pool, a->k_scale, s, h / g, n, K) ||
+      gather(a, a->v_pool, a->v_scale, s, h / g, n, V)) {
+    rc = -1;
+    goto done;
+  }
+  for (int i = 0; i < q_len; ++i) {
+    int64_t row = (int64_t)cu_q[s] + i;
+    int p = n - q_len + i;
+    int lo = (window > 0 && p - window + 1 > 0) ? p - window + 1 : 0;
+    double* o = out + (row * a->num_q_heads + h) * D;
+    double m = -INFINITY;
+    for (int t = lo; t <= p; ++t) {
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) acc += qrow_val(a, row, h, d) * K[(int64_t)t * D + d];
+      z[t] = a->scale * acc;
+      if (z[t] > m) m = z[t];
+    }
+    double l = 0.0;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int t = lo; t <= p; ++t) {
+      double w = exp(z[t] - m);
+      l += w;
+      for (int d = 0; d < D; ++d) o[d] += w * V[(int64_t)t * D + d];
+    }
+    for (int d = 0; d < D; ++d) o[d] /= l;
+  }
+done:
+  free(K);
+  free(V);
+  free(z);
+  return rc;
+}
+
+int oracle_paged_prefill(const void* k_pool, const void* v_pool, int kv_dtype,
+                         const float* k_scale, const float* v_scale, int num_blocks,
+                         int kv_heads, int block_size, int head_dim, const void* q, int q_dtype,
+                         int num_q_heads, const int32_t* cu_q, const int32_t* block_tables,
+                         int max_blocks, const int32_t* context_lens, int batch, double scale,
+                         int window, double* out) {
+  oracle_decode_args a = {k_pool, v_pool, kv_dtype, k_scale, v_scale, num_blocks, kv_heads,
+                          block_size, head_dim, q, q_dtype, num_q_heads, block_tables,
+                          max_blocks, context_lens, batch, scale};
+  int rc = 0;
+  int64_t pairs = (int64_t)batch * num_q_heads;
+#pragma omp parallel for schedule(dynamic, 1) reduction(min : rc)
+  for (int64_t i = 0; i < pairs; ++i) {
+    int r = prefill_one(&a, cu_q, window, (int)(i / num_q_heads), (int)(i % num_q_heads), out);
+    if (r < rc) rc = r;
+  }
+  return rc;
+}
