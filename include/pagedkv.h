@@ -201,6 +201,41 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
                            void* workspace, size_t workspace_bytes, const int32_t* seq_order,
                            kv_stream_t stream);
 
+/* Multi-token attention over the paged cache: the step that processes a
+ * prompt, a chunk of one, or a few drafted tokens before decoding continues
+ * ([PA], and the time-to-first-token discussion of the page's section
+ * "连续批处理：别再等最慢的那个请求了"; the pages give no kernel for it).
+ * Sequence s has n = context_lens[s] tokens in the cache, the last
+ * q_len = cu_seqlens_q[s+1] - cu_seqlens_q[s] of which are its new tokens,
+ * already written (paged_kv_write); new token i sits at position
+ * n - q_len + i and attends causally to positions 0 .. n - q_len + i:
+ *     out[r][h] = sum_{t <= pos} softmax_t(scale * q[r][h] . K_t) V_t,
+ * r = cu_seqlens_q[s] + i, kv head h / (num_q_heads / kv_heads).  q_len = 1
+ * is a decode step; q_len = n a whole prompt.  Runs on the tensor cores
+ * (tcgen05) with fp32 accumulation and softmax.
+ *   pool          f16 or bf16, head_dim 64 or 128 (others: KV_ERR_ARG).
+ *   q             device [total_q][num_q_heads][head_dim] of the pool dtype,
+ *                 16-byte aligned.
+ *   cu_seqlens_q  device int32 [batch + 1], non-decreasing from 0;
+ *                 total_q = cu_seqlens_q[batch] (host copy of it).
+ *   max_q_len     host upper bound on every q_len; it sizes the launch.
+ *   block_tables  device int32 [batch][max_blocks_per_seq].
+ *   context_lens  device int32 [batch].  A sequence with q_len < 0,
+ *                 q_len > n, q_len > max_q_len, rows past total_q, or
+ *                 n > max_blocks_per_seq * block_size is skipped and
+ *                 reported as KV_ERR_BOUNDS by kv_get_device_error, as is a
+ *                 block id outside the pool (that CTA stops).
+ *   scale         finite and > 0.
+ *   out           device [total_q][num_q_heads][head_dim] of out_dtype (the
+ *                 pool dtype or KV_F32), 16-byte aligned.
+ * batch, total_q or max_q_len == 0 enqueues nothing.  No workspace.  Errors:
+ * KV_ERR_ARG, KV_ERR_STATE (layer not bound), KV_ERR_CUDA. */
+int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
+                            int num_q_heads, const int32_t* cu_seqlens_q, int total_q,
+                            int max_q_len, const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int batch, float scale, void* out,
+                            kv_dtype out_dtype, kv_stream_t stream);
+
 /* Largest scratch paged_attention_decode_noalloc can use (16 MiB). */
 #define KV_NOALLOC_WORKSPACE_BYTES (16u << 20)
 

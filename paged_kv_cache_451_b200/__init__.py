@@ -71,6 +71,9 @@ _SIGS = {
     "paged_attention_decode_noalloc": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p,
                                                c_int, c_void_p, c_int, c_int, c_float, c_void_p,
                                                c_int, c_void_p]),
+    "paged_attention_prefill": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int,
+                                        c_int, c_void_p, c_int, c_void_p, c_int, c_float, c_void_p,
+                                        c_int, c_void_p]),
     "kv_selftest_wait_timeout": (c_int, [ctypes.c_uint64, c_void_p]),
     "kv_get_device_error": (c_int, [c_void_p, P(c_int)]),
     "kv_alloc_create": (c_int, [c_int, c_int, c_void_p, P(c_void_p)]),
@@ -194,6 +197,15 @@ def paged_attention_decode(pool, layer, q, q_dtype, num_q_heads, block_tables, m
                                        batch, max_context_len, float(scale), _ptr(out), out_dtype,
                                        _ptr(workspace), int(workspace_bytes), _ptr(seq_order),
                                        _stream(stream)))
+
+
+def paged_attention_prefill(pool, layer, q, q_dtype, num_q_heads, cu_seqlens_q, total_q, max_q_len,
+                            block_tables, max_blocks_per_seq, context_lens, batch, scale, out,
+                            out_dtype, stream=None):
+    _check(_lib.paged_attention_prefill(pool, layer, _ptr(q), q_dtype, num_q_heads,
+                                        _ptr(cu_seqlens_q), int(total_q), int(max_q_len),
+                                        _ptr(block_tables), max_blocks_per_seq, _ptr(context_lens),
+                                        batch, float(scale), _ptr(out), out_dtype, _stream(stream)))
 
 
 KV_NOALLOC_WORKSPACE_BYTES = 16 << 20

@@ -11,7 +11,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpagedkv.so")
-SOURCES = [os.path.join(CSRC, "pagedkv.cu"), os.path.join(CSRC, "alloc.cpp")]
+SOURCES = [os.path.join(CSRC, "pagedkv.cu"), os.path.join(CSRC, "prefill.cu"),
+           os.path.join(CSRC, "alloc.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [
     os.path.join(ROOT, "include", "pagedkv.h")]
 

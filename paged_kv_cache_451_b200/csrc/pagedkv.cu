@@ -284,6 +284,22 @@ int out_kind(kv_dtype t) { return t == KV_F32 ? OUT_F32 : (t == KV_BF16 ? OUT_BF
 
 using namespace pagedkv;
 
+namespace pagedkv {
+
+// Device address of the error word, for kernels built in the library's other
+// translation units (they record into the same word).
+int* device_error_word() {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return static_cast<int*>(p);
+}
+
+}  // namespace pagedkv
+
 extern "C" {
 
 int kv_pool_create(int block_size, int num_blocks, int kv_heads, int head_dim, kv_dtype dtype,

@@ -1,0 +1,476 @@
+// Multi-token attention over the paged cache for sm_100a: the prompt (or a
+// chunk of it, or a few drafted tokens) attends causally to everything the
+// sequence has cached, its own new tokens included.
+//
+// Method: "vLLM 推理加速原理详解：大模型服务吞吐量为何能提升 10 倍", section
+// "PagedAttention：把操作系统的虚拟内存搬进 GPU" (K/V in fixed-size blocks
+// reached through a per-sequence block table) and section
+// "连续批处理：别再等最慢的那个请求了" (prompts are processed before decoding
+// continues; time to first token).  The pages give no kernel for this step.
+// Reading taken: new token i of a sequence with n cached tokens, q_len of
+// them new, sits at position n - q_len + i and attends to positions 0 .. that
+// position.
+//
+// Unlike decode, this is a real dense contraction, so it runs on the
+// fifth-generation tensor cores.  One CTA per (query tile, kv head,
+// sequence); a query tile is 128 rows = 128 / g new tokens x the g query
+// heads of one kv head's group, so each K/V tile read serves the whole group.
+// Per 128-key tile j, with S and O accumulated in tensor memory (TMEM):
+//   S_j = Q . K_j^T          (tcgen05.mma, M 128, N 128, K = head_dim; Q and
+//                            K_j in shared memory, 128-byte swizzled, K-major)
+//   softmax rows in fp32 (one row per thread of warps 0-3, log2 domain, a
+//   lazily moved reference max, causal mask on the diagonal tiles); the
+//   probabilities P_j go back into S_j's TMEM columns as 16-bit values (bf16:
+//   value + rounding residual, about 16 significant bits together)
+//   O += P_j . V_j           (tcgen05.mma with A = P_j from TMEM, B = V_j from
+//                            shared memory, MN-major; bf16: once per half)
+// Warp 4 streams Q and the K/V tiles with 3-D TMA copies straight out of the
+// paged pool (one 16-row box per 16 keys and 64 columns, placed so the tile
+// lands in the canonical swizzled layout the MMA reads); warp 5 issues the
+// MMAs from one thread in the order S_0, S_1, PV_0, S_2, PV_1, ... so the
+// softmax of tile j+1 overlaps P_j . V_j and S_{j+2}.  Completion flows
+// through mbarriers (TMA transaction counts, tcgen05.commit, thread arrives);
+// every wait is bounded and aborts the CTA with KV_ERR_TIMEOUT.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "../../include/pagedkv.h"
+#include "ptx.cuh"
+#include "tcgen05.cuh"
+
+namespace pagedkv {
+
+constexpr int kPfRows = 128;       // query rows per CTA (M of the MMA)
+constexpr int kPfKeys = 128;       // keys per tile (N of Q.K^T, K of P.V)
+constexpr int kPfThreads = 192;    // warps 0-3 softmax, 4 copies, 5 MMA
+constexpr uint32_t kPfTmemCols = 512;  // S double buffer (2 x 128) + O (<= 128)
+constexpr uint64_t kPfWaitNs = 2000000000ull;
+constexpr uint64_t kPfDrainNs = 50000000ull;  // copies and MMAs in flight finish in microseconds
+// reference max moves only when a tile's max exceeds it by more than this
+// many binades: probabilities stay <= 2^8, exact enough in 16 bits + residual
+constexpr float kPfLazyLog2 = 8.f;
+
+enum PrefillOutKind { PF_OUT_F16 = 0, PF_OUT_BF16 = 1, PF_OUT_F32 = 3 };
+
+struct PrefillParams {
+  const int32_t* cu_q;          // [batch + 1] first query row of each sequence
+  const int32_t* block_tables;  // [batch][max_blocks]
+  const int32_t* context_lens;  // [batch] cached tokens, the new ones included
+  void* out;                    // [total_q][num_q_heads][D]
+  int* err;                     // device error word
+  int out_kind;
+  int num_q_heads;
+  int group;                    // query heads per kv head, <= 8
+  int tokens_per_tile;          // 128 / group
+  int num_q_tiles;              // grid x
+  int kv_heads;
+  int block_size;
+  int num_blocks;
+  int max_blocks;
+  int total_q;
+  float scale_log2;             // softmax scale * log2(e), > 0
+};
+
+template <int D, int STAGES>
+struct PrefillShape {
+  static constexpr int NH = D / 64;            // 128-byte column blocks per row
+  static constexpr int HALF = kPfRows * 128;   // one column block of a 128-row tile
+  static constexpr int TILE = NH * HALF;       // a Q, K or V tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + TILE;
+  static constexpr int V_OFF = K_OFF + STAGES * TILE;
+  static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
+  // q, K full/empty and V full/empty per stage, S full, P full, P.V done per
+  // S buffer, and the final MMA drain
+  static constexpr int NBAR = 1 + 4 * STAGES + 6 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // TMEM base, abort flag
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+  static_assert(kPfRows == kPfKeys, "Q, K and V tiles share one byte size");
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+};
+
+namespace pf {
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tensor cores).
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Wait for the phase with `parity`; give up when another role of the CTA
+// has aborted, or after kPfWaitNs (then abort the CTA and record a timeout).
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                     int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kPfWaitNs) {
+      *abort_flag = 1;
+      atomicCAS(err, 0, KV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+}  // namespace pf
+
+template <bool kBf16, int D, int STAGES>
+__global__ void __launch_bounds__(kPfThreads, 1)
+paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap qmap,
+                     const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap) {
+  using S = PrefillShape<D, STAGES>;
+  constexpr int NH = S::NH;
+  constexpr bool kSplit = kBf16;  // bf16 probabilities carry their residual
+  constexpr int KCH = kPfKeys / 16;  // 16-key boxes per tile
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
+  uint8_t* smem = smem_raw + (sbase - raw);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = p.num_q_tiles - 1 - (int)blockIdx.x;  // tiles with the most keys start first
+  const int kvh = blockIdx.y, s = blockIdx.z;
+  const int g = p.group, tq = p.tokens_per_tile;
+
+  const int q0 = p.cu_q[s];
+  const int q_len = p.cu_q[s + 1] - q0;
+  const int n = p.context_lens[s];
+  if (q0 < 0 || q_len < 0 || q_len > n || (int64_t)q0 + q_len > p.total_q ||
+      (int64_t)n > (int64_t)p.max_blocks * p.block_size || q_len > p.num_q_tiles * tq) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) atomicCAS(p.err, 0, KV_ERR_BOUNDS);
+    return;
+  }
+  const int t0 = qt * tq;  // first new token of this tile
+  if (t0 >= q_len) return;
+  const int ntok = min(tq, q_len - t0);
+  const int p0 = n - q_len + t0;   // its position in the sequence
+  const int kend = p0 + ntok;      // keys 0 .. kend - 1 are read
+  const int ntiles = (kend + kPfKeys - 1) / kPfKeys;
+  const int qrows = tq * g;
+
+  const uint32_t bar0 = sbase + S::BAR_OFF;
+  const uint32_t BQ = bar0;
+  auto KF = [&](int i) { return bar0 + 8u * (1 + i); };
+  auto KE = [&](int i) { return bar0 + 8u * (1 + STAGES + i); };
+  auto VF = [&](int i) { return bar0 + 8u * (1 + 2 * STAGES + i); };
+  auto VE = [&](int i) { return bar0 + 8u * (1 + 3 * STAGES + i); };
+  auto SF = [&](int b) { return bar0 + 8u * (1 + 4 * STAGES + b); };
+  auto PF = [&](int b) { return bar0 + 8u * (3 + 4 * STAGES + b); };
+  auto PV = [&](int b) { return bar0 + 8u * (5 + 4 * STAGES + b); };
+  const uint32_t FIN = bar0 + 8u * (7 + 4 * STAGES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::MISC_OFF + 8);
+
+  if (threadIdx.x == 0) {
+    mbar_init(BQ, 1);
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(KF(i), 1);
+      mbar_init(KE(i), 1);
+      mbar_init(VF(i), 1);
+      mbar_init(VE(i), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(SF(b), 1);
+      mbar_init(PF(b), kPfRows);
+      mbar_init(PV(b), 1);
+    }
+    mbar_init(FIN, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  // Query rows past tokens_per_tile * group are not covered by the copy
+  if (threadIdx.x >= qrows && threadIdx.x < kPfRows) {
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      uint4* row = reinterpret_cast<uint4*>(smem + S::Q_OFF + h * S::HALF + threadIdx.x * 128);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) row[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    pf::fence_proxy_async();
+  }
+  if (warp == 4) {
+    __syncwarp();
+    tc::alloc(smem_u32(tmem_slot), kPfTmemCols);
+    tc::relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ copies
+    if (lane == 0) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+      mbar_arrive_expect_tx(BQ, (uint32_t)(NH * qrows * 128));
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+        tma_load_3d(sbase + S::Q_OFF + h * S::HALF, &qmap, BQ, h * 64, kvh * g, q0 + t0);
+      const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks;
+      int nk = 0, nv = 0;  // tiles whose K (V) copies are in flight or done
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = j % STAGES;
+        const uint32_t use = (uint32_t)(j / STAGES);
+        const int key0 = j * kPfKeys;
+        const int nch = min(KCH, (kend - key0 + 15) / 16);
+        int blk[KCH], row[KCH];
+        bool bad = false;
+#pragma unroll
+        for (int c = 0; c < KCH; ++c) {
+          blk[c] = 0;
+          row[c] = 0;
+          if (c < nch) {
+            const int key = key0 + 16 * c;
+            const int b = table[key / p.block_size];
+            bad |= b < 0 || b >= p.num_blocks;
+            blk[c] = b;
+            row[c] = kvh * p.block_size + key % p.block_size;
+          }
+        }
+        if (bad) {
+          atomicCAS(p.err, 0, KV_ERR_BOUNDS);
+          *abort_flag = 1;
+          break;
+        }
+        const uint32_t bytes = (uint32_t)(nch * NH * 16 * 128);
+        if (use > 0 && !pf::wait(KE(st), (use - 1) & 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(KF(st), bytes);
+        for (int c = 0; c < nch; ++c)
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            tma_load_3d(sbase + S::K_OFF + st * S::TILE + h * S::HALF + c * 2048, &kmap, KF(st),
+                        h * 64, row[c], blk[c]);
+        nk = j + 1;
+        if (use > 0 && !pf::wait(VE(st), (use - 1) & 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(VF(st), bytes);
+        for (int c = 0; c < nch; ++c)
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            tma_load_3d(sbase + S::V_OFF + st * S::TILE + h * S::HALF + c * 2048, &vmap, VF(st),
+                        h * 64, row[c], blk[c]);
+        nv = j + 1;
+      }
+      if (*abort_flag) {
+        // let the copies in flight land before the shared memory is released
+        for (int j = max(0, nk - STAGES); j < nk; ++j)
+          (void)mbar_wait_bounded(KF(j % STAGES), (j / STAGES) & 1, kPfDrainNs);
+        for (int j = max(0, nv - STAGES); j < nv; ++j)
+          (void)mbar_wait_bounded(VF(j % STAGES), (j / STAGES) & 1, kPfDrainNs);
+        (void)mbar_wait_bounded(BQ, 0, kPfDrainNs);
+      }
+    }
+  } else if (warp == 5) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t kIdS = tc::idesc_f16(kBf16, kPfRows, kPfKeys, false);
+      constexpr uint32_t kIdO = tc::idesc_f16(kBf16, kPfRows, D, true);
+      const uint32_t dO = tmem + 2 * kPfKeys;
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % STAGES;
+        if (!pf::wait(KF(st), (j / STAGES) & 1, abort_flag, p.err)) return false;
+        tc::fence_after();
+        const uint32_t dS = tmem + (uint32_t)(j & 1) * kPfKeys;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * S::HALF + (kk % 4) * 32;  // 16 columns per step
+          tc::mma_ss(dS, tc::desc_sw128(sbase + S::Q_OFF + off, 16, 1024),
+                     tc::desc_sw128(sbase + S::K_OFF + st * S::TILE + off, 16, 1024), kIdS,
+                     kk > 0 ? 1u : 0u);
+        }
+        tc::commit(KE(st));
+        tc::commit(SF(j & 1));
+        return true;
+      };
+      bool ok = pf::wait(BQ, 0, abort_flag, p.err);
+      tc::fence_after();
+      if (ok) ok = issue_s(0);
+      if (ok && ntiles > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int b = j & 1, st = j % STAGES;
+        if (!pf::wait(PF(b), (j >> 1) & 1, abort_flag, p.err)) break;
+        if (!pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err)) break;
+        tc::fence_after();
+        const uint32_t aP = tmem + (uint32_t)b * kPfKeys;
+#pragma unroll
+        for (int kk = 0; kk < KCH; ++kk) {  // 16 keys per step: 8 TMEM columns of P
+          const uint64_t bV =
+              tc::desc_sw128(sbase + S::V_OFF + st * S::TILE + kk * 2048, S::HALF, 1024);
+          tc::mma_ts(dO, aP + 8 * kk, bV, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
+          if constexpr (kSplit) tc::mma_ts(dO, aP + 64 + 8 * kk, bV, kIdO, 1u);
+        }
+        tc::commit(VE(st));
+        tc::commit(PV(b));
+        if (j + 2 < ntiles && !issue_s(j + 2)) break;
+      }
+      // every MMA issued must finish before TMEM is released
+      tc::commit(FIN);
+      (void)mbar_wait_bounded(FIN, 0, kPfDrainNs);
+    }
+  } else {
+    // ------------------------------------------- softmax: one row a thread
+    const int r = threadIdx.x;
+    const int tok = r / g, head = r - tok * g;
+    const bool valid = r < qrows && tok < ntok;
+    const int prow = valid ? p0 + tok : kend - 1;  // last key this row sees
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const uint32_t tO = tmem + lane_addr + 2 * kPfKeys;
+    const float sl2 = p.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int b = j & 1;
+      ok = __all_sync(0xffffffffu, pf::wait(SF(b), (j >> 1) & 1, abort_flag, p.err));
+      if (!ok) break;
+      tc::fence_after();
+      const uint32_t tS = tmem + lane_addr + (uint32_t)b * kPfKeys;
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::ld32(tS + 32 * c, sr[c]);
+      tc::wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::pin(sr[c]);
+      const int lim = prow - j * kPfKeys;  // columns 0 .. lim are visible
+      if (lim < kPfKeys - 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i > lim) sr[c][i] = __float_as_uint(-INFINITY);
+      }
+      float mx8[8];  // eight independent chains, then a tree
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx8[i % 8] = fmaxf(mx8[i % 8], __uint_as_float(sr[c][i]));
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + w]);
+      const float mt = mx8[0] * sl2;
+      const bool grow = mt > m_ref + kPfLazyLog2;
+      const float m_new = grow ? mt : m_ref;
+      const float alpha = grow ? ex2(m_ref - m_new) : 1.f;
+      __syncwarp();
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O holds P.V up to tile j - 1: wait for it, then rescale in TMEM
+        ok = __all_sync(0xffffffffu,
+                        pf::wait(PV((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.err));
+        if (!ok) break;
+        tc::fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tc::ld32(tO + 32 * c, o);
+          tc::wait_ld();
+          tc::pin(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tc::st32(tO + 32 * c, o);
+        }
+      }
+      m_ref = m_new;
+      float ls[4] = {l * alpha, 0.f, 0.f, 0.f};  // independent partial sums
+      // P_j over S_j's columns: 16-bit pairs, keys 2c and 2c + 1 in column c
+      // (bf16: values in columns 0-63, residuals in 64-127)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = ex2(fmaf(__uint_as_float(sr[c][2 * i]), sl2, -m_ref));
+          const float e = ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, -m_ref));
+          ls[i % 4] += a + e;
+          if constexpr (kSplit) {
+            split2<true>(a, e, hi[i], lo[i]);
+          } else {
+            hi[i] = pack2<false>(a, e);
+            lo[i] = 0u;
+          }
+        }
+        tc::st16(tS + 16 * c, hi);
+        if constexpr (kSplit) tc::st16(tS + 64 + 16 * c, lo);
+      }
+      l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      tc::wait_st();
+      if (j == ntiles - 1 && kend - j * kPfKeys < kPfKeys) {
+        // last tile: zero the V rows past the keys read (stale slots may hold
+        // any bits, and 0 * NaN is NaN)
+        const int st = j % STAGES;
+        ok = __all_sync(0xffffffffu, pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err));
+        if (!ok) break;
+        if (r >= kend - j * kPfKeys) {
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            uint4* row = reinterpret_cast<uint4*>(smem + S::V_OFF + st * S::TILE + h * S::HALF + r * 128);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) row[i] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        pf::fence_proxy_async();
+        __syncwarp();
+      }
+      tc::fence_before();
+      mbar_arrive(PF(b));
+    }
+    if (ok) {
+      const int jl = ntiles - 1;
+      ok = __all_sync(0xffffffffu, pf::wait(PV(jl & 1), (jl >> 1) & 1, abort_flag, p.err));
+    }
+    if (ok) {
+      tc::fence_after();
+      const float inv = 1.f / l;
+      const int64_t orow = ((int64_t)(q0 + t0 + tok) * p.num_q_heads + kvh * g + head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tc::ld32(tO + 32 * c, o);
+        tc::wait_ld();
+        tc::pin(o);
+        if (valid) {
+          if (p.out_kind == PF_OUT_F32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                   __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dst[i] = make_uint4(
+                  pack2<kBf16>(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
+                  pack2<kBf16>(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
+                  pack2<kBf16>(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
+                  pack2<kBf16>(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  // TMEM is released once every role is done with it
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    __syncwarp();
+    tc::fence_after();
+    tc::dealloc(tmem, kPfTmemCols);
+  }
+}
+
+}  // namespace pagedkv

@@ -95,6 +95,14 @@ def test_gpu_entries_reject_bad_arguments_before_launch():
         pk.paged_attention_decode(pool, 3, 16, pk.KV_F16, 2, 16, 1, 16, 1, 16, 0.1, 16, pk.KV_F16, stream=0)
     assert e.value.code == pk.KV_ERR_ARG
     with pytest.raises(pk.KVError) as e:
+        pk.paged_attention_prefill(pool, 0, 16, pk.KV_F16, 2, 16, 4, 4, 16, 1, 16, 1, 0.1, 16,
+                                   pk.KV_F16, stream=0)
+    assert e.value.code == pk.KV_ERR_STATE
+    with pytest.raises(pk.KVError) as e:
+        pk.paged_attention_prefill(pool, -1, 16, pk.KV_F16, 2, 16, 4, 4, 16, 1, 16, 1, 0.1, 16,
+                                   pk.KV_F16, stream=0)
+    assert e.value.code == pk.KV_ERR_ARG
+    with pytest.raises(pk.KVError) as e:
         pk.block_copy(pool, 16, -1, stream=0)
     assert e.value.code == pk.KV_ERR_ARG
     with pytest.raises(pk.KVError):
