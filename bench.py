@@ -35,6 +35,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention: achieved KV-read GB/s (% of HBM peak); decode seqs/s"
+METRIC_PREFILL = "paged multi-token attention: achieved TFLOP/s (% of tensor peak); new tokens/s"
+PREFILL_WORKLOADS = ("prefill_llama13b", "prefill_gqa", "chunked_gqa")
+FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {0: "f16", 1: "bf16", 2: "e4m3"}
 ELEM = {0: 2, 1: 2, 2: 1}
@@ -49,6 +52,15 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:  # noqa: BLE001
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def decode_source_hash():
@@ -517,6 +529,249 @@ def run_e2e(case, torch, pk, flush, stream, K, W):
             "ms_per_step": round(ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+# ------------------------------------------------------ multi-token leg
+
+class PrefillCase:
+    """Device-resident inputs of a multi-token workload: a pool with every
+    sequence's cached prefix, the new tokens' K/V and slots, their queries."""
+
+    def __init__(self, name, rank, torch, pk):
+        from workloads import (WORKLOADS, device_normal_bits, device_pool, pool_blocks,
+                               prefill_lens, scattered_tables)
+        w = WORKLOADS[name]
+        self.w, self.torch, self.pk = w, torch, pk
+        self.prior, self.new = prefill_lens(w)
+        self.lens = (self.prior + self.new).astype(np.int32)
+        self.nb = pool_blocks(w, self.lens)
+        rng = np.random.default_rng([w.seed, 1000 + rank])
+        self.tables = scattered_tables(rng, self.lens, w.block_size, self.nb)
+        dev = torch.device("cuda")
+        seed = w.seed * 7919 + rank
+        self.L = 1
+        self.pool = pk.kv_pool_create(w.block_size, self.nb, w.kv_heads, w.head_dim, w.kv_fmt, 1)
+        k, v, _, _ = device_pool(w, self.nb, dev, seed=seed)
+        self.k, self.v = [k], [v]
+        pk.kv_pool_bind(self.pool, 0, k, v, None, None)
+        T, Hq, Hkv, D = int(self.new.sum()), w.num_q_heads, w.kv_heads, w.head_dim
+        self.T = T
+        self.cu_h = np.concatenate([[0], np.cumsum(self.new)]).astype(np.int32)
+        self.q = device_normal_bits((T, Hq, D), w.q_fmt, dev, seed + 1)
+        self.kn = device_normal_bits((T, Hkv, D), w.q_fmt, dev, seed + 2)
+        self.vn = device_normal_bits((T, Hkv, D), w.q_fmt, dev, seed + 3)
+        pos = np.concatenate([np.arange(p, p + n) for p, n in zip(self.prior, self.new)]).astype(np.int64)
+        seq = np.repeat(np.arange(w.batch), self.new)
+        self.slots_h = self.tables[seq, pos // w.block_size].astype(np.int64) * w.block_size + pos % w.block_size
+        self.slots = torch.from_numpy(self.slots_h).to(dev)
+        self.cu = torch.from_numpy(self.cu_h).to(dev)
+        self.tables_d = torch.from_numpy(self.tables).to(dev)
+        self.lens_d = torch.from_numpy(self.lens).to(dev)
+        self.max_q = int(self.new.max())
+        out_dt = torch.float16 if w.q_fmt == 0 else torch.bfloat16
+        self.out = torch.empty((T, Hq, D), dtype=out_dt, device=dev)
+        # algorithmic work: new token i of s sees prior_s + i + 1 keys; q.K and P.V
+        visible = sum(int(p) * int(n) + int(n) * (int(n) + 1) // 2 for p, n in zip(self.prior, self.new))
+        self.flops = 4.0 * D * Hq * visible
+        e = ELEM[w.q_fmt]
+        self.write_bytes = T * Hkv * D * 2 * (e + ELEM[w.kv_fmt])
+
+    def write(self, kn=None, vn=None, slots=None):
+        self.pk.paged_kv_write(self.pool, 0, self.kn if kn is None else kn, self.vn if vn is None else vn,
+                               self.w.q_fmt, self.slots if slots is None else slots, self.T, None, None)
+
+    def prefill(self, q=None, cu=None, tables=None, lens=None, out=None):
+        w = self.w
+        self.pk.paged_attention_prefill(self.pool, 0, self.q if q is None else q, w.q_fmt, w.num_q_heads,
+                                        self.cu if cu is None else cu, self.T, self.max_q,
+                                        self.tables_d if tables is None else tables, self.tables.shape[1],
+                                        self.lens_d if lens is None else lens, w.batch, w.scale,
+                                        self.out if out is None else out, w.q_fmt)
+
+
+def describe_prefill(w, case=None):
+    names = {
+        "prefill_llama13b": "whole prompts, Llama-2-13B-shaped layer: 40 MHA heads, head_dim 128, fp16, "
+                            "block 16, 16 prompts of U[64,2048] tokens",
+        "prefill_gqa": "whole prompts, GQA 64/8 heads, head_dim 128, bf16, block 16, 16 prompts of U[64,2048] tokens",
+        "chunked_gqa": "prompt chunks, GQA 64/8 heads, head_dim 128, bf16, block 16, 16 sequences x 512 new "
+                       "tokens on U[512,4096] cached",
+    }
+    s = names[w.name]
+    if case is not None:
+        s += f"; {case.T} new tokens; pool {case.nb} blocks"
+    return s
+
+
+def run_prefill(args, rank, world, local_rank):
+    import torch
+    import paged_kv_cache_451_b200 as pk
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    case = PrefillCase(args.workload, rank, torch, pk)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev_w=None, ev_p=None):
+        case.write()
+        if ev_w is not None:
+            ev_w.record(stream)
+        case.prefill()
+        if ev_p is not None:
+            ev_p.record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error during warm-up")
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    evw = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    evp = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev0[i].record(stream)
+            step(evw[i], evp[i])
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    step_ms = [ev0[i].elapsed_time(evp[i]) for i in range(K)]
+    pf_ms = [evw[i].elapsed_time(evp[i]) for i in range(K)]
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
+    ms_per_step = total_ms / K
+    pf_avg = sum(pf_ms) / K
+    e2e = run_e2e_prefill(case, torch, flush, stream, K, args.warmup)
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error during timing")
+    peak, peak_kind = tensor_peak()
+    value = world * case.flops / (ms_per_step * 1e-3) / 1e12
+    achieved = case.flops / (pf_avg * 1e-3) / 1e12
+    w = case.w
+    line = {
+        "metric": METRIC_PREFILL,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": DTYPE_NAME[w.kv_fmt],
+        "data": "synthetic (seeded N(0,1) q/K/V drawn on device; seeded lengths and scattered block placement)",
+        "config": {
+            "workload": describe_prefill(w, case),
+            "global_batch": w.batch * world,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed between steps (256 MiB write)",
+        },
+        "new_tokens_per_s": round(world * case.T / (ms_per_step * 1e-3), 1),
+        "pct_of_tensor_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "paged_attention_prefill",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None,
+            "algorithmic_flops_per_launch": case.flops,
+            "launch_ms": round(pf_avg, 5),
+            "peak_note": f"{peak_kind} dense bf16 GEMM (cuBLAS, burst); f16 runs at the same rate",
+        },
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": 2 * K,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(case, target_s=args.cpu_seconds)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def run_e2e_prefill(case, torch, flush, stream, K, W):
+    """The same step from pinned host memory: H2D of q, new K/V, slots,
+    cu_seqlens, tables and lengths, write + attention, D2H of the output."""
+    hs = [t.cpu().pin_memory() for t in (case.q, case.kn, case.vn, case.slots, case.cu, case.tables_d,
+                                         case.lens_d)]
+    ds = [torch.empty_like(t) for t in (case.q, case.kn, case.vn, case.slots, case.cu, case.tables_d,
+                                        case.lens_d)]
+    hout = torch.empty(case.out.shape, dtype=case.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hs)
+    d2h = hout.numel() * hout.element_size()
+
+    def step():
+        for d, h in zip(ds, hs):
+            d.copy_(h, non_blocking=True)
+        q, kn, vn, slots, cu, tables, lens = ds
+        case.write(kn, vn, slots)
+        case.prefill(q, cu, tables, lens)
+        hout.copy_(case.out, non_blocking=True)
+
+    for _ in range(W):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        a[i].record(stream)
+        step()
+        b[i].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a[i].elapsed_time(b[i]) for i in range(K)) / K
+    return {"value": round(case.flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def cpu_baseline_prefill(case, target_s=15.0):
+    """The oracle, as it stands, on a bounded sample: the shortest sequences
+    first until about target_s of CPU work."""
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    w, bs = case.w, case.w.block_size
+    kh_all = case.k[0]
+    order = np.argsort(case.lens, kind="stable")
+    total_s, flops, tokens, done = 0.0, 0.0, 0, 0
+    qh = case.q.cpu().numpy().view(np.uint16)
+    for s in order:
+        s = int(s)
+        nblk = -(-int(case.lens[s]) // bs)
+        idx = case.torch.tensor(case.tables[s, :nblk].astype(np.int64), device=kh_all.device)
+        kh = case.k[0].index_select(0, idx).cpu().numpy().view(np.uint16)
+        vh = case.v[0].index_select(0, idx).cpu().numpy().view(np.uint16)
+        table = np.arange(nblk, dtype=np.int32)[None, :]
+        rows = slice(int(case.cu_h[s]), int(case.cu_h[s + 1]))
+        cu = np.array([0, int(case.new[s])], np.int32)
+        t0 = time.perf_counter()
+        oracle.paged_prefill(kh, vh, w.kv_fmt, qh[rows], w.q_fmt, cu, table, case.lens[s:s + 1], w.scale, bs)
+        total_s += time.perf_counter() - t0
+        p, n = int(case.prior[s]), int(case.new[s])
+        flops += 4.0 * w.head_dim * w.num_q_heads * (p * n + n * (n + 1) // 2)
+        tokens += n
+        done += 1
+        if total_s >= target_s:
+            break
+    return {"value": round(flops / total_s / 1e12, 6), "unit": "TFLOP/s",
+            "new_tokens_per_s": round(tokens / total_s, 2), "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {w.batch} sequences (shortest first), attention only, fp64 C oracle "
+                      f"(OpenMP over (sequence, head)); {total_s:.1f} s"}
+
+
 # ---------------------------------------------------------- CPU oracle legs
 
 def oracle_sample(case_like, seqs, layer=0):
@@ -585,6 +840,8 @@ def run_reference(args, rank, world):
         return None
     torch.cuda.set_device(0)
     import paged_kv_cache_451_b200 as pk
+    if args.workload in PREFILL_WORKLOADS:
+        return run_reference_prefill(args, world, torch, pk)
     case = Case(args.workload, 0, torch, pk, args)
     per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -612,6 +869,33 @@ def run_reference(args, rank, world):
     }
 
 
+def run_reference_prefill(args, world, torch, pk):
+    case = PrefillCase(args.workload, 0, torch, pk)
+    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline_prefill(case, target_s=per_step)
+    res = cpu_baseline_prefill(case, target_s=per_step * args.steps)
+    return {
+        "impl": "reference",
+        "metric": METRIC_PREFILL,
+        "value": res["value"],
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": None,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": describe_prefill(case.w, case), "global_batch": case.w.batch},
+        "new_tokens_per_s": res["new_tokens_per_s"],
+        "cpu_baseline": res,
+        "e2e": {"value": res["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -619,7 +903,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama13b",
-                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long"])
+                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long", *PREFILL_WORKLOADS])
     ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")
     ap.add_argument("--warps", type=int, default=0, help="warps per decode CTA (0: auto)")
@@ -638,6 +922,8 @@ def main():
         line = run_reference(args, rank, world)
     elif args.workload == "gqa_trace":
         line = run_trace(args, rank, world, local_rank)
+    elif args.workload in PREFILL_WORKLOADS:
+        line = run_prefill(args, rank, world, local_rank)
     else:
         line = run_ours(args, rank, world, local_rank)
     if rank == 0 and line is not None:

@@ -22,6 +22,12 @@ Workloads (sizes from the configurations the library is measured on):
                 sequences sharing a 1024-token prefix, 100-iteration trace.
 * ``fp8_long``  32 MHA heads, head_dim 128, batch 8, context 16384, E4M3 cache
                 with one fp32 scale per (block, kv head), bf16 queries.
+* ``prefill_llama13b`` / ``prefill_gqa``  multi-token attention over whole
+                prompts: 16 prompts of lengths uniform in [64, 2048] (the
+                trace's arrival range), Llama-2-13B layer shape (fp16) or the
+                64/8 GQA shape (bf16).
+* ``chunked_gqa`` 16 sequences, each a 512-token prompt chunk on top of a
+                cached prefix of 512..4096 tokens, 64/8 GQA, bf16.
 
 Values of q, K and V are ~N(0, 1).  Seeds are 451 + the workload's index.
 """
@@ -75,7 +81,28 @@ WORKLOADS = {
                                  "pool_factor": 1.25}),
     "fp8_long": Workload("fp8_long", 4, 1, 32, 32, 128, 16, E4M3, BF16, 8,
                          extra={"ctx": 16384, "pool_factor": 1.25}),
+    # multi-token attention (prompts and prompt chunks)
+    "prefill_llama13b": Workload("prefill_llama13b", 5, 1, 40, 40, 128, 16, F16, F16, 16,
+                                 extra={"new_lo": 64, "new_hi": 2048, "prior_lo": 0, "prior_hi": 0,
+                                        "pool_factor": 1.25}),
+    "prefill_gqa": Workload("prefill_gqa", 6, 1, 64, 8, 128, 16, BF16, BF16, 16,
+                            extra={"new_lo": 64, "new_hi": 2048, "prior_lo": 0, "prior_hi": 0,
+                                   "pool_factor": 1.25}),
+    "chunked_gqa": Workload("chunked_gqa", 7, 1, 64, 8, 128, 16, BF16, BF16, 16,
+                            extra={"new_lo": 512, "new_hi": 512, "prior_lo": 512, "prior_hi": 4096,
+                                   "pool_factor": 1.25}),
 }
+
+
+def prefill_lens(w: Workload):
+    """(cached-before lengths, new-token counts) of a multi-token workload:
+    new tokens uniform in [new_lo, new_hi] (the trace's prompt range for whole
+    prompts), on top of a cached prefix uniform in [prior_lo, prior_hi]."""
+    e = w.extra
+    r = rng_for(w, 3)
+    new = r.integers(e["new_lo"], e["new_hi"] + 1, size=w.batch).astype(np.int32)
+    prior = r.integers(e["prior_lo"], e["prior_hi"] + 1, size=w.batch).astype(np.int32)
+    return prior, new
 
 
 def rng_for(w: Workload, salt: int = 0) -> np.random.Generator:
@@ -98,6 +125,9 @@ def context_lens(w: Workload) -> np.ndarray:
     if w.name == "gqa_trace":
         x = r.lognormal(math.log(w.extra["median"]), w.extra["sigma"], size=w.batch)
         return np.clip(np.rint(x), 1, w.extra["cap"]).astype(np.int32)
+    if "new_lo" in w.extra:  # multi-token workloads: cached prefix + new tokens
+        prior, new = prefill_lens(w)
+        return prior + new
     raise KeyError(w.name)
 
 
