@@ -325,6 +325,52 @@ int kv_alloc_snapshot(const kv_alloc* a, int32_t* free_list, int* n_free, int32_
 int kv_alloc_counters(const kv_alloc* a, int64_t* allocated, int64_t* freed, int64_t* cow);
 int kv_alloc_destroy(kv_alloc* a);
 
+/* Prefix caching: requests that share a prompt prefix (a system prompt, a
+ * document) reuse its KV blocks instead of recomputing them ("vLLM 推理加速
+ * 原理详解", automatic prefix caching among the deployment settings and the
+ * RAG throughput claim; the pages do not describe the lookup).  Reading
+ * taken: only full blocks are cached; block i of a sequence is keyed by
+ * FNV-1a-64 over (key of block i-1 as 8 little-endian bytes, then the block's
+ * token ids as 4 little-endian bytes each), block -1's key being the FNV
+ * offset basis 14695981039346656037; a hit also compares the stored parent
+ * key and token ids, so a hash collision never shares a block.  Freed blocks
+ * keep their key until the free list hands them out again (FIFO; a freed
+ * sequence's blocks are appended deepest first), which evicts the key.
+ * Host only, all O(block_size) per block.
+ *
+ * kv_alloc_enable_prefix_caching: switch caching on; only before any
+ * sequence exists (else KV_ERR_STATE). */
+int kv_alloc_enable_prefix_caching(kv_alloc* a);
+
+/* Allocate a prompt of num_tokens token ids for seq_id: the longest run of
+ * registered blocks matching the prompt from its first block is shared
+ * (refcount + 1; a hit on a free block leaves the free list), at most
+ * (num_tokens - 1) / block_size blocks so that the last prompt token is
+ * always computed; the remaining blocks are taken fresh.  Writes the number
+ * of cached tokens (hit blocks x block_size): the caller writes and attends
+ * only tokens from there on.  The prompt's tokens are remembered for
+ * kv_alloc_commit.  Without caching enabled nothing is shared.  Errors:
+ * KV_ERR_ARG, KV_ERR_STATE (sequence exists), KV_ERR_OOM (nothing changes). */
+int kv_alloc_allocate_prompt(kv_alloc* a, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                             int* num_cached_tokens);
+
+/* kv_alloc_append_slot for a token whose id is known; the id is remembered
+ * while the sequence's known tokens are contiguous from position 0. */
+int kv_alloc_append_token(kv_alloc* a, int64_t seq_id, int32_t token, int64_t* slot,
+                          int32_t* cow_src, int32_t* cow_dst);
+
+/* Register (make findable) every full block of seq_id whose tokens are all
+ * known and not registered yet; call once their KV has been written (or is
+ * ordered before every later reader on the stream).  A block whose key is
+ * already registered to another block stays unregistered.  num_registered
+ * may be NULL. */
+int kv_alloc_commit(kv_alloc* a, int64_t seq_id, int* num_registered);
+
+/* Cumulative hit blocks and evictions, and the number of registered blocks
+ * (each pointer may be NULL). */
+int kv_alloc_prefix_stats(const kv_alloc* a, int64_t* hit_blocks, int64_t* evictions,
+                          int* cached_blocks);
+
 /* --------------------------------------------------------- scheduling step */
 
 /* Continuous-batching scheduler over an allocator ([CB]).  max_num_seqs caps
@@ -336,6 +382,16 @@ int kv_alloc_destroy(kv_alloc* a);
 int kv_sched_create(kv_alloc* a, int max_num_seqs, int min_blocks, kv_sched** out);
 /* Queue a request (FIFO) whose prompt has prompt_len tokens. */
 int kv_sched_add_request(kv_sched* s, int64_t seq_id, int prompt_len);
+
+/* A waiting request with its prompt token ids.  When the allocator has
+ * prefix caching enabled, admission counts only the blocks the request takes
+ * out of the free list (fresh ones plus free cached hits), allocates it with
+ * kv_alloc_allocate_prompt, registers its full prompt blocks at once (the
+ * step's cache write is ordered before any attention of the step), and the
+ * step's slot_mapping holds only its uncached prompt tokens;
+ * kv_sched_admitted_cached gives the cached token counts. */
+int kv_sched_add_request_tokens(kv_sched* s, int64_t seq_id, const int32_t* tokens,
+                                int num_tokens);
 /* Put a sequence that already holds blocks (e.g. a fork) in the running set. */
 int kv_sched_adopt(kv_sched* s, int64_t seq_id);
 
@@ -367,6 +423,10 @@ int kv_sched_outputs(const kv_sched* s, int64_t* running_ids, int32_t* block_tab
                      int32_t* cow_pairs, int64_t* admitted_ids);
 /* [MON]: running and waiting request counts, used and total blocks
  * (cache usage = used / total). */
+/* Cached prompt tokens of each request admitted by the last step, in the
+ * order of admitted_ids (0 without prefix caching). */
+int kv_sched_admitted_cached(const kv_sched* s, int32_t* cached_tokens);
+
 int kv_sched_stats(const kv_sched* s, int* running, int* waiting, int* used_blocks,
                    int* total_blocks);
 int kv_sched_destroy(kv_sched* s);

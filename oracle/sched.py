@@ -167,7 +167,12 @@ class Scheduler:
         self.running: list[int] = []
 
     def add_request(self, seq_id: int, prompt_len: int) -> None:
-        self.waiting.append((seq_id, prompt_len))
+        self.waiting.append((seq_id, prompt_len, None))
+
+    def add_request_tokens(self, seq_id: int, tokens) -> None:
+        """A request whose prompt token ids are known (prefix caching)."""
+        tokens = [int(t) for t in tokens]
+        self.waiting.append((seq_id, len(tokens), tokens))
 
     def adopt(self, seq_id: int) -> None:
         """Put a sequence that already holds blocks (e.g. a fork) in the running set."""
@@ -191,21 +196,35 @@ class Scheduler:
         free_blocks = self.bm.get_num_free_blocks()
         # (3) admit waiting requests, first come first served
         admitted = []
+        cached = []
         prompt_slots = []
+        caching = isinstance(self.bm, PrefixCachingBlockManager)
         while (self.waiting and free_blocks > self._min_blocks()
                and len(self.running) < self.max_num_seqs):
-            sid, plen = self.waiting[0]
+            sid, plen, toks = self.waiting[0]
             reserve = self._min_blocks() + (1 if self.min_blocks is None else 0)
-            if not (self.bm.can_allocate(plen)
-                    and blocks_for(plen, self.bm.block_size) + reserve <= free_blocks):
+            use_cache = caching and toks is not None
+            need = self.bm.admission_cost(toks) if use_cache else blocks_for(plen, self.bm.block_size)
+            if not (need <= free_blocks and need + reserve <= free_blocks):
                 break
+            if sid in self.bm.tables:
+                raise OracleStateError(f"sequence {sid} already exists")
             self.waiting.popleft()
-            self.bm.allocate(sid, plen)
+            if use_cache:
+                hit = self.bm.allocate_prompt(sid, toks)
+                # the step's cache write runs before any attention of the step,
+                # so blocks registered now are written before a later admission
+                # of this step reads them
+                self.bm.commit(sid)
+            else:
+                self.bm.allocate(sid, plen)
+                hit = 0
             self.running.append(sid)
             admitted.append(sid)
+            cached.append(hit)
             table = self.bm.tables[sid]
             bs = self.bm.block_size
-            prompt_slots.extend(table[t // bs] * bs + t % bs for t in range(plen))
+            prompt_slots.extend(table[t // bs] * bs + t % bs for t in range(hit, plen))
             free_blocks = self.bm.get_num_free_blocks()
         # (4) one new token slot per running sequence, then decode
         decode_slots, cow = [], []
@@ -221,8 +240,178 @@ class Scheduler:
             "slot_mapping": prompt_slots + decode_slots,
             "cow_pairs": cow,
             "admitted": admitted,
+            "cached": cached,
         }
 
     def stats(self):
         used = self.bm.num_blocks - self.bm.get_num_free_blocks()
         return len(self.running), len(self.waiting), used, self.bm.num_blocks
+
+
+# ------------------------------------------------------------ prefix caching
+#
+# "vLLM 推理加速原理详解" mentions automatic prefix caching (requests that
+# share a system prompt reuse its KV blocks; the pitfalls section and the
+# deployment flags) without describing the lookup.  Reading taken here (each
+# item also listed in the design doc):
+#
+# * only FULL blocks are cached; block i of a sequence is keyed by
+#   key_i = FNV-1a-64(key_{i-1} as 8 little-endian bytes, then the block's
+#   token ids as 4 little-endian bytes each), key_{-1} = the FNV offset basis
+#   (the FNV-1a definition: for each byte, h ^= byte, h *= 1099511628211 mod
+#   2^64, starting from 14695981039346656037);
+# * a hit requires the stored parent key and token ids to equal the lookup's
+#   (no sharing on a hash collision);
+# * at admission the longest run of hits from block 0 is shared (refcount + 1;
+#   a hit on a free block takes it out of the free list), capped so that at
+#   least the prompt's last token is computed; the rest is allocated fresh;
+# * a block is registered (becomes findable) when the caller commits its
+#   tokens, i.e. once its KV has been written; a block whose key is already
+#   registered to another block stays unregistered;
+# * freed blocks keep their key; the free list stays FIFO, but a sequence's
+#   blocks are appended deepest-first so that shared prefixes leave last;
+#   taking a free block that still holds a key evicts that key.
+
+FNV_OFFSET = 14695981039346656037
+FNV_PRIME = 1099511628211
+_MASK64 = (1 << 64) - 1
+
+
+def fnv1a64(data: bytes, h: int = FNV_OFFSET) -> int:
+    for byte in data:
+        h ^= byte
+        h = (h * FNV_PRIME) & _MASK64
+    return h
+
+
+def block_key(parent: int, tokens) -> int:
+    data = int(parent).to_bytes(8, "little") + b"".join(
+        (int(t) & 0xFFFFFFFF).to_bytes(4, "little") for t in tokens)
+    return fnv1a64(data)
+
+
+class PrefixCachingBlockManager(BlockManager):
+    def __init__(self, num_blocks: int, block_size: int, initial_free_order=None):
+        super().__init__(num_blocks, block_size, initial_free_order)
+        self.cached: dict[int, int] = {}          # key -> block
+        self.key_of: dict[int, tuple] = {}        # block -> (key, parent key, tokens)
+        self.seq_tokens: dict[int, list[int]] = {}
+        self.registered: dict[int, int] = {}      # seq -> leading blocks registered or skipped
+        self.num_hits = 0
+        self.num_evictions = 0
+
+    def _take(self) -> int:
+        if not self.free_list:
+            raise OracleOOM("no free block")
+        b = self.free_list[0]
+        if b in self.key_of:
+            key = self.key_of.pop(b)[0]
+            if self.cached.get(key) == b:
+                del self.cached[key]
+            self.num_evictions += 1
+        return super()._take()
+
+    def _keys(self, tokens):
+        bs = self.block_size
+        keys, parent = [], FNV_OFFSET
+        for i in range(len(tokens) // bs):
+            blk = tuple(int(t) for t in tokens[i * bs:(i + 1) * bs])
+            k = block_key(parent, blk)
+            keys.append((k, parent, blk))
+            parent = k
+        return keys
+
+    def lookup(self, tokens):
+        """Blocks of the longest cached prefix of `tokens` (at most
+        (len - 1) // block_size of them)."""
+        cap = max(0, (len(tokens) - 1) // self.block_size)
+        hits = []
+        for k, parent, blk in self._keys(tokens)[:cap]:
+            b = self.cached.get(k)
+            if b is None or self.key_of.get(b) != (k, parent, blk):
+                break
+            hits.append(b)
+        return hits
+
+    def admission_cost(self, tokens) -> int:
+        """Free blocks an allocate_prompt of `tokens` takes out of the free list."""
+        hits = self.lookup(tokens)
+        fresh = blocks_for(len(tokens), self.block_size) - len(hits)
+        return fresh + sum(1 for b in hits if self.refcount[b] == 0)
+
+    def allocate_prompt(self, seq_id: int, tokens) -> int:
+        """Allocate a prompt, sharing its cached prefix; returns the number
+        of cached tokens (the caller computes only the rest)."""
+        if seq_id in self.tables:
+            raise OracleStateError(f"sequence {seq_id} already exists")
+        tokens = [int(t) for t in tokens]
+        if self.admission_cost(tokens) > len(self.free_list):
+            raise OracleOOM("not enough free blocks")
+        hits = self.lookup(tokens)
+        for b in hits:
+            if self.refcount[b] == 0:
+                self.free_list.remove(b)
+            self.refcount[b] += 1
+        self.num_hits += len(hits)
+        fresh = blocks_for(len(tokens), self.block_size) - len(hits)
+        self.tables[seq_id] = hits + [self._take() for _ in range(fresh)]
+        self.tokens[seq_id] = len(tokens)
+        self.seq_tokens[seq_id] = tokens
+        self.registered[seq_id] = len(hits)
+        return len(hits) * self.block_size
+
+    def allocate(self, seq_id: int, num_tokens: int) -> None:
+        super().allocate(seq_id, num_tokens)
+        self.seq_tokens[seq_id] = []
+        self.registered[seq_id] = 0
+
+    def fork(self, parent: int, child: int) -> None:
+        super().fork(parent, child)
+        self.seq_tokens[child] = list(self.seq_tokens.get(parent, []))
+        self.registered[child] = self.registered.get(parent, 0)
+
+    def append_token(self, seq_id: int, token: int):
+        """append_slot for a token whose id is known (recorded only while the
+        sequence's known tokens are contiguous from position 0)."""
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        toks = self.seq_tokens.setdefault(seq_id, [])
+        contiguous = len(toks) == self.tokens[seq_id]
+        out = self.append_slot(seq_id)
+        if contiguous:
+            toks.append(int(token))
+        return out
+
+    def commit(self, seq_id: int) -> int:
+        """Register every full block whose tokens are all known; returns how
+        many blocks became findable."""
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        toks = self.seq_tokens.get(seq_id, [])
+        keys = self._keys(toks[:self.tokens[seq_id]])
+        table = self.tables[seq_id]
+        done = self.registered.get(seq_id, 0)
+        new = 0
+        for i in range(done, len(keys)):
+            k, parent, blk = keys[i]
+            b = table[i]
+            if k not in self.cached and b not in self.key_of:
+                self.cached[k] = b
+                self.key_of[b] = (k, parent, blk)
+                new += 1
+        self.registered[seq_id] = max(done, len(keys))
+        return new
+
+    def free(self, seq_id: int) -> None:
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        for b in reversed(self.tables.pop(seq_id)):
+            if self.refcount[b] <= 0:
+                raise OracleStateError(f"block {b} freed twice")
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                self.free_list.append(b)
+                self.num_freed += 1
+        del self.tokens[seq_id]
+        self.seq_tokens.pop(seq_id, None)
+        self.registered.pop(seq_id, None)

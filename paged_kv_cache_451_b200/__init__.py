@@ -90,8 +90,16 @@ _SIGS = {
     "kv_alloc_snapshot": (c_int, [c_void_p, c_void_p, P(c_int), c_void_p]),
     "kv_alloc_counters": (c_int, [c_void_p, P(c_int64), P(c_int64), P(c_int64)]),
     "kv_alloc_destroy": (c_int, [c_void_p]),
+    "kv_alloc_enable_prefix_caching": (c_int, [c_void_p]),
+    "kv_alloc_allocate_prompt": (c_int, [c_void_p, c_int64, c_void_p, c_int, P(c_int)]),
+    "kv_alloc_append_token": (c_int, [c_void_p, c_int64, ctypes.c_int32, P(c_int64),
+                                      P(ctypes.c_int32), P(ctypes.c_int32)]),
+    "kv_alloc_commit": (c_int, [c_void_p, c_int64, P(c_int)]),
+    "kv_alloc_prefix_stats": (c_int, [c_void_p, P(c_int64), P(c_int64), P(c_int)]),
     "kv_sched_create": (c_int, [c_void_p, c_int, c_int, P(c_void_p)]),
     "kv_sched_add_request": (c_int, [c_void_p, c_int64, c_int]),
+    "kv_sched_add_request_tokens": (c_int, [c_void_p, c_int64, c_void_p, c_int]),
+    "kv_sched_admitted_cached": (c_int, [c_void_p, c_void_p]),
     "kv_sched_adopt": (c_int, [c_void_p, c_int64]),
     "kv_sched_step": (c_int, [c_void_p, c_void_p, c_int, P(kv_step_info)]),
     "kv_sched_outputs": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
@@ -311,6 +319,38 @@ def kv_alloc_destroy(a):
     _check(_lib.kv_alloc_destroy(a))
 
 
+def kv_alloc_enable_prefix_caching(a):
+    _check(_lib.kv_alloc_enable_prefix_caching(a))
+
+
+def kv_alloc_allocate_prompt(a, seq_id, tokens) -> int:
+    import numpy as np
+    t = np.ascontiguousarray(tokens, np.int32)
+    n = c_int()
+    _check(_lib.kv_alloc_allocate_prompt(a, seq_id, _ptr(t) if t.size else None, int(t.size),
+                                         ctypes.byref(n)))
+    return n.value
+
+
+def kv_alloc_append_token(a, seq_id, token):
+    slot, cs, cd = c_int64(), ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.kv_alloc_append_token(a, seq_id, int(token), ctypes.byref(slot), ctypes.byref(cs),
+                                      ctypes.byref(cd)))
+    return slot.value, cs.value, cd.value
+
+
+def kv_alloc_commit(a, seq_id) -> int:
+    n = c_int()
+    _check(_lib.kv_alloc_commit(a, seq_id, ctypes.byref(n)))
+    return n.value
+
+
+def kv_alloc_prefix_stats(a):
+    h, e, c = c_int64(), c_int64(), c_int()
+    _check(_lib.kv_alloc_prefix_stats(a, ctypes.byref(h), ctypes.byref(e), ctypes.byref(c)))
+    return h.value, e.value, c.value
+
+
 # -------------------------------------------------------------- scheduler
 
 def kv_sched_create(a, max_num_seqs, min_blocks=-1):
@@ -321,6 +361,12 @@ def kv_sched_create(a, max_num_seqs, min_blocks=-1):
 
 def kv_sched_add_request(s, seq_id, prompt_len):
     _check(_lib.kv_sched_add_request(s, seq_id, prompt_len))
+
+
+def kv_sched_add_request_tokens(s, seq_id, tokens):
+    import numpy as np
+    t = np.ascontiguousarray(tokens, np.int32)
+    _check(_lib.kv_sched_add_request_tokens(s, seq_id, _ptr(t) if t.size else None, int(t.size)))
 
 
 def kv_sched_adopt(s, seq_id):
@@ -351,6 +397,8 @@ def kv_sched_outputs(s, info, table_width=None):
     _check(_lib.kv_sched_outputs(s, _ptr(out["running"]), _ptr(out["block_tables"]), w,
                                  _ptr(out["context_lens"]), _ptr(out["slot_mapping"]),
                                  _ptr(out["cow_pairs"]), _ptr(out["admitted"])))
+    out["cached"] = np.empty(info.num_admitted, np.int32)
+    _check(_lib.kv_sched_admitted_cached(s, _ptr(out["cached"])))
     return out
 
 

@@ -17,6 +17,7 @@
 // is admitted only if its prompt blocks fit with that reserve (counting the
 // request) left free, so the appends of the step cannot run out.
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <deque>
@@ -59,21 +60,88 @@ using pagedkv::ok;
 struct SeqState {
   std::vector<int32_t> blocks;
   int64_t tokens = 0;
+  std::vector<int32_t> toks;  // known token ids (prefix caching)
+  int64_t registered = 0;     // leading blocks registered or skipped
+};
+
+// Prefix-caching key of one full block: FNV-1a (64-bit) over the parent
+// key's 8 little-endian bytes, then the block's token ids as 4 little-endian
+// bytes each (the FNV-1a definition: per byte, h ^= byte; h *= 1099511628211
+// mod 2^64; from 14695981039346656037).
+constexpr uint64_t kFnvOffset = 14695981039346656037ull;
+constexpr uint64_t kFnvPrime = 1099511628211ull;
+
+inline uint64_t fnv_bytes(uint64_t h, uint64_t v, int nbytes) {
+  for (int i = 0; i < nbytes; ++i) {
+    h ^= (v >> (8 * i)) & 0xffu;
+    h *= kFnvPrime;
+  }
+  return h;
+}
+
+inline uint64_t block_key(uint64_t parent, const int32_t* tokens, int n) {
+  uint64_t h = fnv_bytes(kFnvOffset, parent, 8);
+  for (int i = 0; i < n; ++i) h = fnv_bytes(h, (uint32_t)tokens[i], 4);
+  return h;
+}
+
+struct CachedBlock {
+  bool valid = false;
+  uint64_t key = 0, parent = 0;
+  std::vector<int32_t> tokens;
 };
 
 struct kv_alloc {
   int num_blocks = 0;
   int block_size = 0;
-  std::deque<int32_t> free_list;
+  // FIFO free list as an intrusive doubly linked list (O(1) removal of a
+  // cached block that a prompt hits)
+  std::vector<int32_t> prev, next;
+  std::vector<char> is_free;
+  int32_t head = -1, tail = -1;
+  int64_t n_free = 0;
   std::vector<int32_t> refcount;
   std::unordered_map<int64_t, SeqState> seqs;
   int64_t n_alloc = 0, n_freed = 0, n_cow = 0;
+  // prefix caching
+  bool caching = false;
+  std::unordered_map<uint64_t, int32_t> cached;
+  std::vector<CachedBlock> key_of;
+  int64_t n_hits = 0, n_evict = 0;
 
   int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
 
+  void push_back(int32_t b) {
+    prev[b] = tail;
+    next[b] = -1;
+    if (tail >= 0) next[tail] = b; else head = b;
+    tail = b;
+    is_free[b] = 1;
+    ++n_free;
+  }
+
+  void unlink(int32_t b) {
+    if (prev[b] >= 0) next[prev[b]] = next[b]; else head = next[b];
+    if (next[b] >= 0) prev[next[b]] = prev[b]; else tail = prev[b];
+    prev[b] = next[b] = -1;
+    is_free[b] = 0;
+    --n_free;
+  }
+
+  void evict(int32_t b) {
+    CachedBlock& c = key_of[b];
+    if (!c.valid) return;
+    auto it = cached.find(c.key);
+    if (it != cached.end() && it->second == b) cached.erase(it);
+    c.valid = false;
+    c.tokens.clear();
+    ++n_evict;
+  }
+
   int32_t take() {
-    int32_t b = free_list.front();
-    free_list.pop_front();
+    int32_t b = head;
+    unlink(b);
+    if (caching) evict(b);
     refcount[b] = 1;
     ++n_alloc;
     return b;
@@ -81,7 +149,7 @@ struct kv_alloc {
 
   void release(int32_t b) {
     if (--refcount[b] == 0) {
-      free_list.push_back(b);
+      push_back(b);
       ++n_freed;
     }
   }
@@ -97,12 +165,12 @@ struct kv_alloc {
     *cs = -1;
     *cd = -1;
     if (pos % block_size == 0) {
-      if (free_list.empty()) return KV_ERR_OOM;
+      if (n_free == 0) return KV_ERR_OOM;
       s.blocks.push_back(take());
     } else {
       int32_t last = s.blocks.back();
       if (refcount[last] > 1) {
-        if (free_list.empty()) return KV_ERR_OOM;
+        if (n_free == 0) return KV_ERR_OOM;
         int32_t fresh = take();
         --refcount[last];
         s.blocks.back() = fresh;
@@ -114,6 +182,63 @@ struct kv_alloc {
     s.tokens = pos + 1;
     *slot = (int64_t)s.blocks[pos / block_size] * block_size + pos % block_size;
     return KV_OK;
+  }
+
+  // Blocks of the longest registered prefix of `tokens`, at most
+  // (n - 1) / block_size of them (the last prompt token is always computed).
+  void lookup(const int32_t* tokens, int n, std::vector<int32_t>* hits) const {
+    hits->clear();
+    if (!caching || n <= 0) return;
+    const int cap = (n - 1) / block_size;
+    uint64_t parent = kFnvOffset;
+    for (int i = 0; i < cap; ++i) {
+      const int32_t* t = tokens + (int64_t)i * block_size;
+      const uint64_t k = block_key(parent, t, block_size);
+      auto it = cached.find(k);
+      if (it == cached.end()) break;
+      const CachedBlock& c = key_of[it->second];
+      if (!c.valid || c.key != k || c.parent != parent ||
+          std::memcmp(c.tokens.data(), t, sizeof(int32_t) * block_size) != 0)
+        break;
+      hits->push_back(it->second);
+      parent = k;
+    }
+  }
+
+  // Free blocks an allocation of `tokens` removes from the free list.
+  int64_t admission_cost(const int32_t* tokens, int n, std::vector<int32_t>* hits) const {
+    lookup(tokens, n, hits);
+    int64_t cost = blocks_for(n) - (int64_t)hits->size();
+    for (int32_t b : *hits) cost += refcount[b] == 0 ? 1 : 0;
+    return cost;
+  }
+
+  // Register every full block of `s` whose tokens are all known.
+  int commit(SeqState& s) {
+    if (!caching) return 0;
+    const int64_t known = std::min<int64_t>((int64_t)s.toks.size(), s.tokens);
+    const int64_t full = known / block_size;
+    uint64_t parent = kFnvOffset;
+    int added = 0;
+    for (int64_t i = 0; i < full; ++i) {
+      const int32_t* t = s.toks.data() + i * block_size;
+      const uint64_t k = block_key(parent, t, block_size);
+      if (i >= s.registered) {
+        const int32_t b = s.blocks[i];
+        if (!cached.count(k) && !key_of[b].valid) {
+          CachedBlock& c = key_of[b];
+          c.valid = true;
+          c.key = k;
+          c.parent = parent;
+          c.tokens.assign(t, t + block_size);
+          cached.emplace(k, b);
+          ++added;
+        }
+      }
+      parent = k;
+    }
+    if (full > s.registered) s.registered = full;
+    return added;
   }
 };
 
@@ -133,6 +258,10 @@ int kv_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_
   a->num_blocks = num_blocks;
   a->block_size = block_size;
   a->refcount.assign(num_blocks, 0);
+  a->prev.assign(num_blocks, -1);
+  a->next.assign(num_blocks, -1);
+  a->is_free.assign(num_blocks, 0);
+  a->key_of.resize(num_blocks);
   if (initial_free_order) {
     std::vector<char> seen(num_blocks, 0);
     for (int i = 0; i < num_blocks; ++i) {
@@ -142,10 +271,10 @@ int kv_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_
         return fail(KV_ERR_ARG, "initial_free_order is not a permutation of 0..%d", num_blocks - 1);
       }
       seen[b] = 1;
-      a->free_list.push_back(b);
+      a->push_back(b);
     }
   } else {
-    for (int i = 0; i < num_blocks; ++i) a->free_list.push_back(i);
+    for (int i = 0; i < num_blocks; ++i) a->push_back(i);
   }
   *out = a;
   return ok();
@@ -158,13 +287,13 @@ int kv_alloc_destroy(kv_alloc* a) {
 
 int kv_alloc_num_free(const kv_alloc* a, int* n) {
   if (!a || !n) return fail(KV_ERR_ARG, "NULL argument");
-  *n = (int)a->free_list.size();
+  *n = (int)a->n_free;
   return ok();
 }
 
 int kv_alloc_can_allocate(const kv_alloc* a, int num_tokens, int* yes) {
   if (!a || !yes || num_tokens < 0) return fail(KV_ERR_ARG, "bad argument");
-  *yes = a->blocks_for(num_tokens) <= (int64_t)a->free_list.size();
+  *yes = a->blocks_for(num_tokens) <= a->n_free;
   return ok();
 }
 
@@ -172,8 +301,8 @@ int kv_alloc_allocate(kv_alloc* a, int64_t seq_id, int num_tokens) {
   if (!a || num_tokens < 0) return fail(KV_ERR_ARG, "bad argument");
   if (a->seqs.count(seq_id)) return fail(KV_ERR_STATE, "sequence %lld already exists", (long long)seq_id);
   int64_t need = a->blocks_for(num_tokens);
-  if (need > (int64_t)a->free_list.size())
-    return fail(KV_ERR_OOM, "need %lld blocks, %zu free", (long long)need, a->free_list.size());
+  if (need > a->n_free)
+    return fail(KV_ERR_OOM, "need %lld blocks, %lld free", (long long)need, (long long)a->n_free);
   SeqState s;
   s.blocks.reserve(need);
   for (int64_t i = 0; i < need; ++i) s.blocks.push_back(a->take());
@@ -207,7 +336,12 @@ int kv_alloc_free(kv_alloc* a, int64_t seq_id) {
   if (!a) return fail(KV_ERR_ARG, "NULL allocator");
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
-  for (int32_t b : it->second.blocks) a->release(b);
+  const auto& blocks = it->second.blocks;
+  if (a->caching) {  // deepest block first: shared prefixes leave the cache last
+    for (auto r = blocks.rbegin(); r != blocks.rend(); ++r) a->release(*r);
+  } else {
+    for (int32_t b : blocks) a->release(b);
+  }
   a->seqs.erase(it);
   return ok();
 }
@@ -238,12 +372,77 @@ int kv_alloc_refcount(const kv_alloc* a, int32_t block, int* rc) {
 
 int kv_alloc_snapshot(const kv_alloc* a, int32_t* free_list, int* n_free, int32_t* refcounts) {
   if (!a) return fail(KV_ERR_ARG, "NULL allocator");
-  if (n_free) *n_free = (int)a->free_list.size();
+  if (n_free) *n_free = (int)a->n_free;
   if (free_list) {
     int i = 0;
-    for (int32_t b : a->free_list) free_list[i++] = b;
+    for (int32_t b = a->head; b >= 0; b = a->next[b]) free_list[i++] = b;
   }
   if (refcounts) std::memcpy(refcounts, a->refcount.data(), sizeof(int32_t) * a->num_blocks);
+  return ok();
+}
+
+int kv_alloc_enable_prefix_caching(kv_alloc* a) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  if (!a->seqs.empty()) return fail(KV_ERR_STATE, "enable prefix caching before any sequence exists");
+  a->caching = true;
+  return ok();
+}
+
+int kv_alloc_allocate_prompt(kv_alloc* a, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                             int* num_cached_tokens) {
+  if (!a || num_tokens < 0 || (num_tokens > 0 && !tokens) || !num_cached_tokens)
+    return fail(KV_ERR_ARG, "bad argument");
+  if (a->seqs.count(seq_id)) return fail(KV_ERR_STATE, "sequence %lld already exists", (long long)seq_id);
+  std::vector<int32_t> hits;
+  const int64_t cost = a->admission_cost(tokens, num_tokens, &hits);
+  if (cost > a->n_free)
+    return fail(KV_ERR_OOM, "need %lld blocks, %lld free", (long long)cost, (long long)a->n_free);
+  SeqState s;
+  s.blocks.reserve(a->blocks_for(num_tokens));
+  for (int32_t b : hits) {
+    if (a->refcount[b] == 0) a->unlink(b);
+    ++a->refcount[b];
+    s.blocks.push_back(b);
+  }
+  a->n_hits += (int64_t)hits.size();
+  const int64_t fresh = a->blocks_for(num_tokens) - (int64_t)hits.size();
+  for (int64_t i = 0; i < fresh; ++i) s.blocks.push_back(a->take());
+  s.tokens = num_tokens;
+  s.toks.assign(tokens, tokens + num_tokens);
+  s.registered = (int64_t)hits.size();
+  a->seqs.emplace(seq_id, std::move(s));
+  *num_cached_tokens = (int)hits.size() * a->block_size;
+  return ok();
+}
+
+int kv_alloc_append_token(kv_alloc* a, int64_t seq_id, int32_t token, int64_t* slot,
+                          int32_t* cow_src, int32_t* cow_dst) {
+  if (!a || !slot || !cow_src || !cow_dst) return fail(KV_ERR_ARG, "NULL argument");
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  SeqState& st = it->second;
+  const bool contiguous = (int64_t)st.toks.size() == st.tokens;
+  int rc = a->append(st, slot, cow_src, cow_dst);
+  if (rc != KV_OK) return fail(rc, "no free block for sequence %lld", (long long)seq_id);
+  if (contiguous) st.toks.push_back(token);
+  return ok();
+}
+
+int kv_alloc_commit(kv_alloc* a, int64_t seq_id, int* num_registered) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  const int n = a->commit(it->second);
+  if (num_registered) *num_registered = n;
+  return ok();
+}
+
+int kv_alloc_prefix_stats(const kv_alloc* a, int64_t* hit_blocks, int64_t* evictions,
+                          int* cached_blocks) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  if (hit_blocks) *hit_blocks = a->n_hits;
+  if (evictions) *evictions = a->n_evict;
+  if (cached_blocks) *cached_blocks = (int)a->cached.size();
   return ok();
 }
 
@@ -262,6 +461,8 @@ int kv_alloc_counters(const kv_alloc* a, int64_t* allocated, int64_t* freed, int
 struct Request {
   int64_t id;
   int prompt_len;
+  bool has_tokens;
+  std::vector<int32_t> tokens;
 };
 
 struct kv_sched {
@@ -277,6 +478,7 @@ struct kv_sched {
   std::vector<int64_t> out_slots;
   std::vector<int32_t> out_cow;
   std::vector<int64_t> out_admitted;
+  std::vector<int32_t> out_cached;
 
   int min_blocks_now() const { return min_blocks < 0 ? (int)running.size() : min_blocks; }
 };
@@ -301,7 +503,13 @@ int kv_sched_destroy(kv_sched* s) {
 
 int kv_sched_add_request(kv_sched* s, int64_t seq_id, int prompt_len) {
   if (!s || prompt_len < 0) return fail(KV_ERR_ARG, "bad argument");
-  s->waiting.push_back({seq_id, prompt_len});
+  s->waiting.push_back({seq_id, prompt_len, false, {}});
+  return ok();
+}
+
+int kv_sched_add_request_tokens(kv_sched* s, int64_t seq_id, const int32_t* tokens, int num_tokens) {
+  if (!s || num_tokens < 0 || (num_tokens > 0 && !tokens)) return fail(KV_ERR_ARG, "bad argument");
+  s->waiting.push_back({seq_id, num_tokens, true, std::vector<int32_t>(tokens, tokens + num_tokens)});
   return ok();
 }
 
@@ -333,6 +541,7 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   s->out_slots.clear();
   s->out_cow.clear();
   s->out_admitted.clear();
+  s->out_cached.clear();
 
   // (1) drop finished requests, return their blocks
   std::vector<int64_t> keep;
@@ -343,25 +552,39 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   for (int i = 0; i < n_finished; ++i) kv_alloc_free(a, finished_ids[i]);
 
   // (2) free block count
-  int64_t free_blocks = (int64_t)a->free_list.size();
+  int64_t free_blocks = a->n_free;
 
   // (3) admit first come first served
   std::vector<int64_t> prompt_slots;
+  std::vector<int32_t> hits;
   while (!s->waiting.empty() && free_blocks > s->min_blocks_now() &&
          (int)s->running.size() < s->max_num_seqs) {
-    const Request req = s->waiting.front();
-    int64_t need = a->blocks_for(req.prompt_len);
-    int64_t reserve = s->min_blocks_now() + (s->min_blocks < 0 ? 1 : 0);
+    const Request& req = s->waiting.front();
+    const bool use_cache = a->caching && req.has_tokens;
+    const int64_t need = use_cache ? a->admission_cost(req.tokens.data(), req.prompt_len, &hits)
+                                   : a->blocks_for(req.prompt_len);
+    const int64_t reserve = s->min_blocks_now() + (s->min_blocks < 0 ? 1 : 0);
     if (need > free_blocks || need + reserve > free_blocks) break;
     if (a->seqs.count(req.id)) return fail(KV_ERR_STATE, "sequence %lld already exists", (long long)req.id);
+    const Request r = req;
     s->waiting.pop_front();
-    kv_alloc_allocate(a, req.id, req.prompt_len);
-    s->running.push_back(req.id);
-    s->out_admitted.push_back(req.id);
-    const SeqState& st = a->seqs[req.id];
-    for (int t = 0; t < req.prompt_len; ++t)
+    int hit = 0;
+    if (use_cache) {
+      // the step's cache write runs before any attention of the step, so a
+      // block registered now is written before a later admission reads it
+      kv_alloc_allocate_prompt(a, r.id, r.tokens.data(), r.prompt_len, &hit);
+      a->commit(a->seqs[r.id]);
+    } else {
+      kv_alloc_allocate(a, r.id, r.prompt_len);
+      if (r.has_tokens) a->seqs[r.id].toks = r.tokens;
+    }
+    s->running.push_back(r.id);
+    s->out_admitted.push_back(r.id);
+    s->out_cached.push_back(hit);
+    const SeqState& st = a->seqs[r.id];
+    for (int t = hit; t < r.prompt_len; ++t)
       prompt_slots.push_back((int64_t)st.blocks[t / a->block_size] * a->block_size + t % a->block_size);
-    free_blocks = (int64_t)a->free_list.size();
+    free_blocks = a->n_free;
   }
 
   // (4) one slot per running sequence; check the whole batch fits first
@@ -380,13 +603,13 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
       int64_t copies = a->refcount[kv.first] - 1;
       need += kv.second < copies ? kv.second : copies;
     }
-    if (need > (int64_t)a->free_list.size()) {
+    if (need > a->n_free) {
       info->batch = (int)s->running.size();
       info->num_tokens = info->num_cow = 0;
       info->num_admitted = (int)s->out_admitted.size();
       info->max_blocks = 0;
-      return fail(KV_ERR_OOM, "appends need %lld blocks, %zu free", (long long)need,
-                  a->free_list.size());
+      return fail(KV_ERR_OOM, "appends need %lld blocks, %lld free", (long long)need,
+                  (long long)a->n_free);
     }
   }
   s->out_slots = prompt_slots;
@@ -442,8 +665,15 @@ int kv_sched_stats(const kv_sched* s, int* running, int* waiting, int* used_bloc
   if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
   if (running) *running = (int)s->running.size();
   if (waiting) *waiting = (int)s->waiting.size();
-  if (used_blocks) *used_blocks = s->a->num_blocks - (int)s->a->free_list.size();
+  if (used_blocks) *used_blocks = s->a->num_blocks - (int)s->a->n_free;
   if (total_blocks) *total_blocks = s->a->num_blocks;
+  return ok();
+}
+
+int kv_sched_admitted_cached(const kv_sched* s, int32_t* cached_tokens) {
+  if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
+  if (cached_tokens)
+    for (size_t i = 0; i < s->out_cached.size(); ++i) cached_tokens[i] = s->out_cached[i];
   return ok();
 }
 
