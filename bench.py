@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode attention: achieved KV-read GB/s (% of HBM peak); decode seqs/s"
 METRIC_PREFILL = "paged multi-token attention: achieved TFLOP/s (% of tensor peak); new tokens/s"
 PREFILL_WORKLOADS = ("prefill_llama13b", "prefill_gqa", "chunked_gqa")
+METRIC_RAG = "retrieval-augmented serving with prefix caching: generated tokens/s (vs no caching)"
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {0: "f16", 1: "bf16", 2: "e4m3"}
@@ -464,6 +465,86 @@ def run_trace(args, rank, world, local_rank):
     }
 
 
+def run_rag(args, rank, world, local_rank):
+    """The retrieval-augmented trace, with and without prefix caching: one
+    step = one iteration (scheduler step, metadata upload, cache write,
+    prefill of the admitted prompts' uncached tokens, decode)."""
+    import torch
+    import paged_kv_cache_451_b200 as pk
+    from workloads import WORKLOADS
+    from workloads.rag_trace import RagTrace, rag_plan
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = WORKLOADS["rag_trace"]
+    plan = rag_plan(w)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    iters = w.extra["iters"]
+    W = min(args.warmup, iters - 1)
+    K = max(1, min(args.steps, iters - W))
+    res = {}
+    for caching in (True, False):
+        tr = RagTrace(w, plan, caching=caching, seed=rank)
+        for it in range(W):
+            tr.iteration(it)
+        torch.cuda.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        gen = prefilled = cached = admitted = 0
+        host_s = 0.0
+
+        def gate_and_start(i):
+            torch.cuda._sleep(2_000_000)  # keep the GPU fed while the host enqueues
+            starts[i].record(stream)
+
+        with ClockSampler(local_rank) as clk:
+            for i in range(K):
+                flush.zero_()
+                t0 = time.perf_counter()
+                fin, arr, pl, *_rest, P = tr.iteration(W + i, before_launch=lambda: gate_and_start(i),
+                                                       after_launch=lambda: ends[i].record(stream))
+                host_s += time.perf_counter() - t0
+                gen += pl["info"].batch
+                prefilled += P
+                cached += int(np.sum(pl["cached"]))
+                admitted += pl["info"].num_admitted
+            torch.cuda.synchronize()
+        if pk.kv_get_device_error() != pk.KV_OK:
+            raise RuntimeError("device error during the trace")
+        total_ms = max_over_ranks(sum(starts[i].elapsed_time(ends[i]) for i in range(K)), dist, "cuda")
+        hits, evictions, nblocks = pk.kv_alloc_prefix_stats(tr.alloc)
+        res[caching] = {"tokens_per_s": world * gen / (total_ms * 1e-3), "ms_per_step": total_ms / K,
+                        "generated": gen, "prefilled_tokens": prefilled, "cached_tokens": cached,
+                        "admitted": admitted, "host_ms_per_step": 1e3 * host_s / K, "clocks": clk.summary(),
+                        "hit_blocks": hits, "evictions": evictions}
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    on, off = res[True], res[False]
+    return {
+        "metric": METRIC_RAG, "value": round(on["tokens_per_s"], 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(on["ms_per_step"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded documents, questions and Poisson arrivals; q/K/V drawn on device)",
+        "config": {"workload": describe(w), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between iterations (256 MiB write)",
+                   "step": "one iteration: scheduler step (prefix lookup), metadata upload, cache write, "
+                           "prefill of uncached prompt tokens, decode of every running sequence"},
+        "no_caching": {"tokens_per_s": round(off["tokens_per_s"], 1), "ms_per_step": round(off["ms_per_step"], 5),
+                       "prefilled_tokens": off["prefilled_tokens"], "admitted": off["admitted"]},
+        "speedup_vs_no_caching": round(on["tokens_per_s"] / off["tokens_per_s"], 3),
+        "prefilled_tokens": on["prefilled_tokens"], "cached_tokens": on["cached_tokens"],
+        "admitted": on["admitted"], "hit_blocks": on["hit_blocks"], "evictions": on["evictions"],
+        "host_iteration_ms_per_step": round(on["host_ms_per_step"], 3),
+        "clocks": on["clocks"],
+    }
+
+
 def describe(w, case=None):
     names = {
         "tiny": "tiny: 1 layer, 4 seqs ctx {2,18,34,101}, 4 MHA heads, head_dim 64, block 16, fp16",
@@ -471,6 +552,9 @@ def describe(w, case=None):
         "kv_example": "KV-size example: 32 layers x 32 heads x head_dim 128, bf16, block 16, batch 32, ctx 2048",
         "gqa_trace": "GQA 64/8 heads, head_dim 128, bf16, block 16, batch 256, lognormal ctx (median 1024, cap 8192)",
         "fp8_long": "long-context FP8: 32 MHA heads, head_dim 128, E4M3 cache + per-(block,head) scales, bf16 q, batch 8, ctx 16384",
+        "rag_trace": "retrieval-augmented serving: GQA 64/8 heads, head_dim 128, bf16, block 16, 8192-block pool, "
+                     "Poisson arrivals (3/iteration) of 2 shared 1536-token documents + U[32,256]-token questions, "
+                     "U[16,64] output tokens, up to 128 running",
     }
     s = names[w.name]
     if case is not None:
@@ -903,7 +987,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama13b",
-                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long", *PREFILL_WORKLOADS])
+                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long", "rag_trace",
+                             *PREFILL_WORKLOADS])
     ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")
     ap.add_argument("--warps", type=int, default=0, help="warps per decode CTA (0: auto)")
@@ -924,6 +1009,8 @@ def main():
         line = run_trace(args, rank, world, local_rank)
     elif args.workload in PREFILL_WORKLOADS:
         line = run_prefill(args, rank, world, local_rank)
+    elif args.workload == "rag_trace":
+        line = run_rag(args, rank, world, local_rank)
     else:
         line = run_ours(args, rank, world, local_rank)
     if rank == 0 and line is not None:

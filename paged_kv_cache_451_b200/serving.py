@@ -10,9 +10,11 @@ the order of the scheduling loop on "vLLM æŽ¨ç†åŠ é€ŸåŽŸç†è¯¦è§£ï¼šå¤§æ¨¡åž‹æœ
 2. upload the step's metadata (block tables, context lengths, slots,
    scheduling order, copy pairs) with one async copy from a pinned buffer;
 3. ``block_copy`` for the copy-on-write pairs;
-4. ``paged_kv_write`` of the step's new tokens (admitted prompts, then one
-   token per running sequence);
-5. ``paged_attention_decode`` over the running set, with the scheduling
+4. ``paged_kv_write`` of the step's new tokens (admitted prompts' uncached
+   tokens, then one token per running sequence);
+5. optionally ``paged_attention_prefill`` over the admitted prompts' uncached
+   tokens (the prompt tokens a prefix-cache hit supplies are only read);
+6. ``paged_attention_decode`` over the running set, with the scheduling
    order of :func:`schedule_order` (it only affects how CTAs are placed on
    the GPU, not the outputs).
 """
@@ -22,7 +24,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import (KV_F32, block_copy, kv_sched_outputs, kv_sched_step, paged_attention_decode,
-               paged_attention_workspace_bytes, paged_kv_write)
+               paged_attention_prefill, paged_attention_workspace_bytes, paged_kv_write)
 
 
 def schedule_order(context_lens, policy="long_first"):
@@ -66,7 +68,7 @@ class DecodeLoop:
         self.q_dtype, self.scale = q_dtype, scale
         self.max_batch, self.max_blocks, self.max_tokens = max_batch, max_blocks, max_tokens
         self.order_policy = order_policy
-        cap = 8 * max_tokens + 4 * (max_batch * max_blocks + 4 * max_batch)
+        cap = 8 * max_tokens + 4 * (max_batch * max_blocks + 6 * max_batch + 1) + 256
         self.cap = (cap + 255) // 256 * 256
         self.h_buf = [torch.empty(self.cap, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.d_buf = [torch.empty(self.cap, dtype=torch.uint8, device=device) for _ in range(2)]
@@ -88,23 +90,38 @@ class DecodeLoop:
         return out
 
     @staticmethod
-    def _layout(b, t, c, width):
+    def _layout(b, t, c, width, a=0):
         off, lay = 0, {}
         for name, n, size in (("slots", t, 8), ("tables", b * width, 4), ("lens", b, 4),
-                              ("order", b, 4), ("cow", 2 * c, 4)):
+                              ("order", b, 4), ("cow", 2 * c, 4), ("cu", a + 1 if a else 0, 4),
+                              ("pf_lens", a, 4)):
             lay[name] = (off, n)
             off += (n * size + 15) // 16 * 16
         return lay, off
 
+    @staticmethod
+    def prefill_sizes(plan):
+        """(admitted count, new tokens per admitted prompt, cached tokens per
+        admitted prompt): admitted sequences are the last rows of the running
+        set, their prompt is their context minus this step's appended token."""
+        a = int(plan["info"].num_admitted)
+        if a == 0:
+            return 0, np.zeros(0, np.int64), np.zeros(0, np.int64)
+        plen = np.asarray(plan["context_lens"][-a:], np.int64) - 1
+        cached = np.asarray(plan.get("cached", np.zeros(a)), np.int64)
+        return a, plen - cached, cached
+
     def launch(self, plan, k_new, v_new, q, out, k_inv=None, v_inv=None, out_dtype=None,
-               layer=0, stream=None):
-        """Upload the plan's metadata and enqueue copy, write and decode."""
+               layer=0, stream=None, prefill_q=None, prefill_out=None):
+        """Upload the plan's metadata and enqueue copy, write, prefill of the
+        admitted prompts (when prefill_q is given) and decode."""
         torch = self.torch
         info = plan["info"]
         b, t, c, w = info.batch, info.num_tokens, info.num_cow, self.max_blocks
+        a, new, _ = self.prefill_sizes(plan) if prefill_q is not None else (0, None, None)
         k = self.it % 2
         self.it += 1
-        lay, nbytes = self._layout(b, t, c, w)
+        lay, nbytes = self._layout(b, t, c, w, a)
         if nbytes > self.cap:
             raise RuntimeError("step metadata exceeds the loop's buffers")
         if self.copy_ev[k] is not None:  # the pinned buffer is reused: its last upload must be done
@@ -121,6 +138,9 @@ class DecodeLoop:
         put("lens", plan["context_lens"], np.int32)
         put("order", schedule_order(plan["context_lens"], self.order_policy), np.int32)
         put("cow", plan["cow_pairs"], np.int32)
+        if a:
+            put("cu", np.concatenate([[0], np.cumsum(new)]), np.int32)
+            put("pf_lens", np.asarray(plan["context_lens"][-a:], np.int64) - 1, np.int32)
         main = torch.cuda.current_stream() if stream is None else stream
         with torch.cuda.stream(self.side):
             if self.done_ev[k] is not None:  # the device buffer is reused after its readers ran
@@ -141,6 +161,12 @@ class DecodeLoop:
         if t:
             paged_kv_write(self.pool, layer, k_new, v_new, self.q_dtype, dview("slots", torch.int64), t,
                            k_inv, v_inv, main)
+        if a and int(new.sum()) > 0:
+            tables = dview("tables", torch.int32).view(b, w)[b - a:]
+            paged_attention_prefill(self.pool, layer, prefill_q, self.q_dtype, self.hq, dview("cu", torch.int32),
+                                    int(new.sum()), int(new.max()), tables, w, dview("pf_lens", torch.int32),
+                                    a, self.scale, prefill_out, KV_F32 if out_dtype is None else out_dtype,
+                                    main)
         if b:
             need = paged_attention_workspace_bytes(self.pool, b, self.hq, max_ctx)
             if need > self.ws_cap:

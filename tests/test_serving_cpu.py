@@ -19,3 +19,25 @@ def test_schedule_orders_are_permutations_with_the_stated_priority():
     assert np.all(np.diff(lens[lf[:n_long]]) <= 0) and np.all(lens[lf[:n_long]] > lens.mean())
     assert np.all(np.diff(lf[n_long:]) > 0)  # the rest keeps batch order
     assert schedule_order(np.zeros(0, np.int32)).size == 0
+
+
+def test_prefill_sizes_take_the_admitted_rows():
+    """Admitted sequences are the last rows of the running set; their prompt
+    is the context minus the step's appended token, less the cached part."""
+    import types
+    from paged_kv_cache_451_b200.serving import DecodeLoop
+    info = types.SimpleNamespace(num_admitted=2)
+    plan = {"info": info, "context_lens": np.array([40, 1601, 70], np.int32), "cached": np.array([1536, 0])}
+    a, new, cached = DecodeLoop.prefill_sizes(plan)
+    assert a == 2 and list(new) == [64, 69] and list(cached) == [1536, 0]
+    info.num_admitted = 0
+    assert DecodeLoop.prefill_sizes(plan)[0] == 0
+
+
+def test_metadata_layout_is_16_byte_aligned_with_prefill_fields():
+    from paged_kv_cache_451_b200.serving import DecodeLoop
+    lay, total = DecodeLoop._layout(5, 77, 3, 9, 2)
+    for name, (off, n) in lay.items():
+        assert off % 16 == 0, name
+    assert lay["cu"][1] == 3 and lay["pf_lens"][1] == 2
+    assert total >= lay["pf_lens"][0] + 8

@@ -28,6 +28,11 @@ Workloads (sizes from the configurations the library is measured on):
                 64/8 GQA shape (bf16).
 * ``chunked_gqa`` 16 sequences, each a 512-token prompt chunk on top of a
                 cached prefix of 512..4096 tokens, 64/8 GQA, bf16.
+* ``rag_trace`` retrieval-augmented serving: Poisson arrivals (3 per
+                iteration, 60 iterations) whose prompt is one of 2 shared
+                1536-token documents plus a U[32,256]-token question, U[16,64]
+                output tokens; 64/8 GQA, bf16, 8192-block pool; prompts are
+                prefilled, then every running sequence decodes each iteration.
 
 Values of q, K and V are ~N(0, 1).  Seeds are 451 + the workload's index.
 """
@@ -91,6 +96,11 @@ WORKLOADS = {
     "chunked_gqa": Workload("chunked_gqa", 7, 1, 64, 8, 128, 16, BF16, BF16, 16,
                             extra={"new_lo": 512, "new_hi": 512, "prior_lo": 512, "prior_hi": 4096,
                                    "pool_factor": 1.25}),
+    # retrieval-augmented requests: a shared document + a question each
+    "rag_trace": Workload("rag_trace", 8, 1, 64, 8, 128, 16, BF16, BF16, 128,
+                          extra={"docs": 2, "doc_len": 1536, "question_lo": 32, "question_hi": 256,
+                                 "out_lo": 16, "out_hi": 64, "arrival_rate": 3.0, "iters": 60,
+                                 "max_num_seqs": 128, "num_blocks": 8192, "vocab": 32000}),
 }
 
 
