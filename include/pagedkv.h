@@ -201,6 +201,17 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
                            void* workspace, size_t workspace_bytes, const int32_t* seq_order,
                            kv_stream_t stream);
 
+/* Sliding-window attention (the long-context remedy named among the
+ * pitfalls of "vLLM 推理加速原理详解"; the page gives no definition): with
+ * window > 0, paged_attention_decode attends, for a sequence of n tokens,
+ * only to its last min(n, window) tokens (positions n - window .. n - 1), and
+ * reads no block before the one holding position n - window, so blocks that
+ * left the window may be released (kv_alloc_release_before).  0 turns the
+ * window off.  Workspace sizes follow the window.  paged_attention_prefill
+ * rejects a pool with a window (KV_ERR_ARG).  Host only; KV_ERR_ARG for a
+ * negative window. */
+int kv_pool_set_sliding_window(kv_pool* pool, int window);
+
 /* Multi-token attention over the paged cache: the step that processes a
  * prompt, a chunk of one, or a few drafted tokens before decoding continues
  * ([PA], and the time-to-first-token discussion of the page's section
@@ -366,6 +377,12 @@ int kv_alloc_append_token(kv_alloc* a, int64_t seq_id, int32_t token, int64_t* s
  * may be NULL. */
 int kv_alloc_commit(kv_alloc* a, int64_t seq_id, int* num_registered);
 
+/* Sliding window: release every block of seq_id wholly before position
+ * `token` (blocks 0 .. token / block_size - 1 not yet released); their table
+ * entries become -1 so logical block indices stay put.  Shared blocks only
+ * lose this sequence's reference.  num_released may be NULL. */
+int kv_alloc_release_before(kv_alloc* a, int64_t seq_id, int64_t token, int* num_released);
+
 /* Cumulative hit blocks and evictions, and the number of registered blocks
  * (each pointer may be NULL). */
 int kv_alloc_prefix_stats(const kv_alloc* a, int64_t* hit_blocks, int64_t* evictions,
@@ -423,6 +440,14 @@ int kv_sched_outputs(const kv_sched* s, int64_t* running_ids, int32_t* block_tab
                      int32_t* cow_pairs, int64_t* admitted_ids);
 /* [MON]: running and waiting request counts, used and total blocks
  * (cache usage = used / total). */
+/* Sliding window for the scheduling step: with window > 0, after its
+ * append in step (4) every running sequence not admitted in this step
+ * releases the blocks wholly before its last `window` positions
+ * (kv_alloc_release_before), which a sliding-window decode never reads;
+ * block tables then hold -1 for released entries.  0 (the default) keeps
+ * every block.  KV_ERR_ARG for a negative window. */
+int kv_sched_set_window(kv_sched* s, int window);
+
 /* Cached prompt tokens of each request admitted by the last step, in the
  * order of admitted_ids (0 without prefix caching). */
 int kv_sched_admitted_cached(const kv_sched* s, int32_t* cached_tokens);

@@ -103,6 +103,8 @@ class BlockManager:
         if seq_id not in self.tables:
             raise OracleStateError(f"sequence {seq_id} is unknown")
         for b in self.tables.pop(seq_id):
+            if b < 0:  # already released (sliding window)
+                continue
             if self.refcount[b] <= 0:
                 raise OracleStateError(f"block {b} freed twice")
             self.refcount[b] -= 1
@@ -120,7 +122,8 @@ class BlockManager:
         self.tables[child] = list(self.tables[parent])
         self.tokens[child] = self.tokens[parent]
         for b in self.tables[child]:
-            self.refcount[b] += 1
+            if b >= 0:
+                self.refcount[b] += 1
 
     def append_slot(self, seq_id: int):
         """Reserve the slot of the sequence's next token.
@@ -147,6 +150,27 @@ class BlockManager:
         slot = table[pos // self.block_size] * self.block_size + pos % self.block_size
         return slot, cow_src, cow_dst
 
+    def release_before(self, seq_id: int, token: int) -> int:
+        """Sliding window: release every block wholly before position
+        `token` (its table entry becomes -1; the table keeps its length so
+        logical block indices stay put).  Returns the number released."""
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        table = self.tables[seq_id]
+        upto = min(max(token, 0) // self.block_size, len(table))
+        n = 0
+        for i in range(upto):
+            b = table[i]
+            if b < 0:
+                continue
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                self.free_list.append(b)
+                self.num_freed += 1
+            table[i] = -1
+            n += 1
+        return n
+
     def block_table(self, seq_id: int) -> list[int]:
         if seq_id not in self.tables:
             raise OracleStateError(f"sequence {seq_id} is unknown")
@@ -159,10 +183,15 @@ class BlockManager:
 class Scheduler:
     """One scheduling iteration per :meth:`step`, in the page's order."""
 
-    def __init__(self, bm: BlockManager, max_num_seqs: int, min_blocks: int | None = None):
+    def __init__(self, bm: BlockManager, max_num_seqs: int, min_blocks: int | None = None,
+                 window: int = 0):
         self.bm = bm
         self.max_num_seqs = max_num_seqs
         self.min_blocks = min_blocks  # None: number of running sequences
+        # > 0: after its append, a running sequence releases the blocks wholly
+        # before its last `window` positions (sliding-window decode reads no
+        # earlier block); one admitted in this step keeps them until the next
+        self.window = window
         self.waiting: deque[tuple[int, int]] = deque()
         self.running: list[int] = []
 
@@ -233,6 +262,8 @@ class Scheduler:
             decode_slots.append(slot)
             if cs >= 0:
                 cow.append((cs, cd))
+            if self.window > 0 and sid not in admitted:
+                self.bm.release_before(sid, self.bm.tokens[sid] - self.window)
         return {
             "running": list(self.running),
             "block_tables": [self.bm.block_table(s) for s in self.running],
@@ -395,7 +426,7 @@ class PrefixCachingBlockManager(BlockManager):
         for i in range(done, len(keys)):
             k, parent, blk = keys[i]
             b = table[i]
-            if k not in self.cached and b not in self.key_of:
+            if b >= 0 and k not in self.cached and b not in self.key_of:
                 self.cached[k] = b
                 self.key_of[b] = (k, parent, blk)
                 new += 1
@@ -406,6 +437,8 @@ class PrefixCachingBlockManager(BlockManager):
         if seq_id not in self.tables:
             raise OracleStateError(f"sequence {seq_id} is unknown")
         for b in reversed(self.tables.pop(seq_id)):
+            if b < 0:
+                continue
             if self.refcount[b] <= 0:
                 raise OracleStateError(f"block {b} freed twice")
             self.refcount[b] -= 1

@@ -60,6 +60,9 @@ _SIGS = {
     "kv_pool_bytes": (c_int, [c_void_p, P(c_size_t), P(c_size_t)]),
     "kv_pool_bind": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "kv_pool_set_decode_config": (c_int, [c_void_p, c_int, c_int, c_int]),
+    "kv_pool_set_sliding_window": (c_int, [c_void_p, c_int]),
+    "kv_alloc_release_before": (c_int, [c_void_p, c_int64, c_int64, P(c_int)]),
+    "kv_sched_set_window": (c_int, [c_void_p, c_int]),
     "kv_pool_destroy": (c_int, [c_void_p]),
     "paged_kv_write": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_int,
                                c_void_p, c_void_p, c_void_p]),
@@ -174,6 +177,20 @@ def kv_pool_bind(pool, layer, k_base, v_base, k_scale=None, v_scale=None):
 
 def kv_pool_set_decode_config(pool, partition_tokens=0, stages=0, warps=0):
     _check(_lib.kv_pool_set_decode_config(pool, partition_tokens, stages, warps))
+
+
+def kv_pool_set_sliding_window(pool, window):
+    _check(_lib.kv_pool_set_sliding_window(pool, int(window)))
+
+
+def kv_alloc_release_before(a, seq_id, token) -> int:
+    n = c_int()
+    _check(_lib.kv_alloc_release_before(a, seq_id, int(token), ctypes.byref(n)))
+    return n.value
+
+
+def kv_sched_set_window(s, window):
+    _check(_lib.kv_sched_set_window(s, int(window)))
 
 
 def kv_pool_destroy(pool):

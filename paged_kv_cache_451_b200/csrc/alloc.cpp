@@ -225,7 +225,7 @@ struct kv_alloc {
       const uint64_t k = block_key(parent, t, block_size);
       if (i >= s.registered) {
         const int32_t b = s.blocks[i];
-        if (!cached.count(k) && !key_of[b].valid) {
+        if (b >= 0 && !cached.count(k) && !key_of[b].valid) {
           CachedBlock& c = key_of[b];
           c.valid = true;
           c.key = k;
@@ -327,7 +327,8 @@ int kv_alloc_fork(kv_alloc* a, int64_t parent, int64_t child) {
   if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)parent);
   if (a->seqs.count(child)) return fail(KV_ERR_STATE, "sequence %lld already exists", (long long)child);
   SeqState s = it->second;
-  for (int32_t b : s.blocks) ++a->refcount[b];
+  for (int32_t b : s.blocks)
+    if (b >= 0) ++a->refcount[b];
   a->seqs.emplace(child, std::move(s));
   return ok();
 }
@@ -338,9 +339,11 @@ int kv_alloc_free(kv_alloc* a, int64_t seq_id) {
   if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
   const auto& blocks = it->second.blocks;
   if (a->caching) {  // deepest block first: shared prefixes leave the cache last
-    for (auto r = blocks.rbegin(); r != blocks.rend(); ++r) a->release(*r);
+    for (auto r = blocks.rbegin(); r != blocks.rend(); ++r)
+      if (*r >= 0) a->release(*r);
   } else {
-    for (int32_t b : blocks) a->release(b);
+    for (int32_t b : blocks)
+      if (b >= 0) a->release(b);
   }
   a->seqs.erase(it);
   return ok();
@@ -446,6 +449,23 @@ int kv_alloc_prefix_stats(const kv_alloc* a, int64_t* hit_blocks, int64_t* evict
   return ok();
 }
 
+int kv_alloc_release_before(kv_alloc* a, int64_t seq_id, int64_t token, int* num_released) {
+  if (!a) return fail(KV_ERR_ARG, "NULL allocator");
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
+  SeqState& st = it->second;
+  const int64_t upto = std::min<int64_t>(token < 0 ? 0 : token / a->block_size, (int64_t)st.blocks.size());
+  int released = 0;
+  for (int64_t i = 0; i < upto; ++i) {
+    if (st.blocks[i] < 0) continue;
+    a->release(st.blocks[i]);
+    st.blocks[i] = -1;
+    ++released;
+  }
+  if (num_released) *num_released = released;
+  return ok();
+}
+
 int kv_alloc_counters(const kv_alloc* a, int64_t* allocated, int64_t* freed, int64_t* cow) {
   if (!a) return fail(KV_ERR_ARG, "NULL allocator");
   if (allocated) *allocated = a->n_alloc;
@@ -469,6 +489,7 @@ struct kv_sched {
   kv_alloc* a = nullptr;
   int max_num_seqs = 0;
   int min_blocks = -1;
+  int window = 0;  // > 0: release blocks that left the window after each step
   std::deque<Request> waiting;
   std::vector<int64_t> running;
   // outputs of the last step
@@ -510,6 +531,12 @@ int kv_sched_add_request(kv_sched* s, int64_t seq_id, int prompt_len) {
 int kv_sched_add_request_tokens(kv_sched* s, int64_t seq_id, const int32_t* tokens, int num_tokens) {
   if (!s || num_tokens < 0 || (num_tokens > 0 && !tokens)) return fail(KV_ERR_ARG, "bad argument");
   s->waiting.push_back({seq_id, num_tokens, true, std::vector<int32_t>(tokens, tokens + num_tokens)});
+  return ok();
+}
+
+int kv_sched_set_window(kv_sched* s, int window) {
+  if (!s || window < 0) return fail(KV_ERR_ARG, "bad argument");
+  s->window = window;
   return ok();
 }
 
@@ -614,6 +641,7 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   }
   s->out_slots = prompt_slots;
   int max_blocks = 0;
+  std::unordered_set<int64_t> admitted(s->out_admitted.begin(), s->out_admitted.end());
   for (int64_t r : s->running) {
     SeqState& st = a->seqs[r];
     int64_t slot;
@@ -623,6 +651,12 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
     if (cs >= 0) {
       s->out_cow.push_back(cs);
       s->out_cow.push_back(cd);
+    }
+    if (s->window > 0 && !admitted.count(r)) {
+      // this step's decode reads positions tokens - window .. tokens - 1: the
+      // blocks wholly before them leave (a sequence admitted in this step
+      // keeps its prompt blocks until the next step, after its prompt write)
+      kv_alloc_release_before(a, r, st.tokens - s->window, nullptr);
     }
     s->out_running.push_back(r);
     s->out_tables.push_back(st.blocks);

@@ -87,6 +87,7 @@ struct DecodeParams {
   int ctx_cap;                  // min(max_blocks * block_size, max_context_len)
   int part_chunks;              // chunks per partition
   int num_parts;
+  int window;                   // > 0: attend only the last `window` tokens
   float scale_log2;             // softmax scale * log2(e)
 };
 
@@ -170,7 +171,11 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
     if (part == 0 && threadIdx.x == 0) record_error(KV_ERR_BOUNDS);
     n = n < 0 ? 0 : p.ctx_cap;
   }
-  const int total_chunks = (n + kChunk - 1) / kChunk;
+  // sliding window: tokens [t_lo, n) only; chunks are counted from cb, the
+  // chunk holding t_lo (blocks wholly before it may already be released)
+  const int t_lo = p.window > 0 ? max(0, n - p.window) : 0;
+  const int cb = t_lo / kChunk;
+  const int total_chunks = (n + kChunk - 1) / kChunk - cb;
   const int c0 = part * p.part_chunks;
   const int c1 = min(c0 + p.part_chunks, total_chunks);
   if (c0 >= c1 && part > 0) return;  // nothing in this partition (uniform per CTA)
@@ -189,7 +194,7 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
     prefetch_tensormap(&vmap);
   }
   for (int i = threadIdx.x; i < nchunks; i += WARPS * 32) {
-    const int c = c0 + i;
+    const int c = cb + c0 + i;
     int32_t b = p.block_tables[(int64_t)seq * p.max_blocks + (c >> cpb_shift)];
     if (b < 0 || b >= p.num_blocks) {
       record_error(KV_ERR_BOUNDS);
@@ -276,7 +281,7 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       mbar_arrive(bar);  // complete the phase without data; the chunk is skipped
       return;
     }
-    const int y = kvh * bs + ((c0 + i) & ((1 << cpb_shift) - 1)) * kChunk;
+    const int y = kvh * bs + ((cb + c0 + i) & ((1 << cpb_shift) - 1)) * kChunk;
     const uint32_t kd = wstage + st * S::STAGEB;
     mbar_arrive_expect_tx(bar, S::STAGEB);
 #pragma unroll
@@ -329,7 +334,9 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
     }
     const int i = warp + li * WARPS;
     if (blk_ids[i] >= 0) {
-      const int vt = min(kChunk, n - (c0 + i) * kChunk);  // valid tokens in the chunk
+      const int ct = (cb + c0 + i) * kChunk;    // first token of the chunk
+      const int vt = min(kChunk, n - ct);        // tokens [lt, vt) of the chunk are attended
+      const int lt = max(0, t_lo - ct);
       const uint32_t kb = wstage + st * S::STAGEB;
       const uint32_t vb = kb + S::TILEB;
 
@@ -366,9 +373,9 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       }
       float z[4] = {(sacc[0][0] + sacc[1][0]) * zsa, (sacc[0][1] + sacc[1][1]) * zsb,
                     (sacc[0][2] + sacc[1][2]) * zsa, (sacc[0][3] + sacc[1][3]) * zsb};
-      if (vt < kChunk) {
-        if (gq >= vt) z[0] = z[1] = -INFINITY;
-        if (gq + 8 >= vt) z[2] = z[3] = -INFINITY;
+      if (vt < kChunk || lt > 0) {
+        if (gq >= vt || gq < lt) z[0] = z[1] = -INFINITY;
+        if (gq + 8 >= vt || gq + 8 < lt) z[2] = z[3] = -INFINITY;
       }
       // A head's max over the chunk is only needed when some value exceeds its
       // reference max by more than 2^kLazyLog2 (the first chunk, rarely later);
@@ -476,11 +483,12 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
           }
         }
       };
-      if (vt == kChunk) {
+      if (vt == kChunk && lt == 0) {
         pv(0u, 0u, std::false_type{});
       } else {
-        const uint32_t mlo = (2 * cq < vt ? 0x0000ffffu : 0u) | (2 * cq + 1 < vt ? 0xffff0000u : 0u);
-        const uint32_t mhi = (8 + 2 * cq < vt ? 0x0000ffffu : 0u) | (9 + 2 * cq < vt ? 0xffff0000u : 0u);
+        auto in = [&](int t) { return t >= lt && t < vt; };
+        const uint32_t mlo = (in(2 * cq) ? 0x0000ffffu : 0u) | (in(2 * cq + 1) ? 0xffff0000u : 0u);
+        const uint32_t mhi = (in(8 + 2 * cq) ? 0x0000ffffu : 0u) | (in(9 + 2 * cq) ? 0xffff0000u : 0u);
         pv(mlo, mhi, std::true_type{});
       }
     }
@@ -592,14 +600,18 @@ __global__ void __launch_bounds__(256)
 lse_reduce_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                   const int32_t* __restrict__ context_lens, void* out, int out_kind,
                   int num_q_heads, int head_dim, int num_parts, int part_tokens, int ctx_cap,
-                  int batch) {
+                  int window, int batch) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t idx = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
   if (idx >= (int64_t)batch * num_q_heads) return;
   const int seq = (int)(idx / num_q_heads);
   int n = context_lens[seq];
   n = n < 0 ? 0 : (n > ctx_cap ? ctx_cap : n);
-  const int np = max(1, (n + part_tokens - 1) / part_tokens);
+  // partitions of the chunks the decode visited (from the window's first chunk)
+  const int cb = window > 0 ? max(0, n - window) / kChunk : 0;
+  const int chunks = (n + kChunk - 1) / kChunk - cb;
+  const int part_chunks = part_tokens / kChunk;
+  const int np = max(1, (chunks + part_chunks - 1) / part_chunks);
   if (np == 1) return;  // written by the decode kernel directly
   const float4* ml = reinterpret_cast<const float4*>(part_ml) + idx * num_parts;
   float Mz = -INFINITY, Mw = -INFINITY;

@@ -187,6 +187,15 @@ int num_parts_for(const kv_pool* pool, int batch, int max_context_len) {
   return std::max(1, (max_context_len + pt - 1) / pt);
 }
 
+// Upper bound on the tokens one decode visits per sequence: with a sliding
+// window of W tokens, the chunks from the one holding the window's first
+// token to the last, i.e. at most 16 * ceil(W / 16) + 16.
+int visited_len(const kv_pool* pool, int max_context_len) {
+  if (pool->window <= 0) return max_context_len;
+  const int64_t w = ((int64_t)pool->window + kChunk - 1) / kChunk * kChunk + kChunk;
+  return (int)std::min<int64_t>(max_context_len, w);
+}
+
 // Resident CTAs per SM of one decode instantiation on the current device
 // (occupancy API; registers and shared memory both count).
 template <int KV, int D, int W, int STAGES>
@@ -384,6 +393,13 @@ int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages, i
   return ok();
 }
 
+int kv_pool_set_sliding_window(kv_pool* pool, int window) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (window < 0) return fail(KV_ERR_ARG, "window %d must be >= 0", window);
+  pool->window = window;
+  return ok();
+}
+
 int kv_pool_destroy(kv_pool* pool) {
   delete pool;
   return ok();
@@ -466,7 +482,7 @@ int block_copy(const kv_pool* pool, const int32_t* pairs, int num_pairs, kv_stre
 size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
                                        int max_context_len) {
   if (!pool || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
-  const int np = num_parts_for(pool, batch, max_context_len);
+  const int np = num_parts_for(pool, batch, visited_len(pool, max_context_len));
   if (np <= 1) return 0;
   return (size_t)batch * num_q_heads * np * (pool->head_dim + 4) * sizeof(float);
 }
@@ -499,8 +515,9 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   if ((int64_t)max_blocks_per_seq * pool->block_size < max_context_len)
     return fail(KV_ERR_ARG, "max_blocks_per_seq %d cannot hold max_context_len %d",
                 max_blocks_per_seq, max_context_len);
-  const int pt = partition_tokens(pool, batch, max_context_len);
-  const int np = num_parts_for(pool, batch, max_context_len);
+  const int visited = visited_len(pool, max_context_len);
+  const int pt = partition_tokens(pool, batch, visited);
+  const int np = num_parts_for(pool, batch, visited);
   if (np > 65535) return fail(KV_ERR_ARG, "too many partitions");
   const size_t need = paged_attention_workspace_bytes(pool, batch, num_q_heads, max_context_len);
   if (need > 0 && (!workspace || workspace_bytes < need))
@@ -531,6 +548,7 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   p.part_chunks = pt / kChunk;
   p.num_parts = np;
   p.ctx_cap = (int)std::min<int64_t>((int64_t)max_blocks_per_seq * pool->block_size, max_context_len);
+  p.window = pool->window;
   p.scale_log2 = scale * 1.4426950408889634f;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -547,7 +565,8 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
     const int64_t rows = (int64_t)batch * num_q_heads;
     const int blocks = (int)((rows + 7) / 8);
     lse_reduce_kernel<<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, context_lens, out, p.out_kind,
-                                             num_q_heads, pool->head_dim, np, pt, p.ctx_cap, batch);
+                                             num_q_heads, pool->head_dim, np, pt, p.ctx_cap,
+                                             p.window, batch);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
   }

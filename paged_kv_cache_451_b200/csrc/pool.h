@@ -34,6 +34,7 @@ struct kv_pool {
   int partition_tokens = 0;  // 0: automatic
   int stages = 0;            // 0: automatic
   int warps = 0;             // 0: automatic
+  int window = 0;            // > 0: decode attends only the last `window` tokens
   std::vector<pagedkv::LayerBinding> layers;
 
   size_t tile_bytes() const { return (size_t)block_size * head_dim * pagedkv::elem_bytes(dtype); }

@@ -104,17 +104,19 @@ int launch(const PrefillParams& p, const CUtensorMap& qmap, const LayerBinding& 
   return KV_OK;
 }
 
-// Stage counts: three K/V stages of 32 KB at head_dim 128, four of 16 KB at
-// 64 (both leave one CTA per SM, which the 512 TMEM columns need).
+// Stage counts: two K/V stages of 32 KB each at head_dim 128 (next to the two
+// 32 KB query tiles), four of 16 KB at 64; both leave one CTA per SM, which
+// the 512 TMEM columns need.
 template <bool kBf16>
 int launch_d(int head_dim, const PrefillParams& p, const CUtensorMap& qmap,
              const LayerBinding& lb, dim3 grid, cudaStream_t stream) {
   return head_dim == 64 ? launch<kBf16, 64, 4>(p, qmap, lb, grid, stream)
-                        : launch<kBf16, 128, 3>(p, qmap, lb, grid, stream);
+                        : launch<kBf16, 128, 2>(p, qmap, lb, grid, stream);
 }
 
-static_assert(PrefillShape<128, 3>::SMEM_BYTES <= 227 * 1024, "prefill shared memory");
+static_assert(PrefillShape<128, 2>::SMEM_BYTES <= 227 * 1024, "prefill shared memory");
 static_assert(PrefillShape<64, 4>::SMEM_BYTES * 2 > 228 * 1024, "one prefill CTA per SM");
+static_assert(PrefillShape<128, 2>::SMEM_BYTES * 2 > 228 * 1024, "one prefill CTA per SM");
 
 }  // namespace
 }  // namespace pagedkv
@@ -136,6 +138,8 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
     return fail(KV_ERR_ARG, "multi-token attention needs an f16 or bf16 pool");
   if (pool->head_dim != 64 && pool->head_dim != 128)
     return fail(KV_ERR_ARG, "multi-token attention needs head_dim 64 or 128");
+  if (pool->window > 0)
+    return fail(KV_ERR_ARG, "multi-token attention over a sliding-window pool is not supported");
   if (q_dtype != pool->dtype) return fail(KV_ERR_ARG, "q dtype must equal the pool dtype");
   if (out_dtype != q_dtype && out_dtype != KV_F32)
     return fail(KV_ERR_ARG, "out dtype must be the q dtype or KV_F32");
@@ -156,8 +160,8 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
 
   const int g = num_q_heads / pool->kv_heads;
   const int tq = kPfRows / g;
-  const int64_t tiles = ((int64_t)max_q_len + tq - 1) / tq;
-  if (tiles > 0x7fffffff) return fail(KV_ERR_ARG, "max_q_len too large");
+  const int64_t pairs = ((int64_t)max_q_len + kPfTiles * tq - 1) / (kPfTiles * tq);
+  if (pairs > 0x7fffffff) return fail(KV_ERR_ARG, "max_q_len too large");
   int* err = error_word_cached();
   if (!err) return fail(KV_ERR_CUDA, "device error word unavailable");
 
@@ -175,7 +179,7 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
   p.num_q_heads = num_q_heads;
   p.group = g;
   p.tokens_per_tile = tq;
-  p.num_q_tiles = (int)tiles;
+  p.num_q_pairs = (int)pairs;
   p.kv_heads = pool->kv_heads;
   p.block_size = pool->block_size;
   p.num_blocks = pool->num_blocks;
@@ -183,7 +187,7 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
   p.total_q = total_q;
   p.scale_log2 = scale * 1.4426950408889634f;
 
-  const dim3 grid((unsigned)tiles, pool->kv_heads, batch);
+  const dim3 grid((unsigned)pairs, pool->kv_heads, batch);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = pool->dtype == KV_BF16 ? launch_d<true>(pool->head_dim, p, qmap, lb, grid, s)
                               : launch_d<false>(pool->head_dim, p, qmap, lb, grid, s);

@@ -45,10 +45,11 @@
 
 namespace pagedkv {
 
-constexpr int kPfRows = 128;       // query rows per CTA (M of the MMA)
-constexpr int kPfKeys = 128;       // keys per tile (N of Q.K^T, K of P.V)
-constexpr int kPfThreads = 192;    // warps 0-3 softmax, 4 copies, 5 MMA
-constexpr uint32_t kPfTmemCols = 512;  // S double buffer (2 x 128) + O (<= 128)
+constexpr int kPfRows = 128;        // query rows per tile (M of the MMA)
+constexpr int kPfKeys = 128;        // keys per tile (N of Q.K^T, K of P.V)
+constexpr int kPfTiles = 2;         // query tiles per CTA, sharing every K/V tile
+constexpr int kPfThreads = 320;     // warps 0-7 softmax (4 per query tile), 8 copies, 9 MMA
+constexpr uint32_t kPfTmemCols = 512;  // S_A, S_B (128 each) + O_A, O_B (<= 128 each)
 constexpr uint64_t kPfWaitNs = 2000000000ull;
 constexpr uint64_t kPfDrainNs = 50000000ull;  // copies and MMAs in flight finish in microseconds
 // reference max moves only when a tile's max exceeds it by more than this
@@ -67,7 +68,7 @@ struct PrefillParams {
   int num_q_heads;
   int group;                    // query heads per kv head, <= 8
   int tokens_per_tile;          // 128 / group
-  int num_q_tiles;              // grid x
+  int num_q_pairs;              // grid x: pairs of query tiles
   int kv_heads;
   int block_size;
   int num_blocks;
@@ -81,17 +82,20 @@ struct PrefillShape {
   static constexpr int NH = D / 64;            // 128-byte column blocks per row
   static constexpr int HALF = kPfRows * 128;   // one column block of a 128-row tile
   static constexpr int TILE = NH * HALF;       // a Q, K or V tile
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE;
+  static constexpr int Q_OFF = 0;              // Q_A, Q_B
+  static constexpr int K_OFF = Q_OFF + kPfTiles * TILE;
   static constexpr int V_OFF = K_OFF + STAGES * TILE;
   static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
-  // q, K full/empty and V full/empty per stage, S full, P full, P.V done per
-  // S buffer, and the final MMA drain
-  static constexpr int NBAR = 1 + 4 * STAGES + 6 + 1;
+  // q; K full/empty and V full/empty per stage; S full, P full and P.V done
+  // per query tile; the final MMA drain
+  static constexpr int NBAR = 1 + 4 * STAGES + 3 * kPfTiles + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // TMEM base, abort flag
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t S_COL = 0;                       // S_X at X * 128
+  static constexpr uint32_t O_COL = kPfTiles * kPfKeys;      // O_X at 256 + X * D
   static_assert(kPfRows == kPfKeys, "Q, K and V tiles share one byte size");
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(O_COL + kPfTiles * D <= kPfTmemCols, "TMEM columns");
 };
 
 namespace pf {
@@ -102,14 +106,28 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Non-suspending probe of a barrier phase (the waits here sit on the
+// critical path between the MMA issuer and the softmax warps).
+__device__ __forceinline__ bool probe(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Wait for the phase with `parity`; give up when another role of the CTA
 // has aborted, or after kPfWaitNs (then abort the CTA and record a timeout).
 __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                      int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (probe(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (probe(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kPfWaitNs) {
       *abort_flag = 1;
@@ -137,7 +155,7 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   uint8_t* smem = smem_raw + (sbase - raw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.num_q_tiles - 1 - (int)blockIdx.x;  // tiles with the most keys start first
+  const int qp = p.num_q_pairs - 1 - (int)blockIdx.x;  // pairs with the most keys start first
   const int kvh = blockIdx.y, s = blockIdx.z;
   const int g = p.group, tq = p.tokens_per_tile;
 
@@ -145,16 +163,24 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   const int q_len = p.cu_q[s + 1] - q0;
   const int n = p.context_lens[s];
   if (q0 < 0 || q_len < 0 || q_len > n || (int64_t)q0 + q_len > p.total_q ||
-      (int64_t)n > (int64_t)p.max_blocks * p.block_size || q_len > p.num_q_tiles * tq) {
+      (int64_t)n > (int64_t)p.max_blocks * p.block_size ||
+      q_len > p.num_q_pairs * kPfTiles * tq) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) atomicCAS(p.err, 0, KV_ERR_BOUNDS);
     return;
   }
-  const int t0 = qt * tq;  // first new token of this tile
+  const int t0 = qp * kPfTiles * tq;  // first new token of query tile A
   if (t0 >= q_len) return;
-  const int ntok = min(tq, q_len - t0);
-  const int p0 = n - q_len + t0;   // its position in the sequence
-  const int kend = p0 + ntok;      // keys 0 .. kend - 1 are read
-  const int ntiles = (kend + kPfKeys - 1) / kPfKeys;
+  // per query tile X (A = 0, B = 1): tokens, key range, key tiles
+  int ntok[kPfTiles], kendx[kPfTiles], ntx[kPfTiles];
+#pragma unroll
+  for (int x = 0; x < kPfTiles; ++x) {
+    const int tx = t0 + x * tq;
+    ntok[x] = tx < q_len ? min(tq, q_len - tx) : 0;
+    kendx[x] = ntok[x] ? n - q_len + tx + ntok[x] : 0;  // keys 0 .. kend - 1
+    ntx[x] = (kendx[x] + kPfKeys - 1) / kPfKeys;
+  }
+  const int kend = max(kendx[0], kendx[1]);
+  const int ntiles = max(ntx[0], ntx[1]);  // K/V tiles read (tile B's when it has tokens)
   const int qrows = tq * g;
 
   const uint32_t bar0 = sbase + S::BAR_OFF;
@@ -163,10 +189,10 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   auto KE = [&](int i) { return bar0 + 8u * (1 + STAGES + i); };
   auto VF = [&](int i) { return bar0 + 8u * (1 + 2 * STAGES + i); };
   auto VE = [&](int i) { return bar0 + 8u * (1 + 3 * STAGES + i); };
-  auto SF = [&](int b) { return bar0 + 8u * (1 + 4 * STAGES + b); };
-  auto PF = [&](int b) { return bar0 + 8u * (3 + 4 * STAGES + b); };
-  auto PV = [&](int b) { return bar0 + 8u * (5 + 4 * STAGES + b); };
-  const uint32_t FIN = bar0 + 8u * (7 + 4 * STAGES);
+  auto SF = [&](int x) { return bar0 + 8u * (1 + 4 * STAGES + x); };
+  auto PF = [&](int x) { return bar0 + 8u * (1 + 4 * STAGES + kPfTiles + x); };
+  auto PV = [&](int x) { return bar0 + 8u * (1 + 4 * STAGES + 2 * kPfTiles + x); };
+  const uint32_t FIN = bar0 + 8u * (1 + 4 * STAGES + 3 * kPfTiles);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::MISC_OFF + 8);
 
@@ -178,26 +204,27 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       mbar_init(VF(i), 1);
       mbar_init(VE(i), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(SF(b), 1);
-      mbar_init(PF(b), kPfRows);
-      mbar_init(PV(b), 1);
+    for (int x = 0; x < kPfTiles; ++x) {
+      mbar_init(SF(x), 1);
+      mbar_init(PF(x), kPfRows);
+      mbar_init(PV(x), 1);
     }
     mbar_init(FIN, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // Query rows past tokens_per_tile * group are not covered by the copy
-  if (threadIdx.x >= qrows && threadIdx.x < kPfRows) {
+  // Query rows past tokens_per_tile * group are not covered by the copies
+  if (threadIdx.x < kPfTiles * kPfRows && (int)(threadIdx.x % kPfRows) >= qrows) {
+    const int x = threadIdx.x / kPfRows, r = threadIdx.x % kPfRows;
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
-      uint4* row = reinterpret_cast<uint4*>(smem + S::Q_OFF + h * S::HALF + threadIdx.x * 128);
+      uint4* row = reinterpret_cast<uint4*>(smem + S::Q_OFF + x * S::TILE + h * S::HALF + r * 128);
 #pragma unroll
       for (int i = 0; i < 8; ++i) row[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     pf::fence_proxy_async();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tc::alloc(smem_u32(tmem_slot), kPfTmemCols);
     tc::relinquish();
@@ -207,16 +234,19 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   tc::fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ copies
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
-      mbar_arrive_expect_tx(BQ, (uint32_t)(NH * qrows * 128));
+      mbar_arrive_expect_tx(BQ, (uint32_t)(kPfTiles * NH * qrows * 128));
 #pragma unroll
-      for (int h = 0; h < NH; ++h)
-        tma_load_3d(sbase + S::Q_OFF + h * S::HALF, &qmap, BQ, h * 64, kvh * g, q0 + t0);
+      for (int x = 0; x < kPfTiles; ++x)
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+          tma_load_3d(sbase + S::Q_OFF + x * S::TILE + h * S::HALF, &qmap, BQ, h * 64, kvh * g,
+                      q0 + t0 + x * tq);
       const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks;
       int nk = 0, nv = 0;  // tiles whose K (V) copies are in flight or done
       for (int j = 0; j < ntiles; ++j) {
@@ -270,91 +300,124 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         (void)mbar_wait_bounded(BQ, 0, kPfDrainNs);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // --------------------------------------------------------------- MMA
+    // Issue order S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) ...:
+    // the softmax of one query tile runs while the tensor cores work on the
+    // other's P.V and next S.
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_f16(kBf16, kPfRows, kPfKeys, false);
       constexpr uint32_t kIdO = tc::idesc_f16(kBf16, kPfRows, D, true);
-      const uint32_t dO = tmem + 2 * kPfKeys;
-      auto issue_s = [&](int j) -> bool {
+      auto issue_s = [&](int x, int j) {
         const int st = j % STAGES;
-        if (!pf::wait(KF(st), (j / STAGES) & 1, abort_flag, p.err)) return false;
-        tc::fence_after();
-        const uint32_t dS = tmem + (uint32_t)(j & 1) * kPfKeys;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * S::HALF + (kk % 4) * 32;  // 16 columns per step
-          tc::mma_ss(dS, tc::desc_sw128(sbase + S::Q_OFF + off, 16, 1024),
+          tc::mma_ss(tmem + S::S_COL + x * kPfKeys,
+                     tc::desc_sw128(sbase + S::Q_OFF + x * S::TILE + off, 16, 1024),
                      tc::desc_sw128(sbase + S::K_OFF + st * S::TILE + off, 16, 1024), kIdS,
                      kk > 0 ? 1u : 0u);
         }
-        tc::commit(KE(st));
-        tc::commit(SF(j & 1));
-        return true;
+        tc::commit(SF(x));
       };
-      bool ok = pf::wait(BQ, 0, abort_flag, p.err);
-      tc::fence_after();
-      if (ok) ok = issue_s(0);
-      if (ok && ntiles > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int b = j & 1, st = j % STAGES;
-        if (!pf::wait(PF(b), (j >> 1) & 1, abort_flag, p.err)) break;
-        if (!pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err)) break;
-        tc::fence_after();
-        const uint32_t aP = tmem + (uint32_t)b * kPfKeys;
+      auto issue_pv = [&](int x, int j) {
+        const int st = j % STAGES;
+        const uint32_t aP = tmem + S::S_COL + x * kPfKeys;
 #pragma unroll
-        for (int kk = 0; kk < KCH; ++kk) {  // 16 keys per step: 8 TMEM columns of P
+        for (int kk = 0; kk < KCH; ++kk) {
+          // keys 16kk..16kk+15: 32-key chunk kk/2 holds its values in 16
+          // columns, then (bf16) its residuals in the next 16
+          const uint32_t col = 32 * (kk / 2) + 8 * (kk % 2);
           const uint64_t bV =
               tc::desc_sw128(sbase + S::V_OFF + st * S::TILE + kk * 2048, S::HALF, 1024);
-          tc::mma_ts(dO, aP + 8 * kk, bV, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
-          if constexpr (kSplit) tc::mma_ts(dO, aP + 64 + 8 * kk, bV, kIdO, 1u);
+          tc::mma_ts(tmem + S::O_COL + x * D, aP + col, bV, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
+          if constexpr (kSplit) tc::mma_ts(tmem + S::O_COL + x * D, aP + col + 16, bV, kIdO, 1u);
         }
+        tc::commit(PV(x));
+      };
+      bool ok = pf::wait(BQ, 0, abort_flag, p.err) && pf::wait(KF(0), 0, abort_flag, p.err);
+      tc::fence_after();
+      if (ok) {
+#pragma unroll
+        for (int x = 0; x < kPfTiles; ++x)
+          if (ntx[x] > 0) issue_s(x, 0);
+        tc::commit(KE(0));
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int st = j % STAGES, sn = (j + 1) % STAGES;
+        const bool more = j + 1 < ntiles;
+        bool waited_k = false;
+        if (!pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err)) break;
+#pragma unroll
+        for (int x = 0; x < kPfTiles; ++x) {
+          if (j < ntx[x]) {
+            if (!pf::wait(PF(x), j & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after();
+            issue_pv(x, j);
+          }
+          if (j + 1 < ntx[x]) {
+            if (!waited_k) {
+              if (!pf::wait(KF(sn), ((j + 1) / STAGES) & 1, abort_flag, p.err)) {
+                ok = false;
+                break;
+              }
+              tc::fence_after();
+              waited_k = true;
+            }
+            issue_s(x, j + 1);
+          }
+        }
+        if (!ok) break;
         tc::commit(VE(st));
-        tc::commit(PV(b));
-        if (j + 2 < ntiles && !issue_s(j + 2)) break;
+        if (more) tc::commit(KE(sn));
       }
       // every MMA issued must finish before TMEM is released
       tc::commit(FIN);
       (void)mbar_wait_bounded(FIN, 0, kPfDrainNs);
     }
   } else {
-    // ------------------------------------------- softmax: one row a thread
-    const int r = threadIdx.x;
+    // ------------------------------------ softmax: one row a thread, warps
+    // 0-3 own query tile A, warps 4-7 tile B
+    const int x = warp / 4;
+    const int r = threadIdx.x % kPfRows;
     const int tok = r / g, head = r - tok * g;
-    const bool valid = r < qrows && tok < ntok;
-    const int prow = valid ? p0 + tok : kend - 1;  // last key this row sees
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    const uint32_t tO = tmem + lane_addr + 2 * kPfKeys;
+    const int nt = x ? ntx[1] : ntx[0];  // selects keep the per-tile values in registers
+    const bool valid = r < qrows && tok < (x ? ntok[1] : ntok[0]);
+    const int prow = valid ? n - q_len + t0 + x * tq + tok : (x ? kendx[1] : kendx[0]) - 1;
+    const uint32_t lane_addr = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + S::S_COL + x * kPfKeys;
+    const uint32_t tO = tmem + lane_addr + S::O_COL + x * D;
     const float sl2 = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, pf::wait(SF(b), (j >> 1) & 1, abort_flag, p.err));
+    for (int j = 0; j < nt; ++j) {
+      ok = __all_sync(0xffffffffu, pf::wait(SF(x), j & 1, abort_flag, p.err));
       if (!ok) break;
       tc::fence_after();
-      const uint32_t tS = tmem + lane_addr + (uint32_t)b * kPfKeys;
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::ld32(tS + 32 * c, sr[c]);
-      tc::wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::pin(sr[c]);
       const int lim = prow - j * kPfKeys;  // columns 0 .. lim are visible
-      if (lim < kPfKeys - 1) {
+      const bool masked = lim < kPfKeys - 1;
+      // pass 1: the row max
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+      {
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::ld32(tS + 32 * c, sr[c]);
+        tc::wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::pin(sr[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * c + i > lim) sr[c][i] = __float_as_uint(-INFINITY);
+          for (int i = 0; i < 32; ++i) {
+            const float v = (masked && 32 * c + i > lim) ? -INFINITY : __uint_as_float(sr[c][i]);
+            mx8[i % 8] = fmaxf(mx8[i % 8], v);
+          }
       }
-      float mx8[8];  // eight independent chains, then a tree
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) mx8[i % 8] = fmaxf(mx8[i % 8], __uint_as_float(sr[c][i]));
 #pragma unroll
       for (int w = 4; w > 0; w >>= 1)
 #pragma unroll
@@ -366,11 +429,10 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       __syncwarp();
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         // O holds P.V up to tile j - 1: wait for it, then rescale in TMEM
-        ok = __all_sync(0xffffffffu,
-                        pf::wait(PV((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.err));
+        ok = __all_sync(0xffffffffu, pf::wait(PV(x), (j - 1) & 1, abort_flag, p.err));
         if (!ok) break;
         tc::fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tc::ld32(tO + 32 * c, o);
@@ -382,16 +444,22 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         }
       }
       m_ref = m_new;
-      float ls[4] = {l * alpha, 0.f, 0.f, 0.f};  // independent partial sums
-      // P_j over S_j's columns: 16-bit pairs, keys 2c and 2c + 1 in column c
-      // (bf16: values in columns 0-63, residuals in 64-127)
-#pragma unroll
+      // pass 2: P over S's own columns, one 32-key chunk at a time: keys
+      // 2i, 2i + 1 of the chunk in its column i (16 columns), then (bf16)
+      // their rounding residuals in the next 16
+      float ls[4] = {l * alpha, 0.f, 0.f, 0.f};
+#pragma unroll 1
       for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32];
+        tc::ld32(tS + 32 * c, sv);
+        tc::wait_ld();
+        tc::pin(sv);
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float a = ex2(fmaf(__uint_as_float(sr[c][2 * i]), sl2, -m_ref));
-          const float e = ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, -m_ref));
+          const bool m0 = masked && 32 * c + 2 * i > lim, m1 = masked && 32 * c + 2 * i + 1 > lim;
+          const float a = m0 ? 0.f : ex2(fmaf(__uint_as_float(sv[2 * i]), sl2, -m_ref));
+          const float e = m1 ? 0.f : ex2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -m_ref));
           ls[i % 4] += a + e;
           if constexpr (kSplit) {
             split2<true>(a, e, hi[i], lo[i]);
@@ -400,14 +468,15 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
             lo[i] = 0u;
           }
         }
-        tc::st16(tS + 16 * c, hi);
-        if constexpr (kSplit) tc::st16(tS + 64 + 16 * c, lo);
+        tc::st16(tS + 32 * c, hi);
+        if constexpr (kSplit) tc::st16(tS + 32 * c + 16, lo);
       }
       l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tc::wait_st();
-      if (j == ntiles - 1 && kend - j * kPfKeys < kPfKeys) {
-        // last tile: zero the V rows past the keys read (stale slots may hold
-        // any bits, and 0 * NaN is NaN)
+      if (j == nt - 1 && kend - j * kPfKeys < kPfKeys) {
+        // this tile's last K/V tile: zero the V rows past every key the CTA
+        // reads (stale slots may hold any bits, and 0 * NaN is NaN); both
+        // query tiles may write the same zeros
         const int st = j % STAGES;
         ok = __all_sync(0xffffffffu, pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err));
         if (!ok) break;
@@ -423,17 +492,14 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         __syncwarp();
       }
       tc::fence_before();
-      mbar_arrive(PF(b));
+      mbar_arrive(PF(x));
     }
-    if (ok) {
-      const int jl = ntiles - 1;
-      ok = __all_sync(0xffffffffu, pf::wait(PV(jl & 1), (jl >> 1) & 1, abort_flag, p.err));
-    }
-    if (ok) {
+    if (ok && nt > 0) ok = __all_sync(0xffffffffu, pf::wait(PV(x), (nt - 1) & 1, abort_flag, p.err));
+    if (ok && nt > 0) {
       tc::fence_after();
       const float inv = 1.f / l;
-      const int64_t orow = ((int64_t)(q0 + t0 + tok) * p.num_q_heads + kvh * g + head) * D;
-#pragma unroll
+      const int64_t orow = ((int64_t)(q0 + t0 + x * tq + tok) * p.num_q_heads + kvh * g + head) * D;
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tc::ld32(tO + 32 * c, o);
@@ -449,13 +515,12 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
           } else {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + 32 * c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 4; ++i)
               dst[i] = make_uint4(
                   pack2<kBf16>(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
                   pack2<kBf16>(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
                   pack2<kBf16>(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
                   pack2<kBf16>(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
-            }
           }
         }
         __syncwarp();
@@ -466,7 +531,7 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   // TMEM is released once every role is done with it
   tc::fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     __syncwarp();
     tc::fence_after();
     tc::dealloc(tmem, kPfTmemCols);

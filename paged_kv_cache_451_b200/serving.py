@@ -76,7 +76,10 @@ class DecodeLoop:
         self.done_ev = [None, None]  # kernels reading buffer k finished
         self.side = torch.cuda.Stream(device=device)
         self.it = 0
-        ws = paged_attention_workspace_bytes(pool, max_batch, num_q_heads, max_context)
+        # the split policy partitions more finely when fewer sequences run, so
+        # the scratch is sized for the largest need over every batch size
+        ws = max(paged_attention_workspace_bytes(pool, b, num_q_heads, max_context)
+                 for b in range(1, max_batch + 1))
         self.ws_cap = max(ws, 16)
         self.d_ws = torch.empty(self.ws_cap, dtype=torch.uint8, device=device)
 
