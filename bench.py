@@ -183,6 +183,9 @@ class Case:
         self.L = w.num_layers
         self.k, self.v, self.ks, self.vs = [], [], [], []
         self.pool = pk.kv_pool_create(w.block_size, nb, w.kv_heads, w.head_dim, w.kv_fmt, self.L)
+        self.window = int(w.extra.get("window", 0))
+        if self.window:
+            pk.kv_pool_set_sliding_window(self.pool, self.window)
         for layer in range(self.L):
             k, v, ks, vs = device_pool(w, nb, dev, seed=seed + 13 * layer)
             self.k.append(k)
@@ -216,7 +219,9 @@ class Case:
         self.split = self.ws_bytes > 0
         e_kv, e_q = ELEM[w.kv_fmt], ELEM[w.q_fmt]
         blocks_touched = int(blocks_needed(self.lens, w.block_size).sum())
-        self.decode_bytes = self.L * (int(self.lens.astype(np.int64).sum()) * Hkv * D * 2 * e_kv
+        # attended tokens per sequence: the whole context, or the window
+        self.attended = np.minimum(self.lens, self.window) if self.window else self.lens
+        self.decode_bytes = self.L * (int(self.attended.astype(np.int64).sum()) * Hkv * D * 2 * e_kv
                                       + B * Hq * D * (e_q + e_q)
                                       + (2 * 4 * blocks_touched * Hkv if w.kv_fmt == 2 else 0))
         self.write_bytes = self.L * B * Hkv * D * 2 * (e_q + e_kv)
@@ -552,6 +557,8 @@ def describe(w, case=None):
         "kv_example": "KV-size example: 32 layers x 32 heads x head_dim 128, bf16, block 16, batch 32, ctx 2048",
         "gqa_trace": "GQA 64/8 heads, head_dim 128, bf16, block 16, batch 256, lognormal ctx (median 1024, cap 8192)",
         "fp8_long": "long-context FP8: 32 MHA heads, head_dim 128, E4M3 cache + per-(block,head) scales, bf16 q, batch 8, ctx 16384",
+        "window_long": "sliding-window decode: 32 MHA heads, head_dim 128, bf16, batch 8, ctx 16384, window 4096 "
+                       "(bytes counted over the window)",
         "rag_trace": "retrieval-augmented serving: GQA 64/8 heads, head_dim 128, bf16, block 16, 8192-block pool, "
                      "Poisson arrivals (3/iteration) of 2 shared 1536-token documents + U[32,256]-token questions, "
                      "U[16,64] output tokens, up to 128 running",
@@ -890,8 +897,12 @@ def cpu_baseline(case, torch, target_s=15.0, steps=1):
     # calibrate on one sequence, then size the sample to ~target_s
     t0 = time.perf_counter()
     args = oracle_sample(case, order[:1])
-    oracle.paged_decode(args[0], args[1], w.kv_fmt, args[4], w.q_fmt, args[5], args[6], w.scale,
-                        w.block_size, args[2], args[3])
+    if case.window:
+        oracle.paged_prefill(args[0], args[1], w.kv_fmt, args[4], w.q_fmt, np.arange(2, dtype=np.int32),
+                             args[5], args[6], w.scale, w.block_size, args[2], args[3], window=case.window)
+    else:
+        oracle.paged_decode(args[0], args[1], w.kv_fmt, args[4], w.q_fmt, args[5], args[6], w.scale,
+                            w.block_size, args[2], args[3])
     one = max(time.perf_counter() - t0, 1e-3)
     n = int(min(w.batch, max(1, target_s / one / max(1, case.L))))
     seqs = order[:n]
@@ -902,9 +913,16 @@ def cpu_baseline(case, torch, target_s=15.0, steps=1):
         for layer in range(case.L):
             kh, vh, ks, vs, q, sub, lens = samples[0] if samples else oracle_sample(case, seqs, layer)
             t0 = time.perf_counter()
-            oracle.paged_decode(kh, vh, w.kv_fmt, q, w.q_fmt, sub, lens, w.scale, w.block_size, ks, vs)
+            if case.window:
+                cu = np.arange(len(lens) + 1, dtype=np.int32)
+                oracle.paged_prefill(kh, vh, w.kv_fmt, q, w.q_fmt, cu, sub, lens, w.scale, w.block_size, ks,
+                                     vs, window=case.window)
+                att = np.minimum(lens, case.window)
+            else:
+                oracle.paged_decode(kh, vh, w.kv_fmt, q, w.q_fmt, sub, lens, w.scale, w.block_size, ks, vs)
+                att = lens
             total_s += time.perf_counter() - t0
-            total_bytes += (int(lens.astype(np.int64).sum()) * w.kv_heads * w.head_dim * 2 * ELEM[w.kv_fmt]
+            total_bytes += (int(att.astype(np.int64).sum()) * w.kv_heads * w.head_dim * 2 * ELEM[w.kv_fmt]
                             + n * w.num_q_heads * w.head_dim * 2 * ELEM[w.q_fmt])
         passes += 1
         if n < w.batch:
@@ -987,7 +1005,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama13b",
-                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long", "rag_trace",
+                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long", "window_long", "rag_trace",
                              *PREFILL_WORKLOADS])
     ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")

@@ -180,10 +180,10 @@ typedef struct {
  * block table ([PA]): token t lives in physical block bt[s][t / block_size]
  * at offset t % block_size.  Values are decoded exactly and, for FP8, times
  * the (block, head) scale.  Returns 0, or -1 on a block id outside the pool. */
-static int gather(const oracle_decode_args* a, const void* pool, const float* scales,
-                  int s, int kvh, int n, double* rows) {
+static int gather_from(const oracle_decode_args* a, const void* pool, const float* scales,
+                       int s, int kvh, int t_first, int n, double* rows) {
   int D = a->head_dim, bs = a->block_size;
-  for (int t = 0; t < n; ++t) {
+  for (int t = t_first; t < n; ++t) {
     int32_t blk = a->block_tables[(int64_t)s * a->max_blocks + t / bs];
     if (blk < 0 || blk >= a->num_blocks) return -1;
     int off = t % bs;
@@ -193,6 +193,11 @@ static int gather(const oracle_decode_args* a, const void* pool, const float* sc
     for (int d = 0; d < D; ++d) rows[(int64_t)t * D + d] = elem(pool, a->kv_dtype, base + d) * sc;
   }
   return 0;
+}
+
+static int gather(const oracle_decode_args* a, const void* pool, const float* scales,
+                  int s, int kvh, int n, double* rows) {
+  return gather_from(a, pool, scales, s, kvh, 0, n, rows);
 }
 
 static double qval(const oracle_decode_args* a, int s, int h, int d) {
@@ -390,8 +395,11 @@ static int prefill_one(const oracle_decode_args* a, const int32_t* cu_q, int win
   double* z = (double*)malloc(sizeof(double) * (size_t)n);
   int rc = 0;
   if (!K || !V || !z) { rc = -2; goto done; }
-  if (gather(a, a->k_pool, a->k_scale, s, h / g, n, K) ||
-      gather(a, a->v_pool, a->v_scale, s, h / g, n, V)) {
+  /* positions before the first row's window are never read (with a sliding
+   * window their blocks may already be released) */
+  int t_first = (window > 0 && n - q_len - window + 1 > 0) ? n - q_len - window + 1 : 0;
+  if (gather_from(a, a->k_pool, a->k_scale, s, h / g, t_first, n, K) ||
+      gather_from(a, a->v_pool, a->v_scale, s, h / g, t_first, n, V)) {
     rc = -1;
     goto done;
   }

@@ -204,3 +204,19 @@ def test_empty_sequences_and_error_cases():
     bad[1, 0] = kp.shape[0]
     with pytest.raises(ValueError):
         oracle.paged_prefill(kp, vp, F16, q, F16, cu, bad, np.array(lens), 0.5, 16)
+
+
+def test_window_reads_no_block_before_it():
+    """With a window, blocks wholly before the first row's window may be
+    released (table entry -1): the result is unchanged."""
+    rng = np.random.default_rng(22)
+    lens, q_lens, bs = [70, 41], [1, 3], 16
+    _, _, kp, vp, tables, cu, q = make_prefill(rng, lens, q_lens, 4, 2, 16, bs, BF16)
+    full = oracle.paged_prefill(kp, vp, BF16, q, BF16, cu, tables, np.array(lens), 0.3, bs, window=20)
+    cut = tables.copy()
+    for s, (n, ql) in enumerate(zip(lens, q_lens)):
+        first = max(0, n - ql - 20 + 1)
+        cut[s, :first // bs] = -1
+    assert (cut < 0).sum() > (tables < 0).sum()
+    got = oracle.paged_prefill(kp, vp, BF16, q, BF16, cu, cut, np.array(lens), 0.3, bs, window=20)
+    assert np.array_equal(full, got)

@@ -22,6 +22,8 @@ Workloads (sizes from the configurations the library is measured on):
                 sequences sharing a 1024-token prefix, 100-iteration trace.
 * ``fp8_long``  32 MHA heads, head_dim 128, batch 8, context 16384, E4M3 cache
                 with one fp32 scale per (block, kv head), bf16 queries.
+* ``window_long`` 32 MHA heads, head_dim 128, bf16, batch 8, context 16384,
+                sliding window of 4096 tokens (decode reads only the window).
 * ``prefill_llama13b`` / ``prefill_gqa``  multi-token attention over whole
                 prompts: 16 prompts of lengths uniform in [64, 2048] (the
                 trace's arrival range), Llama-2-13B layer shape (fp16) or the
@@ -86,6 +88,9 @@ WORKLOADS = {
                                  "pool_factor": 1.25}),
     "fp8_long": Workload("fp8_long", 4, 1, 32, 32, 128, 16, E4M3, BF16, 8,
                          extra={"ctx": 16384, "pool_factor": 1.25}),
+    # sliding-window decode over long contexts
+    "window_long": Workload("window_long", 9, 1, 32, 32, 128, 16, BF16, BF16, 8,
+                            extra={"ctx": 16384, "window": 4096, "pool_factor": 1.25}),
     # multi-token attention (prompts and prompt chunks)
     "prefill_llama13b": Workload("prefill_llama13b", 5, 1, 40, 40, 128, 16, F16, F16, 16,
                                  extra={"new_lo": 64, "new_hi": 2048, "prior_lo": 0, "prior_hi": 0,
@@ -130,7 +135,7 @@ def context_lens(w: Workload) -> np.ndarray:
         return np.asarray(w.extra["cached_lens"], dtype=np.int32) + 1
     if w.name == "llama13b":
         return r.integers(w.extra["ctx_lo"], w.extra["ctx_hi"] + 1, size=w.batch).astype(np.int32)
-    if w.name in ("kv_example", "fp8_long"):
+    if w.name in ("kv_example", "fp8_long", "window_long"):
         return np.full(w.batch, w.extra["ctx"], dtype=np.int32)
     if w.name == "gqa_trace":
         x = r.lognormal(math.log(w.extra["median"]), w.extra["sigma"], size=w.batch)
