@@ -62,6 +62,9 @@ enum {
   KV_ERR_TIMEOUT = -6  /* device-reported: a pipeline wait gave up (bounded spin) */
 };
 
+/* Preemption modes of the scheduling step (kv_sched_set_preemption). */
+typedef enum { KV_PREEMPT_NONE = 0, KV_PREEMPT_SWAP = 1, KV_PREEMPT_RECOMPUTE = 2 } kv_preempt_mode;
+
 typedef struct kv_pool kv_pool;
 typedef struct kv_alloc kv_alloc;
 typedef struct kv_sched kv_sched;
@@ -247,6 +250,26 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
                             const int32_t* context_lens, int batch, float scale, void* out,
                             kv_dtype out_dtype, kv_stream_t stream);
 
+/* Bytes one host swap slot holds: for every layer, K then V, each the
+ * block's kv_heads x block_size x head_dim elements followed (FP8) by its
+ * kv_heads fp32 scales padded to 16 bytes. */
+size_t kv_swap_block_bytes(const kv_pool* pool);
+
+/* Swap copies for preemption, over the host link: the kernel reads or
+ * writes the host swap space directly.  host_swap: pinned host memory
+ * mapped into the device (e.g. cudaHostAlloc / a pinned torch tensor),
+ * num_slots x kv_swap_block_bytes, 16-byte aligned.  pairs: device int32
+ * [num_pairs][2], (device block, host slot) for kv_swap_out and (host slot,
+ * device block) for kv_swap_in; every layer, K, V and FP8 scales move.  An
+ * index out of range is skipped and reported as KV_ERR_BOUNDS by
+ * kv_get_device_error.  Asynchronous on `stream`.  Errors: KV_ERR_ARG (host
+ * memory not mapped, misaligned), KV_ERR_STATE (layer not bound),
+ * KV_ERR_CUDA. */
+int kv_swap_out(const kv_pool* pool, void* host_swap, int num_slots, const int32_t* pairs,
+                int num_pairs, kv_stream_t stream);
+int kv_swap_in(const kv_pool* pool, const void* host_swap, int num_slots, const int32_t* pairs,
+               int num_pairs, kv_stream_t stream);
+
 /* Largest scratch paged_attention_decode_noalloc can use (16 MiB). */
 #define KV_NOALLOC_WORKSPACE_BYTES (16u << 20)
 
@@ -377,6 +400,10 @@ int kv_alloc_append_token(kv_alloc* a, int64_t seq_id, int32_t token, int64_t* s
  * may be NULL. */
 int kv_alloc_commit(kv_alloc* a, int64_t seq_id, int* num_registered);
 
+/* Host swap space of num_slots block slots (FIFO free list), for the
+ * scheduler's swap preemption.  KV_ERR_STATE while a sequence is swapped out. */
+int kv_alloc_set_swap_space(kv_alloc* a, int num_slots);
+
 /* Sliding window: release every block of seq_id wholly before position
  * `token` (blocks 0 .. token / block_size - 1 not yet released); their table
  * entries become -1 so logical block indices stay put.  Shared blocks only
@@ -447,6 +474,39 @@ int kv_sched_outputs(const kv_sched* s, int64_t* running_ids, int32_t* block_tab
  * block tables then hold -1 for released entries.  0 (the default) keeps
  * every block.  KV_ERR_ARG for a negative window. */
 int kv_sched_set_window(kv_sched* s, int window);
+
+/* Preemption when the KV cache runs out ("vLLM 推理加速原理详解" names
+ * preemption and swapping as what an undersized cache leads to; the
+ * mechanism is this library's reading).  With a mode other than
+ * KV_PREEMPT_NONE, each step first checks that the running set's appends fit
+ * the free blocks; while they do not, the most recently scheduled running
+ * sequence is preempted:
+ *   KV_PREEMPT_SWAP: every block it holds alone moves to a host swap slot
+ *     (kv_alloc_set_swap_space) and its device block is freed; blocks it
+ *     shares stay, with its reference; it waits at the front of a swapped
+ *     queue.  If the swap space lacks room it is recomputed instead.
+ *   KV_PREEMPT_RECOMPUTE: its blocks are freed and it goes back to the front
+ *     of the waiting queue with its whole context as the prompt.
+ * In a step without preemption, swapped sequences come back first (first in,
+ * first out) while their host-held blocks fit with the admission reserve;
+ * new requests are admitted only when none is swapped out and nothing was
+ * preempted in the step.  The caller runs
+ * kv_swap_out for the step's swap-out pairs, then kv_swap_in for its swap-in
+ * pairs, before the step's other kernels.  KV_PREEMPT_NONE (default): the
+ * step fails with KV_ERR_OOM when the appends do not fit. */
+int kv_sched_set_preemption(kv_sched* s, int mode);
+
+/* Sizes of the last step's swap outputs, and the number of sequences now
+ * swapped out (any pointer may be NULL). */
+int kv_sched_swap_info(const kv_sched* s, int* num_swap_out, int* num_swap_in, int* num_preempted,
+                       int* num_recomputed, int* num_swapped_in, int* num_swapped);
+
+/* The last step's swap outputs (any pointer may be NULL):
+ * swap_out_pairs[num_swap_out][2] (device block, host slot),
+ * swap_in_pairs[num_swap_in][2] (host slot, device block), the ids swapped
+ * out, recomputed (requeued) and swapped back in. */
+int kv_sched_swap_outputs(const kv_sched* s, int32_t* swap_out_pairs, int32_t* swap_in_pairs,
+                          int64_t* preempted_ids, int64_t* recomputed_ids, int64_t* swapped_in_ids);
 
 /* Cached prompt tokens of each request admitted by the last step, in the
  * order of admitted_ids (0 without prefix caching). */

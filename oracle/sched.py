@@ -71,6 +71,7 @@ class BlockManager:
         self.num_cow = 0
         self.num_alloc = 0
         self.num_freed = 0
+        self.host_free = deque()
 
     # verbs named on the page
     def get_num_free_blocks(self) -> int:
@@ -103,6 +104,9 @@ class BlockManager:
         if seq_id not in self.tables:
             raise OracleStateError(f"sequence {seq_id} is unknown")
         for b in self.tables.pop(seq_id):
+            if b <= -2:  # held in the host swap space
+                self.host_free.append(-b - 2)
+                continue
             if b < 0:  # already released (sliding window)
                 continue
             if self.refcount[b] <= 0:
@@ -171,6 +175,58 @@ class BlockManager:
             n += 1
         return n
 
+    # ------------------------------------------------ swapping (preemption)
+    # Reading taken (the pages only name "preemption and swapping" as what
+    # happens when the KV cache runs out): a swapped-out sequence moves every
+    # block it holds alone to a slot of a host swap space (FIFO free list of
+    # slots) and returns the device block; a block it shares stays on the
+    # device with its reference kept.  Its table entry for a host-held block
+    # is -(2 + slot).  Swapping in takes fresh device blocks for those entries.
+
+    def set_swap_space(self, num_slots: int) -> None:
+        self.host_free = deque(range(int(num_slots)))
+
+    def swap_out_cost(self, seq_id: int) -> int:
+        return sum(1 for b in self.tables[seq_id] if b >= 0 and self.refcount[b] == 1)
+
+    def swap_in_cost(self, seq_id: int) -> int:
+        return sum(1 for b in self.tables[seq_id] if b <= -2)
+
+    def swap_out(self, seq_id: int):
+        """[(device block, host slot)] moved to host; device blocks freed."""
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        table = self.tables[seq_id]
+        if self.swap_out_cost(seq_id) > len(getattr(self, "host_free", ())):
+            raise OracleOOM("not enough host swap slots")
+        pairs = []
+        for i, b in enumerate(table):
+            if b >= 0 and self.refcount[b] == 1:
+                slot = self.host_free.popleft()
+                pairs.append((b, slot))
+                self.refcount[b] = 0
+                self.free_list.append(b)
+                self.num_freed += 1
+                table[i] = -(2 + slot)
+        return pairs
+
+    def swap_in(self, seq_id: int):
+        """[(host slot, device block)] brought back into fresh blocks."""
+        if seq_id not in self.tables:
+            raise OracleStateError(f"sequence {seq_id} is unknown")
+        table = self.tables[seq_id]
+        if self.swap_in_cost(seq_id) > len(self.free_list):
+            raise OracleOOM("not enough free blocks")
+        pairs = []
+        for i, b in enumerate(table):
+            if b <= -2:
+                slot = -b - 2
+                nb = self._take()
+                pairs.append((slot, nb))
+                self.host_free.append(slot)
+                table[i] = nb
+        return pairs
+
     def block_table(self, seq_id: int) -> list[int]:
         if seq_id not in self.tables:
             raise OracleStateError(f"sequence {seq_id} is unknown")
@@ -192,6 +248,10 @@ class Scheduler:
         # before its last `window` positions (sliding-window decode reads no
         # earlier block); one admitted in this step keeps them until the next
         self.window = window
+        # preemption when the running set's appends do not fit: None (the
+        # step fails), "swap" or "recompute"
+        self.preemption = None
+        self.swapped: deque[int] = deque()
         self.waiting: deque[tuple[int, int]] = deque()
         self.running: list[int] = []
 
@@ -221,6 +281,41 @@ class Scheduler:
         self.running = [r for r in self.running if r not in finished]
         for sid in finished_ids:
             self.bm.free(int(sid))
+        # (1b) preemption (reading taken; the pages only name it): while the
+        # running set's appends do not fit, the most recently scheduled
+        # running sequence leaves, swapped out (its exclusive blocks to host
+        # slots; it waits at the front of the swapped queue) or, without room
+        # in the swap space or in recompute mode, freed and put back at the
+        # front of the waiting queue with its whole context as the prompt
+        swap_out, swap_in, preempted, recomputed, swapped_in = [], [], [], [], []
+        if self.preemption is not None:
+            while self.running and self._append_need(self.running) > self.bm.get_num_free_blocks():
+                victim = self.running.pop()
+                if (self.preemption == "swap"
+                        and self.bm.swap_out_cost(victim) <= len(getattr(self.bm, "host_free", ()))):
+                    swap_out += self.bm.swap_out(victim)
+                    self.swapped.appendleft(victim)
+                    preempted.append(victim)
+                else:
+                    n = self.bm.tokens[victim]
+                    toks = getattr(self.bm, "seq_tokens", {}).get(victim)
+                    toks = list(toks) if toks is not None and len(toks) == n else None
+                    self.bm.free(victim)
+                    self.waiting.appendleft((victim, n, toks))
+                    recomputed.append(victim)
+            # (1c) swapped sequences come back first (first in, first out),
+            # each if its host-held blocks fit with the reserve left free;
+            # not in a step that preempted (nor is anything admitted then)
+            while (not preempted and not recomputed and self.swapped
+                   and len(self.running) < self.max_num_seqs):
+                sid = self.swapped[0]
+                reserve = self._min_blocks() + (1 if self.min_blocks is None else 0)
+                if self.bm.swap_in_cost(sid) + reserve > self.bm.get_num_free_blocks():
+                    break
+                self.swapped.popleft()
+                swap_in += self.bm.swap_in(sid)
+                self.running.append(sid)
+                swapped_in.append(sid)
         # (2) free block count
         free_blocks = self.bm.get_num_free_blocks()
         # (3) admit waiting requests, first come first served
@@ -228,8 +323,8 @@ class Scheduler:
         cached = []
         prompt_slots = []
         caching = isinstance(self.bm, PrefixCachingBlockManager)
-        while (self.waiting and free_blocks > self._min_blocks()
-               and len(self.running) < self.max_num_seqs):
+        while (self.waiting and not self.swapped and not preempted and not recomputed
+               and free_blocks > self._min_blocks() and len(self.running) < self.max_num_seqs):
             sid, plen, toks = self.waiting[0]
             reserve = self._min_blocks() + (1 if self.min_blocks is None else 0)
             use_cache = caching and toks is not None
@@ -272,7 +367,28 @@ class Scheduler:
             "cow_pairs": cow,
             "admitted": admitted,
             "cached": cached,
+            "swap_out": swap_out,
+            "swap_in": swap_in,
+            "preempted": preempted,
+            "recomputed": recomputed,
+            "swapped_in": swapped_in,
         }
+
+    def _append_need(self, seqs) -> int:
+        """Fresh blocks the appends of `seqs` take: one per sequence at a
+        block boundary, plus the copies of shared partly filled last blocks
+        (at most refcount - 1 per block)."""
+        bs = self.bm.block_size
+        need, shared = 0, {}
+        for sid in seqs:
+            n, last = self.bm.tokens[sid], self.bm.tables[sid][-1] if self.bm.tables[sid] else -1
+            if n % bs == 0:
+                need += 1
+            elif self.bm.refcount[last] > 1:
+                shared[last] = shared.get(last, 0) + 1
+        for b, k in shared.items():
+            need += min(k, self.bm.refcount[b] - 1)
+        return need
 
     def stats(self):
         used = self.bm.num_blocks - self.bm.get_num_free_blocks()
@@ -437,6 +553,9 @@ class PrefixCachingBlockManager(BlockManager):
         if seq_id not in self.tables:
             raise OracleStateError(f"sequence {seq_id} is unknown")
         for b in reversed(self.tables.pop(seq_id)):
+            if b <= -2:
+                self.host_free.append(-b - 2)
+                continue
             if b < 0:
                 continue
             if self.refcount[b] <= 0:

@@ -15,6 +15,7 @@ import os
 from . import build as _build
 
 KV_F16, KV_BF16, KV_FP8_E4M3, KV_F32 = 0, 1, 2, 3
+KV_PREEMPT_NONE, KV_PREEMPT_SWAP, KV_PREEMPT_RECOMPUTE = 0, 1, 2
 KV_OK, KV_ERR_ARG, KV_ERR_OOM, KV_ERR_STATE, KV_ERR_BOUNDS, KV_ERR_CUDA, KV_ERR_TIMEOUT = (
     0, -1, -2, -3, -4, -5, -6)
 ERROR_NAMES = {0: "KV_OK", -1: "KV_ERR_ARG", -2: "KV_ERR_OOM", -3: "KV_ERR_STATE",
@@ -63,6 +64,13 @@ _SIGS = {
     "kv_pool_set_sliding_window": (c_int, [c_void_p, c_int]),
     "kv_alloc_release_before": (c_int, [c_void_p, c_int64, c_int64, P(c_int)]),
     "kv_sched_set_window": (c_int, [c_void_p, c_int]),
+    "kv_alloc_set_swap_space": (c_int, [c_void_p, c_int]),
+    "kv_sched_set_preemption": (c_int, [c_void_p, c_int]),
+    "kv_sched_swap_info": (c_int, [c_void_p, P(c_int), P(c_int), P(c_int), P(c_int), P(c_int), P(c_int)]),
+    "kv_sched_swap_outputs": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "kv_swap_block_bytes": (c_size_t, [c_void_p]),
+    "kv_swap_out": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p]),
+    "kv_swap_in": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p]),
     "kv_pool_destroy": (c_int, [c_void_p]),
     "paged_kv_write": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_int,
                                c_void_p, c_void_p, c_void_p]),
@@ -191,6 +199,40 @@ def kv_alloc_release_before(a, seq_id, token) -> int:
 
 def kv_sched_set_window(s, window):
     _check(_lib.kv_sched_set_window(s, int(window)))
+
+
+def kv_alloc_set_swap_space(a, num_slots):
+    _check(_lib.kv_alloc_set_swap_space(a, int(num_slots)))
+
+
+def kv_sched_set_preemption(s, mode):
+    _check(_lib.kv_sched_set_preemption(s, int(mode)))
+
+
+def kv_sched_swap_outputs(s):
+    """Last step's swap outputs as numpy arrays (dict) plus the count of
+    sequences now swapped out."""
+    import numpy as np
+    n = [c_int() for _ in range(6)]
+    _check(_lib.kv_sched_swap_info(s, *[ctypes.byref(x) for x in n]))
+    out = {"swap_out": np.empty((n[0].value, 2), np.int32), "swap_in": np.empty((n[1].value, 2), np.int32),
+           "preempted": np.empty(n[2].value, np.int64), "recomputed": np.empty(n[3].value, np.int64),
+           "swapped_in": np.empty(n[4].value, np.int64), "num_swapped": n[5].value}
+    _check(_lib.kv_sched_swap_outputs(s, _ptr(out["swap_out"]), _ptr(out["swap_in"]), _ptr(out["preempted"]),
+                                      _ptr(out["recomputed"]), _ptr(out["swapped_in"])))
+    return out
+
+
+def kv_swap_block_bytes(pool) -> int:
+    return int(_lib.kv_swap_block_bytes(pool))
+
+
+def kv_swap_out(pool, host_swap, num_slots, pairs, num_pairs, stream=None):
+    _check(_lib.kv_swap_out(pool, _ptr(host_swap), int(num_slots), _ptr(pairs), int(num_pairs), _stream(stream)))
+
+
+def kv_swap_in(pool, host_swap, num_slots, pairs, num_pairs, stream=None):
+    _check(_lib.kv_swap_in(pool, _ptr(host_swap), int(num_slots), _ptr(pairs), int(num_pairs), _stream(stream)))
 
 
 def kv_pool_destroy(pool):

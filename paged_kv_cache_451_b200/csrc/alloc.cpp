@@ -108,6 +108,9 @@ struct kv_alloc {
   std::unordered_map<uint64_t, int32_t> cached;
   std::vector<CachedBlock> key_of;
   int64_t n_hits = 0, n_evict = 0;
+  // host swap space: FIFO free list of slots; a table entry -(2 + slot)
+  // marks a block held in a host slot
+  std::deque<int32_t> host_free;
 
   int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
 
@@ -182,6 +185,70 @@ struct kv_alloc {
     s.tokens = pos + 1;
     *slot = (int64_t)s.blocks[pos / block_size] * block_size + pos % block_size;
     return KV_OK;
+  }
+
+  int64_t swap_out_cost(const SeqState& st) const {
+    int64_t c = 0;
+    for (int32_t b : st.blocks) c += (b >= 0 && refcount[b] == 1) ? 1 : 0;
+    return c;
+  }
+
+  int64_t swap_in_cost(const SeqState& st) const {
+    int64_t c = 0;
+    for (int32_t b : st.blocks) c += b <= -2 ? 1 : 0;
+    return c;
+  }
+
+  // Move every block the sequence holds alone to a host slot; shared blocks
+  // stay on the device with the reference kept.  Pairs (device, slot).
+  void swap_out(SeqState& st, std::vector<int32_t>* pairs) {
+    for (auto& b : st.blocks) {
+      if (b >= 0 && refcount[b] == 1) {
+        const int32_t slot = host_free.front();
+        host_free.pop_front();
+        pairs->push_back(b);
+        pairs->push_back(slot);
+        refcount[b] = 0;
+        push_back(b);
+        ++n_freed;
+        b = -(2 + slot);
+      }
+    }
+  }
+
+  // Fresh device blocks for the host-held entries.  Pairs (slot, device).
+  void swap_in(SeqState& st, std::vector<int32_t>* pairs) {
+    for (auto& b : st.blocks) {
+      if (b <= -2) {
+        const int32_t slot = -b - 2;
+        const int32_t nb = take();
+        pairs->push_back(slot);
+        pairs->push_back(nb);
+        host_free.push_back(slot);
+        b = nb;
+      }
+    }
+  }
+
+  // Fresh blocks the appends of `seqs` take: one per sequence at a block
+  // boundary, plus the copies of shared partly filled last blocks (at most
+  // refcount - 1 per block).
+  int64_t append_need(const std::vector<int64_t>& ids) {
+    int64_t need = 0;
+    std::unordered_map<int32_t, int64_t> shared;
+    for (int64_t r : ids) {
+      const SeqState& st = seqs[r];
+      if (st.tokens % block_size == 0) {
+        ++need;
+      } else if (refcount[st.blocks.back()] > 1) {
+        ++shared[st.blocks.back()];
+      }
+    }
+    for (auto& kv : shared) {
+      const int64_t copies = refcount[kv.first] - 1;
+      need += kv.second < copies ? kv.second : copies;
+    }
+    return need;
   }
 
   // Blocks of the longest registered prefix of `tokens`, at most
@@ -339,11 +406,15 @@ int kv_alloc_free(kv_alloc* a, int64_t seq_id) {
   if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
   const auto& blocks = it->second.blocks;
   if (a->caching) {  // deepest block first: shared prefixes leave the cache last
-    for (auto r = blocks.rbegin(); r != blocks.rend(); ++r)
+    for (auto r = blocks.rbegin(); r != blocks.rend(); ++r) {
       if (*r >= 0) a->release(*r);
+      else if (*r <= -2) a->host_free.push_back(-*r - 2);
+    }
   } else {
-    for (int32_t b : blocks)
+    for (int32_t b : blocks) {
       if (b >= 0) a->release(b);
+      else if (b <= -2) a->host_free.push_back(-b - 2);
+    }
   }
   a->seqs.erase(it);
   return ok();
@@ -388,6 +459,16 @@ int kv_alloc_enable_prefix_caching(kv_alloc* a) {
   if (!a) return fail(KV_ERR_ARG, "NULL allocator");
   if (!a->seqs.empty()) return fail(KV_ERR_STATE, "enable prefix caching before any sequence exists");
   a->caching = true;
+  return ok();
+}
+
+int kv_alloc_set_swap_space(kv_alloc* a, int num_slots) {
+  if (!a || num_slots < 0) return fail(KV_ERR_ARG, "bad argument");
+  for (const auto& kv : a->seqs)
+    for (int32_t b : kv.second.blocks)
+      if (b <= -2) return fail(KV_ERR_STATE, "a sequence is swapped out");
+  a->host_free.clear();
+  for (int i = 0; i < num_slots; ++i) a->host_free.push_back(i);
   return ok();
 }
 
@@ -490,6 +571,10 @@ struct kv_sched {
   int max_num_seqs = 0;
   int min_blocks = -1;
   int window = 0;  // > 0: release blocks that left the window after each step
+  int preemption = KV_PREEMPT_NONE;
+  std::deque<int64_t> swapped;
+  std::vector<int32_t> out_swap_out, out_swap_in;  // flattened pairs
+  std::vector<int64_t> out_preempted, out_recomputed, out_swapped_in;
   std::deque<Request> waiting;
   std::vector<int64_t> running;
   // outputs of the last step
@@ -569,6 +654,11 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   s->out_cow.clear();
   s->out_admitted.clear();
   s->out_cached.clear();
+  s->out_swap_out.clear();
+  s->out_swap_in.clear();
+  s->out_preempted.clear();
+  s->out_recomputed.clear();
+  s->out_swapped_in.clear();
 
   // (1) drop finished requests, return their blocks
   std::vector<int64_t> keep;
@@ -578,13 +668,55 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   s->running.swap(keep);
   for (int i = 0; i < n_finished; ++i) kv_alloc_free(a, finished_ids[i]);
 
+  // (1b) preemption: while the running set's appends do not fit, the most
+  // recently scheduled running sequence leaves: swapped out (its exclusive
+  // blocks to host slots; front of the swapped queue) or, without room in the
+  // swap space or in recompute mode, freed and put back at the front of the
+  // waiting queue with its whole context as the prompt
+  if (s->preemption != KV_PREEMPT_NONE) {
+    while (!s->running.empty() && a->append_need(s->running) > a->n_free) {
+      const int64_t victim = s->running.back();
+      s->running.pop_back();
+      SeqState& st = a->seqs[victim];
+      if (s->preemption == KV_PREEMPT_SWAP && a->swap_out_cost(st) <= (int64_t)a->host_free.size()) {
+        a->swap_out(st, &s->out_swap_out);
+        s->swapped.push_front(victim);
+        s->out_preempted.push_back(victim);
+      } else {
+        const int n = (int)st.tokens;
+        const bool known = (int64_t)st.toks.size() == st.tokens;
+        std::vector<int32_t> toks = known ? st.toks : std::vector<int32_t>();
+        kv_alloc_free(a, victim);
+        s->waiting.push_front({victim, n, known, std::move(toks)});
+        s->out_recomputed.push_back(victim);
+      }
+    }
+    // (1c) swapped sequences come back first, first in first out, each if
+    // its host-held blocks fit with the reserve left free; not in a step
+    // that preempted
+    while (s->out_preempted.empty() && s->out_recomputed.empty() && !s->swapped.empty() &&
+           (int)s->running.size() < s->max_num_seqs) {
+      const int64_t sid = s->swapped.front();
+      SeqState& st = a->seqs[sid];
+      const int64_t reserve = s->min_blocks_now() + (s->min_blocks < 0 ? 1 : 0);
+      if (a->swap_in_cost(st) + reserve > a->n_free) break;
+      s->swapped.pop_front();
+      a->swap_in(st, &s->out_swap_in);
+      s->running.push_back(sid);
+      s->out_swapped_in.push_back(sid);
+    }
+  }
+
   // (2) free block count
   int64_t free_blocks = a->n_free;
 
   // (3) admit first come first served
   std::vector<int64_t> prompt_slots;
   std::vector<int32_t> hits;
-  while (!s->waiting.empty() && free_blocks > s->min_blocks_now() &&
+  // nothing is admitted while a sequence is swapped out or in a step that
+  // preempted
+  while (!s->waiting.empty() && s->swapped.empty() && s->out_preempted.empty() &&
+         s->out_recomputed.empty() && free_blocks > s->min_blocks_now() &&
          (int)s->running.size() < s->max_num_seqs) {
     const Request& req = s->waiting.front();
     const bool use_cache = a->caching && req.has_tokens;
@@ -616,20 +748,7 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
 
   // (4) one slot per running sequence; check the whole batch fits first
   {
-    int64_t need = 0;
-    std::unordered_map<int32_t, int64_t> shared_appenders;
-    for (int64_t r : s->running) {
-      const SeqState& st = a->seqs[r];
-      if (st.tokens % a->block_size == 0) {
-        ++need;
-      } else if (a->refcount[st.blocks.back()] > 1) {
-        ++shared_appenders[st.blocks.back()];
-      }
-    }
-    for (auto& kv : shared_appenders) {
-      int64_t copies = a->refcount[kv.first] - 1;
-      need += kv.second < copies ? kv.second : copies;
-    }
+    const int64_t need = a->append_need(s->running);
     if (need > a->n_free) {
       info->batch = (int)s->running.size();
       info->num_tokens = info->num_cow = 0;
@@ -701,6 +820,36 @@ int kv_sched_stats(const kv_sched* s, int* running, int* waiting, int* used_bloc
   if (waiting) *waiting = (int)s->waiting.size();
   if (used_blocks) *used_blocks = s->a->num_blocks - (int)s->a->n_free;
   if (total_blocks) *total_blocks = s->a->num_blocks;
+  return ok();
+}
+
+int kv_sched_set_preemption(kv_sched* s, int mode) {
+  if (!s || (mode != KV_PREEMPT_NONE && mode != KV_PREEMPT_SWAP && mode != KV_PREEMPT_RECOMPUTE))
+    return fail(KV_ERR_ARG, "bad argument");
+  s->preemption = mode;
+  return ok();
+}
+
+int kv_sched_swap_info(const kv_sched* s, int* num_swap_out, int* num_swap_in, int* num_preempted,
+                       int* num_recomputed, int* num_swapped_in, int* num_swapped) {
+  if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
+  if (num_swap_out) *num_swap_out = (int)s->out_swap_out.size() / 2;
+  if (num_swap_in) *num_swap_in = (int)s->out_swap_in.size() / 2;
+  if (num_preempted) *num_preempted = (int)s->out_preempted.size();
+  if (num_recomputed) *num_recomputed = (int)s->out_recomputed.size();
+  if (num_swapped_in) *num_swapped_in = (int)s->out_swapped_in.size();
+  if (num_swapped) *num_swapped = (int)s->swapped.size();
+  return ok();
+}
+
+int kv_sched_swap_outputs(const kv_sched* s, int32_t* swap_out_pairs, int32_t* swap_in_pairs,
+                          int64_t* preempted_ids, int64_t* recomputed_ids, int64_t* swapped_in_ids) {
+  if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
+  if (swap_out_pairs) std::copy(s->out_swap_out.begin(), s->out_swap_out.end(), swap_out_pairs);
+  if (swap_in_pairs) std::copy(s->out_swap_in.begin(), s->out_swap_in.end(), swap_in_pairs);
+  if (preempted_ids) std::copy(s->out_preempted.begin(), s->out_preempted.end(), preempted_ids);
+  if (recomputed_ids) std::copy(s->out_recomputed.begin(), s->out_recomputed.end(), recomputed_ids);
+  if (swapped_in_ids) std::copy(s->out_swapped_in.begin(), s->out_swapped_in.end(), swapped_in_ids);
   return ok();
 }
 

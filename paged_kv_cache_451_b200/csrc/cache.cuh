@@ -118,6 +118,57 @@ __global__ void __launch_bounds__(256) block_copy_kernel(const CopyParams p) {
       sc[(int64_t)dst * p.kv_heads + h] = sc[(int64_t)src * p.kv_heads + h];
 }
 
+// Swap copies between device blocks and a host swap space (pinned host
+// memory mapped into the device address space, written / read directly by
+// the kernel over the host link).  A slot holds, per layer, K then V:
+// block_bytes of data followed (FP8) by the block's kv_heads scales, padded
+// to 16 bytes.  kOut: device block -> slot; else slot -> device block.
+struct SwapParams {
+  const int32_t* pairs;  // [num_pairs][2]: (device block, slot) out, (slot, device block) in
+  int num_pairs;
+  int num_blocks;
+  int num_slots;
+  int kv_heads;
+  int layer0;            // first layer of this launch
+  int num_layers;        // all layers of the pool
+  int64_t block_bytes;
+  int64_t per_bytes;     // block_bytes + padded scale bytes
+  uint8_t* host;         // device-accessible base of the swap space
+  void* k[kCopyLayers];
+  void* v[kCopyLayers];
+  float* ks[kCopyLayers];
+  float* vs[kCopyLayers];
+};
+
+// grid = (num_pairs, layers in this launch, 2 for K and V)
+template <bool kOut>
+__global__ void __launch_bounds__(256) swap_kernel(const SwapParams p) {
+  const int pi = blockIdx.x;
+  const int li = blockIdx.y;
+  const bool is_v = blockIdx.z == 1;
+  const int32_t dev = kOut ? p.pairs[2 * pi] : p.pairs[2 * pi + 1];
+  const int32_t slot = kOut ? p.pairs[2 * pi + 1] : p.pairs[2 * pi];
+  if (dev < 0 || dev >= p.num_blocks || slot < 0 || slot >= p.num_slots) {
+    if (threadIdx.x == 0) record_error(KV_ERR_BOUNDS);
+    return;
+  }
+  const int layer = p.layer0 + li;
+  uint8_t* hb = p.host + ((int64_t)slot * p.num_layers * 2 + layer * 2 + (is_v ? 1 : 0)) * p.per_bytes;
+  uint8_t* db = static_cast<uint8_t*>(is_v ? p.v[li] : p.k[li]) + (int64_t)dev * p.block_bytes;
+  const int64_t n16 = p.block_bytes / 16;
+  uint4* d = reinterpret_cast<uint4*>(kOut ? hb : db);
+  const uint4* s = reinterpret_cast<const uint4*>(kOut ? db : hb);
+  for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) d[i] = s[i];
+  float* sc = is_v ? p.vs[li] : p.ks[li];
+  if (sc != nullptr) {
+    float* hs = reinterpret_cast<float*>(hb + p.block_bytes);
+    for (int h = threadIdx.x; h < p.kv_heads; h += blockDim.x) {
+      if (kOut) hs[h] = sc[(int64_t)dev * p.kv_heads + h];
+      else sc[(int64_t)dev * p.kv_heads + h] = hs[h];
+    }
+  }
+}
+
 // Self-test of the bounded-wait error path used by the decode pipeline: one
 // warp waits on an mbarrier whose phase can never complete (a transaction
 // count that no copy will satisfy).  After limit_ns the wait gives up, the

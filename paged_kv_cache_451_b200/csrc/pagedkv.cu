@@ -479,6 +479,67 @@ int block_copy(const kv_pool* pool, const int32_t* pairs, int num_pairs, kv_stre
   return ok();
 }
 
+size_t kv_swap_block_bytes(const kv_pool* pool) {
+  if (!pool) return 0;
+  const size_t scales = pool->dtype == KV_FP8_E4M3 ? ((size_t)pool->kv_heads * 4 + 15) / 16 * 16 : 0;
+  return (size_t)pool->num_layers * 2 * (pool->block_bytes() + scales);
+}
+
+static int swap_copy(const kv_pool* pool, const void* host_swap, int num_slots, const int32_t* pairs,
+                     int num_pairs, bool out, kv_stream_t stream) {
+  if (!pool) return fail(KV_ERR_ARG, "NULL pool");
+  if (num_pairs < 0 || num_slots < 0) return fail(KV_ERR_ARG, "negative size");
+  if (num_pairs == 0) return ok();
+  if (!pairs || !host_swap) return fail(KV_ERR_ARG, "NULL argument");
+  if ((uintptr_t)host_swap & 15) return fail(KV_ERR_ARG, "host swap space must be 16-byte aligned");
+  for (int l = 0; l < pool->num_layers; ++l)
+    if (!pool->layers[l].bound) return fail(KV_ERR_STATE, "layer %d is not bound", l);
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, host_swap);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+  if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr)
+    return fail(KV_ERR_ARG, "host swap space must be pinned host memory mapped into the device");
+  const int64_t scales = pool->dtype == KV_FP8_E4M3 ? ((int64_t)pool->kv_heads * 4 + 15) / 16 * 16 : 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int l0 = 0; l0 < pool->num_layers; l0 += kCopyLayers) {
+    const int nl = std::min(kCopyLayers, pool->num_layers - l0);
+    SwapParams p;
+    std::memset(&p, 0, sizeof p);
+    p.pairs = pairs;
+    p.num_pairs = num_pairs;
+    p.num_blocks = pool->num_blocks;
+    p.num_slots = num_slots;
+    p.kv_heads = pool->kv_heads;
+    p.layer0 = l0;
+    p.num_layers = pool->num_layers;
+    p.block_bytes = (int64_t)pool->block_bytes();
+    p.per_bytes = p.block_bytes + scales;
+    p.host = static_cast<uint8_t*>(attr.devicePointer);
+    for (int i = 0; i < nl; ++i) {
+      const LayerBinding& lb = pool->layers[l0 + i];
+      p.k[i] = lb.k;
+      p.v[i] = lb.v;
+      p.ks[i] = lb.k_scale;
+      p.vs[i] = lb.v_scale;
+    }
+    if (out) swap_kernel<true><<<dim3(num_pairs, nl, 2), 256, 0, s>>>(p);
+    else swap_kernel<false><<<dim3(num_pairs, nl, 2), 256, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "swap_kernel launch");
+  }
+  return ok();
+}
+
+int kv_swap_out(const kv_pool* pool, void* host_swap, int num_slots, const int32_t* pairs,
+                int num_pairs, kv_stream_t stream) {
+  return swap_copy(pool, host_swap, num_slots, pairs, num_pairs, true, stream);
+}
+
+int kv_swap_in(const kv_pool* pool, const void* host_swap, int num_slots, const int32_t* pairs,
+               int num_pairs, kv_stream_t stream) {
+  return swap_copy(pool, host_swap, num_slots, pairs, num_pairs, false, stream);
+}
+
 size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
                                        int max_context_len) {
   if (!pool || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
