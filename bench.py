@@ -38,6 +38,7 @@ METRIC = "paged decode attention: achieved KV-read GB/s (% of HBM peak); decode 
 METRIC_PREFILL = "paged multi-token attention: achieved TFLOP/s (% of tensor peak); new tokens/s"
 PREFILL_WORKLOADS = ("prefill_llama13b", "prefill_gqa", "chunked_gqa")
 METRIC_RAG = "retrieval-augmented serving with prefix caching: generated tokens/s (vs no caching)"
+METRIC_PREEMPT = "decode under memory pressure with swap preemption: generated tokens/s (vs recompute)"
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {0: "f16", 1: "bf16", 2: "e4m3"}
@@ -550,6 +551,125 @@ def run_rag(args, rank, world, local_rank):
     }
 
 
+def swap_copy_bandwidth(torch, pk, blocks=1024):
+    """kv_swap_out / kv_swap_in of `blocks` blocks (GQA 8 heads, bf16, block
+    16, head_dim 128) against a plain pinned-host cudaMemcpyAsync of the same
+    bytes in each direction (the copy-engine reference), CUDA events."""
+    nb, hkv, bs, d = blocks * 2, 8, 16, 128
+    pool = pk.kv_pool_create(bs, nb, hkv, d, pk.KV_BF16, 1)
+    k = torch.zeros((nb, hkv, bs, d), dtype=torch.int16, device="cuda")
+    v = torch.zeros_like(k)
+    pk.kv_pool_bind(pool, 0, k, v)
+    slot = pk.kv_swap_block_bytes(pool)
+    host = torch.zeros(blocks * slot, dtype=torch.uint8).pin_memory()
+    dev_buf = torch.zeros(blocks * slot, dtype=torch.uint8, device="cuda")
+    out_pairs = torch.stack([torch.arange(0, nb, 2), torch.arange(blocks)], 1).to(torch.int32).cuda()
+    in_pairs = torch.stack([torch.arange(blocks), torch.arange(1, nb, 2)], 1).to(torch.int32).cuda()
+    res = {}
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    nbytes = blocks * slot
+    res["swap_out_gbs"] = nbytes / (timed(lambda: pk.kv_swap_out(pool, host, blocks, out_pairs, blocks)) * 1e-3) / 1e9
+    res["swap_in_gbs"] = nbytes / (timed(lambda: pk.kv_swap_in(pool, host, blocks, in_pairs, blocks)) * 1e-3) / 1e9
+    res["memcpy_d2h_gbs"] = nbytes / (timed(lambda: host.copy_(dev_buf, non_blocking=True)) * 1e-3) / 1e9
+    res["memcpy_h2d_gbs"] = nbytes / (timed(lambda: dev_buf.copy_(host, non_blocking=True)) * 1e-3) / 1e9
+    res["bytes_per_call"] = nbytes
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error in the swap copies")
+    pk.kv_pool_destroy(pool)
+    return {k2: (round(v2, 2) if isinstance(v2, float) else v2) for k2, v2 in res.items()}
+
+
+def run_preempt(args, rank, world, local_rank):
+    """The memory-pressure trace with swap and with recompute preemption: one
+    step = one iteration (scheduler step, metadata upload, swap copies,
+    copy-on-write, cache write, decode)."""
+    import torch
+    import paged_kv_cache_451_b200 as pk
+    from workloads import WORKLOADS
+    from workloads.preempt_trace import PreemptTrace, preempt_plan
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = WORKLOADS["preempt_trace"]
+    plan = preempt_plan(w)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    iters = w.extra["iters"]
+    W = min(args.warmup, iters - 1)
+    K = max(1, min(args.steps, iters - W))
+    res = {}
+    for mode in ("swap", "recompute"):
+        tr = PreemptTrace(w, plan, mode=mode, seed=rank)
+        for it in range(W):
+            tr.iteration(it)
+        torch.cuda.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        gen = pre = rec = swapped_blocks = rewritten = 0
+
+        def gate_and_start(i):
+            torch.cuda._sleep(2_000_000)  # keep the GPU fed while the host enqueues
+            starts[i].record(stream)
+
+        with ClockSampler(local_rank) as clk:
+            for i in range(K):
+                flush.zero_()
+                fin, arr, pl, *_ = tr.iteration(W + i, before_launch=lambda: gate_and_start(i),
+                                               after_launch=lambda: ends[i].record(stream))
+                gen += pl["info"].batch
+                pre += len(pl["preempted"])
+                rec += len(pl["recomputed"])
+                swapped_blocks += len(pl["swap_out"]) + len(pl["swap_in"])
+                rewritten += pl["info"].num_tokens
+            torch.cuda.synchronize()
+        if pk.kv_get_device_error() != pk.KV_OK:
+            raise RuntimeError("device error during the trace")
+        total_ms = max_over_ranks(sum(starts[i].elapsed_time(ends[i]) for i in range(K)), dist, "cuda")
+        res[mode] = {"tokens_per_s": world * gen / (total_ms * 1e-3), "ms_per_step": total_ms / K,
+                     "preempted": pre, "recomputed": rec, "swapped_blocks": swapped_blocks,
+                     "written_tokens": rewritten, "clocks": clk.summary()}
+    swap_bw = swap_copy_bandwidth(torch, pk) if rank == 0 else None
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    sw, rc = res["swap"], res["recompute"]
+    return {
+        "metric": METRIC_PREEMPT, "value": round(sw["tokens_per_s"], 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(sw["ms_per_step"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded prompt / output lengths and Poisson arrivals; q/K/V drawn on device)",
+        "config": {"workload": describe(w), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between iterations (256 MiB write)",
+                   "step": "one iteration: scheduler step (preemption, swap-in), metadata upload, swap copies, "
+                           "copy-on-write, cache write, decode"},
+        "swap": {k2: (round(v2, 3) if isinstance(v2, float) else v2) for k2, v2 in sw.items() if k2 != "clocks"},
+        "recompute": {k2: (round(v2, 3) if isinstance(v2, float) else v2) for k2, v2 in rc.items() if k2 != "clocks"},
+        "swap_copy": swap_bw,
+        "roofline": None if swap_bw is None else {
+            "bound": "host link", "kernel": "kv_swap_out (swap_kernel, device to pinned host)",
+            "achieved": swap_bw["swap_out_gbs"], "peak": swap_bw["memcpy_d2h_gbs"], "unit": "GB/s",
+            "frac": round(swap_bw["swap_out_gbs"] / swap_bw["memcpy_d2h_gbs"], 4), "traffic": None,
+            "peak_note": "pinned cudaMemcpyAsync device-to-host of the same bytes, measured in this run"},
+        "clocks": sw["clocks"],
+    }
+
+
 def describe(w, case=None):
     names = {
         "tiny": "tiny: 1 layer, 4 seqs ctx {2,18,34,101}, 4 MHA heads, head_dim 64, block 16, fp16",
@@ -559,6 +679,9 @@ def describe(w, case=None):
         "fp8_long": "long-context FP8: 32 MHA heads, head_dim 128, E4M3 cache + per-(block,head) scales, bf16 q, batch 8, ctx 16384",
         "window_long": "sliding-window decode: 32 MHA heads, head_dim 128, bf16, batch 8, ctx 16384, window 4096 "
                        "(bytes counted over the window)",
+        "preempt_trace": "decode under memory pressure: GQA 64/8 heads, head_dim 128, bf16, block 16, 3000-block pool, "
+                         "64 initial sequences (prompts U[256,1024]) + Poisson arrivals (0.5/iteration), U[100,400] "
+                         "output tokens, swap space 6000 host blocks",
         "rag_trace": "retrieval-augmented serving: GQA 64/8 heads, head_dim 128, bf16, block 16, 8192-block pool, "
                      "Poisson arrivals (3/iteration) of 2 shared 1536-token documents + U[32,256]-token questions, "
                      "U[16,64] output tokens, up to 128 running",
@@ -1006,6 +1129,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama13b",
                     choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long", "window_long", "rag_trace",
+                             "preempt_trace",
                              *PREFILL_WORKLOADS])
     ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")
@@ -1029,6 +1153,8 @@ def main():
         line = run_prefill(args, rank, world, local_rank)
     elif args.workload == "rag_trace":
         line = run_rag(args, rank, world, local_rank)
+    elif args.workload == "preempt_trace":
+        line = run_preempt(args, rank, world, local_rank)
     else:
         line = run_ours(args, rank, world, local_rank)
     if rank == 0 and line is not None:

@@ -8,8 +8,10 @@ the order of the scheduling loop on "vLLM æŽ¨ç†åŠ é€ŸåŽŸç†è¯¦è§£ï¼šå¤§æ¨¡åž‹æœ
    waiting requests first come first served, append one slot per running
    sequence (copy-on-write pairs where a shared block is written);
 2. upload the step's metadata (block tables, context lengths, slots,
-   scheduling order, copy pairs) with one async copy from a pinned buffer;
-3. ``block_copy`` for the copy-on-write pairs;
+   scheduling order, copy and swap pairs) with one async copy from a pinned
+   buffer;
+3. ``kv_swap_out`` / ``kv_swap_in`` for preempted and resumed sequences,
+   then ``block_copy`` for the copy-on-write pairs;
 4. ``paged_kv_write`` of the step's new tokens (admitted prompts' uncached
    tokens, then one token per running sequence);
 5. optionally ``paged_attention_prefill`` over the admitted prompts' uncached
@@ -23,8 +25,9 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import (KV_F32, block_copy, kv_sched_outputs, kv_sched_step, paged_attention_decode,
-               paged_attention_prefill, paged_attention_workspace_bytes, paged_kv_write)
+from . import (KV_F32, block_copy, kv_sched_outputs, kv_sched_step, kv_sched_swap_outputs, kv_swap_in,
+               kv_swap_out, paged_attention_decode, paged_attention_prefill,
+               paged_attention_workspace_bytes, paged_kv_write)
 
 
 def schedule_order(context_lens, policy="long_first"):
@@ -60,7 +63,7 @@ class DecodeLoop:
 
     def __init__(self, pool, sched, *, num_q_heads, kv_heads, head_dim, block_size, q_dtype,
                  scale, max_batch, max_blocks, max_tokens, max_context, device="cuda",
-                 order_policy="batch"):
+                 order_policy="batch", host_swap=None, swap_slots=0):
         import torch
         self.torch = torch
         self.pool, self.sched = pool, sched
@@ -68,7 +71,10 @@ class DecodeLoop:
         self.q_dtype, self.scale = q_dtype, scale
         self.max_batch, self.max_blocks, self.max_tokens = max_batch, max_blocks, max_tokens
         self.order_policy = order_policy
+        self.host_swap, self.swap_slots = host_swap, swap_slots
         cap = 8 * max_tokens + 4 * (max_batch * max_blocks + 6 * max_batch + 1) + 256
+        if swap_slots:
+            cap += 16 * swap_slots + 64
         self.cap = (cap + 255) // 256 * 256
         self.h_buf = [torch.empty(self.cap, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
         self.d_buf = [torch.empty(self.cap, dtype=torch.uint8, device=device) for _ in range(2)]
@@ -89,15 +95,16 @@ class DecodeLoop:
         if info.batch > self.max_batch or info.num_tokens > self.max_tokens:
             raise RuntimeError("step exceeds the loop's buffers")
         out = kv_sched_outputs(self.sched, info, self.max_blocks)
+        out.update(kv_sched_swap_outputs(self.sched))
         out["info"] = info
         return out
 
     @staticmethod
-    def _layout(b, t, c, width, a=0):
+    def _layout(b, t, c, width, a=0, so=0, si=0):
         off, lay = 0, {}
         for name, n, size in (("slots", t, 8), ("tables", b * width, 4), ("lens", b, 4),
                               ("order", b, 4), ("cow", 2 * c, 4), ("cu", a + 1 if a else 0, 4),
-                              ("pf_lens", a, 4)):
+                              ("pf_lens", a, 4), ("swo", 2 * so, 4), ("swi", 2 * si, 4)):
             lay[name] = (off, n)
             off += (n * size + 15) // 16 * 16
         return lay, off
@@ -122,9 +129,13 @@ class DecodeLoop:
         info = plan["info"]
         b, t, c, w = info.batch, info.num_tokens, info.num_cow, self.max_blocks
         a, new, _ = self.prefill_sizes(plan) if prefill_q is not None else (0, None, None)
+        so = len(plan.get("swap_out", ()))
+        si = len(plan.get("swap_in", ()))
+        if (so or si) and self.host_swap is None:
+            raise RuntimeError("the step swaps but the loop has no host swap space")
         k = self.it % 2
         self.it += 1
-        lay, nbytes = self._layout(b, t, c, w, a)
+        lay, nbytes = self._layout(b, t, c, w, a, so, si)
         if nbytes > self.cap:
             raise RuntimeError("step metadata exceeds the loop's buffers")
         if self.copy_ev[k] is not None:  # the pinned buffer is reused: its last upload must be done
@@ -141,6 +152,10 @@ class DecodeLoop:
         put("lens", plan["context_lens"], np.int32)
         put("order", schedule_order(plan["context_lens"], self.order_policy), np.int32)
         put("cow", plan["cow_pairs"], np.int32)
+        if so:
+            put("swo", plan["swap_out"], np.int32)
+        if si:
+            put("swi", plan["swap_in"], np.int32)
         if a:
             put("cu", np.concatenate([[0], np.cumsum(new)]), np.int32)
             put("pf_lens", np.asarray(plan["context_lens"][-a:], np.int64) - 1, np.int32)
@@ -159,6 +174,10 @@ class DecodeLoop:
             return self.d_buf[k][off:off + n * (8 if dtype == torch.int64 else 4)].view(dtype)
 
         max_ctx = int(plan["context_lens"].max()) if b else 0
+        if so:  # before this step's writes can reuse the freed blocks
+            kv_swap_out(self.pool, self.host_swap, self.swap_slots, dview("swo", torch.int32), so, main)
+        if si:
+            kv_swap_in(self.pool, self.host_swap, self.swap_slots, dview("swi", torch.int32), si, main)
         if c:
             block_copy(self.pool, dview("cow", torch.int32), c, main)
         if t:

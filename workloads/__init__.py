@@ -30,6 +30,11 @@ Workloads (sizes from the configurations the library is measured on):
                 64/8 GQA shape (bf16).
 * ``chunked_gqa`` 16 sequences, each a 512-token prompt chunk on top of a
                 cached prefix of 512..4096 tokens, 64/8 GQA, bf16.
+* ``preempt_trace`` decode under memory pressure: 64 initial sequences
+                (prompts U[256,1024]) plus Poisson arrivals (0.5 per
+                iteration), U[100,400] output tokens, a 3000-block pool that
+                the running set outgrows; preempted sequences are swapped to
+                a 6000-slot host space or recomputed; 64/8 GQA, bf16.
 * ``rag_trace`` retrieval-augmented serving: Poisson arrivals (3 per
                 iteration, 60 iterations) whose prompt is one of 2 shared
                 1536-token documents plus a U[32,256]-token question, U[16,64]
@@ -101,6 +106,11 @@ WORKLOADS = {
     "chunked_gqa": Workload("chunked_gqa", 7, 1, 64, 8, 128, 16, BF16, BF16, 16,
                             extra={"new_lo": 512, "new_hi": 512, "prior_lo": 512, "prior_hi": 4096,
                                    "pool_factor": 1.25}),
+    # decode under memory pressure: sequences outgrow the pool and are preempted
+    "preempt_trace": Workload("preempt_trace", 10, 1, 64, 8, 128, 16, BF16, BF16, 64,
+                              extra={"prompt_lo": 256, "prompt_hi": 1024, "out_lo": 100, "out_hi": 400,
+                                     "arrival_rate": 0.5, "iters": 150, "max_num_seqs": 96,
+                                     "num_blocks": 3000, "swap_slots": 6000}),
     # retrieval-augmented requests: a shared document + a question each
     "rag_trace": Workload("rag_trace", 8, 1, 64, 8, 128, 16, BF16, BF16, 128,
                           extra={"docs": 2, "doc_len": 1536, "question_lo": 32, "question_hi": 256,
