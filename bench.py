@@ -74,16 +74,25 @@ def decode_source_hash():
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload):
-    """DRAM bytes per decode launch from a committed ncu capture, if it was
-    taken on the current decode source."""
+def prefill_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_451_b200", "csrc")
+    for f in ("prefill.cuh", "tcgen05.cuh", "ptx.cuh", "prefill.cu"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload, source_hash=None):
+    """DRAM bytes per launch of the workload's dominant kernel from a
+    committed ncu capture, if it was taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f).get(workload)
     except Exception:  # noqa: BLE001
         return None
-    if not rec or rec.get("source_hash") != decode_source_hash():
+    if not rec or rec.get("source_hash") != (source_hash or decode_source_hash()):
         return None
     return rec.get("bytes_per_launch")
 
@@ -898,7 +907,7 @@ def run_prefill(args, rank, world, local_rank):
             "peak": peak,
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None,
+            "traffic": committed_traffic(args.workload, prefill_source_hash()),
             "algorithmic_flops_per_launch": case.flops,
             "launch_ms": round(pf_avg, 5),
             "peak_note": f"{peak_kind} dense bf16 GEMM (cuBLAS, burst); f16 runs at the same rate",

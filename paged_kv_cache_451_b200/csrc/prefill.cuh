@@ -38,6 +38,7 @@
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "../../include/pagedkv.h"
 #include "ptx.cuh"
@@ -118,6 +119,13 @@ __device__ __forceinline__ bool probe(uint32_t bar, uint32_t parity) {
       : "r"(bar), "r"(parity)
       : "memory");
   return done != 0;
+}
+
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Wait for the phase with `parity`; give up when another role of the CTA
@@ -399,7 +407,9 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       tc::fence_after();
       const int lim = prow - j * kPfKeys;  // columns 0 .. lim are visible
       const bool masked = lim < kPfKeys - 1;
-      // pass 1: the row max
+      // pass 1: the row max.  Only tiles on the causal diagonal mask
+      // anything; a warp takes the masked code only when one of its rows needs it.
+      const bool wmask = __any_sync(0xffffffffu, masked);
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
@@ -410,13 +420,21 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         tc::wait_ld();
 #pragma unroll
         for (int c = 0; c < 4; ++c) tc::pin(sr[c]);
+        auto row_max = [&](auto kMask) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float v = (masked && 32 * c + i > lim) ? -INFINITY : __uint_as_float(sr[c][i]);
-            mx8[i % 8] = fmaxf(mx8[i % 8], v);
-          }
+            for (int i = 0; i < 32; i += 2) {
+              float v0 = __uint_as_float(sr[c][i]), v1 = __uint_as_float(sr[c][i + 1]);
+              if constexpr (decltype(kMask)::value) {
+                if (32 * c + i > lim) v0 = -INFINITY;
+                if (32 * c + i + 1 > lim) v1 = -INFINITY;
+              }
+              mx8[(i / 2) % 8] = pf::max3(mx8[(i / 2) % 8], v0, v1);
+            }
+        };
+        if (wmask) row_max(std::true_type{});
+        else row_max(std::false_type{});
       }
 #pragma unroll
       for (int w = 4; w > 0; w >>= 1)
@@ -448,29 +466,36 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       // 2i, 2i + 1 of the chunk in its column i (16 columns), then (bf16)
       // their rounding residuals in the next 16
       float ls[4] = {l * alpha, 0.f, 0.f, 0.f};
+      auto probs = [&](auto kMask) {
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32];
-        tc::ld32(tS + 32 * c, sv);
-        tc::wait_ld();
-        tc::pin(sv);
-        uint32_t hi[16], lo[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32];
+          tc::ld32(tS + 32 * c, sv);
+          tc::wait_ld();
+          tc::pin(sv);
+          uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const bool m0 = masked && 32 * c + 2 * i > lim, m1 = masked && 32 * c + 2 * i + 1 > lim;
-          const float a = m0 ? 0.f : ex2(fmaf(__uint_as_float(sv[2 * i]), sl2, -m_ref));
-          const float e = m1 ? 0.f : ex2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -m_ref));
-          ls[i % 4] += a + e;
-          if constexpr (kSplit) {
-            split2<true>(a, e, hi[i], lo[i]);
-          } else {
-            hi[i] = pack2<false>(a, e);
-            lo[i] = 0u;
+          for (int i = 0; i < 16; ++i) {
+            float a = ex2(fmaf(__uint_as_float(sv[2 * i]), sl2, -m_ref));
+            float e = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -m_ref));
+            if constexpr (decltype(kMask)::value) {
+              if (32 * c + 2 * i > lim) a = 0.f;
+              if (32 * c + 2 * i + 1 > lim) e = 0.f;
+            }
+            ls[i % 4] += a + e;
+            if constexpr (kSplit) {
+              split2<true>(a, e, hi[i], lo[i]);
+            } else {
+              hi[i] = pack2<false>(a, e);
+              lo[i] = 0u;
+            }
           }
+          tc::st16(tS + 32 * c, hi);
+          if constexpr (kSplit) tc::st16(tS + 32 * c + 16, lo);
         }
-        tc::st16(tS + 32 * c, hi);
-        if constexpr (kSplit) tc::st16(tS + 32 * c + 16, lo);
-      }
+      };
+      if (wmask) probs(std::true_type{});
+      else probs(std::false_type{});
       l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tc::wait_st();
       if (j == nt - 1 && kend - j * kPfKeys < kPfKeys) {
