@@ -1076,6 +1076,10 @@ def run_reference(args, rank, world):
     import paged_kv_cache_451_b200 as pk
     if args.workload in PREFILL_WORKLOADS:
         return run_reference_prefill(args, world, torch, pk)
+    if args.workload in ("gqa_trace", "rag_trace", "preempt_trace"):
+        return {"impl": "reference", "metric": METRIC, "workload": args.workload,
+                "unavailable": "the CPU oracle has no serving-trace leg (the GPU line reports the host "
+                               "scheduling time per iteration); time decode workloads instead"}
     case = Case(args.workload, 0, torch, pk, args)
     per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
