@@ -1076,7 +1076,7 @@ def run_reference(args, rank, world):
     import paged_kv_cache_451_b200 as pk
     if args.workload in PREFILL_WORKLOADS:
         return run_reference_prefill(args, world, torch, pk)
-    if args.workload in ("gqa_trace", "rag_trace", "preempt_trace"):
+    if args.workload in ("rag_trace", "preempt_trace"):
         return {"impl": "reference", "metric": METRIC, "workload": args.workload,
                 "unavailable": "the CPU oracle has no serving-trace leg (the GPU line reports the host "
                                "scheduling time per iteration); time decode workloads instead"}
