@@ -209,10 +209,11 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
  * window > 0, paged_attention_decode attends, for a sequence of n tokens,
  * only to its last min(n, window) tokens (positions n - window .. n - 1), and
  * reads no block before the one holding position n - window, so blocks that
- * left the window may be released (kv_alloc_release_before).  0 turns the
- * window off.  Workspace sizes follow the window.  paged_attention_prefill
- * rejects a pool with a window (KV_ERR_ARG).  Host only; KV_ERR_ARG for a
- * negative window. */
+ * left the window may be released (kv_alloc_release_before).
+ * paged_attention_prefill applies the same band to every new token (it
+ * attends to its own last `window` positions) and reads no block wholly
+ * before the first new token's window.  0 turns the window off.  Workspace
+ * sizes follow the window.  Host only; KV_ERR_ARG for a negative window. */
 int kv_pool_set_sliding_window(kv_pool* pool, int window);
 
 /* Multi-token attention over the paged cache: the step that processes a

@@ -138,8 +138,6 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
     return fail(KV_ERR_ARG, "multi-token attention needs an f16 or bf16 pool");
   if (pool->head_dim != 64 && pool->head_dim != 128)
     return fail(KV_ERR_ARG, "multi-token attention needs head_dim 64 or 128");
-  if (pool->window > 0)
-    return fail(KV_ERR_ARG, "multi-token attention over a sliding-window pool is not supported");
   if (q_dtype != pool->dtype) return fail(KV_ERR_ARG, "q dtype must equal the pool dtype");
   if (out_dtype != q_dtype && out_dtype != KV_F32)
     return fail(KV_ERR_ARG, "out dtype must be the q dtype or KV_F32");
@@ -185,6 +183,7 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
   p.num_blocks = pool->num_blocks;
   p.max_blocks = max_blocks_per_seq;
   p.total_q = total_q;
+  p.window = pool->window;
   p.scale_log2 = scale * 1.4426950408889634f;
 
   const dim3 grid((unsigned)pairs, pool->kv_heads, batch);

@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <climits>
 #include <cstdint>
 #include <type_traits>
 
@@ -75,6 +76,7 @@ struct PrefillParams {
   int num_blocks;
   int max_blocks;
   int total_q;
+  int window;                   // > 0: each token attends only to its last `window` positions
   float scale_log2;             // softmax scale * log2(e), > 0
 };
 
@@ -178,14 +180,18 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   }
   const int t0 = qp * kPfTiles * tq;  // first new token of query tile A
   if (t0 >= q_len) return;
+  // Key tiles start at kb: 0, or with a sliding window the 16-key chunk
+  // holding the first position any row of this CTA sees (no block before it
+  // is read: it may already be released).
+  const int kb = p.window > 0 ? max(0, n - q_len + t0 - p.window + 1) / 16 * 16 : 0;
   // per query tile X (A = 0, B = 1): tokens, key range, key tiles
   int ntok[kPfTiles], kendx[kPfTiles], ntx[kPfTiles];
 #pragma unroll
   for (int x = 0; x < kPfTiles; ++x) {
     const int tx = t0 + x * tq;
     ntok[x] = tx < q_len ? min(tq, q_len - tx) : 0;
-    kendx[x] = ntok[x] ? n - q_len + tx + ntok[x] : 0;  // keys 0 .. kend - 1
-    ntx[x] = (kendx[x] + kPfKeys - 1) / kPfKeys;
+    kendx[x] = ntok[x] ? n - q_len + tx + ntok[x] : 0;  // keys .. kend - 1
+    ntx[x] = ntok[x] ? (kendx[x] - kb + kPfKeys - 1) / kPfKeys : 0;
   }
   const int kend = max(kendx[0], kendx[1]);
   const int ntiles = max(ntx[0], ntx[1]);  // K/V tiles read (tile B's when it has tokens)
@@ -260,7 +266,7 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % STAGES;
         const uint32_t use = (uint32_t)(j / STAGES);
-        const int key0 = j * kPfKeys;
+        const int key0 = kb + j * kPfKeys;
         const int nch = min(KCH, (kend - key0 + 15) / 16);
         int blk[KCH], row[KCH];
         bool bad = false;
@@ -405,8 +411,9 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       ok = __all_sync(0xffffffffu, pf::wait(SF(x), j & 1, abort_flag, p.err));
       if (!ok) break;
       tc::fence_after();
-      const int lim = prow - j * kPfKeys;  // columns 0 .. lim are visible
-      const bool masked = lim < kPfKeys - 1;
+      const int lim = prow - kb - j * kPfKeys;  // columns wlo .. lim are visible
+      const int wlo = p.window > 0 ? lim - p.window + 1 : INT_MIN;
+      const bool masked = lim < kPfKeys - 1 || wlo > 0;
       // pass 1: the row max.  Only tiles on the causal diagonal mask
       // anything; a warp takes the masked code only when one of its rows needs it.
       const bool wmask = __any_sync(0xffffffffu, masked);
@@ -427,8 +434,8 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
             for (int i = 0; i < 32; i += 2) {
               float v0 = __uint_as_float(sr[c][i]), v1 = __uint_as_float(sr[c][i + 1]);
               if constexpr (decltype(kMask)::value) {
-                if (32 * c + i > lim) v0 = -INFINITY;
-                if (32 * c + i + 1 > lim) v1 = -INFINITY;
+                if (32 * c + i > lim || 32 * c + i < wlo) v0 = -INFINITY;
+                if (32 * c + i + 1 > lim || 32 * c + i + 1 < wlo) v1 = -INFINITY;
               }
               mx8[(i / 2) % 8] = pf::max3(mx8[(i / 2) % 8], v0, v1);
             }
@@ -479,8 +486,8 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
             float a = ex2(fmaf(__uint_as_float(sv[2 * i]), sl2, -m_ref));
             float e = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -m_ref));
             if constexpr (decltype(kMask)::value) {
-              if (32 * c + 2 * i > lim) a = 0.f;
-              if (32 * c + 2 * i + 1 > lim) e = 0.f;
+              if (32 * c + 2 * i > lim || 32 * c + 2 * i < wlo) a = 0.f;
+              if (32 * c + 2 * i + 1 > lim || 32 * c + 2 * i + 1 < wlo) e = 0.f;
             }
             ls[i % 4] += a + e;
             if constexpr (kSplit) {
@@ -498,14 +505,14 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       else probs(std::false_type{});
       l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tc::wait_st();
-      if (j == nt - 1 && kend - j * kPfKeys < kPfKeys) {
+      if (j == nt - 1 && kend - kb - j * kPfKeys < kPfKeys) {
         // this tile's last K/V tile: zero the V rows past every key the CTA
         // reads (stale slots may hold any bits, and 0 * NaN is NaN); both
         // query tiles may write the same zeros
         const int st = j % STAGES;
         ok = __all_sync(0xffffffffu, pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err));
         if (!ok) break;
-        if (r >= kend - j * kPfKeys) {
+        if (r >= kend - kb - j * kPfKeys) {
 #pragma unroll
           for (int h = 0; h < NH; ++h) {
             uint4* row = reinterpret_cast<uint4*>(smem + S::V_OFF + st * S::TILE + h * S::HALF + r * 128);

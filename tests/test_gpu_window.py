@@ -91,3 +91,42 @@ def test_window_off_restores_full_attention():
     assert max_abs(out.cpu().numpy(), ref) <= TOL[F16]
     with pytest.raises(pk.KVError):
         pk.kv_pool_set_sliding_window(pool.h, -1)
+
+
+def run_prefill_case(fmt, d, bs, hq, hkv, lens, q_lens, window, seed=0):
+    """Multi-token attention over a windowed pool; blocks wholly before each
+    sequence's first-row window are released (-1) and hold NaN bits."""
+    rng = np.random.default_rng(seed)
+    lens, q_lens = np.asarray(lens, np.int32), np.asarray(q_lens, np.int32)
+    nb = int(sum(-(-int(n) // bs) for n in lens)) + 3
+    shape = (nb, hkv, bs, d)
+    kh, vh = normal_bits(rng, shape, fmt), normal_bits(rng, shape, fmt)
+    tables = scattered_tables(rng, lens, bs, nb, pad_to=int(np.max(-(-lens // bs))) + 1)
+    for s, (n, ql) in enumerate(zip(lens, q_lens)):
+        first = max(0, int(n) - int(ql) - window + 1)
+        for i in range(first // bs):
+            kh[tables[s, i]] = NAN[fmt]
+            vh[tables[s, i]] = NAN[fmt]
+            tables[s, i] = -1
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q = normal_bits(rng, (int(cu[-1]), hq, d), fmt)
+    pool = DevicePool(nb, hkv, d, bs, fmt, k=[dev(kh)], v=[dev(vh)])
+    pk.kv_pool_set_sliding_window(pool.h, window)
+    out = torch.full((int(cu[-1]), hq, d), float("nan"), dtype=torch.float32, device="cuda")
+    pk.paged_attention_prefill(pool.h, 0, dev(q), fmt, hq, dev(cu), int(cu[-1]), int(q_lens.max()),
+                               dev(tables), tables.shape[1], dev(lens), len(lens), 1 / math.sqrt(d), out,
+                               pk.KV_F32)
+    torch.cuda.synchronize()
+    assert pk.kv_get_device_error() == pk.KV_OK
+    ref = oracle.paged_prefill(kh, vh, fmt, q, fmt, cu, tables, lens, 1 / math.sqrt(d), bs, window=window)
+    return out.cpu().numpy(), ref
+
+
+@pytest.mark.parametrize("window", [1, 16, 17, 100, 128, 129, 300, 2000])
+@pytest.mark.parametrize("fmt,d,hq,hkv", [(BF16, 128, 16, 2), (F16, 64, 4, 4)])
+def test_window_prefill_matches_oracle(window, fmt, d, hq, hkv):
+    lens = [1, 129, 700, 1500, 300]
+    q_lens = [1, 129, 300, 256, 1]  # whole prompts, chunks on cached prefixes, a decode row
+    out, ref = run_prefill_case(fmt, d, 16, hq, hkv, lens, q_lens, window, seed=window + d)
+    assert not np.isnan(out).any()
+    assert max_abs(out, ref) <= TOL[fmt]
