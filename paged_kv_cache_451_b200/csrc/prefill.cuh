@@ -12,25 +12,28 @@
 // position.
 //
 // Unlike decode, this is a real dense contraction, so it runs on the
-// fifth-generation tensor cores.  One CTA per (query tile, kv head,
-// sequence); a query tile is 128 rows = 128 / g new tokens x the g query
-// heads of one kv head's group, so each K/V tile read serves the whole group.
-// Per 128-key tile j, with S and O accumulated in tensor memory (TMEM):
+// fifth-generation tensor cores.  One CTA per (pair of query tiles A, B, kv
+// head, sequence), pairs with the most keys launched first; a query tile is
+// 128 rows = 128 / g new tokens x the g query heads of one kv head's group,
+// and both tiles share every K/V tile read.  Per 128-key tile j, with S and O
+// of each query tile in tensor memory (TMEM, 4 x 128 columns):
 //   S_j = Q . K_j^T          (tcgen05.mma, M 128, N 128, K = head_dim; Q and
 //                            K_j in shared memory, 128-byte swizzled, K-major)
-//   softmax rows in fp32 (one row per thread of warps 0-3, log2 domain, a
-//   lazily moved reference max, causal mask on the diagonal tiles); the
-//   probabilities P_j go back into S_j's TMEM columns as 16-bit values (bf16:
-//   value + rounding residual, about 16 significant bits together)
+//   softmax rows in fp32 (one row per thread, warps 0-3 tile A, 4-7 tile B;
+//   log2 domain, a lazily moved reference max, causal and sliding-window
+//   masks only on the tiles that need them); the probabilities P_j go back
+//   into S_j's TMEM columns as 16-bit values (bf16: value + rounding
+//   residual, about 16 significant bits together)
 //   O += P_j . V_j           (tcgen05.mma with A = P_j from TMEM, B = V_j from
 //                            shared memory, MN-major; bf16: once per half)
-// Warp 4 streams Q and the K/V tiles with 3-D TMA copies straight out of the
+// Warp 8 streams Q and the K/V tiles with 3-D TMA copies straight out of the
 // paged pool (one 16-row box per 16 keys and 64 columns, placed so the tile
-// lands in the canonical swizzled layout the MMA reads); warp 5 issues the
-// MMAs from one thread in the order S_0, S_1, PV_0, S_2, PV_1, ... so the
-// softmax of tile j+1 overlaps P_j . V_j and S_{j+2}.  Completion flows
-// through mbarriers (TMA transaction counts, tcgen05.commit, thread arrives);
-// every wait is bounded and aborts the CTA with KV_ERR_TIMEOUT.
+// lands in the canonical swizzled layout the MMA reads); warp 9 issues the
+// MMAs from one thread in the order S_A(0) S_B(0) PV_A(0) S_A(1) PV_B(0)
+// S_B(1) ..., so one tile's softmax runs while the tensor cores work on the
+// other's.  Completion flows through mbarriers (TMA transaction counts,
+// tcgen05.commit, thread arrives); every wait is bounded and aborts the CTA
+// with KV_ERR_TIMEOUT.
 #pragma once
 
 #include <cuda.h>
