@@ -319,6 +319,9 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the C ABI with host buffers (pinned), copies timed
     e2e = run_e2e(case, torch, pk, flush, stream, K, args.warmup)
+    e2e_ms = max_over_ranks(e2e["ms_per_step"] * K, dist, "cuda") / K
+    e2e["ms_per_step"] = round(e2e_ms, 5)
+    e2e["value"] = round(job_value(case.step_bytes, world, e2e_ms), 2)
     if pk.kv_get_device_error() != pk.KV_OK:
         raise RuntimeError("device error during timing")
 
@@ -702,54 +705,85 @@ def describe(w, case=None):
 
 
 def run_e2e(case, torch, pk, flush, stream, K, W):
-    """Same step, inputs from pinned host memory: H2D of q, new K/V, slots,
-    tables and lengths, then the write and decode, then D2H of the output."""
-    w = case.w
-    hq = [t.cpu().pin_memory() for t in case.q]
-    hk = [t.cpu().pin_memory() for t in case.kn]
-    hv = [t.cpu().pin_memory() for t in case.vn]
-    hs = torch.from_numpy(case.slots_h).pin_memory()
-    ht = torch.from_numpy(case.tables).pin_memory()
-    hl = torch.from_numpy(case.lens).pin_memory()
-    ho = torch.from_numpy(case.order_h).pin_memory()
-    hout = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in case.out]
-    dq = [torch.empty_like(t) for t in case.q]
-    dk = [torch.empty_like(t) for t in case.kn]
-    dv = [torch.empty_like(t) for t in case.vn]
-    ds, dt, dl = torch.empty_like(case.slots), torch.empty_like(case.tables_d), torch.empty_like(case.lens_d)
-    do = torch.empty_like(case.order_d)
-    h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv) + sum(
-        t.numel() * t.element_size() for t in (hs, ht, hl, ho))
-    d2h = sum(t.numel() * t.element_size() for t in hout)
+    """The same step through the C ABI from pinned host memory, pipelined the
+    way a serving loop runs it: each step's inputs (q, new K/V of every
+    layer, slots, tables, lengths, order) are packed in one pinned buffer and
+    uploaded with one copy on a copy stream into one of two device buffers,
+    the step's write + decode kernels wait for that upload, and the output
+    goes back to pinned host memory on the copy stream.  The upload of step
+    i + 1 overlaps the kernels of step i.  K steps are timed as one region
+    (CUDA events on the compute stream, every copy inside it).  The decode
+    reads more than L2 holds each step, so there is no flush in between."""
+    ins = list(case.q) + list(case.kn) + list(case.vn) + [case.slots, case.tables_d, case.lens_d, case.order_d]
+    offs, off = [], 0
+    for t in ins:
+        offs.append(off)
+        off += (t.numel() * t.element_size() + 255) // 256 * 256
+    h2d = sum(t.numel() * t.element_size() for t in ins)
+    hbuf = torch.empty(off, dtype=torch.uint8).pin_memory()
+    for t, o in zip(ins, offs):
+        n = t.numel() * t.element_size()
+        hbuf[o:o + n].copy_(t.contiguous().view(-1).view(torch.uint8).cpu())
+    dbuf = [torch.empty(off, dtype=torch.uint8, device="cuda") for _ in range(2)]
 
-    def step():
-        ds.copy_(hs, non_blocking=True)
-        dt.copy_(ht, non_blocking=True)
-        dl.copy_(hl, non_blocking=True)
-        do.copy_(ho, non_blocking=True)
-        for layer in range(case.L):
-            dq[layer].copy_(hq[layer], non_blocking=True)
-            dk[layer].copy_(hk[layer], non_blocking=True)
-            dv[layer].copy_(hv[layer], non_blocking=True)
-            case.write(layer, dk[layer], dv[layer], ds)
-            case.decode(layer, dq[layer], dt, dl, order=do)
-            hout[layer].copy_(case.out[layer], non_blocking=True)
+    def views(k):
+        out = []
+        for t, o in zip(ins, offs):
+            n = t.numel() * t.element_size()
+            out.append(dbuf[k][o:o + n].view(t.dtype).view(t.shape))
+        return out
 
-    for _ in range(W):
-        flush.zero_()
-        step()
+    dv = [views(k) for k in range(2)]
+    L = case.L
+    dout = [[torch.empty_like(o) for o in case.out] for _ in range(2)]
+    hout = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in case.out] for _ in range(2)]
+    d2h = sum(o.numel() * o.element_size() for o in case.out)
+    cs = torch.cuda.Stream()
+    up = [torch.cuda.Event() for _ in range(2)]
+    comp = [None, None]   # kernels that read device buffer k (and wrote dout[k])
+    down = [None, None]   # read-back of dout[k]
+
+    def step(i):
+        k = i % 2
+        with torch.cuda.stream(cs):
+            if comp[k] is not None:
+                cs.wait_event(comp[k])  # buffer k's previous readers are done
+            dbuf[k].copy_(hbuf, non_blocking=True)
+            up[k].record(cs)
+        stream.wait_event(up[k])
+        if down[k] is not None:
+            stream.wait_event(down[k])  # dout[k] was read back
+        v = dv[k]
+        for layer in range(L):
+            case.write(layer, v[L + layer], v[2 * L + layer], v[3 * L])
+            case.decode(layer, v[layer], v[3 * L + 1], v[3 * L + 2], out=dout[k][layer], order=v[3 * L + 3])
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        comp[k] = ev
+        with torch.cuda.stream(cs):
+            cs.wait_event(ev)
+            for layer in range(L):
+                hout[k][layer].copy_(dout[k][layer], non_blocking=True)
+            dn = torch.cuda.Event()
+            dn.record(cs)
+            down[k] = dn
+
+    for i in range(W):
+        step(i)
     torch.cuda.synchronize()
-    a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    cs.wait_event(a)  # the first upload starts inside the region
     for i in range(K):
-        flush.zero_()
-        a[i].record(stream)
-        step()
-        b[i].record(stream)
+        step(W + i)
+    stream.wait_event(down[(W + K - 1) % 2])  # the last read-back is inside the region
+    b.record(stream)
     torch.cuda.synchronize()
-    ms = sum(a[i].elapsed_time(b[i]) for i in range(K)) / K
+    ms = a.elapsed_time(b) / K
     return {"value": round(case.step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "ms_per_step": round(ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "ms_per_step": round(ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "mode": "pipelined: one packed upload per step on a copy stream (double-buffered), "
+                    "read-back of every step's output; K steps timed as one region"}
 
 
 # ------------------------------------------------------ multi-token leg
