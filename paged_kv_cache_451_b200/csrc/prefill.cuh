@@ -21,14 +21,19 @@
 //                            K_j in shared memory, 128-byte swizzled, K-major)
 //   softmax rows in fp32 (one row per thread, warps 0-3 tile A, 4-7 tile B;
 //   log2 domain, a lazily moved reference max, causal and sliding-window
-//   masks only on the tiles that need them); the probabilities P_j go back
-//   into S_j's TMEM columns as 16-bit values (bf16: value + rounding
-//   residual, about 16 significant bits together)
+//   masks only on the tiles that need them; pairs of keys through the
+//   .f32x2 add / fma; S read 16 columns at a time with the next 16 in
+//   flight); the probabilities P_j go back into S_j's TMEM columns as
+//   16-bit values (bf16: value + rounding residual, about 16 significant
+//   bits together)
 //   O += P_j . V_j           (tcgen05.mma with A = P_j from TMEM, B = V_j from
 //                            shared memory, MN-major; bf16: once per half)
 // Warp 8 streams Q and the K/V tiles with 3-D TMA copies straight out of the
 // paged pool (one 16-row box per 16 keys and 64 columns, placed so the tile
-// lands in the canonical swizzled layout the MMA reads); warp 9 issues the
+// lands in the canonical swizzled layout the MMA reads; each lane owns one
+// box of every tile, so a tile's copies go out in one instruction: issued
+// from a single thread they came out one every ~60 cycles and set the pace
+// of the whole pipeline); warp 9 issues the
 // MMAs from one thread in the order S_A(0) S_B(0) PV_A(0) S_A(1) PV_B(0)
 // S_B(1) ..., so one tile's softmax runs while the tensor cores work on the
 // other's.  Completion flows through mbarriers (TMA transaction counts,
@@ -124,6 +129,32 @@ __device__ __forceinline__ bool probe(uint32_t bar, uint32_t parity) {
       : "r"(bar), "r"(parity)
       : "memory");
   return done != 0;
+}
+
+// Two fp32 values in one 64-bit register pair: sm_100 executes add, sub and
+// fma on both halves with one instruction (.f32x2).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 // max of three (one instruction on sm_100)
@@ -253,69 +284,69 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
 
   if (warp == 8) {
     // ------------------------------------------------------------ copies
+    // The whole warp streams: lane c + KCH * h owns 16-key chunk c, column
+    // block h of every tile (its block id, its box), so one instruction puts
+    // a tile's NH * KCH box copies in flight; lane 0 sets the transaction
+    // counts.  Every lane takes the same waits and branches.
+    constexpr int NBOX = NH * KCH;  // 16 (head_dim 128) or 8 (64) boxes per tile
+    const int c = lane % KCH, h = lane / KCH;
+    const bool boxer = lane < NBOX;
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
       mbar_arrive_expect_tx(BQ, (uint32_t)(kPfTiles * NH * qrows * 128));
-#pragma unroll
-      for (int x = 0; x < kPfTiles; ++x)
-#pragma unroll
-        for (int h = 0; h < NH; ++h)
-          tma_load_3d(sbase + S::Q_OFF + x * S::TILE + h * S::HALF, &qmap, BQ, h * 64, kvh * g,
-                      q0 + t0 + x * tq);
-      const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks;
-      int nk = 0, nv = 0;  // tiles whose K (V) copies are in flight or done
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = j % STAGES;
-        const uint32_t use = (uint32_t)(j / STAGES);
-        const int key0 = kb + j * kPfKeys;
-        const int nch = min(KCH, (kend - key0 + 15) / 16);
-        int blk[KCH], row[KCH];
-        bool bad = false;
-#pragma unroll
-        for (int c = 0; c < KCH; ++c) {
-          blk[c] = 0;
-          row[c] = 0;
-          if (c < nch) {
-            const int key = key0 + 16 * c;
-            const int b = table[key / p.block_size];
-            bad |= b < 0 || b >= p.num_blocks;
-            blk[c] = b;
-            row[c] = kvh * p.block_size + key % p.block_size;
-          }
-        }
-        if (bad) {
+    }
+    __syncwarp();
+    if (lane < kPfTiles * NH)
+      tma_load_3d(sbase + S::Q_OFF + (lane / NH) * S::TILE + (lane % NH) * S::HALF, &qmap, BQ,
+                  (lane % NH) * 64, kvh * g, q0 + t0 + (lane / NH) * tq);
+    const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks;
+    int nk = 0, nv = 0;  // tiles whose K (V) copies are in flight or done
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j % STAGES;
+      const uint32_t use = (uint32_t)(j / STAGES);
+      const int key0 = kb + j * kPfKeys;
+      const int nch = min(KCH, (kend - key0 + 15) / 16);
+      const bool mine = boxer && c < nch;
+      int blk = 0, row = 0;
+      bool bad = false;
+      if (mine) {
+        const int key = key0 + 16 * c;
+        blk = table[key / p.block_size];
+        bad = blk < 0 || blk >= p.num_blocks;
+        row = kvh * p.block_size + key % p.block_size;
+      }
+      if (__any_sync(0xffffffffu, bad)) {
+        if (lane == 0) {
           atomicCAS(p.err, 0, KV_ERR_BOUNDS);
           *abort_flag = 1;
-          break;
         }
-        const uint32_t bytes = (uint32_t)(nch * NH * 16 * 128);
-        if (use > 0 && !pf::wait(KE(st), (use - 1) & 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(KF(st), bytes);
-        for (int c = 0; c < nch; ++c)
-#pragma unroll
-          for (int h = 0; h < NH; ++h)
-            tma_load_3d(sbase + S::K_OFF + st * S::TILE + h * S::HALF + c * 2048, &kmap, KF(st),
-                        h * 64, row[c], blk[c]);
-        nk = j + 1;
-        if (use > 0 && !pf::wait(VE(st), (use - 1) & 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(VF(st), bytes);
-        for (int c = 0; c < nch; ++c)
-#pragma unroll
-          for (int h = 0; h < NH; ++h)
-            tma_load_3d(sbase + S::V_OFF + st * S::TILE + h * S::HALF + c * 2048, &vmap, VF(st),
-                        h * 64, row[c], blk[c]);
-        nv = j + 1;
+        break;
       }
-      if (*abort_flag) {
-        // let the copies in flight land before the shared memory is released
-        for (int j = max(0, nk - STAGES); j < nk; ++j)
-          (void)mbar_wait_bounded(KF(j % STAGES), (j / STAGES) & 1, kPfDrainNs);
-        for (int j = max(0, nv - STAGES); j < nv; ++j)
-          (void)mbar_wait_bounded(VF(j % STAGES), (j / STAGES) & 1, kPfDrainNs);
-        (void)mbar_wait_bounded(BQ, 0, kPfDrainNs);
-      }
+      const uint32_t bytes = (uint32_t)(nch * NH * 16 * 128);
+      if (use > 0 && !__all_sync(0xffffffffu, pf::wait(KE(st), (use - 1) & 1, abort_flag, p.err))) break;
+      if (lane == 0) mbar_arrive_expect_tx(KF(st), bytes);
+      __syncwarp();
+      if (mine)
+        tma_load_3d(sbase + S::K_OFF + st * S::TILE + h * S::HALF + c * 2048, &kmap, KF(st), h * 64,
+                    row, blk);
+      nk = j + 1;
+      if (use > 0 && !__all_sync(0xffffffffu, pf::wait(VE(st), (use - 1) & 1, abort_flag, p.err))) break;
+      if (lane == 0) mbar_arrive_expect_tx(VF(st), bytes);
+      __syncwarp();
+      if (mine)
+        tma_load_3d(sbase + S::V_OFF + st * S::TILE + h * S::HALF + c * 2048, &vmap, VF(st), h * 64,
+                    row, blk);
+      nv = j + 1;
+    }
+    if (lane == 0 && *abort_flag) {
+      // let the copies in flight land before the shared memory is released
+      for (int jj = max(0, nk - STAGES); jj < nk; ++jj)
+        (void)mbar_wait_bounded(KF(jj % STAGES), (jj / STAGES) & 1, kPfDrainNs);
+      for (int jj = max(0, nv - STAGES); jj < nv; ++jj)
+        (void)mbar_wait_bounded(VF(jj % STAGES), (jj / STAGES) & 1, kPfDrainNs);
+      (void)mbar_wait_bounded(BQ, 0, kPfDrainNs);
     }
   } else if (warp == 9) {
     // --------------------------------------------------------------- MMA
@@ -342,13 +373,13 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         const uint32_t aP = tmem + S::S_COL + x * kPfKeys;
 #pragma unroll
         for (int kk = 0; kk < KCH; ++kk) {
-          // keys 16kk..16kk+15: 32-key chunk kk/2 holds its values in 16
-          // columns, then (bf16) its residuals in the next 16
-          const uint32_t col = 32 * (kk / 2) + 8 * (kk % 2);
+          // keys 16kk..16kk+15: their 16-bit values in columns 16kk..16kk+7,
+          // (bf16) the residuals in the next 8
+          const uint32_t col = 16 * kk;
           const uint64_t bV =
               tc::desc_sw128(sbase + S::V_OFF + st * S::TILE + kk * 2048, S::HALF, 1024);
           tc::mma_ts(tmem + S::O_COL + x * D, aP + col, bV, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
-          if constexpr (kSplit) tc::mma_ts(tmem + S::O_COL + x * D, aP + col + 16, bV, kIdO, 1u);
+          if constexpr (kSplit) tc::mma_ts(tmem + S::O_COL + x * D, aP + col + 8, bV, kIdO, 1u);
         }
         tc::commit(PV(x));
       };
@@ -472,41 +503,70 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         }
       }
       m_ref = m_new;
-      // pass 2: P over S's own columns, one 32-key chunk at a time: keys
-      // 2i, 2i + 1 of the chunk in its column i (16 columns), then (bf16)
-      // their rounding residuals in the next 16
-      float ls[4] = {l * alpha, 0.f, 0.f, 0.f};
+      // pass 2: P over S's own columns, 16 keys at a time: keys 16m + 2i,
+      // 16m + 2i + 1 go to column 16m + i as a 16-bit pair, (bf16) their
+      // rounding residuals to column 16m + 8 + i.  Pairs of keys run through
+      // the .f32x2 instructions.
+      const uint64_t sl2x2 = pf::f2(sl2, sl2), negm = pf::f2(-m_ref, -m_ref);
+      uint64_t ls2[2] = {pf::f2(l * alpha, 0.f), pf::f2(0.f, 0.f)};
       auto probs = [&](auto kMask) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32];
-          tc::ld32(tS + 32 * c, sv);
-          tc::wait_ld();
-          tc::pin(sv);
-          uint32_t hi[16], lo[16];
+        // 16 keys (16 columns of S) at a time; the next 16 are loading while
+        // these are computed
+        uint32_t sv0[16], sv1[16];
+        auto chunk = [&](const uint32_t(&cur)[16], int m) {
+          uint32_t hi[8], lo[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float a = ex2(fmaf(__uint_as_float(sv[2 * i]), sl2, -m_ref));
-            float e = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -m_ref));
+          for (int i = 0; i < 8; ++i) {
+            const uint64_t t = pf::fma2(pf::f2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])),
+                                        sl2x2, negm);
+            float ta, tb;
+            pf::f2_split(t, ta, tb);
+            float a = ex2(ta), e = ex2(tb);
             if constexpr (decltype(kMask)::value) {
-              if (32 * c + 2 * i > lim || 32 * c + 2 * i < wlo) a = 0.f;
-              if (32 * c + 2 * i + 1 > lim || 32 * c + 2 * i + 1 < wlo) e = 0.f;
+              if (16 * m + 2 * i > lim || 16 * m + 2 * i < wlo) a = 0.f;
+              if (16 * m + 2 * i + 1 > lim || 16 * m + 2 * i + 1 < wlo) e = 0.f;
             }
-            ls[i % 4] += a + e;
+            const uint64_t ae = pf::f2(a, e);
+            ls2[i % 2] = pf::add2(ls2[i % 2], ae);
             if constexpr (kSplit) {
-              split2<true>(a, e, hi[i], lo[i]);
+              hi[i] = pack2<true>(a, e);
+              float ra, rb;
+              pf::f2_split(pf::sub2(ae, pf::f2(__uint_as_float(hi[i] << 16),
+                                               __uint_as_float(hi[i] & 0xffff0000u))), ra, rb);
+              lo[i] = pack2<true>(ra, rb);
             } else {
               hi[i] = pack2<false>(a, e);
               lo[i] = 0u;
             }
           }
-          tc::st16(tS + 32 * c, hi);
-          if constexpr (kSplit) tc::st16(tS + 32 * c + 16, lo);
+          tc::st8(tS + 16 * m, hi);
+          if constexpr (kSplit) tc::st8(tS + 16 * m + 8, lo);
+        };
+        tc::ld16(tS, sv0);
+        tc::wait_ld();
+        tc::pin(sv0);
+#pragma unroll 1
+        for (int m = 0; m < kPfKeys / 16; m += 2) {
+          tc::ld16(tS + 16 * (m + 1), sv1);
+          chunk(sv0, m);
+          tc::wait_ld();
+          tc::pin(sv1);
+          if (m + 2 < kPfKeys / 16) tc::ld16(tS + 16 * (m + 2), sv0);
+          chunk(sv1, m + 1);
+          if (m + 2 < kPfKeys / 16) {
+            tc::wait_ld();
+            tc::pin(sv0);
+          }
         }
       };
       if (wmask) probs(std::true_type{});
       else probs(std::false_type{});
-      l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      {
+        float s0, s1, s2, s3;
+        pf::f2_split(ls2[0], s0, s1);
+        pf::f2_split(ls2[1], s2, s3);
+        l = (s0 + s1) + (s2 + s3);
+      }
       tc::wait_st();
       if (j == nt - 1 && kend - kb - j * kPfKeys < kPfKeys) {
         // this tile's last K/V tile: zero the V rows past every key the CTA
