@@ -185,8 +185,13 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
   p.total_q = total_q;
   p.window = pool->window;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.batch = batch;
+  p.num_items = pairs * pool->kv_heads * batch;
+  if (p.num_items > 0x7fffffff) return fail(KV_ERR_ARG, "too many query tiles");
 
-  const dim3 grid((unsigned)pairs, pool->kv_heads, batch);
+  // one CTA per work item, heaviest first; a CTA that finishes an item
+  // cancels the launch of a CTA not yet started and takes over its item
+  const dim3 grid((unsigned)p.num_items);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = pool->dtype == KV_BF16 ? launch_d<true>(pool->head_dim, p, qmap, lb, grid, s)
                               : launch_d<false>(pool->head_dim, p, qmap, lb, grid, s);

@@ -12,11 +12,16 @@
 // position.
 //
 // Unlike decode, this is a real dense contraction, so it runs on the
-// fifth-generation tensor cores.  One CTA per (pair of query tiles A, B, kv
-// head, sequence), pairs with the most keys launched first; a query tile is
-// 128 rows = 128 / g new tokens x the g query heads of one kv head's group,
-// and both tiles share every K/V tile read.  Per 128-key tile j, with S and O
-// of each query tile in tensor memory (TMEM, 4 x 128 columns):
+// fifth-generation tensor cores.  A work item is a pair of query tiles A, B
+// of one (kv head, sequence); a query tile is 128 rows = 128 / g new tokens x
+// the g query heads of one kv head's group, and both tiles share every K/V
+// tile read.  The grid has one CTA per item, but CTAs persist (one per SM):
+// a CTA that starts an item asks the hardware (cluster launch control) to
+// cancel the launch of a CTA that has not started yet and takes over its
+// item next, so the copies and first MMAs of the next item overlap the end
+// of the current one and no CTA is set up per item.  Barrier phases run on
+// counters across items.  Per 128-key tile j, with S and O of each query
+// tile in tensor memory (TMEM, 4 x 128 columns):
 //   S_j = Q . K_j^T          (tcgen05.mma, M 128, N 128, K = head_dim; Q and
 //                            K_j in shared memory, 128-byte swizzled, K-major)
 //   softmax rows in fp32 (one row per thread, warps 0-3 tile A, 4-7 tile B;
@@ -62,6 +67,7 @@ constexpr int kPfThreads = 320;     // warps 0-7 softmax (4 per query tile), 8 c
 constexpr uint32_t kPfTmemCols = 512;  // S_A, S_B (128 each) + O_A, O_B (<= 128 each)
 constexpr uint64_t kPfWaitNs = 2000000000ull;
 constexpr uint64_t kPfDrainNs = 50000000ull;  // copies and MMAs in flight finish in microseconds
+constexpr int kPfSlots = 4;         // launch-control responses in flight or unread
 // reference max moves only when a tile's max exceeds it by more than this
 // many binades: probabilities stay <= 2^8, exact enough in 16 bits + residual
 constexpr float kPfLazyLog2 = 8.f;
@@ -78,7 +84,7 @@ struct PrefillParams {
   int num_q_heads;
   int group;                    // query heads per kv head, <= 8
   int tokens_per_tile;          // 128 / group
-  int num_q_pairs;              // grid x: pairs of query tiles
+  int num_q_pairs;              // pairs of query tiles per (kv head, sequence), max over sequences
   int kv_heads;
   int block_size;
   int num_blocks;
@@ -86,6 +92,8 @@ struct PrefillParams {
   int total_q;
   int window;                   // > 0: each token attends only to its last `window` positions
   float scale_log2;             // softmax scale * log2(e), > 0
+  int batch;
+  int64_t num_items;            // num_q_pairs * kv_heads * batch
 };
 
 template <int D, int STAGES>
@@ -97,11 +105,13 @@ struct PrefillShape {
   static constexpr int K_OFF = Q_OFF + kPfTiles * TILE;
   static constexpr int V_OFF = K_OFF + STAGES * TILE;
   static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
-  // q; K full/empty and V full/empty per stage; S full, P full and P.V done
-  // per query tile; the final MMA drain
-  static constexpr int NBAR = 1 + 4 * STAGES + 3 * kPfTiles + 1;
+  // q full and q empty; K full/empty and V full/empty per stage; S full,
+  // P full, P.V done and O free per query tile; the final MMA drain;
+  // launch-control response full and read per slot
+  static constexpr int NBAR = 2 + 4 * STAGES + 4 * kPfTiles + 1 + 2 * kPfSlots;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // TMEM base, abort flag
-  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+  static constexpr int RESP_OFF = (MISC_OFF + 16 + 15) / 16 * 16;  // 16-byte responses
+  static constexpr int SMEM_BYTES = RESP_OFF + 16 * kPfSlots + 1024;  // + alignment slack
   static constexpr uint32_t S_COL = 0;                       // S_X at X * 128
   static constexpr uint32_t O_COL = kPfTiles * kPfKeys;      // O_X at 256 + X * D
   static_assert(kPfRows == kPfKeys, "Q, K and V tiles share one byte size");
@@ -181,6 +191,79 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, volatile int
   }
 }
 
+// Cluster launch control (sm_100): cancel the launch of a CTA of this grid
+// that has not started and take over its work.  The 16-byte response lands
+// in shared memory at `resp` and completes 16 transaction bytes on `bar`.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], "
+      "[%1];" ::"r"(resp),
+      "r"(bar)
+      : "memory");
+}
+
+// The CTA index (x) a response names, or -1 when no launch was cancelled
+// (every CTA of the grid has started: no work is left to take over).
+__device__ __forceinline__ int64_t clc_item(uint32_t resp) {
+  uint32_t ok, x = 0;
+  asm volatile(
+      "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+      : "=r"(ok), "+r"(x)
+      : "r"(resp)
+      : "memory");
+  return ok ? (int64_t)x : -1;
+}
+
+// One work item: a pair of query tiles (A, B) of one (kv head, sequence).
+struct Item {
+  int s, kvh, q0, q_len, n, t0, kb, kend, ntiles;
+  int ntok[kPfTiles], kendx[kPfTiles], ntx[kPfTiles];
+};
+
+// Geometry of item v.  Items run sequence by sequence (CTAs working side by
+// side then read the same sequence's K/V tiles, from L2 after the first),
+// and within a sequence heaviest first: its last pair of query tiles for
+// every kv head, then the pairs before.  False
+// when the item has no tokens, or its sequence's lengths are out of range
+// (then `report` records KV_ERR_BOUNDS, once per sequence).
+__device__ __forceinline__ bool item_at(const PrefillParams& p, int64_t v, bool report, Item& it) {
+  const int64_t per_seq = (int64_t)p.kv_heads * p.num_q_pairs;
+  it.s = (int)(v / per_seq);
+  const int local = (int)(v - (int64_t)it.s * per_seq);
+  const int qp = p.num_q_pairs - 1 - local / p.kv_heads;
+  it.kvh = local % p.kv_heads;
+  const int tq = p.tokens_per_tile;
+  it.q0 = p.cu_q[it.s];
+  it.q_len = p.cu_q[it.s + 1] - it.q0;
+  it.n = p.context_lens[it.s];
+  if (it.q0 < 0 || it.q_len < 0 || it.q_len > it.n || (int64_t)it.q0 + it.q_len > p.total_q ||
+      (int64_t)it.n > (int64_t)p.max_blocks * p.block_size ||
+      it.q_len > p.num_q_pairs * kPfTiles * tq) {
+    if (report && qp == p.num_q_pairs - 1 && it.kvh == 0) atomicCAS(p.err, 0, KV_ERR_BOUNDS);
+    return false;
+  }
+  it.t0 = qp * kPfTiles * tq;
+  if (it.t0 >= it.q_len) return false;
+  // Key tiles start at kb: 0, or with a sliding window the 16-key chunk
+  // holding the first position any row of the item sees (no block before
+  // it is read: it may already be released).
+  it.kb = p.window > 0 ? max(0, it.n - it.q_len + it.t0 - p.window + 1) / 16 * 16 : 0;
+#pragma unroll
+  for (int x = 0; x < kPfTiles; ++x) {
+    const int tx = it.t0 + x * tq;
+    it.ntok[x] = tx < it.q_len ? min(tq, it.q_len - tx) : 0;
+    it.kendx[x] = it.ntok[x] ? it.n - it.q_len + tx + it.ntok[x] : 0;  // keys .. kend - 1
+    it.ntx[x] = it.ntok[x] ? (it.kendx[x] - it.kb + kPfKeys - 1) / kPfKeys : 0;
+  }
+  it.kend = max(it.kendx[0], it.kendx[1]);
+  it.ntiles = max(it.ntx[0], it.ntx[1]);  // K/V tiles read (tile B's when it has tokens)
+  return true;
+}
+
 }  // namespace pf
 
 template <bool kBf16, int D, int STAGES>
@@ -199,53 +282,30 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   uint8_t* smem = smem_raw + (sbase - raw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qp = p.num_q_pairs - 1 - (int)blockIdx.x;  // pairs with the most keys start first
-  const int kvh = blockIdx.y, s = blockIdx.z;
   const int g = p.group, tq = p.tokens_per_tile;
-
-  const int q0 = p.cu_q[s];
-  const int q_len = p.cu_q[s + 1] - q0;
-  const int n = p.context_lens[s];
-  if (q0 < 0 || q_len < 0 || q_len > n || (int64_t)q0 + q_len > p.total_q ||
-      (int64_t)n > (int64_t)p.max_blocks * p.block_size ||
-      q_len > p.num_q_pairs * kPfTiles * tq) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) atomicCAS(p.err, 0, KV_ERR_BOUNDS);
-    return;
-  }
-  const int t0 = qp * kPfTiles * tq;  // first new token of query tile A
-  if (t0 >= q_len) return;
-  // Key tiles start at kb: 0, or with a sliding window the 16-key chunk
-  // holding the first position any row of this CTA sees (no block before it
-  // is read: it may already be released).
-  const int kb = p.window > 0 ? max(0, n - q_len + t0 - p.window + 1) / 16 * 16 : 0;
-  // per query tile X (A = 0, B = 1): tokens, key range, key tiles
-  int ntok[kPfTiles], kendx[kPfTiles], ntx[kPfTiles];
-#pragma unroll
-  for (int x = 0; x < kPfTiles; ++x) {
-    const int tx = t0 + x * tq;
-    ntok[x] = tx < q_len ? min(tq, q_len - tx) : 0;
-    kendx[x] = ntok[x] ? n - q_len + tx + ntok[x] : 0;  // keys .. kend - 1
-    ntx[x] = ntok[x] ? (kendx[x] - kb + kPfKeys - 1) / kPfKeys : 0;
-  }
-  const int kend = max(kendx[0], kendx[1]);
-  const int ntiles = max(ntx[0], ntx[1]);  // K/V tiles read (tile B's when it has tokens)
   const int qrows = tq * g;
 
   const uint32_t bar0 = sbase + S::BAR_OFF;
-  const uint32_t BQ = bar0;
-  auto KF = [&](int i) { return bar0 + 8u * (1 + i); };
-  auto KE = [&](int i) { return bar0 + 8u * (1 + STAGES + i); };
-  auto VF = [&](int i) { return bar0 + 8u * (1 + 2 * STAGES + i); };
-  auto VE = [&](int i) { return bar0 + 8u * (1 + 3 * STAGES + i); };
-  auto SF = [&](int x) { return bar0 + 8u * (1 + 4 * STAGES + x); };
-  auto PF = [&](int x) { return bar0 + 8u * (1 + 4 * STAGES + kPfTiles + x); };
-  auto PV = [&](int x) { return bar0 + 8u * (1 + 4 * STAGES + 2 * kPfTiles + x); };
-  const uint32_t FIN = bar0 + 8u * (1 + 4 * STAGES + 3 * kPfTiles);
+  const uint32_t BQ = bar0;        // query tiles loaded
+  const uint32_t QE = bar0 + 8u;   // query tiles free (every S of the item issued and done)
+  auto KF = [&](int i) { return bar0 + 8u * (2 + i); };
+  auto KE = [&](int i) { return bar0 + 8u * (2 + STAGES + i); };
+  auto VF = [&](int i) { return bar0 + 8u * (2 + 2 * STAGES + i); };
+  auto VE = [&](int i) { return bar0 + 8u * (2 + 3 * STAGES + i); };
+  auto SF = [&](int x) { return bar0 + 8u * (2 + 4 * STAGES + x); };
+  auto PF = [&](int x) { return bar0 + 8u * (2 + 4 * STAGES + kPfTiles + x); };
+  auto PV = [&](int x) { return bar0 + 8u * (2 + 4 * STAGES + 2 * kPfTiles + x); };
+  auto OF = [&](int x) { return bar0 + 8u * (2 + 4 * STAGES + 3 * kPfTiles + x); };
+  const uint32_t FIN = bar0 + 8u * (2 + 4 * STAGES + 4 * kPfTiles);
+  auto CF = [&](int i) { return FIN + 8u * (1 + i); };             // response i landed
+  auto CR = [&](int i) { return FIN + 8u * (1 + kPfSlots + i); };  // response i read by all
+  auto RESP = [&](int i) { return sbase + (uint32_t)S::RESP_OFF + 16u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::MISC_OFF + 8);
 
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
+    mbar_init(QE, 1);
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(KF(i), 1);
       mbar_init(KE(i), 1);
@@ -256,12 +316,17 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       mbar_init(SF(x), 1);
       mbar_init(PF(x), kPfRows);
       mbar_init(PV(x), 1);
+      mbar_init(OF(x), kPfRows);
     }
     mbar_init(FIN, 1);
+    for (int i = 0; i < kPfSlots; ++i) {
+      mbar_init(CF(i), 1);
+      mbar_init(CR(i), 1 + kPfTiles * kPfRows / 32);  // the MMA warp + 8 softmax warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // Query rows past tokens_per_tile * group are not covered by the copies
+  // Query rows past tokens_per_tile * group are never written by the copies
   if (threadIdx.x < kPfTiles * kPfRows && (int)(threadIdx.x % kPfRows) >= qrows) {
     const int x = threadIdx.x / kPfRows, r = threadIdx.x % kPfRows;
 #pragma unroll
@@ -282,12 +347,22 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
   tc::fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Work items of this CTA: item 0 is its own (blockIdx.x); item k >= 1 is
+  // the CTA whose launch the copy warp cancelled when it began item k - 1
+  // (response slot (k - 1) % kPfSlots; -1: none left).  Every role walks the
+  // same items and keeps running counters, so barrier phases continue across
+  // items: ic items with work, kc K/V tiles (stage kc % STAGES), per query
+  // tile sc[x] S tiles and oc[x] items that used it.
+  auto slot_of = [](uint32_t k) { return (int)((k - 1) % kPfSlots); };
+  auto use_of = [](uint32_t k) { return ((k - 1) / kPfSlots) & 1u; };
+
   if (warp == 8) {
     // ------------------------------------------------------------ copies
     // The whole warp streams: lane c + KCH * h owns 16-key chunk c, column
     // block h of every tile (its block id, its box), so one instruction puts
     // a tile's NH * KCH box copies in flight; lane 0 sets the transaction
-    // counts.  Every lane takes the same waits and branches.
+    // counts and asks for the next item.  Every lane takes the same waits
+    // and branches.
     constexpr int NBOX = NH * KCH;  // 16 (head_dim 128) or 8 (64) boxes per tile
     const int c = lane % KCH, h = lane / KCH;
     const bool boxer = lane < NBOX;
@@ -295,69 +370,110 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
-      mbar_arrive_expect_tx(BQ, (uint32_t)(kPfTiles * NH * qrows * 128));
     }
-    __syncwarp();
-    if (lane < kPfTiles * NH)
-      tma_load_3d(sbase + S::Q_OFF + (lane / NH) * S::TILE + (lane % NH) * S::HALF, &qmap, BQ,
-                  (lane % NH) * 64, kvh * g, q0 + t0 + (lane / NH) * tq);
-    const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks;
-    int nk = 0, nv = 0;  // tiles whose K (V) copies are in flight or done
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j % STAGES;
-      const uint32_t use = (uint32_t)(j / STAGES);
-      const int key0 = kb + j * kPfKeys;
-      const int nch = min(KCH, (kend - key0 + 15) / 16);
-      const bool mine = boxer && c < nch;
-      int blk = 0, row = 0;
-      bool bad = false;
-      if (mine) {
-        const int key = key0 + 16 * c;
-        blk = table[key / p.block_size];
-        bad = blk < 0 || blk >= p.num_blocks;
-        row = kvh * p.block_size + key % p.block_size;
+    uint32_t ic = 0, kc = 0;
+    uint32_t nk = 0, nv = 0;   // tiles whose K (V) copies were issued
+    int64_t q_last = -1;       // index (in ic) of the last query copy issued
+    uint32_t asked = 0, read = 0;  // items requested / responses read
+    for (uint32_t k = 0;; ++k) {
+      int64_t v = blockIdx.x;
+      if (k > 0) {
+        if (!__all_sync(0xffffffffu, pf::wait(CF(slot_of(k)), use_of(k), abort_flag, p.err))) break;
+        read = k;
+        v = pf::clc_item(RESP(slot_of(k)));
       }
-      if (__any_sync(0xffffffffu, bad)) {
-        if (lane == 0) {
-          atomicCAS(p.err, 0, KV_ERR_BOUNDS);
-          *abort_flag = 1;
-        }
+      if (v < 0) break;  // every CTA of the grid has started: no item left
+      // ask for item k + 1 now: the answer is back long before this item's
+      // copies are issued.  Its slot was last used by item k + 1 - kPfSlots.
+      if (k >= kPfSlots &&
+          !__all_sync(0xffffffffu, pf::wait(CR(slot_of(k + 1)), use_of(k + 1) ^ 1u, abort_flag, p.err)))
         break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(CF(slot_of(k + 1)), 16u);
+        pf::clc_try_cancel(RESP(slot_of(k + 1)), CF(slot_of(k + 1)));
       }
-      const uint32_t bytes = (uint32_t)(nch * NH * 16 * 128);
-      if (use > 0 && !__all_sync(0xffffffffu, pf::wait(KE(st), (use - 1) & 1, abort_flag, p.err))) break;
-      if (lane == 0) mbar_arrive_expect_tx(KF(st), bytes);
+      asked = k + 1;
+      pf::Item it;
+      if (!pf::item_at(p, v, lane == 0, it)) continue;
+      // the previous item's S MMAs must be done before its query tiles are replaced
+      if (ic > 0 && !__all_sync(0xffffffffu, pf::wait(QE, (ic - 1) & 1, abort_flag, p.err))) break;
+      if (lane == 0) mbar_arrive_expect_tx(BQ, (uint32_t)(kPfTiles * NH * qrows * 128));
       __syncwarp();
-      if (mine)
-        tma_load_3d(sbase + S::K_OFF + st * S::TILE + h * S::HALF + c * 2048, &kmap, KF(st), h * 64,
-                    row, blk);
-      nk = j + 1;
-      if (use > 0 && !__all_sync(0xffffffffu, pf::wait(VE(st), (use - 1) & 1, abort_flag, p.err))) break;
-      if (lane == 0) mbar_arrive_expect_tx(VF(st), bytes);
-      __syncwarp();
-      if (mine)
-        tma_load_3d(sbase + S::V_OFF + st * S::TILE + h * S::HALF + c * 2048, &vmap, VF(st), h * 64,
-                    row, blk);
-      nv = j + 1;
+      q_last = ic;
+      if (lane < kPfTiles * NH)
+        tma_load_3d(sbase + S::Q_OFF + (lane / NH) * S::TILE + (lane % NH) * S::HALF, &qmap, BQ,
+                    (lane % NH) * 64, it.kvh * g, it.q0 + it.t0 + (lane / NH) * tq);
+      const int32_t* table = p.block_tables + (int64_t)it.s * p.max_blocks;
+      bool stop = false;
+      for (int j = 0; j < it.ntiles; ++j, ++kc) {
+        const int st = kc % STAGES;
+        const uint32_t use = kc / STAGES;
+        const int key0 = it.kb + j * kPfKeys;
+        const int nch = min(KCH, (it.kend - key0 + 15) / 16);
+        const bool mine = boxer && c < nch;
+        int blk = 0, row = 0;
+        bool bad = false;
+        if (mine) {
+          const int key = key0 + 16 * c;
+          blk = table[key / p.block_size];
+          bad = blk < 0 || blk >= p.num_blocks;
+          row = it.kvh * p.block_size + key % p.block_size;
+        }
+        if (__any_sync(0xffffffffu, bad)) {
+          if (lane == 0) {
+            atomicCAS(p.err, 0, KV_ERR_BOUNDS);
+            *abort_flag = 1;
+          }
+          stop = true;
+          break;
+        }
+        const uint32_t bytes = (uint32_t)(nch * NH * 16 * 128);
+        if (use > 0 &&
+            !__all_sync(0xffffffffu, pf::wait(KE(st), (use - 1) & 1, abort_flag, p.err))) {
+          stop = true;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(KF(st), bytes);
+        __syncwarp();
+        if (mine)
+          tma_load_3d(sbase + S::K_OFF + st * S::TILE + h * S::HALF + c * 2048, &kmap, KF(st),
+                      h * 64, row, blk);
+        nk = kc + 1;
+        if (use > 0 &&
+            !__all_sync(0xffffffffu, pf::wait(VE(st), (use - 1) & 1, abort_flag, p.err))) {
+          stop = true;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(VF(st), bytes);
+        __syncwarp();
+        if (mine)
+          tma_load_3d(sbase + S::V_OFF + st * S::TILE + h * S::HALF + c * 2048, &vmap, VF(st),
+                      h * 64, row, blk);
+        nv = kc + 1;
+      }
+      if (stop) break;
+      ++ic;
     }
     if (lane == 0 && *abort_flag) {
-      // let the copies in flight land before the shared memory is released
-      for (int jj = max(0, nk - STAGES); jj < nk; ++jj)
-        (void)mbar_wait_bounded(KF(jj % STAGES), (jj / STAGES) & 1, kPfDrainNs);
-      for (int jj = max(0, nv - STAGES); jj < nv; ++jj)
-        (void)mbar_wait_bounded(VF(jj % STAGES), (jj / STAGES) & 1, kPfDrainNs);
-      (void)mbar_wait_bounded(BQ, 0, kPfDrainNs);
+      // let the copies and the launch-control answer in flight land before
+      // the shared memory is released
+      for (uint32_t kk = nk > STAGES ? nk - STAGES : 0; kk < nk; ++kk)
+        (void)mbar_wait_bounded(KF(kk % STAGES), (kk / STAGES) & 1, kPfDrainNs);
+      for (uint32_t kk = nv > STAGES ? nv - STAGES : 0; kk < nv; ++kk)
+        (void)mbar_wait_bounded(VF(kk % STAGES), (kk / STAGES) & 1, kPfDrainNs);
+      if (q_last >= 0) (void)mbar_wait_bounded(BQ, (uint32_t)q_last & 1, kPfDrainNs);
+      if (asked > read) (void)mbar_wait_bounded(CF(slot_of(asked)), use_of(asked), kPfDrainNs);
     }
   } else if (warp == 9) {
     // --------------------------------------------------------------- MMA
-    // Issue order S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) ...:
+    // Per item: S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) ...:
     // the softmax of one query tile runs while the tensor cores work on the
     // other's P.V and next S.
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_f16(kBf16, kPfRows, kPfKeys, false);
       constexpr uint32_t kIdO = tc::idesc_f16(kBf16, kPfRows, D, true);
-      auto issue_s = [&](int x, int j) {
-        const int st = j % STAGES;
+      auto issue_s = [&](int x, uint32_t kt) {
+        const int st = kt % STAGES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * S::HALF + (kk % 4) * 32;  // 16 columns per step
@@ -368,8 +484,8 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         }
         tc::commit(SF(x));
       };
-      auto issue_pv = [&](int x, int j) {
-        const int st = j % STAGES;
+      auto issue_pv = [&](int x, uint32_t kt, bool first) {
+        const int st = kt % STAGES;
         const uint32_t aP = tmem + S::S_COL + x * kPfKeys;
 #pragma unroll
         for (int kk = 0; kk < KCH; ++kk) {
@@ -378,49 +494,83 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
           const uint32_t col = 16 * kk;
           const uint64_t bV =
               tc::desc_sw128(sbase + S::V_OFF + st * S::TILE + kk * 2048, S::HALF, 1024);
-          tc::mma_ts(tmem + S::O_COL + x * D, aP + col, bV, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(tmem + S::O_COL + x * D, aP + col, bV, kIdO, (!first || kk > 0) ? 1u : 0u);
           if constexpr (kSplit) tc::mma_ts(tmem + S::O_COL + x * D, aP + col + 8, bV, kIdO, 1u);
         }
         tc::commit(PV(x));
       };
-      bool ok = pf::wait(BQ, 0, abort_flag, p.err) && pf::wait(KF(0), 0, abort_flag, p.err);
-      tc::fence_after();
-      if (ok) {
+      uint32_t ic = 0, kc = 0, sc[kPfTiles] = {0, 0}, oc[kPfTiles] = {0, 0};
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        int64_t v = blockIdx.x;
+        if (k > 0) {
+          if (!pf::wait(CF(slot_of(k)), use_of(k), abort_flag, p.err)) break;
+          v = pf::clc_item(RESP(slot_of(k)));
+          mbar_arrive(CR(slot_of(k)));
+        }
+        if (v < 0) break;
+        pf::Item it;
+        if (!pf::item_at(p, v, false, it)) continue;
+        ok = pf::wait(BQ, ic & 1, abort_flag, p.err) &&
+             pf::wait(KF(kc % STAGES), (kc / STAGES) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc::fence_after();
 #pragma unroll
         for (int x = 0; x < kPfTiles; ++x)
-          if (ntx[x] > 0) issue_s(x, 0);
-        tc::commit(KE(0));
-      }
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int st = j % STAGES, sn = (j + 1) % STAGES;
-        const bool more = j + 1 < ntiles;
-        bool waited_k = false;
-        if (!pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err)) break;
-#pragma unroll
-        for (int x = 0; x < kPfTiles; ++x) {
-          if (j < ntx[x]) {
-            if (!pf::wait(PF(x), j & 1, abort_flag, p.err)) {
-              ok = false;
-              break;
-            }
-            tc::fence_after();
-            issue_pv(x, j);
+          if (it.ntx[x] > 0) issue_s(x, kc);
+        tc::commit(KE(kc % STAGES));
+        if (it.ntiles == 1) tc::commit(QE);  // the item's last S: its query tiles may be replaced
+        for (int j = 0; ok && j < it.ntiles; ++j) {
+          const uint32_t kt = kc + j, kn = kt + 1;
+          const int st = kt % STAGES;
+          bool waited_k = false;
+          if (!pf::wait(VF(st), (kt / STAGES) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
           }
-          if (j + 1 < ntx[x]) {
-            if (!waited_k) {
-              if (!pf::wait(KF(sn), ((j + 1) / STAGES) & 1, abort_flag, p.err)) {
+#pragma unroll
+          for (int x = 0; x < kPfTiles; ++x) {
+            if (j < it.ntx[x]) {
+              // the first P.V of an item overwrites O_x: the previous item's
+              // output must have been read
+              if (j == 0 && oc[x] > 0 && !pf::wait(OF(x), (oc[x] - 1) & 1, abort_flag, p.err)) {
+                ok = false;
+                break;
+              }
+              if (!pf::wait(PF(x), (sc[x] + j) & 1, abort_flag, p.err)) {
                 ok = false;
                 break;
               }
               tc::fence_after();
-              waited_k = true;
+              issue_pv(x, kt, j == 0);
             }
-            issue_s(x, j + 1);
+            if (j + 1 < it.ntx[x]) {
+              if (!waited_k) {
+                if (!pf::wait(KF(kn % STAGES), (kn / STAGES) & 1, abort_flag, p.err)) {
+                  ok = false;
+                  break;
+                }
+                tc::fence_after();
+                waited_k = true;
+              }
+              issue_s(x, kn);
+            }
+          }
+          if (!ok) break;
+          tc::commit(VE(st));
+          if (j + 1 < it.ntiles) {
+            tc::commit(KE(kn % STAGES));
+            if (j + 2 == it.ntiles) tc::commit(QE);
           }
         }
         if (!ok) break;
-        tc::commit(VE(st));
-        if (more) tc::commit(KE(sn));
+#pragma unroll
+        for (int x = 0; x < kPfTiles; ++x) {
+          sc[x] += it.ntx[x];
+          oc[x] += it.ntx[x] > 0 ? 1 : 0;
+        }
+        kc += it.ntiles;
+        ++ic;
       }
       // every MMA issued must finish before TMEM is released
       tc::commit(FIN);
@@ -432,20 +582,37 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
     const int x = warp / 4;
     const int r = threadIdx.x % kPfRows;
     const int tok = r / g, head = r - tok * g;
-    const int nt = x ? ntx[1] : ntx[0];  // selects keep the per-tile values in registers
-    const bool valid = r < qrows && tok < (x ? ntok[1] : ntok[0]);
-    const int prow = valid ? n - q_len + t0 + x * tq + tok : (x ? kendx[1] : kendx[0]) - 1;
     const uint32_t lane_addr = (uint32_t)((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + lane_addr + S::S_COL + x * kPfKeys;
     const uint32_t tO = tmem + lane_addr + S::O_COL + x * D;
     const float sl2 = p.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
+    uint32_t sc = 0, kc = 0;  // this query tile's S tiles so far; K/V tiles so far
     bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+    int64_t v = blockIdx.x;
+    if (k > 0) {
+      ok = __all_sync(0xffffffffu, pf::wait(CF(slot_of(k)), use_of(k), abort_flag, p.err));
+      if (!ok) break;
+      v = pf::clc_item(RESP(slot_of(k)));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(CR(slot_of(k)));
+    }
+    if (v < 0) break;
+    pf::Item it;
+    if (!pf::item_at(p, v, false, it)) continue;
+    const int nt = x ? it.ntx[1] : it.ntx[0];  // selects keep the per-tile values in registers
+    if (nt == 0) {
+      kc += it.ntiles;
+      continue;
+    }
+    const bool valid = r < qrows && tok < (x ? it.ntok[1] : it.ntok[0]);
+    const int prow = valid ? it.n - it.q_len + it.t0 + x * tq + tok : (x ? it.kendx[1] : it.kendx[0]) - 1;
+    float m_ref = -INFINITY, l = 0.f;
     for (int j = 0; j < nt; ++j) {
-      ok = __all_sync(0xffffffffu, pf::wait(SF(x), j & 1, abort_flag, p.err));
+      ok = __all_sync(0xffffffffu, pf::wait(SF(x), (sc + j) & 1, abort_flag, p.err));
       if (!ok) break;
       tc::fence_after();
-      const int lim = prow - kb - j * kPfKeys;  // columns wlo .. lim are visible
+      const int lim = prow - it.kb - j * kPfKeys;  // columns wlo .. lim are visible
       const int wlo = p.window > 0 ? lim - p.window + 1 : INT_MIN;
       const bool masked = lim < kPfKeys - 1 || wlo > 0;
       // pass 1: the row max.  Only tiles on the causal diagonal mask
@@ -488,7 +655,7 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       __syncwarp();
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         // O holds P.V up to tile j - 1: wait for it, then rescale in TMEM
-        ok = __all_sync(0xffffffffu, pf::wait(PV(x), (j - 1) & 1, abort_flag, p.err));
+        ok = __all_sync(0xffffffffu, pf::wait(PV(x), (sc + j - 1) & 1, abort_flag, p.err));
         if (!ok) break;
         tc::fence_after();
 #pragma unroll 1
@@ -568,14 +735,15 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         l = (s0 + s1) + (s2 + s3);
       }
       tc::wait_st();
-      if (j == nt - 1 && kend - kb - j * kPfKeys < kPfKeys) {
+      if (j == nt - 1 && it.kend - it.kb - j * kPfKeys < kPfKeys) {
         // this tile's last K/V tile: zero the V rows past every key the CTA
         // reads (stale slots may hold any bits, and 0 * NaN is NaN); both
         // query tiles may write the same zeros
-        const int st = j % STAGES;
-        ok = __all_sync(0xffffffffu, pf::wait(VF(st), (j / STAGES) & 1, abort_flag, p.err));
+        const uint32_t kt = kc + j;
+        const int st = kt % STAGES;
+        ok = __all_sync(0xffffffffu, pf::wait(VF(st), (kt / STAGES) & 1, abort_flag, p.err));
         if (!ok) break;
-        if (r >= kend - kb - j * kPfKeys) {
+        if (r >= it.kend - it.kb - j * kPfKeys) {
 #pragma unroll
           for (int h = 0; h < NH; ++h) {
             uint4* row = reinterpret_cast<uint4*>(smem + S::V_OFF + st * S::TILE + h * S::HALF + r * 128);
@@ -589,11 +757,12 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       tc::fence_before();
       mbar_arrive(PF(x));
     }
-    if (ok && nt > 0) ok = __all_sync(0xffffffffu, pf::wait(PV(x), (nt - 1) & 1, abort_flag, p.err));
-    if (ok && nt > 0) {
+    if (ok) ok = __all_sync(0xffffffffu, pf::wait(PV(x), (sc + nt - 1) & 1, abort_flag, p.err));
+    if (ok) {
       tc::fence_after();
       const float inv = 1.f / l;
-      const int64_t orow = ((int64_t)(q0 + t0 + x * tq + tok) * p.num_q_heads + kvh * g + head) * D;
+      const int64_t orow =
+          ((int64_t)(it.q0 + it.t0 + x * tq + tok) * p.num_q_heads + it.kvh * g + head) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -620,6 +789,12 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
         }
         __syncwarp();
       }
+      // O_x is read: the next item's first P.V may overwrite it
+      tc::fence_before();
+      mbar_arrive(OF(x));
+    }
+    sc += nt;
+    kc += it.ntiles;
     }
   }
 
