@@ -108,7 +108,7 @@ int kv_pool_bind(kv_pool* pool, int layer, void* k_base, void* v_base, float* k_
  * merged by a log-sum-exp reduce (see paged_attention_decode).  0 chooses
  * automatically: partitions of at most 4096 tokens; if batch * kv_heads is
  * under three waves of resident CTAs, enough partitions (of at least 512
- * tokens) for eight waves.  A context that fits one partition is written
+ * tokens) for four waves.  A context that fits one partition is written
  * directly and skips the reduce.  stages: shared-memory pipeline
  * depth per warp, 0 for automatic, else 2, 3, 4, 6 or 8; warps: warps per
  * CTA, 0 for automatic, else 4 or 8.  Automatic: 4 warps x 3 stages for

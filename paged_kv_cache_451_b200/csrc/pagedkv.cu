@@ -161,10 +161,12 @@ int decode_slots(const kv_pool* pool) {
 // further, into enough partitions (of at least kMinPartition tokens) for
 // kWavesSplit waves.  Measured on B200: unsplit 2K-token contexts with 1024
 // units (32-layer example, 3.5 waves), 4K-token partitions for a 256-sequence
-// lognormal batch (few long contexts; the others skip the reduce), 1-2K-token
-// partitions for 8 x 16K-token FP8 contexts (256 units).
+// lognormal batch (few long contexts; the others skip the reduce), ~2K-token
+// partitions for 8 x 16K-token FP8 contexts (256 units) and ~1K-token ones
+// for a 4K-token window over 8 x 16K-token bf16 contexts (shorter partitions
+// lose more to each CTA's start than they gain in balance).
 constexpr int kWavesKeep = 3;
-constexpr int kWavesSplit = 8;
+constexpr int kWavesSplit = 4;
 constexpr int kAutoPartition = 4096;
 constexpr int kMinPartition = 512;
 
