@@ -704,17 +704,17 @@ def describe(w, case=None):
     return s
 
 
-def run_e2e(case, torch, pk, flush, stream, K, W):
-    """The same step through the C ABI from pinned host memory, pipelined the
-    way a serving loop runs it: each step's inputs (q, new K/V of every
-    layer, slots, tables, lengths, order) are packed in one pinned buffer and
-    uploaded with one copy on a copy stream into one of two device buffers,
-    the step's write + decode kernels wait for that upload, and the output
-    goes back to pinned host memory on the copy stream.  The upload of step
-    i + 1 overlaps the kernels of step i.  K steps are timed as one region
-    (CUDA events on the compute stream, every copy inside it).  The decode
-    reads more than L2 holds each step, so there is no flush in between."""
-    ins = list(case.q) + list(case.kn) + list(case.vn) + [case.slots, case.tables_d, case.lens_d, case.order_d]
+def pipelined_e2e(torch, stream, ins, outs, launch, K, W):
+    """Time K steps of a serving-style loop from pinned host memory: each
+    step's inputs (the device tensors `ins`, copied once to the host) are
+    packed in one pinned buffer and uploaded with one copy on an upload
+    stream into one of two device buffers; `launch(views, outs_k)` enqueues
+    the step's kernels on `stream` over those views, writing per-buffer
+    copies of `outs`; the outputs go back to pinned host memory on a
+    read-back stream.  The upload of step i + 1 overlaps the kernels of step
+    i, and the read-back of step i the kernels of step i + 1.  The K steps
+    are timed as one region (CUDA events on `stream`, every copy inside).
+    Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
     offs, off = [], 0
     for t in ins:
         offs.append(off)
@@ -725,47 +725,36 @@ def run_e2e(case, torch, pk, flush, stream, K, W):
         n = t.numel() * t.element_size()
         hbuf[o:o + n].copy_(t.contiguous().view(-1).view(torch.uint8).cpu())
     dbuf = [torch.empty(off, dtype=torch.uint8, device="cuda") for _ in range(2)]
-
-    def views(k):
-        out = []
-        for t, o in zip(ins, offs):
-            n = t.numel() * t.element_size()
-            out.append(dbuf[k][o:o + n].view(t.dtype).view(t.shape))
-        return out
-
-    dv = [views(k) for k in range(2)]
-    L = case.L
-    dout = [[torch.empty_like(o) for o in case.out] for _ in range(2)]
-    hout = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in case.out] for _ in range(2)]
-    d2h = sum(o.numel() * o.element_size() for o in case.out)
-    cs = torch.cuda.Stream()
+    views = [[dbuf[k][o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+              for t, o in zip(ins, offs)] for k in range(2)]
+    dout = [[torch.empty_like(o) for o in outs] for _ in range(2)]
+    hout = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _ in range(2)]
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    cs_up, cs_dn = torch.cuda.Stream(), torch.cuda.Stream()
     up = [torch.cuda.Event() for _ in range(2)]
     comp = [None, None]   # kernels that read device buffer k (and wrote dout[k])
     down = [None, None]   # read-back of dout[k]
 
     def step(i):
         k = i % 2
-        with torch.cuda.stream(cs):
+        with torch.cuda.stream(cs_up):
             if comp[k] is not None:
-                cs.wait_event(comp[k])  # buffer k's previous readers are done
+                cs_up.wait_event(comp[k])  # buffer k's previous readers are done
             dbuf[k].copy_(hbuf, non_blocking=True)
-            up[k].record(cs)
+            up[k].record(cs_up)
         stream.wait_event(up[k])
         if down[k] is not None:
             stream.wait_event(down[k])  # dout[k] was read back
-        v = dv[k]
-        for layer in range(L):
-            case.write(layer, v[L + layer], v[2 * L + layer], v[3 * L])
-            case.decode(layer, v[layer], v[3 * L + 1], v[3 * L + 2], out=dout[k][layer], order=v[3 * L + 3])
+        launch(views[k], dout[k])
         ev = torch.cuda.Event()
         ev.record(stream)
         comp[k] = ev
-        with torch.cuda.stream(cs):
-            cs.wait_event(ev)
-            for layer in range(L):
-                hout[k][layer].copy_(dout[k][layer], non_blocking=True)
+        with torch.cuda.stream(cs_dn):
+            cs_dn.wait_event(ev)
+            for h, d in zip(hout[k], dout[k]):
+                h.copy_(d, non_blocking=True)
             dn = torch.cuda.Event()
-            dn.record(cs)
+            dn.record(cs_dn)
             down[k] = dn
 
     for i in range(W):
@@ -773,17 +762,36 @@ def run_e2e(case, torch, pk, flush, stream, K, W):
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    cs.wait_event(a)  # the first upload starts inside the region
+    cs_up.wait_event(a)  # the first upload starts inside the region
     for i in range(K):
         step(W + i)
     stream.wait_event(down[(W + K - 1) % 2])  # the last read-back is inside the region
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / K
+    return a.elapsed_time(b) / K, h2d, d2h
+
+
+PIPELINE_MODE = ("pipelined: one packed upload per step on an upload stream (double-buffered), "
+                 "read-back of every step's output on a read-back stream; K steps timed as one region")
+
+
+def run_e2e(case, torch, pk, flush, stream, K, W):
+    """The decode step through the C ABI from pinned host memory, pipelined
+    the way a serving loop runs it (pipelined_e2e): inputs are q, the new
+    K/V of every layer, slots, tables, lengths and order.  The decode reads
+    more than L2 holds each step, so there is no flush in between."""
+    L = case.L
+    ins = list(case.q) + list(case.kn) + list(case.vn) + [case.slots, case.tables_d, case.lens_d, case.order_d]
+
+    def launch(v, outs):
+        for layer in range(L):
+            case.write(layer, v[L + layer], v[2 * L + layer], v[3 * L])
+            case.decode(layer, v[layer], v[3 * L + 1], v[3 * L + 2], out=outs[layer], order=v[3 * L + 3])
+
+    ms, h2d, d2h = pipelined_e2e(torch, stream, ins, list(case.out), launch, K, W)
     return {"value": round(case.step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "mode": "pipelined: one packed upload per step on a copy stream (double-buffered), "
-                    "read-back of every step's output; K steps timed as one region"}
+            "mode": PIPELINE_MODE}
 
 
 # ------------------------------------------------------ multi-token leg
@@ -907,6 +915,9 @@ def run_prefill(args, rank, world, local_rank):
     ms_per_step = total_ms / K
     pf_avg = sum(pf_ms) / K
     e2e = run_e2e_prefill(case, torch, flush, stream, K, args.warmup)
+    e2e_ms = max_over_ranks(e2e["ms_per_step"] * K, dist, "cuda") / K
+    e2e["ms_per_step"] = round(e2e_ms, 5)
+    e2e["value"] = round(world * case.flops / (e2e_ms * 1e-3) / 1e12, 2)
     if pk.kv_get_device_error() != pk.KV_OK:
         raise RuntimeError("device error during timing")
     peak, peak_kind = tensor_peak()
@@ -959,39 +970,20 @@ def run_prefill(args, rank, world, local_rank):
 
 
 def run_e2e_prefill(case, torch, flush, stream, K, W):
-    """The same step from pinned host memory: H2D of q, new K/V, slots,
-    cu_seqlens, tables and lengths, write + attention, D2H of the output."""
-    hs = [t.cpu().pin_memory() for t in (case.q, case.kn, case.vn, case.slots, case.cu, case.tables_d,
-                                         case.lens_d)]
-    ds = [torch.empty_like(t) for t in (case.q, case.kn, case.vn, case.slots, case.cu, case.tables_d,
-                                        case.lens_d)]
-    hout = torch.empty(case.out.shape, dtype=case.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in hs)
-    d2h = hout.numel() * hout.element_size()
+    """The multi-token step from pinned host memory, pipelined like the
+    decode leg (pipelined_e2e): inputs are q, the new K/V, slots,
+    cu_seqlens, tables and lengths; the output comes back every step.  The
+    step moves hundreds of MB over PCIe, more than L2 holds."""
+    ins = [case.q, case.kn, case.vn, case.slots, case.cu, case.tables_d, case.lens_d]
 
-    def step():
-        for d, h in zip(ds, hs):
-            d.copy_(h, non_blocking=True)
-        q, kn, vn, slots, cu, tables, lens = ds
+    def launch(v, outs):
+        q, kn, vn, slots, cu, tables, lens = v
         case.write(kn, vn, slots)
-        case.prefill(q, cu, tables, lens)
-        hout.copy_(case.out, non_blocking=True)
+        case.prefill(q, cu, tables, lens, out=outs[0])
 
-    for _ in range(W):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    for i in range(K):
-        flush.zero_()
-        a[i].record(stream)
-        step()
-        b[i].record(stream)
-    torch.cuda.synchronize()
-    ms = sum(a[i].elapsed_time(b[i]) for i in range(K)) / K
+    ms, h2d, d2h = pipelined_e2e(torch, stream, ins, [case.out], launch, K, W)
     return {"value": round(case.flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "mode": PIPELINE_MODE}
 
 
 def cpu_baseline_prefill(case, target_s=15.0):

@@ -100,6 +100,22 @@ def test_prefill_long_prompts_many_tiles(hq, hkv, n):
     assert max_abs(out.cpu().numpy(), ref) <= TOL[BF16]
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_many_items_per_persistent_cta(d):
+    """Far more work items than SMs, so every persistent CTA takes over the
+    items of CTAs whose launch it cancels and its barrier phases carry across
+    items of different lengths; most sequences are much shorter than the
+    longest, so runs of items without tokens are skipped in between."""
+    rng = np.random.default_rng(77 + d)
+    q_lens = rng.integers(1, 120, size=48).astype(np.int32)
+    q_lens[[5, 30]] = [600, 400]
+    prior = rng.integers(0, 300, size=48).astype(np.int32)
+    out, ref = run_case(BF16, d, 16, 32, 4, prior + q_lens, q_lens, seed=11 + d)
+    got = out.cpu().numpy()
+    assert not np.isnan(got).any()
+    assert max_abs(got, ref) <= TOL[BF16]
+
+
 def test_prefill_large_logits_move_the_reference_max():
     """A scale that makes logits span many binades forces rescales of O."""
     out, ref = run_case(F16, 64, 16, 4, 2, [600, 300], [600, 150], seed=9, scale=0.9)
