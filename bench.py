@@ -173,6 +173,24 @@ def job_value(bytes_per_rank, world, max_ms):
     return world * bytes_per_rank / (max_ms * 1e-3) / 1e9
 
 
+class L2Flush:
+    """Evicts L2 (126 MB on B200) between timed steps: zero_() writes a
+    256 MiB buffer and then reads another 256 MiB, so the dirty lines the
+    write leaves are written back before the next step starts (otherwise
+    the step pays for ~126 MB of write-backs that are not its own work)."""
+
+    def __init__(self, torch):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(64 << 20, dtype=torch.float32, device="cuda")
+
+    def zero_(self):
+        self.w.zero_()
+        self.r.sum()
+
+
+L2_NOTE = "flushed between steps (256 MiB write, then 256 MiB read: no dirty lines left)"
+
+
 # --------------------------------------------------------------- workloads
 
 class Case:
@@ -273,7 +291,7 @@ def run_ours(args, rank, world, local_rank):
         case.ws = torch.empty(max(case.ws_bytes, 16), dtype=torch.uint8, device="cuda")
         case.split = case.ws_bytes > 0
         case.launches_per_step = case.L * (2 + (1 if case.split else 0))
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+    flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
 
     def step(ev_write=None, ev_dec=None):
@@ -318,7 +336,17 @@ def run_ours(args, rank, world, local_rank):
     dec_bytes_per_launch = case.decode_bytes / case.L
 
     # end to end through the C ABI with host buffers (pinned), copies timed
-    e2e = run_e2e(case, torch, pk, flush, stream, K, args.warmup)
+    # a second replica with its own pool for the end-to-end loop (see
+    # run_e2e); with several layers consecutive decodes already read
+    # different pools
+    twin = case
+    if case.L == 1:
+        twin = Case(args.workload, rank, torch, pk, args)
+        if args.partition or args.stages or args.warps:
+            pk.kv_pool_set_decode_config(twin.pool, args.partition, args.stages, args.warps)
+            twin.ws_bytes, twin.ws, twin.split = case.ws_bytes, case.ws, case.split
+    e2e = run_e2e(case, twin, torch, pk, flush, stream, K, args.warmup)
+    del twin
     e2e_ms = max_over_ranks(e2e["ms_per_step"] * K, dist, "cuda") / K
     e2e["ms_per_step"] = round(e2e_ms, 5)
     e2e["value"] = round(job_value(case.step_bytes, world, e2e_ms), 2)
@@ -346,7 +374,7 @@ def run_ours(args, rank, world, local_rank):
             "workload": describe(w, case),
             "global_batch": w.batch * world,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": "flushed between steps (256 MiB write)",
+            "l2": L2_NOTE,
             "split_k": bool(case.split),
             "order": args.order or "longest",
         },
@@ -412,7 +440,7 @@ def run_trace(args, rank, world, local_rank):
     plan = gqa_trace_plan(w)
     tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
                   order_policy=args.order or "batch")
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
     iters = w.extra["iters"]
     W = min(args.warmup, iters - 1)
@@ -472,7 +500,7 @@ def run_trace(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded lognormal lengths, shared prefix, Poisson arrivals; q/K/V drawn on device)",
         "config": {"workload": describe(w), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between iterations (256 MiB write)",
+                   "l2": L2_NOTE.replace("steps", "iterations"),
                    "step": "one trace iteration: native scheduler step, metadata upload, copy-on-write block copies, cache write, decode"},
         "logical_gbs": round(logical, 2),
         "unique_bytes_per_step": int((uniq_b + other_b) / K), "logical_bytes_per_step": int((logi_b + other_b) / K),
@@ -500,7 +528,7 @@ def run_rag(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = WORKLOADS["rag_trace"]
     plan = rag_plan(w)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
     iters = w.extra["iters"]
     W = min(args.warmup, iters - 1)
@@ -550,7 +578,7 @@ def run_rag(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded documents, questions and Poisson arrivals; q/K/V drawn on device)",
         "config": {"workload": describe(w), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between iterations (256 MiB write)",
+                   "l2": L2_NOTE.replace("steps", "iterations"),
                    "step": "one iteration: scheduler step (prefix lookup), metadata upload, cache write, "
                            "prefill of uncached prompt tokens, decode of every running sequence"},
         "no_caching": {"tokens_per_s": round(off["tokens_per_s"], 1), "ms_per_step": round(off["ms_per_step"], 5),
@@ -620,7 +648,7 @@ def run_preempt(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = WORKLOADS["preempt_trace"]
     plan = preempt_plan(w)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
     iters = w.extra["iters"]
     W = min(args.warmup, iters - 1)
@@ -667,7 +695,7 @@ def run_preempt(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded prompt / output lengths and Poisson arrivals; q/K/V drawn on device)",
         "config": {"workload": describe(w), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between iterations (256 MiB write)",
+                   "l2": L2_NOTE.replace("steps", "iterations"),
                    "step": "one iteration: scheduler step (preemption, swap-in), metadata upload, swap copies, "
                            "copy-on-write, cache write, decode"},
         "swap": {k2: (round(v2, 3) if isinstance(v2, float) else v2) for k2, v2 in sw.items() if k2 != "clocks"},
@@ -714,6 +742,7 @@ def pipelined_e2e(torch, stream, ins, outs, launch, K, W):
     read-back stream.  The upload of step i + 1 overlaps the kernels of step
     i, and the read-back of step i the kernels of step i + 1.  The K steps
     are timed as one region (CUDA events on `stream`, every copy inside).
+    `launch(k, views, outs)` also gets the buffer index k (0 or 1).
     Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
     offs, off = [], 0
     for t in ins:
@@ -745,7 +774,7 @@ def pipelined_e2e(torch, stream, ins, outs, launch, K, W):
         stream.wait_event(up[k])
         if down[k] is not None:
             stream.wait_event(down[k])  # dout[k] was read back
-        launch(views[k], dout[k])
+        launch(k, views[k], dout[k])
         ev = torch.cuda.Event()
         ev.record(stream)
         comp[k] = ev
@@ -775,18 +804,24 @@ PIPELINE_MODE = ("pipelined: one packed upload per step on an upload stream (dou
                  "read-back of every step's output on a read-back stream; K steps timed as one region")
 
 
-def run_e2e(case, torch, pk, flush, stream, K, W):
+def run_e2e(case, twin, torch, pk, flush, stream, K, W):
     """The decode step through the C ABI from pinned host memory, pipelined
     the way a serving loop runs it (pipelined_e2e): inputs are q, the new
-    K/V of every layer, slots, tables, lengths and order.  The decode reads
-    more than L2 holds each step, so there is no flush in between."""
+    K/V of every layer, slots, tables, lengths and order.  Consecutive steps
+    alternate between `case` and `twin`, a replica with its own pool memory
+    (the same inputs address it): in a model, consecutive decode calls read
+    different layers' pools, and each step reads more than L2 holds, so
+    nothing one step leaves in L2 serves the next and no flush is needed in
+    between."""
     L = case.L
     ins = list(case.q) + list(case.kn) + list(case.vn) + [case.slots, case.tables_d, case.lens_d, case.order_d]
+    cases = (case, twin)
 
-    def launch(v, outs):
+    def launch(k, v, outs):
+        c = cases[k]
         for layer in range(L):
-            case.write(layer, v[L + layer], v[2 * L + layer], v[3 * L])
-            case.decode(layer, v[layer], v[3 * L + 1], v[3 * L + 2], out=outs[layer], order=v[3 * L + 3])
+            c.write(layer, v[L + layer], v[2 * L + layer], v[3 * L])
+            c.decode(layer, v[layer], v[3 * L + 1], v[3 * L + 2], out=outs[layer], order=v[3 * L + 3])
 
     ms, h2d, d2h = pipelined_e2e(torch, stream, ins, list(case.out), launch, K, W)
     return {"value": round(case.step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
@@ -877,7 +912,7 @@ def run_prefill(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     case = PrefillCase(args.workload, rank, torch, pk)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
 
     def step(ev_w=None, ev_p=None):
@@ -941,7 +976,7 @@ def run_prefill(args, rank, world, local_rank):
             "workload": describe_prefill(w, case),
             "global_batch": w.batch * world,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": "flushed between steps (256 MiB write)",
+            "l2": L2_NOTE,
         },
         "new_tokens_per_s": round(world * case.T / (ms_per_step * 1e-3), 1),
         "pct_of_tensor_peak": round(100.0 * value / world / peak, 2),
@@ -976,7 +1011,7 @@ def run_e2e_prefill(case, torch, flush, stream, K, W):
     step moves hundreds of MB over PCIe, more than L2 holds."""
     ins = [case.q, case.kn, case.vn, case.slots, case.cu, case.tables_d, case.lens_d]
 
-    def launch(v, outs):
+    def launch(k, v, outs):
         q, kn, vn, slots, cu, tables, lens = v
         case.write(kn, vn, slots)
         case.prefill(q, cu, tables, lens, out=outs[0])
