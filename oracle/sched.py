@@ -15,7 +15,7 @@ Written from "vLLM æ¨ç†åŠ é€ŸåŸç†è¯¦è§£ï¼šå¤§æ¨¡å‹æœåŠ¡ååé‡ä¸ºä½•èƒ½æ
   allocate it, allocate and move it to the running set, (4) decode the
   running set.
 
-Readings where the page leaves a step open (each also listed in the design doc):
+Readings where the page leaves a step open:
 
 * sharing implies a reference count per physical block; a block returns to
   the free list when its count reaches zero;
@@ -399,8 +399,7 @@ class Scheduler:
 #
 # "vLLM æ¨ç†åŠ é€ŸåŸç†è¯¦è§£" mentions automatic prefix caching (requests that
 # share a system prompt reuse its KV blocks; the pitfalls section and the
-# deployment flags) without describing the lookup.  Reading taken here (each
-# item also listed in the design doc):
+# deployment flags) without describing the lookup.  Reading taken here:
 #
 # * only FULL blocks are cached; block i of a sequence is keyed by
 #   key_i = FNV-1a-64(key_{i-1} as 8 little-endian bytes, then the block's
