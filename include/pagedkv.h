@@ -239,7 +239,10 @@ int kv_pool_set_sliding_window(kv_pool* pool, int window);
  *                 q_len > n, q_len > max_q_len, rows past total_q, or
  *                 n > max_blocks_per_seq * block_size is skipped and
  *                 reported as KV_ERR_BOUNDS by kv_get_device_error, as is a
- *                 block id outside the pool (that CTA stops).
+ *                 block id outside the pool (the CTA that meets it stops; the
+ *                 rows of its current work item, and of the one it had
+ *                 already claimed, are left unwritten).  A pipeline wait that
+ *                 runs out (2 s) records KV_ERR_TIMEOUT the same way.
  *   scale         finite and > 0.
  *   out           device [total_q][num_q_heads][head_dim] of out_dtype (the
  *                 pool dtype or KV_F32), 16-byte aligned.
