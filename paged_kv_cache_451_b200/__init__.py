@@ -218,8 +218,9 @@ def kv_sched_swap_outputs(s):
     out = {"swap_out": np.empty((n[0].value, 2), np.int32), "swap_in": np.empty((n[1].value, 2), np.int32),
            "preempted": np.empty(n[2].value, np.int64), "recomputed": np.empty(n[3].value, np.int64),
            "swapped_in": np.empty(n[4].value, np.int64), "num_swapped": n[5].value}
-    _check(_lib.kv_sched_swap_outputs(s, _ptr(out["swap_out"]), _ptr(out["swap_in"]), _ptr(out["preempted"]),
-                                      _ptr(out["recomputed"]), _ptr(out["swapped_in"])))
+    if n[0].value or n[1].value or n[2].value or n[3].value or n[4].value:  # else nothing to copy
+        _check(_lib.kv_sched_swap_outputs(s, _ptr(out["swap_out"]), _ptr(out["swap_in"]), _ptr(out["preempted"]),
+                                          _ptr(out["recomputed"]), _ptr(out["swapped_in"])))
     return out
 
 
