@@ -345,7 +345,7 @@ def run_ours(args, rank, world, local_rank):
         if args.partition or args.stages or args.warps:
             pk.kv_pool_set_decode_config(twin.pool, args.partition, args.stages, args.warps)
             twin.ws_bytes, twin.ws, twin.split = case.ws_bytes, case.ws, case.split
-    e2e = run_e2e(case, twin, torch, pk, flush, stream, K, args.warmup)
+    e2e = run_e2e(case, twin, torch, stream, K, args.warmup)
     del twin
     e2e_ms = max_over_ranks(e2e["ms_per_step"] * K, dist, "cuda") / K
     e2e["ms_per_step"] = round(e2e_ms, 5)
@@ -804,7 +804,7 @@ PIPELINE_MODE = ("pipelined: one packed upload per step on an upload stream (dou
                  "read-back of every step's output on a read-back stream; K steps timed as one region")
 
 
-def run_e2e(case, twin, torch, pk, flush, stream, K, W):
+def run_e2e(case, twin, torch, stream, K, W):
     """The decode step through the C ABI from pinned host memory, pipelined
     the way a serving loop runs it (pipelined_e2e): inputs are q, the new
     K/V of every layer, slots, tables, lengths and order.  Consecutive steps
@@ -949,7 +949,7 @@ def run_prefill(args, rank, world, local_rank):
     total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / K
     pf_avg = sum(pf_ms) / K
-    e2e = run_e2e_prefill(case, torch, flush, stream, K, args.warmup)
+    e2e = run_e2e_prefill(case, torch, stream, K, args.warmup)
     e2e_ms = max_over_ranks(e2e["ms_per_step"] * K, dist, "cuda") / K
     e2e["ms_per_step"] = round(e2e_ms, 5)
     e2e["value"] = round(world * case.flops / (e2e_ms * 1e-3) / 1e12, 2)
@@ -1004,7 +1004,7 @@ def run_prefill(args, rank, world, local_rank):
     return line
 
 
-def run_e2e_prefill(case, torch, flush, stream, K, W):
+def run_e2e_prefill(case, torch, stream, K, W):
     """The multi-token step from pinned host memory, pipelined like the
     decode leg (pipelined_e2e): inputs are q, the new K/V, slots,
     cu_seqlens, tables and lengths; the output comes back every step.  The
