@@ -3,14 +3,24 @@
 One step = the cache write of the step's new tokens (paged_kv_write) and one
 PagedAttention decode over every sequence (paged_attention_decode, with its
 split-K reduce when contexts are split), all through the C ABI, on inputs
-resident in HBM.  Default workload: one Llama-2-13B-shaped layer (40 MHA
-heads, head_dim 128, fp16, block 16, batch 64, context lengths uniform in
-[128, 2048]).
+resident in HBM.  Default workload: the pages' KV-size example — 32 layers x
+32 heads x head_dim 128, bf16, block 16, 32 sequences of 2048 tokens (about
+1.07 GB of K/V per request, 34 GB in all) — one step covering all 32 layers.
 
 Prints one JSON line (rank 0).  ``value`` is achieved GB/s of algorithmic
 bytes (K/V read + q read + output write + the step's cache-write bytes) over
-the device-timed step, summed over ranks; ``--impl reference`` times the CPU
-oracle on the same workload instead.
+the device-timed step, summed over ranks; ``seqs_per_s`` is decode sequences
+per second (a step decodes every sequence through all its layers).  On one
+GPU the line also carries ``per_config``: the other measured decode
+workloads (the Llama-2-13B-shaped layer, the GQA continuous-batching trace,
+long-context FP8 under the automatic split and under 512-token partitions),
+each timed for at least a second with its own roofline, end-to-end figure and
+clock record.  ``--impl reference`` times the CPU oracle on the same workload
+instead.
+
+The CPU-baseline leg runs the oracle on sampled sequences of each workload,
+times it, and checks the GPU outputs of those sequences against it (outside
+every timed region); a mismatch makes the run exit non-zero.
 
 Multi-GPU: ``torchrun --nproc-per-node N bench.py --gpus N``: every rank runs
 an independent replica (decode shards by sequence with no exchange), time is
@@ -37,12 +47,14 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode attention: achieved KV-read GB/s (% of HBM peak); decode seqs/s"
 METRIC_PREFILL = "paged multi-token attention: achieved TFLOP/s (% of tensor peak); new tokens/s"
 PREFILL_WORKLOADS = ("prefill_llama13b", "prefill_gqa", "chunked_gqa")
+DECODE_WORKLOADS = ("tiny", "llama13b", "kv_example", "fp8_long", "window_long")
 METRIC_RAG = "retrieval-augmented serving with prefix caching: generated tokens/s (vs no caching)"
 METRIC_PREEMPT = "decode under memory pressure with swap preemption: generated tokens/s (vs recompute)"
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {0: "f16", 1: "bf16", 2: "e4m3"}
 ELEM = {0: 2, 1: 2, 2: 1}
+MIN_TIMED_S = 1.0  # every per-config measurement times at least this much device work
 
 
 # ------------------------------------------------------------------ helpers
@@ -65,25 +77,24 @@ def tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def decode_source_hash():
+def source_hash(files):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_451_b200", "csrc")
-    for f in ("decode.cuh", "ptx.cuh", "pagedkv.cu"):
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def decode_source_hash():
+    return source_hash(("decode.cuh", "ptx.cuh", "pagedkv.cu"))
 
 
 def prefill_source_hash():
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "paged_kv_cache_451_b200", "csrc")
-    for f in ("prefill.cuh", "tcgen05.cuh", "ptx.cuh", "prefill.cu"):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
-    return h.hexdigest()[:16]
+    return source_hash(("prefill.cuh", "tcgen05.cuh", "ptx.cuh", "prefill.cu"))
 
 
-def committed_traffic(workload, source_hash=None):
+def committed_traffic(workload, source_hash_=None):
     """DRAM bytes per launch of the workload's dominant kernel from a
     committed ncu capture, if it was taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -92,14 +103,16 @@ def committed_traffic(workload, source_hash=None):
             rec = json.load(f).get(workload)
     except Exception:  # noqa: BLE001
         return None
-    if not rec or rec.get("source_hash") != (source_hash or decode_source_hash()):
+    if not rec or rec.get("source_hash") != (source_hash_ or decode_source_hash()):
         return None
     return rec.get("bytes_per_launch")
 
 
 class ClockSampler:
-    """Polls NVML (the library nvidia-smi reads) for SM clock and throttle
-    reasons while the timed region runs.  Read-only."""
+    """Polls NVML (the library nvidia-smi reads) for the SM clock and the
+    throttle reasons every 2 ms from start() to stop(), keeping a host
+    timestamp with each sample; summary(t0, t1) describes the samples taken
+    while a timed region ran.  Read-only: it changes no setting."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -109,7 +122,7 @@ class ClockSampler:
     }
 
     def __init__(self, device_index):
-        self.samples, self.reasons = [], 0
+        self.samples = []  # (t, sm_mhz, reasons)
         self.ok = False
         self.max_mhz = None
         try:
@@ -129,33 +142,41 @@ class ClockSampler:
         except Exception:  # noqa: BLE001
             pass
         self._stop = threading.Event()
+        self.t = None
 
     def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
-                self.reasons |= self.get_reasons(self.h)
+                t = time.perf_counter()
+                mhz = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+                self.samples.append((t, mhz, int(self.get_reasons(self.h))))
             except Exception:  # noqa: BLE001
                 pass
             time.sleep(0.002)
 
-    def __enter__(self):
-        if self.ok:
+    def start(self):
+        if self.ok and self.t is None:
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
 
-    def __exit__(self, *a):
-        if self.ok:
+    def stop(self):
+        if self.t is not None:
             self._stop.set()
             self.t.join()
+            self.t = None
 
-    def summary(self):
-        if not self.ok or not self.samples:
+    def summary(self, t0, t1):
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not self.ok or not sel:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples), "source": "nvml"}
+        bits = 0
+        for s in sel:
+            bits |= s[2]
+        names = [n for bit, n in self.REASONS.items() if bits & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": self.max_mhz,
+                "sm_min_mhz": min(s[1] for s in sel), "reasons": names, "samples": len(sel),
+                "region_s": round(t1 - t0, 3), "source": "nvml, 2 ms polling during the timed region"}
 
 
 def max_over_ranks(value, dist, device):
@@ -191,67 +212,57 @@ class L2Flush:
 L2_NOTE = "flushed between steps (256 MiB write, then 256 MiB read: no dirty lines left)"
 
 
-# --------------------------------------------------------------- workloads
+def init_dist(world):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+# ------------------------------------------------------- single-step decode
 
 class Case:
-    """Device-resident inputs of one workload replica."""
+    """Device-resident inputs of one decode workload replica (drawn by
+    workloads.decode_inputs) bound to a pool of the product library."""
 
-    def __init__(self, name, rank, torch, pk, W):
-        from workloads import (WORKLOADS, blocks_needed, context_lens, device_normal_bits,
-                               device_pool, pool_blocks, scattered_tables, rng_for)
-        w = WORKLOADS[name]
-        self.w, self.torch, self.pk = w, torch, pk
-        self.lens = context_lens(w)
-        nb = pool_blocks(w, self.lens)
-        self.nb = nb
-        rng = np.random.default_rng([w.seed, 1000 + rank])
-        self.tables = scattered_tables(rng, self.lens, w.block_size, nb)
-        dev = torch.device("cuda")
-        seed = w.seed * 7919 + rank
-        self.L = w.num_layers
-        self.k, self.v, self.ks, self.vs = [], [], [], []
-        self.pool = pk.kv_pool_create(w.block_size, nb, w.kv_heads, w.head_dim, w.kv_fmt, self.L)
-        self.window = int(w.extra.get("window", 0))
+    def __init__(self, name, rank, torch, pk, args=None, layers=None, partition=None):
+        from paged_kv_cache_451_b200.serving import schedule_order
+        from workloads.decode_inputs import DecodeInputs
+        inp = DecodeInputs(name, rank, layers)
+        self.inp = inp
+        self.w, self.torch, self.pk = inp.w, torch, pk
+        w = self.w
+        self.lens, self.nb, self.tables, self.L, self.window = inp.lens, inp.nb, inp.tables, inp.L, inp.window
+        self.k, self.v, self.ks, self.vs = inp.k, inp.v, inp.ks, inp.vs
+        self.q, self.kn, self.vn, self.inv = inp.q, inp.kn, inp.vn, inp.inv
+        self.slots, self.tables_d, self.lens_d, self.max_ctx = inp.slots, inp.tables_d, inp.lens_d, inp.max_ctx
+        self.pool = pk.kv_pool_create(w.block_size, self.nb, w.kv_heads, w.head_dim, w.kv_fmt, self.L)
         if self.window:
             pk.kv_pool_set_sliding_window(self.pool, self.window)
         for layer in range(self.L):
-            k, v, ks, vs = device_pool(w, nb, dev, seed=seed + 13 * layer)
-            self.k.append(k)
-            self.v.append(v)
-            self.ks.append(ks)
-            self.vs.append(vs)
-            pk.kv_pool_bind(self.pool, layer, k, v, ks, vs)
+            pk.kv_pool_bind(self.pool, layer, self.k[layer], self.v[layer], self.ks[layer], self.vs[layer])
+        part = getattr(args, "partition", 0) if partition is None else partition
+        stages, warps = getattr(args, "stages", 0), getattr(args, "warps", 0)
+        if part or stages or warps:
+            pk.kv_pool_set_decode_config(self.pool, part, stages, warps)
+        self.partition = part
         B, Hq, Hkv, D = w.batch, w.num_q_heads, w.kv_heads, w.head_dim
-        self.q = [device_normal_bits((B, Hq, D), w.q_fmt, dev, seed + 1 + 17 * l) for l in range(self.L)]
-        self.kn = [device_normal_bits((B, Hkv, D), w.q_fmt, dev, seed + 2 + 17 * l) for l in range(self.L)]
-        self.vn = [device_normal_bits((B, Hkv, D), w.q_fmt, dev, seed + 3 + 17 * l) for l in range(self.L)]
-        # the step writes each sequence's last token (position len-1)
-        pos = self.lens.astype(np.int64) - 1
-        self.slots_h = (self.tables[np.arange(B), pos // w.block_size].astype(np.int64) * w.block_size
-                        + pos % w.block_size)
-        self.slots = torch.from_numpy(self.slots_h).to(dev)
-        self.tables_d = torch.from_numpy(self.tables).to(dev)
-        self.lens_d = torch.from_numpy(self.lens).to(dev)
         # the caller's scheduling order (placement only): long contexts first
-        from paged_kv_cache_451_b200.serving import schedule_order
-        self.order_h = schedule_order(self.lens, getattr(W, "order", None) or "longest")
-        self.order_d = torch.from_numpy(self.order_h).to(dev)
-        self.inv = None
-        if w.kv_fmt == 2:
-            self.inv = [(1.0 / self.ks[l], 1.0 / self.vs[l]) for l in range(self.L)]
-        self.max_ctx = int(self.lens.max())
-        out_dt = torch.float16 if w.q_fmt == 0 else torch.bfloat16
-        self.out = [torch.empty((B, Hq, D), dtype=out_dt, device=dev) for _ in range(self.L)]
+        self.order_name = getattr(args, "order", None) or "longest"
+        self.order_h = schedule_order(self.lens, self.order_name)
+        self.order_d = torch.from_numpy(self.order_h).to("cuda")
+        self.out = [torch.empty((B, Hq, D), dtype=inp.out_torch_dtype, device="cuda") for _ in range(self.L)]
         self.ws_bytes = pk.paged_attention_workspace_bytes(self.pool, B, Hq, self.max_ctx)
-        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device="cuda")
         self.split = self.ws_bytes > 0
+        self.num_parts = self.ws_bytes // (B * Hq * (D + 4) * 4) if self.split else 1
         e_kv, e_q = ELEM[w.kv_fmt], ELEM[w.q_fmt]
-        blocks_touched = int(blocks_needed(self.lens, w.block_size).sum())
-        # attended tokens per sequence: the whole context, or the window
-        self.attended = np.minimum(self.lens, self.window) if self.window else self.lens
+        self.attended = inp.attended
         self.decode_bytes = self.L * (int(self.attended.astype(np.int64).sum()) * Hkv * D * 2 * e_kv
                                       + B * Hq * D * (e_q + e_q)
-                                      + (2 * 4 * blocks_touched * Hkv if w.kv_fmt == 2 else 0))
+                                      + (2 * 4 * inp.blocks_touched * Hkv if w.kv_fmt == 2 else 0))
         self.write_bytes = self.L * B * Hkv * D * 2 * (e_q + e_kv)
         self.step_bytes = self.decode_bytes + self.write_bytes
         self.launches_per_step = self.L * (2 + (1 if self.split else 0))
@@ -272,99 +283,138 @@ class Case:
                                   w.q_fmt, self.ws, self.ws_bytes,
                                   seq_order=self.order_d if order is None else order)
 
+    def destroy(self):
+        self.pk.kv_pool_destroy(self.pool)
+
+
+def timed_steps(case, K, flush, stream, clk):
+    """K device-timed steps (L2 flushed before each): returns (step ms list,
+    decode-launch ms list, clock summary).  A step is, for every layer, the
+    cache write then the decode (and its reduce)."""
+    torch = case.torch
+    L = case.L
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    evw = [[torch.cuda.Event(enable_timing=True) for _ in range(L)] for _ in range(K)]
+    evd = [[torch.cuda.Event(enable_timing=True) for _ in range(L)] for _ in range(K)]
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        ev0[i].record(stream)
+        for layer in range(L):
+            case.write(layer)
+            evw[i][layer].record(stream)
+            case.decode(layer)
+            evd[i][layer].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    step_ms = [ev0[i].elapsed_time(evd[i][-1]) for i in range(K)]
+    dec_ms = [evw[i][l].elapsed_time(evd[i][l]) for i in range(K) for l in range(L)]
+    return step_ms, dec_ms, clk.summary(t0, t1)
+
+
+def decode_roofline(case, dec_ms, workload_key):
+    peak, peak_kind = hbm_peak()
+    dec_avg = sum(dec_ms) / len(dec_ms)
+    per_launch = case.decode_bytes / case.L
+    achieved = per_launch / (dec_avg * 1e-3) / 1e9
+    return {
+        "bound": "hbm",
+        "kernel": "paged_attention_decode (decode kernel" + (" + LSE reduce)" if case.split else ")"),
+        "achieved": round(achieved, 2),
+        "peak": peak,
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "traffic": committed_traffic(workload_key),
+        "algorithmic_bytes_per_launch": per_launch,
+        "launch_ms": round(dec_avg, 5),
+        "peak_note": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback copy bandwidth",
+    }
+
+
+def measure_decode(case, args, stream, flush, clk, dist, world, K=None, min_s=None, key=None):
+    """Warm-up, then the device-timed steps (exactly K, or enough for min_s
+    seconds of device time), the end-to-end loop with host buffers, and the
+    roofline of the decode kernel.  Returns a dict of figures."""
+    torch, pk = case.torch, case.pk
+    W = args.warmup
+    for _ in range(W):
+        flush.zero_()
+        for layer in range(case.L):
+            case.write(layer)
+            case.decode(layer)
+    torch.cuda.synchronize()
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error during warm-up")
+    if K is None:  # calibrate: enough steps for min_s seconds of device time
+        cal, _, _ = timed_steps(case, 5, flush, stream, clk)
+        K = max(5, int(math.ceil(min_s * 1e3 / (sum(cal) / len(cal)))))
+    if dist:
+        dist.barrier()
+    step_ms, dec_ms, clocks = timed_steps(case, K, flush, stream, clk)
+    if dist:
+        dist.barrier()
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
+    ms_per_step = total_ms / K
+    # end to end through the C ABI with host buffers (pinned), copies timed; a
+    # second replica with its own pool alternates with this one when the step
+    # has a single layer (see run_e2e); with several layers consecutive
+    # decodes already read different pools
+    twin = case
+    if case.L == 1:
+        twin = Case(case.w.name, 0, torch, pk, args, partition=case.partition)
+        twin.ws_bytes, twin.ws, twin.split = case.ws_bytes, case.ws, case.split
+    K_e2e = K if min_s is None else max(K, 5)
+    e2e = run_e2e(case, twin, torch, stream, K_e2e, W, clk)
+    if twin is not case:
+        twin.destroy()
+    del twin
+    e2e_ms = max_over_ranks(e2e["ms_per_step"] * K_e2e, dist, "cuda") / K_e2e
+    e2e["ms_per_step"] = round(e2e_ms, 5)
+    e2e["value"] = round(job_value(case.step_bytes, world, e2e_ms), 2)
+    e2e["steps"] = K_e2e
+    if pk.kv_get_device_error() != pk.KV_OK:
+        raise RuntimeError("device error during timing")
+    peak, _ = hbm_peak()
+    value = job_value(case.step_bytes, world, ms_per_step)
+    return {
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "steps": K,
+        "ms_per_step": round(ms_per_step, 5),
+        "timed_device_s": round(total_ms / 1e3, 4),
+        "seqs_per_s": round(world * case.w.batch / (ms_per_step * 1e-3), 1),
+        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
+        "roofline": decode_roofline(case, dec_ms, key or case.w.name),
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": case.launches_per_step * K,
+        "split_k": {"partitions": case.num_parts, "partition_tokens": case.partition or "auto"},
+    }
+
 
 def run_ours(args, rank, world, local_rank):
     import torch
     import paged_kv_cache_451_b200 as pk
 
     torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    case = Case(args.workload, rank, torch, pk, args)
-    if args.partition or args.stages or args.warps:
-        pk.kv_pool_set_decode_config(case.pool, args.partition, args.stages, args.warps)
-        case.ws_bytes = pk.paged_attention_workspace_bytes(case.pool, case.w.batch, case.w.num_q_heads, case.max_ctx)
-        case.ws = torch.empty(max(case.ws_bytes, 16), dtype=torch.uint8, device="cuda")
-        case.split = case.ws_bytes > 0
-        case.launches_per_step = case.L * (2 + (1 if case.split else 0))
+    dist = init_dist(world)
+    clk = ClockSampler(local_rank).start()
     flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
-
-    def step(ev_write=None, ev_dec=None):
-        for layer in range(case.L):
-            case.write(layer)
-            if ev_write is not None:
-                ev_write[layer].record(stream)
-            case.decode(layer)
-            if ev_dec is not None:
-                ev_dec[layer].record(stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    if pk.kv_get_device_error() != pk.KV_OK:
-        raise RuntimeError("device error during warm-up")
-
-    K = args.steps
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    evw = [[torch.cuda.Event(enable_timing=True) for _ in range(case.L)] for _ in range(K)]
-    evd = [[torch.cuda.Event(enable_timing=True) for _ in range(case.L)] for _ in range(K)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        for i in range(K):
-            flush.zero_()
-            ev0[i].record(stream)
-            step(evw[i], evd[i])
-        torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    step_ms = [ev0[i].elapsed_time(evd[i][-1]) for i in range(K)]
-    dec_ms = []
-    for i in range(K):
-        for layer in range(case.L):
-            dec_ms.append(evw[i][layer].elapsed_time(evd[i][layer]))
-    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
-    ms_per_step = total_ms / K
-    dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    dec_bytes_per_launch = case.decode_bytes / case.L
-
-    # end to end through the C ABI with host buffers (pinned), copies timed
-    # a second replica with its own pool for the end-to-end loop (see
-    # run_e2e); with several layers consecutive decodes already read
-    # different pools
-    twin = case
-    if case.L == 1:
-        twin = Case(args.workload, rank, torch, pk, args)
-        if args.partition or args.stages or args.warps:
-            pk.kv_pool_set_decode_config(twin.pool, args.partition, args.stages, args.warps)
-            twin.ws_bytes, twin.ws, twin.split = case.ws_bytes, case.ws, case.split
-    e2e = run_e2e(case, twin, torch, stream, K, args.warmup)
-    del twin
-    e2e_ms = max_over_ranks(e2e["ms_per_step"] * K, dist, "cuda") / K
-    e2e["ms_per_step"] = round(e2e_ms, 5)
-    e2e["value"] = round(job_value(case.step_bytes, world, e2e_ms), 2)
-    if pk.kv_get_device_error() != pk.KV_OK:
-        raise RuntimeError("device error during timing")
-
-    peak, peak_kind = hbm_peak()
-    value = job_value(case.step_bytes, world, ms_per_step)
-    achieved = dec_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
+    case = Case(args.workload, rank, torch, pk, args, layers=args.layers)
+    key = args.workload if args.layers is None else f"{args.workload}_layers{args.layers}"
+    m = measure_decode(case, args, stream, flush, clk, dist, world, K=args.steps, key=key)
     w = case.w
     line = {
         "metric": METRIC,
-        "value": round(value, 2),
+        "value": m["value"],
         "unit": "GB/s",
         "n_gpus": world,
-        "steps": K,
+        "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 5),
+        "ms_per_step": m["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -373,39 +423,66 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": describe(w, case),
             "global_batch": w.batch * world,
+            "layers_per_step": case.L,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": L2_NOTE,
             "split_k": bool(case.split),
-            "order": args.order or "longest",
+            "order": case.order_name,
         },
-        "seqs_per_s": round(world * w.batch / (ms_per_step * 1e-3), 1),
-        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
-        "hbm_peak_gbs": peak,
-        "hbm_peak_kind": peak_kind,
-        "roofline": {
-            "bound": "hbm",
-            "kernel": "paged_attention_decode (decode kernel" + (" + LSE reduce)" if case.split else ")"),
-            "achieved": round(achieved, 2),
-            "peak": peak,
-            "unit": "GB/s",
-            "frac": round(achieved / peak, 4),
-            "traffic": committed_traffic(args.workload),
-            "algorithmic_bytes_per_launch": dec_bytes_per_launch,
-            "launch_ms": round(dec_avg_ms, 5),
-            "peak_note": f"{peak_kind} copy bandwidth",
-        },
-        "e2e": e2e,
-        "clocks": clk.summary(),
-        "gpu_launches": case.launches_per_step * K,
+        "seqs_per_s": m["seqs_per_s"],
+        "pct_of_hbm_peak": m["pct_of_hbm_peak"],
+        "hbm_peak_gbs": hbm_peak()[0],
+        "hbm_peak_kind": hbm_peak()[1],
+        "roofline": m["roofline"],
+        "e2e": m["e2e"],
+        "clocks": m["clocks"],
+        "gpu_launches": m["gpu_launches"],
     }
-    if dist:
-        dist.barrier()
+    # the same step repeated for at least a second, for a sustained figure
+    # and a clock record over a long region
+    if not args.no_extras:
+        K_s = max(args.steps, int(math.ceil(MIN_TIMED_S * 1e3 / m["ms_per_step"])))
+        if dist:
+            dist.barrier()
+        step_ms, _, clocks = timed_steps(case, K_s, flush, stream, clk)
+        if dist:
+            dist.barrier()
+        tot = max_over_ranks(sum(step_ms), dist, "cuda")
+        line["sustained"] = {"steps": K_s, "ms_per_step": round(tot / K_s, 5),
+                             "value": round(job_value(case.step_bytes, world, tot / K_s), 2),
+                             "timed_device_s": round(tot / 1e3, 3), "clocks": clocks}
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(case, torch, target_s=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(case, target_s=args.cpu_seconds, check=True)
+    case.destroy()
+    del case
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extras and args.workload == "kv_example":
+        line["per_config"] = per_config(args, torch, pk, stream, flush, clk)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+    clk.stop()
     return line
+
+
+def per_config(args, torch, pk, stream, flush, clk):
+    """The other measured decode workloads, each timed for at least
+    MIN_TIMED_S seconds of device time, with its own roofline, end-to-end
+    figure, clock record and (CPU-baseline leg) sampled oracle check."""
+    res = {}
+    for name, label, part in (("llama13b", "llama13b", None), ("fp8_long", "fp8_long", None),
+                              ("fp8_long", "fp8_long_partition512", 512)):
+        case = Case(name, 0, torch, pk, args, partition=part or 0)
+        m = measure_decode(case, args, stream, flush, clk, None, 1, min_s=MIN_TIMED_S, key=label)
+        m["workload"] = describe(case.w, case)
+        if not args.no_cpu_baseline:
+            m["oracle_check"] = cpu_baseline(case, target_s=0.0, check=True)["check"]
+        case.destroy()
+        del case
+        torch.cuda.empty_cache()
+        res[label] = m
+    res["gqa_trace"] = trace_measure(args, 0, 1, 0, None, clk, flush, stream, min_s=MIN_TIMED_S)
+    return res
 
 
 def unique_and_logical_tokens(tables, lens, block_size):
@@ -423,92 +500,143 @@ def unique_and_logical_tokens(tables, lens, block_size):
     return sum(best.values()), logical
 
 
-def run_trace(args, rank, world, local_rank):
-    """The GQA continuous-batching trace: one step = one trace iteration."""
+def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s=None):
+    """The GQA continuous-batching trace: one step = one trace iteration
+    (native scheduler step, metadata upload, copy-on-write block copies,
+    cache write, decode).  The trace's iterations after the warm-up are
+    timed; with min_s the trace is replayed (same seed, a fresh pool each
+    pass) until the timed regions span at least min_s seconds."""
     import torch
     import paged_kv_cache_451_b200 as pk
     from workloads import WORKLOADS, gqa_trace_plan
     from workloads.gqa_trace import GqaTrace
 
-    torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = WORKLOADS["gqa_trace"]
     plan = gqa_trace_plan(w)
-    tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
-                  order_policy=args.order or "batch")
-    flush = L2Flush(torch)
-    stream = torch.cuda.current_stream()
     iters = w.extra["iters"]
     W = min(args.warmup, iters - 1)
-    K = max(1, min(args.steps, iters - W))
-    e = w.extra
+    K = max(1, min(args.steps, iters - W)) if min_s is None else iters - W
     hq, hkv, d = w.num_q_heads, w.kv_heads, w.head_dim
-    for it in range(W):
-        flush.zero_()
-        tr.iteration(it, out_dtype=w.q_fmt)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    uniq_b = logi_b = other_b = 0
-    launches = 0
+    per_tok = hkv * d * 2 * 2
+    tot_ms = dec_ms = 0.0
+    uniq_b = logi_b = other_b = dec_b = 0
+    launches = steps = 0
     host_s = sched_s = 0.0
+    regions = []
+    passes = 0
+    while True:
+        tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
+                      order_policy=args.order or "batch")
+        for it in range(W):
+            flush.zero_()
+            tr.iteration(it, out_dtype=w.q_fmt)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        mids = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
 
-    def gate_and_start(i):
-        # keep the GPU busy (~1 ms device sleep) while the host enqueues the
-        # iteration, so the timed interval is the fed-GPU time of the step
-        torch.cuda._sleep(2_000_000)
-        starts[i].record(stream)
+        def gate_and_start(i):
+            # keep the GPU busy (~1 ms device sleep) while the host enqueues
+            # the iteration, so the timed interval is the fed-GPU time of the step
+            torch.cuda._sleep(2_000_000)
+            starts[i].record(stream)
 
-    with ClockSampler(local_rank) as clk:
+        t0 = time.perf_counter()
         for i in range(K):
             flush.zero_()
-            t0 = time.perf_counter()
+            h0 = time.perf_counter()
             fin, arr, pl, q, kn, vn, out = tr.iteration(W + i, out_dtype=w.q_fmt,
                                                         before_launch=lambda: gate_and_start(i),
-                                                        after_launch=lambda: ends[i].record(stream))
-            host_s += time.perf_counter() - t0
+                                                        after_launch=lambda: ends[i].record(stream),
+                                                        before_decode=lambda s: mids[i].record(s))
+            host_s += time.perf_counter() - h0
             sched_s += tr.last_schedule_s
             info = pl["info"]
             u, l = unique_and_logical_tokens(pl["block_tables"], pl["context_lens"], w.block_size)
-            per_tok = hkv * d * 2 * 2
             uniq_b += u * per_tok
             logi_b += l * per_tok
-            other_b += (info.batch * hq * d * 4 + info.num_tokens * hkv * d * 2 * 4
+            qo = info.batch * hq * d * 4
+            dec_b += u * per_tok + qo
+            other_b += (qo + info.num_tokens * hkv * d * 2 * 4
                         + info.num_cow * hkv * w.block_size * d * 2 * 2 * 2)
             launches += 2 + (1 if info.num_cow else 0) + (
                 1 if pk.paged_attention_workspace_bytes(tr.pool, info.batch, hq, int(pl["context_lens"].max())) else 0)
         torch.cuda.synchronize()
-    if pk.kv_get_device_error() != pk.KV_OK:
-        raise RuntimeError("device error during the trace")
-    total_ms = max_over_ranks(sum(starts[i].elapsed_time(ends[i]) for i in range(K)), dist, "cuda")
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
-    ms = total_ms / K
+        t1 = time.perf_counter()
+        regions.append((t0, t1))
+        if pk.kv_get_device_error() != pk.KV_OK:
+            raise RuntimeError("device error during the trace")
+        tot_ms += sum(starts[i].elapsed_time(ends[i]) for i in range(K))
+        dec_ms += sum(mids[i].elapsed_time(ends[i]) for i in range(K))
+        steps += K
+        passes += 1
+        del tr
+        if min_s is None or sum(b - a for a, b in regions) >= min_s or passes >= 8:
+            break
+    total_ms = max_over_ranks(tot_ms, dist, "cuda")
+    ms = total_ms / steps
     peak, peak_kind = hbm_peak()
     value = world * (uniq_b + other_b) / (total_ms * 1e-3) / 1e9
     logical = world * (logi_b + other_b) / (total_ms * 1e-3) / 1e9
+    achieved = dec_b / (dec_ms * 1e-3) / 1e9
+    # clocks over every pass's timed region
+    samples = [s for a, b in regions for s in clk.samples if a <= s[0] <= b]
+    clocks = clk.summary(regions[0][0], regions[-1][1]) if samples else clk.summary(0, -1)
+    if samples:
+        clocks["samples"] = len(samples)
+        clocks["sm_mhz"] = statistics.median(s[1] for s in samples)
+        clocks["region_s"] = round(sum(b - a for a, b in regions), 3)
     return {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
-        "warmup": W, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "value": round(value, 2), "unit": "GB/s", "steps": steps, "passes": passes, "warmup": W,
+        "ms_per_step": round(ms, 5), "timed_device_s": round(total_ms / 1e3, 4),
+        "workload": describe(w),
+        "logical_gbs": round(logical, 2),
+        "unique_bytes_per_step": int((uniq_b + other_b) / steps),
+        "logical_bytes_per_step": int((logi_b + other_b) / steps),
+        "host_scheduler_ms_per_step": round(1e3 * sched_s / steps, 3),
+        "host_iteration_ms_per_step": round(1e3 * host_s / steps, 3),
+        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {
+            "bound": "hbm", "kernel": "paged_attention_decode (decode kernel, + LSE reduce when split)",
+            "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": committed_traffic("gqa_trace"),
+            "algorithmic_bytes_per_launch": int(dec_b / steps),
+            "launch_ms": round(dec_ms / steps, 5),
+            "bytes_note": "unique physical K/V bytes (shared prefix blocks counted once) + q + out",
+            "peak_note": f"{peak_kind} copy bandwidth"},
+        "clocks": clocks, "gpu_launches": launches,
+        "step": "one trace iteration: native scheduler step, metadata upload, copy-on-write block copies, "
+                "cache write, decode",
+    }
+
+
+def run_trace(args, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    dist = init_dist(world)
+    clk = ClockSampler(local_rank).start()
+    flush = L2Flush(torch)
+    stream = torch.cuda.current_stream()
+    m = trace_measure(args, rank, world, local_rank, dist, clk, flush, stream)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    clk.stop()
+    line = {
+        "metric": METRIC, "value": m["value"], "unit": "GB/s", "n_gpus": world, "steps": m["steps"],
+        "warmup": m["warmup"], "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded lognormal lengths, shared prefix, Poisson arrivals; q/K/V drawn on device)",
-        "config": {"workload": describe(w), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": L2_NOTE.replace("steps", "iterations"),
-                   "step": "one trace iteration: native scheduler step, metadata upload, copy-on-write block copies, cache write, decode"},
-        "logical_gbs": round(logical, 2),
-        "unique_bytes_per_step": int((uniq_b + other_b) / K), "logical_bytes_per_step": int((logi_b + other_b) / K),
-        "host_scheduler_ms_per_step": round(1e3 * sched_s / K, 3),
-        "host_iteration_ms_per_step": round(1e3 * host_s / K, 3),
-        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2), "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
-        "clocks": clk.summary(), "gpu_launches": launches,
+        "config": {"workload": m["workload"], "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": L2_NOTE.replace("steps", "iterations"), "step": m["step"]},
     }
+    for k in ("logical_gbs", "unique_bytes_per_step", "logical_bytes_per_step", "host_scheduler_ms_per_step",
+              "host_iteration_ms_per_step", "pct_of_hbm_peak", "roofline", "clocks", "gpu_launches"):
+        line[k] = m[k]
+    line["hbm_peak_gbs"], line["hbm_peak_kind"] = hbm_peak()
+    return line
 
 
 def run_rag(args, rank, world, local_rank):
@@ -521,11 +649,8 @@ def run_rag(args, rank, world, local_rank):
     from workloads.rag_trace import RagTrace, rag_plan
 
     torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist = init_dist(world)
+    clk = ClockSampler(local_rank).start()
     w = WORKLOADS["rag_trace"]
     plan = rag_plan(w)
     flush = L2Flush(torch)
@@ -548,29 +673,31 @@ def run_rag(args, rank, world, local_rank):
             torch.cuda._sleep(2_000_000)  # keep the GPU fed while the host enqueues
             starts[i].record(stream)
 
-        with ClockSampler(local_rank) as clk:
-            for i in range(K):
-                flush.zero_()
-                t0 = time.perf_counter()
-                fin, arr, pl, *_rest, P = tr.iteration(W + i, before_launch=lambda: gate_and_start(i),
-                                                       after_launch=lambda: ends[i].record(stream))
-                host_s += time.perf_counter() - t0
-                gen += pl["info"].batch
-                prefilled += P
-                cached += int(np.sum(pl["cached"]))
-                admitted += pl["info"].num_admitted
-            torch.cuda.synchronize()
+        r0 = time.perf_counter()
+        for i in range(K):
+            flush.zero_()
+            t0 = time.perf_counter()
+            fin, arr, pl, *_rest, P = tr.iteration(W + i, before_launch=lambda: gate_and_start(i),
+                                                   after_launch=lambda: ends[i].record(stream))
+            host_s += time.perf_counter() - t0
+            gen += pl["info"].batch
+            prefilled += P
+            cached += int(np.sum(pl["cached"]))
+            admitted += pl["info"].num_admitted
+        torch.cuda.synchronize()
+        clocks = clk.summary(r0, time.perf_counter())
         if pk.kv_get_device_error() != pk.KV_OK:
             raise RuntimeError("device error during the trace")
         total_ms = max_over_ranks(sum(starts[i].elapsed_time(ends[i]) for i in range(K)), dist, "cuda")
         hits, evictions, nblocks = pk.kv_alloc_prefix_stats(tr.alloc)
         res[caching] = {"tokens_per_s": world * gen / (total_ms * 1e-3), "ms_per_step": total_ms / K,
                         "generated": gen, "prefilled_tokens": prefilled, "cached_tokens": cached,
-                        "admitted": admitted, "host_ms_per_step": 1e3 * host_s / K, "clocks": clk.summary(),
+                        "admitted": admitted, "host_ms_per_step": 1e3 * host_s / K, "clocks": clocks,
                         "hit_blocks": hits, "evictions": evictions}
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+    clk.stop()
     on, off = res[True], res[False]
     return {
         "metric": METRIC_RAG, "value": round(on["tokens_per_s"], 1), "unit": "tokens/s", "n_gpus": world,
@@ -641,11 +768,8 @@ def run_preempt(args, rank, world, local_rank):
     from workloads.preempt_trace import PreemptTrace, preempt_plan
 
     torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist = init_dist(world)
+    clk = ClockSampler(local_rank).start()
     w = WORKLOADS["preempt_trace"]
     plan = preempt_plan(w)
     flush = L2Flush(torch)
@@ -667,27 +791,29 @@ def run_preempt(args, rank, world, local_rank):
             torch.cuda._sleep(2_000_000)  # keep the GPU fed while the host enqueues
             starts[i].record(stream)
 
-        with ClockSampler(local_rank) as clk:
-            for i in range(K):
-                flush.zero_()
-                fin, arr, pl, *_ = tr.iteration(W + i, before_launch=lambda: gate_and_start(i),
-                                               after_launch=lambda: ends[i].record(stream))
-                gen += pl["info"].batch
-                pre += len(pl["preempted"])
-                rec += len(pl["recomputed"])
-                swapped_blocks += len(pl["swap_out"]) + len(pl["swap_in"])
-                rewritten += pl["info"].num_tokens
-            torch.cuda.synchronize()
+        r0 = time.perf_counter()
+        for i in range(K):
+            flush.zero_()
+            fin, arr, pl, *_ = tr.iteration(W + i, before_launch=lambda: gate_and_start(i),
+                                           after_launch=lambda: ends[i].record(stream))
+            gen += pl["info"].batch
+            pre += len(pl["preempted"])
+            rec += len(pl["recomputed"])
+            swapped_blocks += len(pl["swap_out"]) + len(pl["swap_in"])
+            rewritten += pl["info"].num_tokens
+        torch.cuda.synchronize()
+        clocks = clk.summary(r0, time.perf_counter())
         if pk.kv_get_device_error() != pk.KV_OK:
             raise RuntimeError("device error during the trace")
         total_ms = max_over_ranks(sum(starts[i].elapsed_time(ends[i]) for i in range(K)), dist, "cuda")
         res[mode] = {"tokens_per_s": world * gen / (total_ms * 1e-3), "ms_per_step": total_ms / K,
                      "preempted": pre, "recomputed": rec, "swapped_blocks": swapped_blocks,
-                     "written_tokens": rewritten, "clocks": clk.summary()}
+                     "written_tokens": rewritten, "clocks": clocks}
     swap_bw = swap_copy_bandwidth(torch, pk) if rank == 0 else None
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+    clk.stop()
     sw, rc = res["swap"], res["recompute"]
     return {
         "metric": METRIC_PREEMPT, "value": round(sw["tokens_per_s"], 1), "unit": "tokens/s", "n_gpus": world,
@@ -743,7 +869,8 @@ def pipelined_e2e(torch, stream, ins, outs, launch, K, W):
     i, and the read-back of step i the kernels of step i + 1.  The K steps
     are timed as one region (CUDA events on `stream`, every copy inside).
     `launch(k, views, outs)` also gets the buffer index k (0 or 1).
-    Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
+    Returns (ms per step, H2D bytes per step, D2H bytes per step, host
+    time span of the timed region)."""
     offs, off = [], 0
     for t in ins:
         offs.append(off)
@@ -789,6 +916,7 @@ def pipelined_e2e(torch, stream, ins, outs, launch, K, W):
     for i in range(W):
         step(i)
     torch.cuda.synchronize()
+    t0 = time.perf_counter()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     cs_up.wait_event(a)  # the first upload starts inside the region
@@ -797,14 +925,14 @@ def pipelined_e2e(torch, stream, ins, outs, launch, K, W):
     stream.wait_event(down[(W + K - 1) % 2])  # the last read-back is inside the region
     b.record(stream)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / K, h2d, d2h
+    return a.elapsed_time(b) / K, h2d, d2h, (t0, time.perf_counter())
 
 
 PIPELINE_MODE = ("pipelined: one packed upload per step on an upload stream (double-buffered), "
                  "read-back of every step's output on a read-back stream; K steps timed as one region")
 
 
-def run_e2e(case, twin, torch, stream, K, W):
+def run_e2e(case, twin, torch, stream, K, W, clk):
     """The decode step through the C ABI from pinned host memory, pipelined
     the way a serving loop runs it (pipelined_e2e): inputs are q, the new
     K/V of every layer, slots, tables, lengths and order.  Consecutive steps
@@ -823,17 +951,19 @@ def run_e2e(case, twin, torch, stream, K, W):
             c.write(layer, v[L + layer], v[2 * L + layer], v[3 * L])
             c.decode(layer, v[layer], v[3 * L + 1], v[3 * L + 2], out=outs[layer], order=v[3 * L + 3])
 
-    ms, h2d, d2h = pipelined_e2e(torch, stream, ins, list(case.out), launch, K, W)
+    ms, h2d, d2h, span = pipelined_e2e(torch, stream, ins, list(case.out), launch, K, W)
     return {"value": round(case.step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "mode": PIPELINE_MODE}
+            "mode": PIPELINE_MODE, "clocks": clk.summary(*span)}
 
 
 # ------------------------------------------------------ multi-token leg
 
 class PrefillCase:
     """Device-resident inputs of a multi-token workload: a pool with every
-    sequence's cached prefix, the new tokens' K/V and slots, their queries."""
+    sequence's cached prefix, the new tokens' K/V and slots, their queries.
+    With pk None (the reference arm) the inputs are drawn with torch alone
+    and no pool of the product library is created."""
 
     def __init__(self, name, rank, torch, pk):
         from workloads import (WORKLOADS, device_normal_bits, device_pool, pool_blocks,
@@ -848,10 +978,12 @@ class PrefillCase:
         dev = torch.device("cuda")
         seed = w.seed * 7919 + rank
         self.L = 1
-        self.pool = pk.kv_pool_create(w.block_size, self.nb, w.kv_heads, w.head_dim, w.kv_fmt, 1)
         k, v, _, _ = device_pool(w, self.nb, dev, seed=seed)
         self.k, self.v = [k], [v]
-        pk.kv_pool_bind(self.pool, 0, k, v, None, None)
+        self.pool = None
+        if pk is not None:
+            self.pool = pk.kv_pool_create(w.block_size, self.nb, w.kv_heads, w.head_dim, w.kv_fmt, 1)
+            pk.kv_pool_bind(self.pool, 0, k, v, None, None)
         T, Hq, Hkv, D = int(self.new.sum()), w.num_q_heads, w.kv_heads, w.head_dim
         self.T = T
         self.cu_h = np.concatenate([[0], np.cumsum(self.new)]).astype(np.int32)
@@ -906,11 +1038,8 @@ def run_prefill(args, rank, world, local_rank):
     import paged_kv_cache_451_b200 as pk
 
     torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist = init_dist(world)
+    clk = ClockSampler(local_rank).start()
     case = PrefillCase(args.workload, rank, torch, pk)
     flush = L2Flush(torch)
     stream = torch.cuda.current_stream()
@@ -936,12 +1065,13 @@ def run_prefill(args, rank, world, local_rank):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        for i in range(K):
-            flush.zero_()
-            ev0[i].record(stream)
-            step(evw[i], evp[i])
-        torch.cuda.synchronize()
+    r0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        ev0[i].record(stream)
+        step(evw[i], evp[i])
+    torch.cuda.synchronize()
+    clocks = clk.summary(r0, time.perf_counter())
     if dist:
         dist.barrier()
     step_ms = [ev0[i].elapsed_time(evp[i]) for i in range(K)]
@@ -949,7 +1079,7 @@ def run_prefill(args, rank, world, local_rank):
     total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / K
     pf_avg = sum(pf_ms) / K
-    e2e = run_e2e_prefill(case, torch, stream, K, args.warmup)
+    e2e = run_e2e_prefill(case, torch, stream, K, args.warmup, clk)
     e2e_ms = max_over_ranks(e2e["ms_per_step"] * K, dist, "cuda") / K
     e2e["ms_per_step"] = round(e2e_ms, 5)
     e2e["value"] = round(world * case.flops / (e2e_ms * 1e-3) / 1e12, 2)
@@ -993,7 +1123,7 @@ def run_prefill(args, rank, world, local_rank):
             "peak_note": f"{peak_kind} dense bf16 GEMM (cuBLAS, burst); f16 runs at the same rate",
         },
         "e2e": e2e,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "gpu_launches": 2 * K,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -1001,10 +1131,11 @@ def run_prefill(args, rank, world, local_rank):
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+    clk.stop()
     return line
 
 
-def run_e2e_prefill(case, torch, stream, K, W):
+def run_e2e_prefill(case, torch, stream, K, W, clk):
     """The multi-token step from pinned host memory, pipelined like the
     decode leg (pipelined_e2e): inputs are q, the new K/V, slots,
     cu_seqlens, tables and lengths; the output comes back every step.  The
@@ -1016,9 +1147,107 @@ def run_e2e_prefill(case, torch, stream, K, W):
         case.write(kn, vn, slots)
         case.prefill(q, cu, tables, lens, out=outs[0])
 
-    ms, h2d, d2h = pipelined_e2e(torch, stream, ins, [case.out], launch, K, W)
+    ms, h2d, d2h, span = pipelined_e2e(torch, stream, ins, [case.out], launch, K, W)
     return {"value": round(case.flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "mode": PIPELINE_MODE}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "mode": PIPELINE_MODE,
+            "clocks": clk.summary(*span)}
+
+
+# ---------------------------------------------------------- CPU oracle legs
+
+PARITY_FAILURES = []
+
+
+def oracle_decode_sample(oracle, inp, seqs, layer):
+    """The oracle on the sampled sequences of one layer: their blocks as
+    the device holds them, with the step's cache write redone by the
+    oracle's own mirror (so the slot the GPU wrote is replaced by the
+    oracle's value and no input comes from the product path).  Returns
+    (fp64 output [n][Hq][D], attended tokens, seconds spent in the oracle's
+    attention)."""
+    w = inp.w
+    s = inp.host_sample(seqs, layer)
+    oracle.kv_write(s["k"], s["v"], w.kv_fmt, s["k_new"], s["v_new"], w.q_fmt, s["slots"], w.block_size,
+                    s["k_inv"], s["v_inv"])
+    t0 = time.perf_counter()
+    if inp.window:
+        cu = np.arange(len(seqs) + 1, dtype=np.int32)
+        ref = oracle.paged_prefill(s["k"], s["v"], w.kv_fmt, s["q"], w.q_fmt, cu, s["tables"], s["lens"],
+                                   w.scale, w.block_size, s["k_scale"], s["v_scale"], window=inp.window)
+        att = np.minimum(s["lens"], inp.window)
+    else:
+        ref = oracle.paged_decode(s["k"], s["v"], w.kv_fmt, s["q"], w.q_fmt, s["tables"], s["lens"], w.scale,
+                                  w.block_size, s["k_scale"], s["v_scale"])
+        att = s["lens"]
+    return ref, att, time.perf_counter() - t0
+
+
+def check_outputs(got, ref, q_fmt, kv_fmt):
+    """GPU outputs in the query dtype against the fp64 oracle: max-abs 2e-3
+    (16-bit caches) or 1e-2 (FP8 cache), plus one rounding of the output
+    format (2u|ref|).  Returns (passed, worst excess over the bound, max
+    abs error)."""
+    tol = 1e-2 if kv_fmt == 2 else 2e-3
+    u = 2.0 ** -8 if q_fmt == 1 else 2.0 ** -11
+    err = np.abs(got - ref)
+    excess = float(np.max(err - (tol + 2 * u * np.abs(ref)))) if err.size else -tol
+    return excess <= 0, excess, float(err.max()) if err.size else 0.0
+
+
+def cpu_baseline(case, target_s=15.0, check=False, steps=1):
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    sequences in batch order until about target_s seconds of CPU work (all
+    layers of each sampled sequence).  With ``check`` (``case`` is a Case
+    whose step has run), the GPU outputs of the sampled sequences — and of
+    the longest and shortest sequences, through every layer — are compared
+    with the oracle's; a mismatch is recorded and makes bench.py exit
+    non-zero after printing its line."""
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    import oracle
+    inp = getattr(case, "inp", case)
+    w = inp.w
+    L = inp.L
+    # calibrate on one sequence of one layer, then size the sample
+    _, _, one = oracle_decode_sample(oracle, inp, [0], 0)
+    n = int(min(w.batch, max(1, target_s / max(one, 1e-3) / max(1, L)))) if target_s > 0 else 0
+    seqs = list(range(n))
+    total_s, total_bytes, passes = 0.0, 0, 0
+    worst, max_err, checked = -1.0, 0.0, 0
+    extra = sorted({int(np.argmax(inp.lens)), int(np.argmin(inp.lens))} - set(seqs)) if check else []
+    while n and (passes < steps or total_s < 0.5 * target_s):
+        for layer in range(L):
+            ref, att, dt = oracle_decode_sample(oracle, inp, seqs, layer)
+            total_s += dt
+            total_bytes += (int(att.astype(np.int64).sum()) * w.kv_heads * w.head_dim * 2 * ELEM[w.kv_fmt]
+                            + n * w.num_q_heads * w.head_dim * 2 * ELEM[w.q_fmt])
+            if check and passes == 0:
+                got = case.out[layer][seqs].float().cpu().numpy().astype(np.float64)
+                ok, exc, err = check_outputs(got, ref, w.q_fmt, w.kv_fmt)
+                worst, max_err, checked = max(worst, exc), max(max_err, err), checked + 1
+        passes += 1
+        if n < w.batch:
+            break
+    if check and extra:
+        for layer in range(L):
+            ref, _, _ = oracle_decode_sample(oracle, inp, extra, layer)
+            got = case.out[layer][extra].float().cpu().numpy().astype(np.float64)
+            ok, exc, err = check_outputs(got, ref, w.q_fmt, w.kv_fmt)
+            worst, max_err, checked = max(worst, exc), max(max_err, err), checked + 1
+    res = {"cores": cores, "kind": "oracle"}
+    if n:
+        res.update({"value": round(total_bytes / total_s / 1e9, 4), "unit": "GB/s",
+                    "seqs_per_s": round(passes * n / total_s, 3),
+                    "sample": f"{n} of {w.batch} sequences x {L} layer(s), decode only, fp64 C oracle "
+                              f"(OpenMP over (sequence, head)); {total_s:.1f} s"})
+    if check:
+        passed = worst <= 0
+        res["check"] = {"passed": passed, "sequences": sorted(set(seqs) | set(extra)), "layers": L,
+                        "max_abs_err": round(max_err, 6), "worst_excess_over_bound": round(worst, 6),
+                        "bound": "max-abs 2e-3 (16-bit cache) / 1e-2 (FP8) + one output rounding, vs fp64 oracle"}
+        if not passed:
+            PARITY_FAILURES.append((w.name, res["check"]))
+    return res
 
 
 def cpu_baseline_prefill(case, target_s=15.0):
@@ -1056,97 +1285,27 @@ def cpu_baseline_prefill(case, target_s=15.0):
                       f"(OpenMP over (sequence, head)); {total_s:.1f} s"}
 
 
-# ---------------------------------------------------------- CPU oracle legs
-
-def oracle_sample(case_like, seqs, layer=0):
-    """Host inputs of the sampled sequences (their blocks, remapped tables)."""
-    import torch
-    w = case_like.w
-    bs = w.block_size
-    used, sub = [], np.full((len(seqs), case_like.tables.shape[1]), -1, np.int32)
-    for i, s in enumerate(seqs):
-        for j in range(-(-int(case_like.lens[s]) // bs)):
-            sub[i, j] = len(used)
-            used.append(int(case_like.tables[s, j]))
-    idx = torch.tensor(used, dtype=torch.long, device=case_like.k[layer].device)
-    raw = np.uint8 if w.kv_fmt == 2 else np.uint16
-    kh = case_like.k[layer].index_select(0, idx).cpu().numpy().view(raw)
-    vh = case_like.v[layer].index_select(0, idx).cpu().numpy().view(raw)
-    ks = vs = None
-    if w.kv_fmt == 2:
-        ks = case_like.ks[layer].index_select(0, idx).cpu().numpy()
-        vs = case_like.vs[layer].index_select(0, idx).cpu().numpy()
-    q = case_like.q[layer].cpu().numpy().view(np.uint16)[list(seqs)]
-    return kh, vh, ks, vs, q, sub, case_like.lens[list(seqs)].astype(np.int32)
-
-
-def cpu_baseline(case, torch, target_s=15.0, steps=1):
-    """The oracle, as it stands, on a bounded sample of the same workload."""
-    cores = len(os.sched_getaffinity(0))
-    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
-    import oracle
-    w = case.w
-    order = list(range(w.batch))
-    # calibrate on one sequence, then size the sample to ~target_s
-    t0 = time.perf_counter()
-    args = oracle_sample(case, order[:1])
-    if case.window:
-        oracle.paged_prefill(args[0], args[1], w.kv_fmt, args[4], w.q_fmt, np.arange(2, dtype=np.int32),
-                             args[5], args[6], w.scale, w.block_size, args[2], args[3], window=case.window)
-    else:
-        oracle.paged_decode(args[0], args[1], w.kv_fmt, args[4], w.q_fmt, args[5], args[6], w.scale,
-                            w.block_size, args[2], args[3])
-    one = max(time.perf_counter() - t0, 1e-3)
-    n = int(min(w.batch, max(1, target_s / one / max(1, case.L))))
-    seqs = order[:n]
-    total_s, total_bytes, passes = 0.0, 0, 0
-    samples = [oracle_sample(case, seqs, layer) for layer in range(case.L)] if case.L == 1 else None
-    # repeat the sample until about target_s of CPU work (at least `steps` passes)
-    while passes < steps or total_s < 0.5 * target_s:
-        for layer in range(case.L):
-            kh, vh, ks, vs, q, sub, lens = samples[0] if samples else oracle_sample(case, seqs, layer)
-            t0 = time.perf_counter()
-            if case.window:
-                cu = np.arange(len(lens) + 1, dtype=np.int32)
-                oracle.paged_prefill(kh, vh, w.kv_fmt, q, w.q_fmt, cu, sub, lens, w.scale, w.block_size, ks,
-                                     vs, window=case.window)
-                att = np.minimum(lens, case.window)
-            else:
-                oracle.paged_decode(kh, vh, w.kv_fmt, q, w.q_fmt, sub, lens, w.scale, w.block_size, ks, vs)
-                att = lens
-            total_s += time.perf_counter() - t0
-            total_bytes += (int(att.astype(np.int64).sum()) * w.kv_heads * w.head_dim * 2 * ELEM[w.kv_fmt]
-                            + n * w.num_q_heads * w.head_dim * 2 * ELEM[w.q_fmt])
-        passes += 1
-        if n < w.batch:
-            break
-    steps = passes
-    return {"value": round(total_bytes / total_s / 1e9, 4), "unit": "GB/s",
-            "seqs_per_s": round(steps * n / total_s, 3), "cores": cores, "kind": "oracle",
-            "sample": f"{n} of {w.batch} sequences x {case.L} layer(s), decode only, fp64 C oracle "
-                      f"(OpenMP over (sequence, head)); {total_s:.1f} s"}
-
-
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle timed on the host cores, each step a
-    bounded sample of the same workload."""
+    bounded sample of the same workload.  The inputs are drawn with torch
+    alone (the GPU arm's generators); the product library is not loaded."""
     import torch
     if rank != 0:
         return None
     torch.cuda.set_device(0)
-    import paged_kv_cache_451_b200 as pk
     if args.workload in PREFILL_WORKLOADS:
-        return run_reference_prefill(args, world, torch, pk)
-    if args.workload in ("rag_trace", "preempt_trace"):
+        return run_reference_prefill(args, world, torch)
+    if args.workload in ("rag_trace", "preempt_trace", "gqa_trace"):
         return {"impl": "reference", "metric": METRIC, "workload": args.workload,
                 "unavailable": "the CPU oracle has no serving-trace leg (the GPU line reports the host "
-                               "scheduling time per iteration); time decode workloads instead"}
-    case = Case(args.workload, 0, torch, pk, args)
+                               "scheduling time per iteration); time the single-step decode workloads instead"}
+    from workloads.decode_inputs import DecodeInputs
+    inp = DecodeInputs(args.workload, 0, args.layers)
     per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_baseline(case, torch, target_s=per_step)
-    res = cpu_baseline(case, torch, target_s=per_step * args.steps, steps=1)
-    w = case.w
+        cpu_baseline(inp, target_s=per_step)
+    res = cpu_baseline(inp, target_s=per_step * args.steps, steps=1)
+    w = inp.w
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -1161,15 +1320,15 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (same seeded inputs as the GPU arm)",
-        "config": {"workload": describe(w, case), "global_batch": w.batch},
+        "config": {"workload": describe(w, inp), "global_batch": w.batch, "layers_per_step": inp.L},
         "seqs_per_s": res["seqs_per_s"],
         "cpu_baseline": res,
         "e2e": {"value": res["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-def run_reference_prefill(args, world, torch, pk):
-    case = PrefillCase(args.workload, 0, torch, pk)
+def run_reference_prefill(args, world, torch):
+    case = PrefillCase(args.workload, 0, torch, None)
     per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline_prefill(case, target_s=per_step)
@@ -1198,13 +1357,13 @@ def run_reference_prefill(args, world, torch, pk):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama13b",
-                    choices=["tiny", "llama13b", "kv_example", "gqa_trace", "fp8_long", "window_long", "rag_trace",
-                             "preempt_trace",
-                             *PREFILL_WORKLOADS])
+    ap.add_argument("--workload", default="kv_example",
+                    choices=[*DECODE_WORKLOADS, "gqa_trace", "rag_trace", "preempt_trace", *PREFILL_WORKLOADS])
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode workloads: time only the first N layers (a small case for profiling)")
     ap.add_argument("--partition", type=int, default=0, help="decode partition tokens (0: auto)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline stages per warp (0: auto)")
     ap.add_argument("--warps", type=int, default=0, help="warps per decode CTA (0: auto)")
@@ -1212,6 +1371,8 @@ def main():
                     help="decode scheduling order (default: longest first for one decode step, "
                          "batch order for the continuous-batching trace)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the sustained loop and the per-config measurements")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -1233,6 +1394,9 @@ def main():
         line = run_ours(args, rank, world, local_rank)
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
+    if PARITY_FAILURES:
+        print(f"oracle check failed: {PARITY_FAILURES}", file=sys.stderr, flush=True)
+        sys.exit(3)
 
 
 if __name__ == "__main__":

@@ -295,7 +295,9 @@ int kv_swap_in(const kv_pool* pool, const void* host_swap, int num_slots, const 
  *   that needs fewer partials).
  *   The first call on a device looks up the scratch array's device address
  *   (once per device, with that device current); make that first call before
- *   any stream capture.
+ *   any stream capture.  The address is kept until the process exits: after
+ *   cudaDeviceReset the library's device memory is reloaded elsewhere, so a
+ *   process that resets a device must not call this entry point again on it.
  *   All calls share the one array, which keeps whatever the last call wrote;
  *   nothing in it has to start at zero, because every partial a call reads
  *   was written earlier in that same call.  Calls whose kernels can overlap

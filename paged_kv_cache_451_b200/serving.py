@@ -122,9 +122,11 @@ class DecodeLoop:
         return a, plen - cached, cached
 
     def launch(self, plan, k_new, v_new, q, out, k_inv=None, v_inv=None, out_dtype=None,
-               layer=0, stream=None, prefill_q=None, prefill_out=None):
+               layer=0, stream=None, prefill_q=None, prefill_out=None, before_decode=None):
         """Upload the plan's metadata and enqueue copy, write, prefill of the
-        admitted prompts (when prefill_q is given) and decode."""
+        admitted prompts (when prefill_q is given) and decode.
+        ``before_decode(stream)``, if given, is called right before the
+        decode is enqueued (e.g. to record a timing event)."""
         torch = self.torch
         info = plan["info"]
         b, t, c, w = info.batch, info.num_tokens, info.num_cow, self.max_blocks
@@ -193,6 +195,8 @@ class DecodeLoop:
             need = paged_attention_workspace_bytes(self.pool, b, self.hq, max_ctx)
             if need > self.ws_cap:
                 raise RuntimeError("decode workspace too small")
+            if before_decode is not None:
+                before_decode(main)
             paged_attention_decode(self.pool, layer, q, self.q_dtype, self.hq, dview("tables", torch.int32),
                                    w, dview("lens", torch.int32), b, max_ctx, self.scale, out,
                                    KV_F32 if out_dtype is None else out_dtype, self.d_ws, need, main,

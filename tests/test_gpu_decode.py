@@ -216,3 +216,36 @@ def test_scheduling_order_does_not_change_outputs():
     pk.paged_attention_decode(pool.h, 0, dev(q), BF16, hq, dev(tables), tables.shape[1], dev(lens), len(lens),
                               int(lens.max()), 0.09, out, pk.KV_F32, ws, wsb, seq_order=dev(bad))
     assert pk.kv_get_device_error() == pk.KV_ERR_BOUNDS
+
+
+@pytest.mark.parametrize("kv_fmt,q_fmt", [(BF16, BF16), (E4M3, BF16)])
+def test_every_layer_decodes_its_own_pool(kv_fmt, q_fmt):
+    """A 5-layer pool whose layers hold different values: decoding layers 0,
+    1 and 4 each matches the oracle on that layer's arrays (a wrong per-layer
+    binding or tensor map would read another layer's values)."""
+    rng = np.random.default_rng(77)
+    L, nb, hkv, hq, bs, d = 5, 40, 2, 8, 16, 128
+    lens = np.array([1, 100, 333, 17], np.int32)
+    shape = (nb, hkv, bs, d)
+    ks_h = vs_h = [None] * L
+    if kv_fmt == E4M3:
+        kh = [e4m3_codes(rng, shape) for _ in range(L)]
+        vh = [e4m3_codes(rng, shape) for _ in range(L)]
+        ks_h = [fp8_scales(rng, (nb, hkv)) for _ in range(L)]
+        vs_h = [fp8_scales(rng, (nb, hkv)) for _ in range(L)]
+    else:
+        kh = [normal_bits(rng, shape, kv_fmt) for _ in range(L)]
+        vh = [normal_bits(rng, shape, kv_fmt) for _ in range(L)]
+    tables = scattered_tables(rng, lens, bs, nb)
+    pool = DevicePool(nb, hkv, d, bs, kv_fmt, num_layers=L, k=[dev(a) for a in kh], v=[dev(a) for a in vh],
+                      k_scale=None if ks_h[0] is None else [dev(a) for a in ks_h],
+                      v_scale=None if vs_h[0] is None else [dev(a) for a in vs_h], partition=128)
+    for layer in (0, 1, L - 1):
+        q = normal_bits(rng, (len(lens), hq, d), q_fmt)
+        out = decode(pool, dev(q), q_fmt, hq, dev(tables), dev(lens), int(lens.max()), 0.1, layer=layer)
+        torch.cuda.synchronize()
+        assert pk.kv_get_device_error() == pk.KV_OK
+        ref = oracle.paged_decode(kh[layer], vh[layer], kv_fmt, q, q_fmt, tables, lens, 0.1, bs,
+                                  ks_h[layer], vs_h[layer])
+        assert max_abs(out.cpu().numpy(), ref) <= TOL[kv_fmt], layer
+

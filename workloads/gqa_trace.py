@@ -112,7 +112,8 @@ class GqaTrace:
             out.append((sid, plen))
         return out
 
-    def iteration(self, it, out_dtype=None, out=None, before_launch=None, after_launch=None):
+    def iteration(self, it, out_dtype=None, out=None, before_launch=None, after_launch=None,
+                  before_decode=None):
         """One trace iteration: returns (finished, arrivals, plan, q, k_new,
         v_new, out) with device tensors of this step's inputs and output.
         before_launch / after_launch are called right around the library
@@ -135,7 +136,7 @@ class GqaTrace:
             out = torch.empty((max(B, 1), w.num_q_heads, w.head_dim), dtype=dt, device=self.device)
         if before_launch is not None:
             before_launch()
-        self.loop.launch(plan, k_new, v_new, q, out, out_dtype=out_dtype)
+        self.loop.launch(plan, k_new, v_new, q, out, out_dtype=out_dtype, before_decode=before_decode)
         if after_launch is not None:
             after_launch()
         for s in self.running:
