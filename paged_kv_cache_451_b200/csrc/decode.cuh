@@ -116,13 +116,20 @@ struct DecodeShape {
   static constexpr int MERGE_BYTES = WARPS * kMaxGroup * D * 4;
   static constexpr int BUF_BYTES = STAGES_BYTES > MERGE_BYTES ? STAGES_BYTES : MERGE_BYTES;
   static constexpr int BAR_OFF = BUF_BYTES;
-  static constexpr int BLK_OFF = BAR_OFF + WARPS * STAGES * 8;
-  static constexpr int SCALE_ENTRIES = kFp8 ? kMaxPartChunks : 0;  // FP8 scale tables only
-  static constexpr int KSC_OFF = BLK_OFF + kMaxPartChunks * 4;
-  static constexpr int VSC_OFF = KSC_OFF + SCALE_ENTRIES * 4;
-  static constexpr int VSG_OFF = VSC_OFF + SCALE_ENTRIES * 4;
-  static constexpr int ML_OFF = VSG_OFF + SCALE_ENTRIES * 4;
-  static constexpr int SMEM_BYTES = ML_OFF + WARPS * kMaxGroup * 16 + 1024;  // + alignment slack
+  static constexpr int ML_OFF = BAR_OFF + WARPS * STAGES * 8;
+  // per-chunk tables, sized at launch by the partition's chunk count: block
+  // id, and for FP8 the K scale, log2 |V scale| and the V scale's sign
+  // ML: per (warp, head) m_z, l, m_w and the warp's merge weight; then per
+  // head the output factor, M_z, L and M_w of the merged CTA
+  static constexpr int TAB_OFF = (ML_OFF + (WARPS + 1) * kMaxGroup * 16 + 15) / 16 * 16;
+  static constexpr int TAB_ENTRY = kFp8 ? 16 : 4;
+  __host__ __device__ static constexpr int tab_cap(int chunks) { return (chunks + 3) / 4 * 4; }
+  // dynamic shared memory of a launch whose partitions hold `chunks` chunks
+  // (+ 1024 bytes of alignment slack)
+  __host__ __device__ static constexpr int smem_bytes(int chunks) {
+    return TAB_OFF + tab_cap(chunks) * TAB_ENTRY + 1024;
+  }
+  static constexpr int MAX_SMEM_BYTES = smem_bytes(kMaxPartChunks);
   static_assert(BOXB == 128 || BOXB == 64, "row bytes must be 64 or a multiple of 128");
 };
 
@@ -135,8 +142,15 @@ __device__ __forceinline__ uint32_t tile_off(int row, int chunk16) {
   return box * (kChunk * S::BOXB) + (lin ^ (((lin >> 7) & S::SWZ) << 4));
 }
 
+// Resident CTAs per SM the register allocation is sized for: FP8 tiles
+// need half the shared memory of 16-bit ones, so four 4-warp CTAs fit.
+template <int KV, int WARPS>
+constexpr int decode_min_blocks() {
+  return WARPS == 8 ? 2 : (KV == KV_KIND_E4M3 ? 4 : 1);
+}
+
 template <int KV, int D, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32, WARPS == 8 ? 2 : 1)
+__global__ void __launch_bounds__(WARPS * 32, decode_min_blocks<KV, WARPS>())
 paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap) {
   using S = DecodeShape<KV, D, WARPS, STAGES>;
@@ -183,10 +197,11 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bars = sbase + S::BAR_OFF;
-  int32_t* blk_ids = reinterpret_cast<int32_t*>(smem + S::BLK_OFF);
-  float* ksc = reinterpret_cast<float*>(smem + S::KSC_OFF);
-  float* vsc = reinterpret_cast<float*>(smem + S::VSC_OFF);  // log2 |V scale|
-  float* vsg = reinterpret_cast<float*>(smem + S::VSG_OFF);  // sign of the V scale
+  const int tab = S::tab_cap(p.part_chunks);
+  int32_t* blk_ids = reinterpret_cast<int32_t*>(smem + S::TAB_OFF);
+  float* ksc = reinterpret_cast<float*>(smem + S::TAB_OFF) + tab;  // FP8: K scale
+  float* vsc = ksc + tab;                                           // FP8: log2 |V scale|
+  float* vsg = vsc + tab;                                           // FP8: sign of the V scale
   float* mls = reinterpret_cast<float*>(smem + S::ML_OFF);
 
   if (threadIdx.x == 0) {
@@ -473,10 +488,12 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint32_t lo = h ? r2 : r0, hi = h ? r3 : r1;
-              const uint32_t a0 = e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0020));
-              const uint32_t a1 = e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x0031));
-              const uint32_t a2 = e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0020));
-              const uint32_t a3 = e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x0031));
+              // the even bytes (dim d0 of tokens 2c, 2c+1) and the odd bytes (dim
+              // d0 + 1) of both registers, one permute each; each 16-bit half
+              // then converts to an f16 pair
+              uint32_t a0, a1, a2, a3;
+              e4m3x4_to_f16x4(__byte_perm(lo, hi, 0x6420), a0, a2);
+              e4m3x4_to_f16x4(__byte_perm(lo, hi, 0x7531), a1, a3);
               mma_16816<false>(o[2 * cp + h], a0, a1, a2, a3, bh0, bh1);
               mma_16816<false>(o[2 * cp + h], a0, a1, a2, a3, bl0, bl1);
             }
@@ -552,38 +569,54 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
   }
   __syncthreads();
 
-  // a context that fits one partition is finished here even in split mode;
-  // the reduce kernel skips it
-  const bool split = p.num_parts > 1 && total_chunks > p.part_chunks;
-  for (int idx = threadIdx.x; idx < p.group * D; idx += WARPS * 32) {
-    const int g = idx / D;
-    const int d = idx - g * D;
+  // Merge weights, once per head: with Mz = max over warps of m_z, Mw = max
+  // of m_w, warp w's output enters with weight 2^(m_w,w - Mw), its sum with
+  // 2^(m_z,w - Mz); the head's result is O * 2^(Mw - Mz) / L.
+  float* hd = mls + WARPS * kMaxGroup * 4;  // per head: factor, Mz, L, Mw
+  if (threadIdx.x < p.group) {
+    const int g = threadIdx.x;
     float Mz = -INFINITY, Mw = -INFINITY;
 #pragma unroll
     for (int w = 0; w < WARPS; ++w) {
       Mz = fmaxf(Mz, mls[(w * kMaxGroup + g) * 4 + 0]);
       Mw = fmaxf(Mw, mls[(w * kMaxGroup + g) * 4 + 2]);
     }
-    float O = 0.f, L = 0.f;
+    float L = 0.f;
 #pragma unroll
     for (int w = 0; w < WARPS; ++w) {
-      const float* ml = mls + (w * kMaxGroup + g) * 4;
+      float* ml = mls + (w * kMaxGroup + g) * 4;
       if (ml[0] != -INFINITY) L += ml[1] * ex2(ml[0] - Mz);
-      if (ml[2] != -INFINITY) O += obuf[(w * kMaxGroup + g) * D + d] * ex2(ml[2] - Mw);
+      ml[3] = ml[2] != -INFINITY ? ex2(ml[2] - Mw) : 0.f;
     }
+    float fin = 0.f;
+    if (L > 0.f && Mw != -INFINITY) fin = (kFp8 ? ex2(Mw - Mz) : 1.f) / L;
+    hd[g * 4 + 0] = fin;
+    hd[g * 4 + 1] = Mz;
+    hd[g * 4 + 2] = L;
+    hd[g * 4 + 3] = Mw;
+  }
+  __syncthreads();
+
+  // a context that fits one partition is finished here even in split mode;
+  // the reduce kernel skips it
+  const bool split = p.num_parts > 1 && total_chunks > p.part_chunks;
+  for (int idx = threadIdx.x; idx < p.group * D; idx += WARPS * 32) {
+    const int g = idx / D;
+    const int d = idx - g * D;
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) O += obuf[(w * kMaxGroup + g) * D + d] * mls[(w * kMaxGroup + g) * 4 + 3];
     const int h = kvh * p.group + g;
     const int64_t sh = (int64_t)seq * p.num_q_heads + h;
     if (!split) {
-      float r = 0.f;
-      if (L > 0.f && Mw != -INFINITY) r = kFp8 ? (O / L) * ex2(Mw - Mz) : O / L;
-      store_out(p.out, p.out_kind, sh * D + d, r);
+      store_out(p.out, p.out_kind, sh * D + d, O * hd[g * 4]);
     } else {
       const int64_t pi = sh * p.num_parts + part;
       p.part_o[pi * D + d] = O;
       if (d == 0) {
-        p.part_ml[pi * 4 + 0] = Mz;
-        p.part_ml[pi * 4 + 1] = L;
-        p.part_ml[pi * 4 + 2] = Mw;
+        p.part_ml[pi * 4 + 0] = hd[g * 4 + 1];
+        p.part_ml[pi * 4 + 1] = hd[g * 4 + 2];
+        p.part_ml[pi * 4 + 2] = hd[g * 4 + 3];
         p.part_ml[pi * 4 + 3] = 0.f;
       }
     }

@@ -90,18 +90,21 @@ int ensure_smem(K kernel, int bytes, std::atomic<uint64_t>& done) {
 }
 
 // Pipeline shape: warps per CTA and stages per warp.  4 warps of 3 stages of
-// 8 KB (16-bit, D 128: two CTAs per SM); 3 stages of 4 KB (FP8 D 128, 16-bit
-// D 64: three CTAs per SM, the register limit); 6 stages of 2 KB.  Measured
-// on B200: more warps per CTA or deeper rings were slower for every format.
+// 8 KB (16-bit, D 128: two CTAs per SM) for single heads and small groups;
+// 2 stages (three CTAs per SM) for GQA groups of 4 or more, whose shared
+// prefixes are read from L2 with shorter latency and whose CTAs cover fewer
+// chunks; 3 stages of 4 KB (FP8 D 128, 16-bit D 64: four and three CTAs per
+// SM); 6 stages of 2 KB.  Measured on B200: more warps per CTA or deeper rings
+// were slower for every format.
 struct PipeShape {
   int warps;
   int stages;
 };
 
-PipeShape pipe_for(kv_dtype dtype, int head_dim, int stages, int warps) {
+PipeShape pipe_for(kv_dtype dtype, int head_dim, int group, int stages, int warps) {
   const int stage_bytes = 2 * kChunk * head_dim * elem_bytes(dtype);
   PipeShape ps;
-  if (stage_bytes >= 8192) ps = {4, 3};
+  if (stage_bytes >= 8192) ps = {4, group >= 4 ? 2 : 3};
   else if (stage_bytes >= 4096) ps = {4, 3};
   else ps = {4, 6};
   if (warps > 0) ps.warps = warps;
@@ -109,18 +112,18 @@ PipeShape pipe_for(kv_dtype dtype, int head_dim, int stages, int warps) {
   return ps;
 }
 
-PipeShape pipe_for(const kv_pool* pool) {
-  return pipe_for(pool->dtype, pool->head_dim, pool->stages, pool->warps);
+PipeShape pipe_for(const kv_pool* pool, int group) {
+  return pipe_for(pool->dtype, pool->head_dim, group, pool->stages, pool->warps);
 }
 
 template <int KV, int D, int W>
 int smem_bytes_w(int stages) {
   switch (stages) {
-    case 2: return DecodeShape<KV, D, W, 2>::SMEM_BYTES;
-    case 3: return DecodeShape<KV, D, W, 3>::SMEM_BYTES;
-    case 4: return DecodeShape<KV, D, W, 4>::SMEM_BYTES;
-    case 6: return DecodeShape<KV, D, W, 6>::SMEM_BYTES;
-    default: return DecodeShape<KV, D, W, 8>::SMEM_BYTES;
+    case 2: return DecodeShape<KV, D, W, 2>::MAX_SMEM_BYTES;
+    case 3: return DecodeShape<KV, D, W, 3>::MAX_SMEM_BYTES;
+    case 4: return DecodeShape<KV, D, W, 4>::MAX_SMEM_BYTES;
+    case 6: return DecodeShape<KV, D, W, 6>::MAX_SMEM_BYTES;
+    default: return DecodeShape<KV, D, W, 8>::MAX_SMEM_BYTES;
   }
 }
 
@@ -137,10 +140,10 @@ int smem_bytes(kv_dtype dtype, int head_dim, PipeShape ps) {
   }
 }
 
-int decode_occupancy(const kv_pool* pool);  // defined with the launchers below
+int decode_occupancy(const kv_pool* pool, int group);  // defined with the launchers below
 
 // Resident decode CTAs the current device holds at once.
-int decode_slots(const kv_pool* pool) {
+int decode_slots(const kv_pool* pool, int group) {
   static std::atomic<int> sm_count[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
@@ -152,7 +155,7 @@ int decode_slots(const kv_pool* pool) {
     }
     sm_count[dev % kMaxDevices].store(sms, std::memory_order_relaxed);
   }
-  return sms * decode_occupancy(pool);
+  return sms * decode_occupancy(pool, group);
 }
 
 // Partition length in tokens.  Automatic: contexts are cut into partitions
@@ -170,11 +173,11 @@ constexpr int kWavesSplit = 4;
 constexpr int kAutoPartition = 4096;
 constexpr int kMinPartition = 512;
 
-int partition_tokens(const kv_pool* pool, int batch, int max_context_len) {
+int partition_tokens(const kv_pool* pool, int batch, int max_context_len, int group) {
   if (pool->partition_tokens > 0) return pool->partition_tokens;
   const int ctx = std::max(max_context_len, 1);
   const int64_t units = std::max<int64_t>(1, (int64_t)batch * pool->kv_heads);
-  const int64_t slots = decode_slots(pool);
+  const int64_t slots = decode_slots(pool, group);
   int64_t np = (ctx + kAutoPartition - 1) / kAutoPartition;
   if (units < (int64_t)kWavesKeep * slots) {
     np = std::max<int64_t>(np, (kWavesSplit * slots + units - 1) / units);
@@ -184,8 +187,8 @@ int partition_tokens(const kv_pool* pool, int batch, int max_context_len) {
   return (int)std::min<int64_t>(kChunk * kMaxPartChunks, (per + kChunk - 1) / kChunk * kChunk);
 }
 
-int num_parts_for(const kv_pool* pool, int batch, int max_context_len) {
-  const int pt = partition_tokens(pool, batch, max_context_len);
+int num_parts_for(const kv_pool* pool, int batch, int max_context_len, int group) {
+  const int pt = partition_tokens(pool, batch, max_context_len, group);
   return std::max(1, (max_context_len + pt - 1) / pt);
 }
 
@@ -199,7 +202,8 @@ int visited_len(const kv_pool* pool, int max_context_len) {
 }
 
 // Resident CTAs per SM of one decode instantiation on the current device
-// (occupancy API; registers and shared memory both count).
+// (occupancy API; registers and shared memory both count), with the chunk
+// tables of the automatic policy's longest partition.
 template <int KV, int D, int W, int STAGES>
 int decode_occupancy() {
   using Shape = DecodeShape<KV, D, W, STAGES>;
@@ -209,13 +213,13 @@ int decode_occupancy() {
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
   int v = cached[dev % kMaxDevices].load(std::memory_order_relaxed);
   if (v > 0) return v;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Shape::SMEM_BYTES) !=
+  const int smem = Shape::smem_bytes(kAutoPartition / kChunk);
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Shape::MAX_SMEM_BYTES) !=
           cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, W * 32, Shape::SMEM_BYTES) !=
-          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, W * 32, smem) != cudaSuccess ||
       v <= 0) {
     (void)cudaGetLastError();
-    v = std::max(1, kMaxSmemPerCta / Shape::SMEM_BYTES);  // no device: shared-memory bound
+    v = std::max(1, kMaxSmemPerCta / smem);  // no device: shared-memory bound
   }
   cached[dev % kMaxDevices].store(v, std::memory_order_relaxed);
   return v;
@@ -237,8 +241,8 @@ int occupancy_d(PipeShape ps) {
   return ps.warps == 8 ? occupancy_w<KV, D, 8>(ps.stages) : occupancy_w<KV, D, 4>(ps.stages);
 }
 
-int decode_occupancy(const kv_pool* pool) {
-  const PipeShape ps = pipe_for(pool);
+int decode_occupancy(const kv_pool* pool, int group) {
+  const PipeShape ps = pipe_for(pool, group);
   const bool d64 = pool->head_dim == 64;
   switch (pool->dtype) {
     case KV_FP8_E4M3: return d64 ? occupancy_d<KV_KIND_E4M3, 64>(ps) : occupancy_d<KV_KIND_E4M3, 128>(ps);
@@ -252,9 +256,9 @@ int launch_decode_t(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cu
   using Shape = DecodeShape<KV, D, W, STAGES>;
   auto kernel = paged_decode_kernel<KV, D, W, STAGES>;
   static std::atomic<uint64_t> done{0};  // one flag word per instantiation
-  int rc = ensure_smem(kernel, Shape::SMEM_BYTES, done);
+  int rc = ensure_smem(kernel, Shape::MAX_SMEM_BYTES, done);
   if (rc != KV_OK) return rc;
-  kernel<<<grid, W * 32, Shape::SMEM_BYTES, stream>>>(p, lb.k_map, lb.v_map);
+  kernel<<<grid, W * 32, Shape::smem_bytes(p.part_chunks), stream>>>(p, lb.k_map, lb.v_map);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
   return KV_OK;
@@ -384,7 +388,7 @@ int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages, i
     return fail(KV_ERR_ARG, "stages %d must be 0, 2, 3, 4, 6 or 8", stages);
   if (warps != 0 && warps != 4 && warps != 8)
     return fail(KV_ERR_ARG, "warps %d must be 0, 4 or 8", warps);
-  const PipeShape ps = pipe_for(pool->dtype, pool->head_dim, stages, warps);
+  const PipeShape ps = pipe_for(pool->dtype, pool->head_dim, 1, stages, warps);
   const int need = smem_bytes(pool->dtype, pool->head_dim, ps);
   if (need > kMaxSmemPerCta)
     return fail(KV_ERR_ARG, "%d warps x %d stages need %d bytes of shared memory per CTA, above %d",
@@ -545,7 +549,8 @@ int kv_swap_in(const kv_pool* pool, const void* host_swap, int num_slots, const 
 size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
                                        int max_context_len) {
   if (!pool || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
-  const int np = num_parts_for(pool, batch, visited_len(pool, max_context_len));
+  const int group = num_q_heads % pool->kv_heads == 0 ? num_q_heads / pool->kv_heads : 1;
+  const int np = num_parts_for(pool, batch, visited_len(pool, max_context_len), group);
   if (np <= 1) return 0;
   return (size_t)batch * num_q_heads * np * (pool->head_dim + 4) * sizeof(float);
 }
@@ -579,8 +584,9 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
     return fail(KV_ERR_ARG, "max_blocks_per_seq %d cannot hold max_context_len %d",
                 max_blocks_per_seq, max_context_len);
   const int visited = visited_len(pool, max_context_len);
-  const int pt = partition_tokens(pool, batch, visited);
-  const int np = num_parts_for(pool, batch, visited);
+  const int group = num_q_heads / pool->kv_heads;
+  const int pt = partition_tokens(pool, batch, visited, group);
+  const int np = num_parts_for(pool, batch, visited, group);
   if (np > 65535) return fail(KV_ERR_ARG, "too many partitions");
   const size_t need = paged_attention_workspace_bytes(pool, batch, num_q_heads, max_context_len);
   if (need > 0 && (!workspace || workspace_bytes < need))
@@ -616,7 +622,7 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(np, pool->kv_heads, batch);
-  const PipeShape ps = pipe_for(pool);
+  const PipeShape ps = pipe_for(pool, group);
   int rc;
   switch (pool->dtype) {
     case KV_F16: rc = launch_decode_kv<KV_KIND_F16>(pool->head_dim, ps, p, lb, grid, s); break;

@@ -249,3 +249,26 @@ def test_every_layer_decodes_its_own_pool(kv_fmt, q_fmt):
                                   ks_h[layer], vs_h[layer])
         assert max_abs(out.cpu().numpy(), ref) <= TOL[kv_fmt], layer
 
+
+@pytest.mark.parametrize("q_fmt", [BF16, F16])
+def test_fp8_queries_spanning_many_binades(q_fmt):
+    """FP8 caches take the query as a sum of E4M3 terms (exact for bf16
+    queries, and for f16 ones up to components far below the head's largest):
+    queries whose components span 2^-24 .. 2^6 in magnitude, with a few huge
+    and many tiny values per head, still match the oracle."""
+    rng = np.random.default_rng(31)
+    nb, hkv, hq, bs, d = 64, 2, 8, 16, 128
+    kh, vh = e4m3_codes(rng, (nb, hkv, bs, d)), e4m3_codes(rng, (nb, hkv, bs, d))
+    ks, vs = fp8_scales(rng, (nb, hkv)), fp8_scales(rng, (nb, hkv))
+    lens = np.array([1, 40, 300, 513], np.int32)
+    tables = scattered_tables(rng, lens, bs, nb)
+    mag = np.exp2(rng.uniform(-24, 6, (len(lens), hq, d))) * rng.choice([-1.0, 1.0], (len(lens), hq, d))
+    mag[:, 3, :] = 0.0  # an all-zero head
+    x = torch.from_numpy(mag.astype(np.float32)).to(torch.float16 if q_fmt == F16 else torch.bfloat16)
+    q = x.view(torch.int16).numpy().view(np.uint16)
+    pool = DevicePool(nb, hkv, d, bs, E4M3, k=[dev(kh)], v=[dev(vh)], k_scale=[dev(ks)], v_scale=[dev(vs)],
+                      partition=256)
+    for scale in (1.0 / math.sqrt(d), 1e-3):
+        out = decode(pool, dev(q), q_fmt, hq, dev(tables), dev(lens), int(lens.max()), scale).cpu().numpy()
+        ref = oracle.paged_decode(kh, vh, E4M3, q, q_fmt, tables, lens, scale, bs, ks, vs)
+        assert max_abs(out, ref) <= TOL[E4M3], scale
