@@ -577,6 +577,7 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
             break
     total_ms = max_over_ranks(tot_ms, dist, "cuda")
     ms = total_ms / steps
+    e2e = trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, dist, world)
     peak, peak_kind = hbm_peak()
     value = world * (uniq_b + other_b) / (total_ms * 1e-3) / 1e9
     logical = world * (logi_b + other_b) / (total_ms * 1e-3) / 1e9
@@ -606,10 +607,66 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
             "launch_ms": round(dec_ms / steps, 5),
             "bytes_note": "unique physical K/V bytes (shared prefix blocks counted once) + q + out",
             "peak_note": f"{peak_kind} copy bandwidth"},
-        "clocks": clocks, "gpu_launches": launches,
+        "clocks": clocks, "gpu_launches": launches, "e2e": e2e,
         "step": "one trace iteration: native scheduler step, metadata upload, copy-on-write block copies, "
                 "cache write, decode",
     }
+
+
+def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, dist, world):
+    """The trace end to end from host buffers: the same iterations, run back
+    to back as a serving loop runs them (no device-side gate), each one
+    uploading its queries and new K/V rows from pinned host memory and
+    reading its output back; the K iterations are timed as one region, host
+    scheduling included.  Bytes per step are the device-timed run's."""
+    import torch
+    from workloads.gqa_trace import GqaTrace
+    e = w.extra
+    hq, hkv, d = w.num_q_heads, w.kv_heads, w.head_dim
+    tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
+                  order_policy=args.order or "batch")
+    max_b, max_t = e["max_num_seqs"], tr.loop.max_tokens
+    g = torch.Generator().manual_seed(w.seed * 31 + rank)
+    host = {n: torch.randn(m, generator=g).to(torch.bfloat16).view(torch.int16).pin_memory()
+            for n, m in (("q", max_b * hq * d), ("k", max_t * hkv * d), ("v", max_t * hkv * d))}
+    devb = {n: torch.empty_like(t, device="cuda") for n, t in host.items()}
+    hout = torch.empty(max_b * hq * d, dtype=torch.bfloat16).pin_memory()
+    moved = {"h2d": 0, "d2h": 0}
+
+    def inputs(T, B):
+        views = []
+        for n, rows, heads in (("q", B, hq), ("k", T, hkv), ("v", T, hkv)):
+            m = rows * heads * d
+            devb[n][:m].copy_(host[n][:m], non_blocking=True)
+            moved["h2d"] += 2 * m
+            views.append(devb[n][:m].view(rows, heads, d))
+        return views[0], views[1], views[2]
+
+    for it in range(W):
+        tr.iteration(it, out_dtype=w.q_fmt, inputs=inputs)
+    torch.cuda.synchronize()
+    moved["h2d"] = 0
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record(stream)
+    for i in range(K):
+        *_r, out = tr.iteration(W + i, out_dtype=w.q_fmt, inputs=inputs)
+        n = out.numel()
+        hout[:n].copy_(out.view(-1), non_blocking=True)
+        moved["d2h"] += 2 * n
+    b.record(stream)
+    torch.cuda.synchronize()
+    span = (t0, time.perf_counter())
+    ms = max_over_ranks(a.elapsed_time(b), dist, "cuda") / K
+    del tr
+    return {"value": round(world * (uniq_b + other_b) / steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 5), "steps": K, "h2d_bytes_per_step": int(moved["h2d"] / K),
+            "d2h_bytes_per_step": int(moved["d2h"] / K),
+            "mode": "serving loop from host memory: per iteration the native scheduler step, the packed "
+                    "metadata upload, the upload of the step's q and new K/V rows from pinned host memory, "
+                    "the kernels, and the output read back; K iterations timed as one region (host "
+                    "scheduling and Python sequencing included)",
+            "clocks": clk.summary(*span)}
 
 
 def run_trace(args, rank, world, local_rank):
@@ -633,7 +690,7 @@ def run_trace(args, rank, world, local_rank):
                    "l2": L2_NOTE.replace("steps", "iterations"), "step": m["step"]},
     }
     for k in ("logical_gbs", "unique_bytes_per_step", "logical_bytes_per_step", "host_scheduler_ms_per_step",
-              "host_iteration_ms_per_step", "pct_of_hbm_peak", "roofline", "clocks", "gpu_launches"):
+              "host_iteration_ms_per_step", "pct_of_hbm_peak", "roofline", "e2e", "clocks", "gpu_launches"):
         line[k] = m[k]
     line["hbm_peak_gbs"], line["hbm_peak_kind"] = hbm_peak()
     return line

@@ -113,11 +113,14 @@ class GqaTrace:
         return out
 
     def iteration(self, it, out_dtype=None, out=None, before_launch=None, after_launch=None,
-                  before_decode=None):
+                  before_decode=None, inputs=None):
         """One trace iteration: returns (finished, arrivals, plan, q, k_new,
         v_new, out) with device tensors of this step's inputs and output.
         before_launch / after_launch are called right around the library
-        calls (after the inputs are drawn), e.g. to record timing events."""
+        calls (after the inputs are drawn), e.g. to record timing events.
+        ``inputs(T, B)``, if given, supplies (q, k_new, v_new) instead of the
+        seeded draws (e.g. views of buffers it uploads from host memory); it
+        is called after before_launch."""
         torch, w = self.torch, self.w
         import time
         fin = self.finished()
@@ -128,14 +131,17 @@ class GqaTrace:
         info = plan["info"]
         self.running = [int(x) for x in plan["running"]]
         T, B = info.num_tokens, info.batch
-        k_new = self.draw((max(T, 1), w.kv_heads, w.head_dim), w.kv_fmt, self.device, self._seed(it, 0))
-        v_new = self.draw((max(T, 1), w.kv_heads, w.head_dim), w.kv_fmt, self.device, self._seed(it, 1))
-        q = self.draw((max(B, 1), w.num_q_heads, w.head_dim), w.q_fmt, self.device, self._seed(it, 2))
+        if inputs is None:
+            k_new = self.draw((max(T, 1), w.kv_heads, w.head_dim), w.kv_fmt, self.device, self._seed(it, 0))
+            v_new = self.draw((max(T, 1), w.kv_heads, w.head_dim), w.kv_fmt, self.device, self._seed(it, 1))
+            q = self.draw((max(B, 1), w.num_q_heads, w.head_dim), w.q_fmt, self.device, self._seed(it, 2))
         if out is None:
             dt = torch.float32 if out_dtype is None else {0: torch.float16, 1: torch.bfloat16}[out_dtype]
             out = torch.empty((max(B, 1), w.num_q_heads, w.head_dim), dtype=dt, device=self.device)
         if before_launch is not None:
             before_launch()
+        if inputs is not None:
+            q, k_new, v_new = inputs(max(T, 1), max(B, 1))
         self.loop.launch(plan, k_new, v_new, q, out, out_dtype=out_dtype, before_decode=before_decode)
         if after_launch is not None:
             after_launch()
