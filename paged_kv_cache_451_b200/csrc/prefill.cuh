@@ -472,30 +472,35 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_f16(kBf16, kPfRows, kPfKeys, false);
       constexpr uint32_t kIdO = tc::idesc_f16(kBf16, kPfRows, D, true);
+      // Shared-memory descriptors of the Q, K and V regions, built once: the
+      // start-address field (address >> 4, bits 0-13) of a position inside a
+      // region is the region's plus (offset >> 4), as shared-memory addresses
+      // stay below 256 KB and the field never carries; each MMA then costs
+      // the issuing thread one add per operand.
+      const uint64_t dQ = tc::desc_sw128(sbase + S::Q_OFF, 16, 1024);
+      const uint64_t dK = tc::desc_sw128(sbase + S::K_OFF, 16, 1024);
+      const uint64_t dV = tc::desc_sw128(sbase + S::V_OFF, S::HALF, 1024);
       auto issue_s = [&](int x, uint32_t kt) {
-        const int st = kt % STAGES;
+        const uint64_t q0 = dQ + (uint64_t)((x * S::TILE) >> 4);
+        const uint64_t k0 = dK + (uint64_t)(((kt % STAGES) * S::TILE) >> 4);
+        const uint32_t d = tmem + S::S_COL + x * kPfKeys;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * S::HALF + (kk % 4) * 32;  // 16 columns per step
-          tc::mma_ss(tmem + S::S_COL + x * kPfKeys,
-                     tc::desc_sw128(sbase + S::Q_OFF + x * S::TILE + off, 16, 1024),
-                     tc::desc_sw128(sbase + S::K_OFF + st * S::TILE + off, 16, 1024), kIdS,
-                     kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * S::HALF + (kk % 4) * 32) >> 4;  // 16 columns per step
+          tc::mma_ss(d, q0 + off, k0 + off, kIdS, kk > 0 ? 1u : 0u);
         }
         tc::commit(SF(x));
       };
       auto issue_pv = [&](int x, uint32_t kt, bool first) {
-        const int st = kt % STAGES;
-        const uint32_t aP = tmem + S::S_COL + x * kPfKeys;
+        const uint64_t v0 = dV + (uint64_t)(((kt % STAGES) * S::TILE) >> 4);
+        const uint32_t aP = tmem + S::S_COL + x * kPfKeys, d = tmem + S::O_COL + x * D;
 #pragma unroll
         for (int kk = 0; kk < KCH; ++kk) {
           // keys 16kk..16kk+15: their 16-bit values in columns 16kk..16kk+7,
           // (bf16) the residuals in the next 8
-          const uint32_t col = 16 * kk;
-          const uint64_t bV =
-              tc::desc_sw128(sbase + S::V_OFF + st * S::TILE + kk * 2048, S::HALF, 1024);
-          tc::mma_ts(tmem + S::O_COL + x * D, aP + col, bV, kIdO, (!first || kk > 0) ? 1u : 0u);
-          if constexpr (kSplit) tc::mma_ts(tmem + S::O_COL + x * D, aP + col + 8, bV, kIdO, 1u);
+          const uint64_t bV = v0 + (uint64_t)((kk * 2048) >> 4);
+          tc::mma_ts(d, aP + 16 * kk, bV, kIdO, (!first || kk > 0) ? 1u : 0u);
+          if constexpr (kSplit) tc::mma_ts(d, aP + 16 * kk + 8, bV, kIdO, 1u);
         }
         tc::commit(PV(x));
       };
