@@ -265,7 +265,9 @@ class Case:
                                       + (2 * 4 * inp.blocks_touched * Hkv if w.kv_fmt == 2 else 0))
         self.write_bytes = self.L * B * Hkv * D * 2 * (e_q + e_kv)
         self.step_bytes = self.decode_bytes + self.write_bytes
-        self.launches_per_step = self.L * (2 + (1 if self.split else 0))
+        # the cache write and the decode (split partials are merged by the decode's
+        # last partition CTA; the merge counters are zeroed by a memset)
+        self.launches_per_step = self.L * 2
 
     def write(self, layer, kn=None, vn=None, slots=None):
         w, pk = self.w, self.pk
@@ -320,7 +322,8 @@ def decode_roofline(case, dec_ms, workload_key):
     achieved = per_launch / (dec_avg * 1e-3) / 1e9
     return {
         "bound": "hbm",
-        "kernel": "paged_attention_decode (decode kernel" + (" + LSE reduce)" if case.split else ")"),
+        "kernel": "paged_attention_decode (decode kernel" + (", split partials merged by its last partition CTA)"
+                                                            if case.split else ")"),
         "achieved": round(achieved, 2),
         "peak": peak,
         "unit": "GB/s",
@@ -500,7 +503,7 @@ def unique_and_logical_tokens(tables, lens, block_size):
     return sum(best.values()), logical
 
 
-def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s=None):
+def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s=None, shared_prefix=None):
     """The GQA continuous-batching trace: one step = one trace iteration
     (native scheduler step, metadata upload, copy-on-write block copies,
     cache write, decode).  The trace's iterations after the warm-up are
@@ -513,6 +516,8 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
 
     w = WORKLOADS["gqa_trace"]
     plan = gqa_trace_plan(w)
+    if shared_prefix is None:
+        shared_prefix = args.shared_prefix
     iters = w.extra["iters"]
     W = min(args.warmup, iters - 1)
     K = max(1, min(args.steps, iters - W)) if min_s is None else iters - W
@@ -526,7 +531,7 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
     passes = 0
     while True:
         tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
-                      order_policy=args.order or "batch")
+                      order_policy=args.order or "batch", shared_prefix=shared_prefix)
         for it in range(W):
             flush.zero_()
             tr.iteration(it, out_dtype=w.q_fmt)
@@ -561,8 +566,7 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
             dec_b += u * per_tok + qo
             other_b += (qo + info.num_tokens * hkv * d * 2 * 4
                         + info.num_cow * hkv * w.block_size * d * 2 * 2 * 2)
-            launches += 2 + (1 if info.num_cow else 0) + (
-                1 if pk.paged_attention_workspace_bytes(tr.pool, info.batch, hq, int(pl["context_lens"].max())) else 0)
+            launches += 2 + (1 if info.num_cow else 0)
         torch.cuda.synchronize()
         t1 = time.perf_counter()
         regions.append((t0, t1))
@@ -577,7 +581,7 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
             break
     total_ms = max_over_ranks(tot_ms, dist, "cuda")
     ms = total_ms / steps
-    e2e = trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, dist, world)
+    e2e = trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, dist, world, shared_prefix)
     peak, peak_kind = hbm_peak()
     value = world * (uniq_b + other_b) / (total_ms * 1e-3) / 1e9
     logical = world * (logi_b + other_b) / (total_ms * 1e-3) / 1e9
@@ -600,7 +604,7 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
         "host_iteration_ms_per_step": round(1e3 * host_s / steps, 3),
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
         "roofline": {
-            "bound": "hbm", "kernel": "paged_attention_decode (decode kernel, + LSE reduce when split)",
+            "bound": "hbm", "kernel": "paged_attention_decode (decode kernel; split partials merged in it)",
             "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
             "traffic": committed_traffic("gqa_trace"),
             "algorithmic_bytes_per_launch": int(dec_b / steps),
@@ -609,11 +613,14 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
             "peak_note": f"{peak_kind} copy bandwidth"},
         "clocks": clocks, "gpu_launches": launches, "e2e": e2e,
         "step": "one trace iteration: native scheduler step, metadata upload, copy-on-write block copies, "
-                "cache write, decode",
+                "cache write, decode" + (" (shared-prefix decode: the sharers' common blocks once per kv head "
+                                         "on the tensor cores, merged with each sequence's own tokens)"
+                                         if shared_prefix else ""),
+        "shared_prefix_decode": bool(shared_prefix),
     }
 
 
-def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, dist, world):
+def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, dist, world, shared_prefix):
     """The trace end to end from host buffers: the same iterations, run back
     to back as a serving loop runs them (no device-side gate), each one
     uploading its queries and new K/V rows from pinned host memory and
@@ -624,7 +631,7 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
     e = w.extra
     hq, hkv, d = w.num_q_heads, w.kv_heads, w.head_dim
     tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
-                  order_policy=args.order or "batch")
+                  order_policy=args.order or "batch", shared_prefix=shared_prefix)
     max_b, max_t = e["max_num_seqs"], tr.loop.max_tokens
     g = torch.Generator().manual_seed(w.seed * 31 + rank)
     host = {n: torch.randn(m, generator=g).to(torch.bfloat16).view(torch.int16).pin_memory()
@@ -690,7 +697,8 @@ def run_trace(args, rank, world, local_rank):
                    "l2": L2_NOTE.replace("steps", "iterations"), "step": m["step"]},
     }
     for k in ("logical_gbs", "unique_bytes_per_step", "logical_bytes_per_step", "host_scheduler_ms_per_step",
-              "host_iteration_ms_per_step", "pct_of_hbm_peak", "roofline", "e2e", "clocks", "gpu_launches"):
+              "host_iteration_ms_per_step", "pct_of_hbm_peak", "roofline", "e2e", "clocks", "gpu_launches",
+              "shared_prefix_decode"):
         line[k] = m[k]
     line["hbm_peak_gbs"], line["hbm_peak_kind"] = hbm_peak()
     return line
@@ -717,7 +725,7 @@ def run_rag(args, rank, world, local_rank):
     K = max(1, min(args.steps, iters - W))
     res = {}
     for caching in (True, False):
-        tr = RagTrace(w, plan, caching=caching, seed=rank)
+        tr = RagTrace(w, plan, caching=caching, seed=rank, shared_prefix=args.shared_prefix and caching)
         for it in range(W):
             tr.iteration(it)
         torch.cuda.synchronize()
@@ -1428,6 +1436,9 @@ def main():
                     help="decode scheduling order (default: longest first for one decode step, "
                          "batch order for the continuous-batching trace)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shared-prefix", action="store_true",
+                    help="serving traces: the shared-prefix decode for the largest group of sequences "
+                         "sharing leading blocks (default: the plain decode)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the sustained loop and the per-config measurements")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -274,6 +274,46 @@ int kv_swap_out(const kv_pool* pool, void* host_swap, int num_slots, const int32
 int kv_swap_in(const kv_pool* pool, const void* host_swap, int num_slots, const int32_t* pairs,
                int num_pairs, kv_stream_t stream);
 
+/* Decode for a batch in which some sequences share their first prefix_len
+ * tokens through the same physical blocks (forked sequences, a common
+ * system prompt or document; [PA]: blocks shared by reference count).  The
+ * result is that of paged_attention_decode on the same arguments; only the
+ * work is split: the shared prefix is attended once for all sharing
+ * sequences on the tensor cores (their queries are the rows of one
+ * multi-token pass over the prefix's blocks, no causal mask), each
+ * sequence's own tokens by the decode kernel, and the two partial results
+ * are merged by the log-sum-exp reduce.  The prefix's blocks are then read
+ * once per kv head instead of once per sequence and kv head.
+ *   Arguments as paged_attention_decode, plus:
+ *   prefix_seqs    device int32 [num_sharers]: batch indices of the
+ *                  sequences that share the prefix (each once).
+ *   prefix_blocks  device int32 [prefix_len / block_size]: its blocks; for
+ *                  every sharer s, block_tables[s][0 ..] starts with them and
+ *                  context_lens[s] >= prefix_len (not checked: other tables
+ *                  give another result).
+ *   prefix_len     tokens of the prefix, whole blocks (0: plain decode).
+ *   skip_lens      device int32 [batch]: prefix_len for the sharers, 0 for
+ *                  every other sequence.
+ *   workspace      device, 16-byte aligned, at least
+ *                  paged_attention_shared_prefix_workspace_bytes(pool, batch,
+ *                  num_q_heads, max_context_len, num_sharers) bytes (always
+ *                  needed); q must be 16-byte aligned.
+ *   Pools: f16 or bf16, no sliding window (others: KV_ERR_ARG).  Enqueues a
+ *   row gather, one multi-token launch, the decode and the reduce on
+ *   `stream`.  Device-side errors as paged_attention_decode (a sharer index
+ *   outside the batch or a skip length that is not a multiple of 16 within
+ *   the context: KV_ERR_BOUNDS). */
+size_t paged_attention_shared_prefix_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
+                                                     int max_context_len, int num_sharers);
+int paged_attention_decode_shared_prefix(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
+                                         int num_q_heads, const int32_t* block_tables,
+                                         int max_blocks_per_seq, const int32_t* context_lens, int batch,
+                                         int max_context_len, const int32_t* prefix_seqs, int num_sharers,
+                                         const int32_t* prefix_blocks, int prefix_len,
+                                         const int32_t* skip_lens, float scale, void* out,
+                                         kv_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                         const int32_t* seq_order, kv_stream_t stream);
+
 /* Largest scratch paged_attention_decode_noalloc can use (16 MiB). */
 #define KV_NOALLOC_WORKSPACE_BYTES (16u << 20)
 

@@ -79,6 +79,11 @@ _SIGS = {
     "paged_attention_decode": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int,
                                        c_void_p, c_int, c_int, c_float, c_void_p, c_int, c_void_p,
                                        c_size_t, c_void_p, c_void_p]),
+    "paged_attention_shared_prefix_workspace_bytes": (c_size_t, [c_void_p, c_int, c_int, c_int, c_int]),
+    "paged_attention_decode_shared_prefix": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p, c_int,
+                                                     c_void_p, c_int, c_int, c_void_p, c_int, c_void_p, c_int,
+                                                     c_void_p, c_float, c_void_p, c_int, c_void_p, c_size_t,
+                                                     c_void_p, c_void_p]),
     "paged_attention_decode_noalloc": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_void_p,
                                                c_int, c_void_p, c_int, c_int, c_float, c_void_p,
                                                c_int, c_void_p]),
@@ -274,6 +279,22 @@ def paged_attention_prefill(pool, layer, q, q_dtype, num_q_heads, cu_seqlens_q, 
                                         _ptr(cu_seqlens_q), int(total_q), int(max_q_len),
                                         _ptr(block_tables), max_blocks_per_seq, _ptr(context_lens),
                                         batch, float(scale), _ptr(out), out_dtype, _stream(stream)))
+
+
+def paged_attention_shared_prefix_workspace_bytes(pool, batch, num_q_heads, max_context_len, num_sharers) -> int:
+    return int(_lib.paged_attention_shared_prefix_workspace_bytes(pool, batch, num_q_heads, max_context_len,
+                                                                  num_sharers))
+
+
+def paged_attention_decode_shared_prefix(pool, layer, q, q_dtype, num_q_heads, block_tables, max_blocks_per_seq,
+                                         context_lens, batch, max_context_len, prefix_seqs, num_sharers,
+                                         prefix_blocks, prefix_len, skip_lens, scale, out, out_dtype,
+                                         workspace, workspace_bytes, stream=None, seq_order=None):
+    _check(_lib.paged_attention_decode_shared_prefix(
+        pool, layer, _ptr(q), q_dtype, num_q_heads, _ptr(block_tables), max_blocks_per_seq,
+        _ptr(context_lens), batch, max_context_len, _ptr(prefix_seqs), num_sharers, _ptr(prefix_blocks),
+        prefix_len, _ptr(skip_lens), float(scale), _ptr(out), out_dtype, _ptr(workspace), workspace_bytes,
+        _ptr(seq_order), _stream(stream)))
 
 
 KV_NOALLOC_WORKSPACE_BYTES = 16 << 20

@@ -69,6 +69,14 @@ struct DecodeParams {
   const void* q;                // [batch][num_q_heads][D] f16 / bf16
   const int32_t* block_tables;  // [batch][max_blocks]
   const int32_t* context_lens;  // [batch]
+  // NULL or [batch]: leading tokens of each sequence attended elsewhere (a
+  // shared prefix, a multiple of 16).  Such a sequence's decode starts after
+  // them and always writes split partials, at partition index + 1 (partition
+  // 0 holds the prefix's).
+  const int32_t* skip;
+  // NULL, or [batch][kv_heads] zeroed counters: the last CTA of a split
+  // (sequence, kv head) to finish merges its partials into the output
+  int* counters;
   const int32_t* seq_order;     // NULL or [batch]: sequence of grid row z
   const float* k_scale;         // FP8: [num_blocks][kv_heads]
   const float* v_scale;
@@ -142,6 +150,104 @@ __device__ __forceinline__ uint32_t tile_off(int row, int chunk16) {
   return box * (kChunk * S::BOXB) + (lin ^ (((lin >> 7) & S::SWZ) << 4));
 }
 
+// Merge of one (sequence, query head)'s split partials by one warp: with
+// partition p holding (o_p, m_z,p, l_p, m_w,p) in the log2 domain,
+//   Mz = max m_z,p,  L = sum l_p 2^(m_z,p - Mz),
+//   Mw = max m_w,p,  O = sum o_p 2^(m_w,p - Mw),   out = (O / L) 2^(Mw - Mz).
+// (For 16-bit caches m_w = m_z.)  idx = sequence * num_q_heads + head; np
+// partials of the num_parts slots are used; head_dim 64 or 128.  kL2: read
+// the partials through L2 only (other SMs of the same launch wrote them);
+// otherwise through the read-only path (a separate launch: the (m, l)
+// slots, read three times, may also hit in L1).
+template <bool kL2>
+__device__ __forceinline__ float4 ld_part(const float4* p) {
+  if constexpr (kL2) return __ldcg(p);
+  else return __ldg(p);
+}
+template <bool kL2>
+__device__ __forceinline__ float2 ld_part(const float2* p) {
+  if constexpr (kL2) return __ldcg(p);
+  else return __ldg(p);
+}
+
+template <bool kL2, int PER>
+__device__ __forceinline__ void merge_head_partials_t(const float* __restrict__ part_o,
+                                                      const float* __restrict__ part_ml, int64_t idx,
+                                                      int num_parts, int np, void* out, int out_kind,
+                                                      int lane) {
+  constexpr int HD = PER * 32;  // each lane owns PER consecutive dims
+  using Vec = typename std::conditional<PER == 4, float4, float2>::type;
+  const float4* ml = reinterpret_cast<const float4*>(part_ml) + idx * num_parts;
+  // the first 32 partitions' (m_z, l, m_w): one load per lane, kept
+  const float4 m0 = lane < np ? ld_part<kL2>(ml + lane) : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+  float Mz = m0.x, Mw = m0.z;
+  for (int q = lane + 32; q < np; q += 32) {
+    const float4 v = ld_part<kL2>(ml + q);
+    Mz = fmaxf(Mz, v.x);
+    Mw = fmaxf(Mw, v.z);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Mz = fmaxf(Mz, __shfl_xor_sync(0xffffffffu, Mz, o));
+    Mw = fmaxf(Mw, __shfl_xor_sync(0xffffffffu, Mw, o));
+  }
+  float L = m0.x != -INFINITY ? m0.y * ex2(m0.x - Mz) : 0.f;
+  for (int q = lane + 32; q < np; q += 32) {
+    const float4 v = ld_part<kL2>(ml + q);
+    if (v.x != -INFINITY) L += v.y * ex2(v.x - Mz);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const bool empty = !(L > 0.f) || Mw == -INFINITY;
+  const float scale = empty ? 0.f : ex2(Mw - Mz) / L;
+  // partition weights computed once per 32 partitions and broadcast; the
+  // partial rows are loaded 8 at a time so their latencies overlap (the sum
+  // still runs in partition order)
+  const float* po = part_o + idx * num_parts * HD + lane * PER;
+  float acc[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+  if (!empty) {
+    for (int q0 = 0; q0 < np; q0 += 32) {
+      float mq = m0.z;
+      if (q0 > 0) mq = q0 + lane < np ? ld_part<kL2>(ml + q0 + lane).z : -INFINITY;
+      const float wq = mq == -INFINITY ? 0.f : ex2(mq - Mw);
+      const int nq = min(32, np - q0);
+      for (int j0 = 0; j0 < nq; j0 += 8) {
+        Vec v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (j0 + u < nq) v[u] = ld_part<kL2>(reinterpret_cast<const Vec*>(po + (int64_t)(q0 + j0 + u) * HD));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u < nq) {  // uniform over the warp
+            const float wj = __shfl_sync(0xffffffffu, wq, j0 + u);
+            acc[0] += wj * v[u].x;
+            acc[1] += wj * v[u].y;
+            if constexpr (PER == 4) {
+              acc[2] += wj * v[u].z;
+              acc[3] += wj * v[u].w;
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < PER; ++k) store_out(out, out_kind, idx * HD + lane * PER + k, acc[k] * scale);
+}
+
+// head_dim 64 or 128
+template <bool kL2>
+__device__ __forceinline__ void merge_head_partials(const float* part_o, const float* part_ml, int64_t idx,
+                                                    int num_parts, int np, int head_dim, void* out,
+                                                    int out_kind, int lane) {
+  if (head_dim == 128)
+    merge_head_partials_t<kL2, 4>(part_o, part_ml, idx, num_parts, np, out, out_kind, lane);
+  else
+    merge_head_partials_t<kL2, 2>(part_o, part_ml, idx, num_parts, np, out, out_kind, lane);
+}
+
 // Resident CTAs per SM the register allocation is sized for: FP8 tiles
 // need half the shared memory of 16-bit ones, so four 4-warp CTAs fit.
 template <int KV, int WARPS>
@@ -149,7 +255,9 @@ constexpr int decode_min_blocks() {
   return WARPS == 8 ? 2 : (KV == KV_KIND_E4M3 ? 4 : 1);
 }
 
-template <int KV, int D, int WARPS, int STAGES>
+// EXT: the instantiation honours DecodeParams::skip and ::counters (16-bit
+// caches only); without it both are ignored and compiled out.
+template <int KV, int D, int WARPS, int STAGES, bool EXT>
 __global__ void __launch_bounds__(WARPS * 32, decode_min_blocks<KV, WARPS>())
 paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap) {
@@ -185,9 +293,22 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
     if (part == 0 && threadIdx.x == 0) record_error(KV_ERR_BOUNDS);
     n = n < 0 ? 0 : p.ctx_cap;
   }
+  // Skipped prefixes and the in-kernel merge: 16-bit caches only (the
+  // shared-prefix decode takes 16-bit pools, and FP8 contexts long enough to
+  // split run faster with the separate reduce)
+  constexpr bool kExt = EXT && !kFp8;
+  int skip = 0;
+  if (kExt && p.skip != nullptr) {
+    skip = p.skip[seq];
+    if (skip < 0 || skip > n || (skip & (kChunk - 1))) {
+      if (part == 0 && threadIdx.x == 0) record_error(KV_ERR_BOUNDS);
+      skip = skip < 0 ? 0 : min(skip, n) & ~(kChunk - 1);
+    }
+  }
   // sliding window: tokens [t_lo, n) only; chunks are counted from cb, the
-  // chunk holding t_lo (blocks wholly before it may already be released)
-  const int t_lo = p.window > 0 ? max(0, n - p.window) : 0;
+  // chunk holding t_lo (blocks wholly before it may already be released);
+  // a skipped prefix starts the visited range the same way
+  const int t_lo = p.window > 0 ? max(0, n - p.window) : skip;
   const int cb = t_lo / kChunk;
   const int total_chunks = (n + kChunk - 1) / kChunk - cb;
   const int c0 = part * p.part_chunks;
@@ -599,7 +720,8 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
 
   // a context that fits one partition is finished here even in split mode;
   // the reduce kernel skips it
-  const bool split = p.num_parts > 1 && total_chunks > p.part_chunks;
+  const bool split = (p.num_parts > 1 && total_chunks > p.part_chunks) || skip > 0;
+  const int pidx = part + (skip > 0 ? 1 : 0);  // partition 0 of a skipping sequence is its prefix's
   for (int idx = threadIdx.x; idx < p.group * D; idx += WARPS * 32) {
     const int g = idx / D;
     const int d = idx - g * D;
@@ -611,7 +733,7 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
     if (!split) {
       store_out(p.out, p.out_kind, sh * D + d, O * hd[g * 4]);
     } else {
-      const int64_t pi = sh * p.num_parts + part;
+      const int64_t pi = sh * p.num_parts + pidx;
       p.part_o[pi * D + d] = O;
       if (d == 0) {
         p.part_ml[pi * 4 + 0] = hd[g * 4 + 1];
@@ -621,83 +743,73 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
       }
     }
   }
+  if (kExt && split && p.counters != nullptr && skip == 0) {
+    // the last of this (sequence, kv head)'s partition CTAs merges them all
+    __shared__ int s_last;
+    const int np_seq = (total_chunks + p.part_chunks - 1) / p.part_chunks;
+    __threadfence();  // this thread's partials are visible to every SM
+    __syncthreads();
+    if (threadIdx.x == 0)
+      s_last = atomicAdd(p.counters + (int64_t)seq * p.kv_heads + kvh, 1) == np_seq - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int g = warp; g < p.group; g += WARPS)
+        merge_head_partials<true>(p.part_o, p.part_ml, (int64_t)seq * p.num_q_heads + kvh * p.group + g,
+                            p.num_parts, np_seq, D, p.out, p.out_kind, lane);
+    }
+  }
 }
 
-// Merge of split partials: for each (sequence, query head), with partition p
-// holding (o_p, m_z,p, l_p, m_w,p) in the log2 domain,
-//   Mz = max m_z,p,  L = sum l_p 2^(m_z,p - Mz),
-//   Mw = max m_w,p,  O = sum o_p 2^(m_w,p - Mw),   out = (O / L) 2^(Mw - Mz).
-// (For 16-bit caches m_w = m_z.)  One warp per (sequence, head); head_dim is
-// 64 or 128.
+// Merge of split partials (merge_head_partials), one warp per (sequence,
+// head), as a separate launch: used when the decode was not asked to merge
+// in its last partition CTA (shared-prefix decode, whose prefix partials
+// come from another kernel).
 __global__ void __launch_bounds__(256)
 lse_reduce_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                   const int32_t* __restrict__ context_lens, void* out, int out_kind,
                   int num_q_heads, int head_dim, int num_parts, int part_tokens, int ctx_cap,
-                  int window, int batch) {
+                  int window, int batch, const int32_t* __restrict__ skip_lens) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t idx = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
   if (idx >= (int64_t)batch * num_q_heads) return;
   const int seq = (int)(idx / num_q_heads);
   int n = context_lens[seq];
   n = n < 0 ? 0 : (n > ctx_cap ? ctx_cap : n);
-  // partitions of the chunks the decode visited (from the window's first chunk)
-  const int cb = window > 0 ? max(0, n - window) / kChunk : 0;
+  int skip = skip_lens != nullptr ? skip_lens[seq] : 0;
+  skip = skip < 0 ? 0 : min(skip, n) & ~(kChunk - 1);
+  // partitions of the chunks the decode visited (from the window's first
+  // chunk, or after a skipped prefix, whose partials come first)
+  const int cb = window > 0 ? max(0, n - window) / kChunk : skip / kChunk;
   const int chunks = (n + kChunk - 1) / kChunk - cb;
   const int part_chunks = part_tokens / kChunk;
-  const int np = max(1, (chunks + part_chunks - 1) / part_chunks);
+  const int np = max(1, (chunks + part_chunks - 1) / part_chunks) + (skip > 0 ? 1 : 0);
   if (np == 1) return;  // written by the decode kernel directly
-  const float4* ml = reinterpret_cast<const float4*>(part_ml) + idx * num_parts;
-  float Mz = -INFINITY, Mw = -INFINITY;
-  for (int q = lane; q < np; q += 32) {
-    const float4 v = ml[q];
-    Mz = fmaxf(Mz, v.x);
-    Mw = fmaxf(Mw, v.z);
+  merge_head_partials<false>(part_o, part_ml, idx, num_parts, np, head_dim, out, out_kind, lane);
+}
+
+// Rows of the sequences that share a prefix, gathered into consecutive
+// rows for the multi-token kernel: dst[i] = q[rows[i]] (num_q_heads * D
+// 16-bit values each, 16-byte chunks); also writes that kernel's one-sequence
+// metadata: cu = {0, num_rows}, ctx = {prefix_len}.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint4* __restrict__ q, const int32_t* __restrict__ rows, int num_rows,
+                   int batch, int chunks_per_row, uint4* __restrict__ dst, int32_t* meta, int prefix_len) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i == 0) {
+    meta[0] = 0;
+    meta[1] = num_rows;
+    meta[2] = prefix_len;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    Mz = fmaxf(Mz, __shfl_xor_sync(0xffffffffu, Mz, o));
-    Mw = fmaxf(Mw, __shfl_xor_sync(0xffffffffu, Mw, o));
+  if (i >= (int64_t)num_rows * chunks_per_row) return;
+  const int r = (int)(i / chunks_per_row), c = (int)(i - (int64_t)r * chunks_per_row);
+  const int src = rows[r];
+  if (src < 0 || src >= batch) {
+    record_error(KV_ERR_BOUNDS);
+    dst[i] = make_uint4(0u, 0u, 0u, 0u);
+    return;
   }
-  float L = 0.f;
-  for (int q = lane; q < np; q += 32) {
-    const float4 v = ml[q];
-    if (v.x != -INFINITY) L += v.y * ex2(v.x - Mz);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const bool empty = !(L > 0.f) || Mw == -INFINITY;
-  const float scale = empty ? 0.f : ex2(Mw - Mz) / L;
-  // each lane owns head_dim / 32 consecutive dims; partition weights are
-  // computed once per 32 partitions and broadcast
-  const int per = head_dim / 32;  // 2 or 4
-  const float* po = part_o + idx * num_parts * head_dim + lane * per;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (!empty) {
-    for (int q0 = 0; q0 < np; q0 += 32) {
-      float wq = 0.f;
-      if (q0 + lane < np) {
-        const float mq = ml[q0 + lane].z;
-        wq = mq == -INFINITY ? 0.f : ex2(mq - Mw);
-      }
-      const int nq = min(32, np - q0);
-      for (int j = 0; j < nq; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, wq, j);
-        const float* src = po + (int64_t)(q0 + j) * head_dim;
-        if (per == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(src);
-          acc[0] += wj * v.x;
-          acc[1] += wj * v.y;
-          acc[2] += wj * v.z;
-          acc[3] += wj * v.w;
-        } else {
-          const float2 v = *reinterpret_cast<const float2*>(src);
-          acc[0] += wj * v.x;
-          acc[1] += wj * v.y;
-        }
-      }
-    }
-  }
-  for (int k = 0; k < per; ++k) store_out(out, out_kind, idx * head_dim + lane * per + k, acc[k] * scale);
+  dst[i] = q[(int64_t)src * chunks_per_row + c];
 }
 
 }  // namespace pagedkv

@@ -168,6 +168,7 @@ int decode_slots(const kv_pool* pool, int group) {
 // partitions for 8 x 16K-token FP8 contexts (256 units) and ~1K-token ones
 // for a 4K-token window over 8 x 16K-token bf16 contexts (shorter partitions
 // lose more to each CTA's start than they gain in balance).
+constexpr int kFusedMergeMaxParts = 4;  // measured: GQA trace (3) +3%, FP8 16K contexts (10, 32) -1%, -6%
 constexpr int kWavesKeep = 3;
 constexpr int kWavesSplit = 4;
 constexpr int kAutoPartition = 4096;
@@ -207,7 +208,7 @@ int visited_len(const kv_pool* pool, int max_context_len) {
 template <int KV, int D, int W, int STAGES>
 int decode_occupancy() {
   using Shape = DecodeShape<KV, D, W, STAGES>;
-  auto kernel = paged_decode_kernel<KV, D, W, STAGES>;
+  auto kernel = paged_decode_kernel<KV, D, W, STAGES, false>;
   static std::atomic<int> cached[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
@@ -251,10 +252,10 @@ int decode_occupancy(const kv_pool* pool, int group) {
   }
 }
 
-template <int KV, int D, int W, int STAGES>
-int launch_decode_t(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cudaStream_t stream) {
+template <int KV, int D, int W, int STAGES, bool EXT>
+int launch_decode_x(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cudaStream_t stream) {
   using Shape = DecodeShape<KV, D, W, STAGES>;
-  auto kernel = paged_decode_kernel<KV, D, W, STAGES>;
+  auto kernel = paged_decode_kernel<KV, D, W, STAGES, EXT>;
   static std::atomic<uint64_t> done{0};  // one flag word per instantiation
   int rc = ensure_smem(kernel, Shape::MAX_SMEM_BYTES, done);
   if (rc != KV_OK) return rc;
@@ -262,6 +263,19 @@ int launch_decode_t(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cu
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "paged_decode_kernel launch");
   return KV_OK;
+}
+
+// Decodes that skip prefixes or merge their own partials run the extended
+// instantiation (16-bit caches; FP8 callers pass neither)
+template <int KV, int D, int W, int STAGES>
+int launch_decode_t(const DecodeParams& p, const LayerBinding& lb, dim3 grid, cudaStream_t stream) {
+  if constexpr (KV != KV_KIND_E4M3) {
+    if (p.skip != nullptr || p.counters != nullptr)
+      return launch_decode_x<KV, D, W, STAGES, true>(p, lb, grid, stream);
+  } else {
+    if (p.skip != nullptr || p.counters != nullptr) return fail(KV_ERR_ARG, "FP8 decode takes no skip or counters");
+  }
+  return launch_decode_x<KV, D, W, STAGES, false>(p, lb, grid, stream);
 }
 
 template <int KV, int D, int W>
@@ -552,18 +566,23 @@ size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q
   const int group = num_q_heads % pool->kv_heads == 0 ? num_q_heads / pool->kv_heads : 1;
   const int np = num_parts_for(pool, batch, visited_len(pool, max_context_len), group);
   if (np <= 1) return 0;
-  return (size_t)batch * num_q_heads * np * (pool->head_dim + 4) * sizeof(float);
+  // partials, then one merge counter per (sequence, kv head)
+  return (size_t)batch * num_q_heads * np * (pool->head_dim + 4) * sizeof(float) +
+         ((size_t)batch * pool->kv_heads * sizeof(int) + 15) / 16 * 16;
 }
 
-int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
-                           int num_q_heads, const int32_t* block_tables, int max_blocks_per_seq,
-                           const int32_t* context_lens, int batch, int max_context_len,
-                           float scale, void* out, kv_dtype out_dtype, void* workspace,
-                           size_t workspace_bytes, const int32_t* seq_order, kv_stream_t stream) {
+}  // extern "C"
+
+namespace pagedkv {
+namespace {
+
+// Argument checks shared by the decode entry points.
+int check_decode_args(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype, int num_q_heads,
+                      const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                      int batch, int max_context_len, float scale, void* out, kv_dtype out_dtype) {
   if (!pool) return fail(KV_ERR_ARG, "NULL pool");
   if (layer < 0 || layer >= pool->num_layers) return fail(KV_ERR_ARG, "layer %d out of range", layer);
-  const LayerBinding& lb = pool->layers[layer];
-  if (!lb.bound) return fail(KV_ERR_STATE, "layer %d is not bound", layer);
+  if (!pool->layers[layer].bound) return fail(KV_ERR_STATE, "layer %d is not bound", layer);
   if (batch < 0 || max_context_len < 0 || max_blocks_per_seq < 0)
     return fail(KV_ERR_ARG, "negative size");
   if (batch > 65535) return fail(KV_ERR_ARG, "batch %d above 65535", batch);
@@ -577,12 +596,93 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   if (out_dtype != q_dtype && out_dtype != KV_F32)
     return fail(KV_ERR_ARG, "out dtype must be the q dtype or KV_F32");
   if (!std::isfinite(scale)) return fail(KV_ERR_ARG, "scale is not finite");
-  if (batch == 0) return ok();
+  if (batch == 0) return KV_OK;
   if (!q || !block_tables || !context_lens || !out) return fail(KV_ERR_ARG, "NULL input");
   if ((uintptr_t)q & 7) return fail(KV_ERR_ARG, "q must be 8-byte aligned");
   if ((int64_t)max_blocks_per_seq * pool->block_size < max_context_len)
     return fail(KV_ERR_ARG, "max_blocks_per_seq %d cannot hold max_context_len %d",
                 max_blocks_per_seq, max_context_len);
+  return KV_OK;
+}
+
+// The decode launch (and the reduce when more than one partition exists):
+// `grid_parts` partitions per sequence in the grid, `stride_parts` partials
+// per (sequence, head) in part_o / part_ml, `skip` as in DecodeParams.
+int enqueue_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype, int num_q_heads,
+                   const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                   int batch, int max_context_len, float scale, void* out, kv_dtype out_dtype,
+                   float* part_o, float* part_ml, int grid_parts, int stride_parts, int part_tokens,
+                   const int32_t* skip, int* counters, const int32_t* seq_order, cudaStream_t s) {
+  const LayerBinding& lb = pool->layers[layer];
+  const int group = num_q_heads / pool->kv_heads;
+  DecodeParams p;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.skip = skip;
+  p.counters = counters;
+  p.seq_order = seq_order;
+  p.k_scale = lb.k_scale;
+  p.v_scale = lb.v_scale;
+  p.out = out;
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.q_bf16 = q_dtype == KV_BF16;
+  p.out_kind = out_kind(out_dtype);
+  p.num_q_heads = num_q_heads;
+  p.group = group;
+  p.kv_heads = pool->kv_heads;
+  p.block_size = pool->block_size;
+  p.cpb_shift = 0;
+  while ((kChunk << p.cpb_shift) < pool->block_size) ++p.cpb_shift;
+  p.num_blocks = pool->num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.part_chunks = part_tokens / kChunk;
+  p.num_parts = stride_parts;
+  p.ctx_cap = (int)std::min<int64_t>((int64_t)max_blocks_per_seq * pool->block_size, max_context_len);
+  p.window = pool->window;
+  p.scale_log2 = scale * 1.4426950408889634f;
+
+  const dim3 grid(grid_parts, pool->kv_heads, batch);
+  const PipeShape ps = pipe_for(pool, group);
+  if (counters != nullptr && stride_parts > 1) {
+    // the merge counters start at zero in every call (the workspace is the caller's)
+    cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)batch * pool->kv_heads * sizeof(int), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (merge counters)");
+  }
+  int rc;
+  switch (pool->dtype) {
+    case KV_F16: rc = launch_decode_kv<KV_KIND_F16>(pool->head_dim, ps, p, lb, grid, s); break;
+    case KV_BF16: rc = launch_decode_kv<KV_KIND_BF16>(pool->head_dim, ps, p, lb, grid, s); break;
+    default: rc = launch_decode_kv<KV_KIND_E4M3>(pool->head_dim, ps, p, lb, grid, s); break;
+  }
+  if (rc != KV_OK) return rc;
+  if (stride_parts > 1 && counters == nullptr) {  // merged by a separate launch
+    const int64_t rows = (int64_t)batch * num_q_heads;
+    const int blocks = (int)((rows + 7) / 8);
+    lse_reduce_kernel<<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, context_lens, out, p.out_kind,
+                                             num_q_heads, pool->head_dim, stride_parts, part_tokens,
+                                             p.ctx_cap, p.window, batch, skip);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
+  }
+  return KV_OK;
+}
+
+}  // namespace
+}  // namespace pagedkv
+
+extern "C" {
+
+int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
+                           int num_q_heads, const int32_t* block_tables, int max_blocks_per_seq,
+                           const int32_t* context_lens, int batch, int max_context_len,
+                           float scale, void* out, kv_dtype out_dtype, void* workspace,
+                           size_t workspace_bytes, const int32_t* seq_order, kv_stream_t stream) {
+  int rc = check_decode_args(pool, layer, q, q_dtype, num_q_heads, block_tables, max_blocks_per_seq,
+                             context_lens, batch, max_context_len, scale, out, out_dtype);
+  if (rc != KV_OK) return rc;
+  if (batch == 0) return ok();
   const int visited = visited_len(pool, max_context_len);
   const int group = num_q_heads / pool->kv_heads;
   const int pt = partition_tokens(pool, batch, visited, group);
@@ -592,53 +692,94 @@ int paged_attention_decode(const kv_pool* pool, int layer, const void* q, kv_dty
   if (need > 0 && (!workspace || workspace_bytes < need))
     return fail(KV_ERR_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
   if (need > 0 && ((uintptr_t)workspace & 15)) return fail(KV_ERR_ARG, "workspace must be 16-byte aligned");
-
-  DecodeParams p;
-  p.q = q;
-  p.block_tables = block_tables;
-  p.context_lens = context_lens;
-  p.seq_order = seq_order;
-  p.k_scale = lb.k_scale;
-  p.v_scale = lb.v_scale;
-  p.out = out;
   float* ws = static_cast<float*>(workspace);
-  p.part_o = need ? ws : nullptr;
-  p.part_ml = need ? ws + (size_t)batch * num_q_heads * np * pool->head_dim : nullptr;
-  p.q_bf16 = q_dtype == KV_BF16;
-  p.out_kind = out_kind(out_dtype);
-  p.num_q_heads = num_q_heads;
-  p.group = num_q_heads / pool->kv_heads;
-  p.kv_heads = pool->kv_heads;
-  p.block_size = pool->block_size;
-  p.cpb_shift = 0;
-  while ((kChunk << p.cpb_shift) < pool->block_size) ++p.cpb_shift;
-  p.num_blocks = pool->num_blocks;
-  p.max_blocks = max_blocks_per_seq;
-  p.part_chunks = pt / kChunk;
-  p.num_parts = np;
-  p.ctx_cap = (int)std::min<int64_t>((int64_t)max_blocks_per_seq * pool->block_size, max_context_len);
-  p.window = pool->window;
-  p.scale_log2 = scale * 1.4426950408889634f;
-
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const dim3 grid(np, pool->kv_heads, batch);
-  const PipeShape ps = pipe_for(pool, group);
-  int rc;
-  switch (pool->dtype) {
-    case KV_F16: rc = launch_decode_kv<KV_KIND_F16>(pool->head_dim, ps, p, lb, grid, s); break;
-    case KV_BF16: rc = launch_decode_kv<KV_KIND_BF16>(pool->head_dim, ps, p, lb, grid, s); break;
-    default: rc = launch_decode_kv<KV_KIND_E4M3>(pool->head_dim, ps, p, lb, grid, s); break;
-  }
+  float* part_o = need ? ws : nullptr;
+  float* part_ml = need ? ws + (size_t)batch * num_q_heads * np * pool->head_dim : nullptr;
+  // the decode merges its own partials when contexts are split into few
+  // partitions (few split sequences: a separate reduce launch would mostly
+  // find nothing to do); with many partitions per sequence the separate
+  // reduce, spread over every SM, is faster than the last CTAs' merges (FP8
+  // decodes always use the separate reduce)
+  int* counters = need && np <= kFusedMergeMaxParts && pool->dtype != KV_FP8_E4M3
+                      ? reinterpret_cast<int*>(part_ml + (size_t)batch * num_q_heads * np * 4)
+                      : nullptr;
+  rc = enqueue_decode(pool, layer, q, q_dtype, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
+                      batch, max_context_len, scale, out, out_dtype, part_o, part_ml, np, np, pt, nullptr,
+                      counters, seq_order, reinterpret_cast<cudaStream_t>(stream));
   if (rc != KV_OK) return rc;
-  if (np > 1) {
-    const int64_t rows = (int64_t)batch * num_q_heads;
-    const int blocks = (int)((rows + 7) / 8);
-    lse_reduce_kernel<<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, context_lens, out, p.out_kind,
-                                             num_q_heads, pool->head_dim, np, pt, p.ctx_cap,
-                                             p.window, batch);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "lse_reduce_kernel launch");
-  }
+  return ok();
+}
+
+size_t paged_attention_shared_prefix_workspace_bytes(const kv_pool* pool, int batch, int num_q_heads,
+                                                     int max_context_len, int num_sharers) {
+  if (!pool || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0 || num_sharers < 0) return 0;
+  const int group = num_q_heads % pool->kv_heads == 0 ? num_q_heads / pool->kv_heads : 1;
+  const int np = num_parts_for(pool, batch, max_context_len, group) + 1;
+  const size_t parts = (size_t)batch * num_q_heads * np * (pool->head_dim + 4) * sizeof(float);
+  const size_t rows = (size_t)num_sharers * num_q_heads * pool->head_dim * 2;
+  return parts + (rows + 15) / 16 * 16 + 16;
+}
+
+int paged_attention_decode_shared_prefix(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
+                                         int num_q_heads, const int32_t* block_tables,
+                                         int max_blocks_per_seq, const int32_t* context_lens, int batch,
+                                         int max_context_len, const int32_t* prefix_seqs, int num_sharers,
+                                         const int32_t* prefix_blocks, int prefix_len,
+                                         const int32_t* skip_lens, float scale, void* out,
+                                         kv_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                         const int32_t* seq_order, kv_stream_t stream) {
+  int rc = check_decode_args(pool, layer, q, q_dtype, num_q_heads, block_tables, max_blocks_per_seq,
+                             context_lens, batch, max_context_len, scale, out, out_dtype);
+  if (rc != KV_OK) return rc;
+  if (pool->dtype != KV_F16 && pool->dtype != KV_BF16)
+    return fail(KV_ERR_ARG, "shared-prefix decode needs an f16 or bf16 pool");
+  if (pool->window > 0) return fail(KV_ERR_ARG, "shared-prefix decode does not take a sliding window");
+  if (num_sharers < 0 || prefix_len < 0 || num_sharers > batch)
+    return fail(KV_ERR_ARG, "bad shared prefix: %d sequences, %d tokens", num_sharers, prefix_len);
+  if (prefix_len % pool->block_size != 0 || prefix_len > max_context_len)
+    return fail(KV_ERR_ARG, "prefix_len %d must be whole blocks within max_context_len %d", prefix_len,
+                max_context_len);
+  if (!(scale > 0.f)) return fail(KV_ERR_ARG, "scale must be > 0");
+  if (batch == 0) return ok();
+  if (num_sharers == 0 || prefix_len == 0)  // nothing shared: the plain decode
+    return paged_attention_decode(pool, layer, q, q_dtype, num_q_heads, block_tables, max_blocks_per_seq,
+                                  context_lens, batch, max_context_len, scale, out, out_dtype, workspace,
+                                  workspace_bytes, seq_order, stream);
+  if (!prefix_seqs || !prefix_blocks || !skip_lens) return fail(KV_ERR_ARG, "NULL shared-prefix input");
+  if ((uintptr_t)q & 15) return fail(KV_ERR_ARG, "q must be 16-byte aligned for shared-prefix decode");
+  const size_t need = paged_attention_shared_prefix_workspace_bytes(pool, batch, num_q_heads, max_context_len,
+                                                                    num_sharers);
+  if (!workspace || workspace_bytes < need)
+    return fail(KV_ERR_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if ((uintptr_t)workspace & 15) return fail(KV_ERR_ARG, "workspace must be 16-byte aligned");
+  const int group = num_q_heads / pool->kv_heads;
+  const int pt = partition_tokens(pool, batch, max_context_len, group);
+  const int np = num_parts_for(pool, batch, max_context_len, group);
+  if (np + 1 > 65535) return fail(KV_ERR_ARG, "too many partitions");
+  const int npa = np + 1;
+  float* part_o = static_cast<float*>(workspace);
+  float* part_ml = part_o + (size_t)batch * num_q_heads * npa * pool->head_dim;
+  uint8_t* rows = reinterpret_cast<uint8_t*>(part_ml + (size_t)batch * num_q_heads * npa * 4);
+  const size_t row_bytes = (size_t)num_sharers * num_q_heads * pool->head_dim * 2;
+  int32_t* meta = reinterpret_cast<int32_t*>(rows + (row_bytes + 15) / 16 * 16);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // 1. the sharers' query rows, consecutive
+  const int chunks_per_row = num_q_heads * pool->head_dim * 2 / 16;
+  const int64_t threads = (int64_t)num_sharers * chunks_per_row;
+  gather_rows_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+      static_cast<const uint4*>(q), prefix_seqs, num_sharers, batch, chunks_per_row,
+      reinterpret_cast<uint4*>(rows), meta, prefix_len);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gather_rows_kernel launch");
+  // 2. the prefix once for every sharer, on the tensor cores: partition 0
+  rc = prefix_partials(pool, layer, rows, num_sharers, num_q_heads, prefix_blocks,
+                       prefix_len / pool->block_size, meta, scale, part_o, part_ml, prefix_seqs, npa, stream);
+  if (rc != KV_OK) return rc;
+  // 3. every sequence's own tokens (after the prefix for sharers), then the merge
+  rc = enqueue_decode(pool, layer, q, q_dtype, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
+                      batch, max_context_len, scale, out, out_dtype, part_o, part_ml, np, npa, pt, skip_lens,
+                      nullptr, seq_order, s);
+  if (rc != KV_OK) return rc;
   return ok();
 }
 

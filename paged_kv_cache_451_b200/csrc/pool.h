@@ -24,6 +24,23 @@ inline int elem_bytes(kv_dtype t) { return t == KV_FP8_E4M3 ? 1 : (t == KV_F32 ?
 
 }  // namespace pagedkv
 
+struct kv_pool;
+
+namespace pagedkv {
+
+// Shared-prefix partials on the tensor cores (prefill.cu): rows of q_rows
+// ([num_rows][num_q_heads][head_dim], the pool dtype) attend to the
+// prefix_len tokens held by prefix_blocks; row r writes partition 0 of
+// sequence prefix_rows[r] in part_o / part_ml (num_parts per (sequence,
+// head)).  meta: device int32 {0, num_rows, prefix_len}.  Enqueues one
+// launch on `stream`; returns a KV_* status.
+int prefix_partials(const kv_pool* pool, int layer, const void* q_rows, int num_rows, int num_q_heads,
+                    const int32_t* prefix_blocks, int num_prefix_blocks, const int32_t* meta,
+                    float scale, float* part_o, float* part_ml, const int32_t* prefix_rows,
+                    int num_parts, kv_stream_t stream);
+
+}  // namespace pagedkv
+
 struct kv_pool {
   int block_size = 0;
   int num_blocks = 0;

@@ -119,6 +119,50 @@ static_assert(PrefillShape<64, 4>::SMEM_BYTES * 2 > 228 * 1024, "one prefill CTA
 static_assert(PrefillShape<128, 2>::SMEM_BYTES * 2 > 228 * 1024, "one prefill CTA per SM");
 
 }  // namespace
+
+int prefix_partials(const kv_pool* pool, int layer, const void* q_rows, int num_rows, int num_q_heads,
+                    const int32_t* prefix_blocks, int num_prefix_blocks, const int32_t* meta,
+                    float scale, float* part_o, float* part_ml, const int32_t* prefix_rows,
+                    int num_parts, kv_stream_t stream) {
+  const LayerBinding& lb = pool->layers[layer];
+  const int g = num_q_heads / pool->kv_heads;
+  const int tq = kPfRows / g;
+  const int64_t pairs = ((int64_t)num_rows + kPfTiles * tq - 1) / (kPfTiles * tq);
+  int* err = error_word_cached();
+  if (!err) return fail(KV_ERR_CUDA, "device error word unavailable");
+  CUtensorMap qmap;
+  int rc = make_q_map(q_rows, num_rows, num_q_heads, pool->head_dim, g, tq, &qmap);
+  if (rc != KV_OK) return rc;
+  PrefillParams p;
+  p.cu_q = meta;              // {0, num_rows}: one sequence of num_rows new tokens
+  p.block_tables = prefix_blocks;
+  p.context_lens = meta + 2;  // {prefix_len}
+  p.out = part_o;             // unused: the epilogue writes partials
+  p.err = err;
+  p.out_kind = PF_OUT_F32;
+  p.num_q_heads = num_q_heads;
+  p.group = g;
+  p.tokens_per_tile = tq;
+  p.num_q_pairs = (int)pairs;
+  p.kv_heads = pool->kv_heads;
+  p.block_size = pool->block_size;
+  p.num_blocks = pool->num_blocks;
+  p.max_blocks = num_prefix_blocks;
+  p.total_q = num_rows;
+  p.window = 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.batch = 1;
+  p.num_items = pairs * pool->kv_heads;
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.prefix_rows = prefix_rows;
+  p.num_parts = num_parts;
+  const dim3 grid((unsigned)p.num_items);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return pool->dtype == KV_BF16 ? launch_d<true>(pool->head_dim, p, qmap, lb, grid, s)
+                                : launch_d<false>(pool->head_dim, p, qmap, lb, grid, s);
+}
+
 }  // namespace pagedkv
 
 using namespace pagedkv;
@@ -188,6 +232,10 @@ int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dt
   p.batch = batch;
   p.num_items = pairs * pool->kv_heads * batch;
   if (p.num_items > 0x7fffffff) return fail(KV_ERR_ARG, "too many query tiles");
+  p.part_o = nullptr;
+  p.part_ml = nullptr;
+  p.prefix_rows = nullptr;
+  p.num_parts = 0;
 
   // one CTA per work item, heaviest first; a CTA that finishes an item
   // cancels the launch of a CTA not yet started and takes over its item

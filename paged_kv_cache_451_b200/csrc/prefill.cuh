@@ -94,6 +94,17 @@ struct PrefillParams {
   float scale_log2;             // softmax scale * log2(e), > 0
   int batch;
   int64_t num_items;            // num_q_pairs * kv_heads * batch
+  // Shared-prefix mode (part_o != NULL): one virtual sequence whose new
+  // tokens are the decode queries of the sequences sharing a prefix (one q
+  // row each) and whose keys are the prefix's context_lens[0] tokens; every
+  // row attends to all of them (no causal mask, no window), and the
+  // epilogue writes split-K partials of partition 0 of the row's sequence
+  // prefix_rows[row] (unnormalised O, its reference max and sum) in place
+  // of an output row.
+  float* part_o;                // [B][num_q_heads][num_parts][D]
+  float* part_ml;               // [B][num_q_heads][num_parts][4]: m_z, l, m_w, 0
+  const int32_t* prefix_rows;   // [total_q]
+  int num_parts;
 };
 
 template <int D, int STAGES>
@@ -240,7 +251,8 @@ __device__ __forceinline__ bool item_at(const PrefillParams& p, int64_t v, bool 
   it.q0 = p.cu_q[it.s];
   it.q_len = p.cu_q[it.s + 1] - it.q0;
   it.n = p.context_lens[it.s];
-  if (it.q0 < 0 || it.q_len < 0 || it.q_len > it.n || (int64_t)it.q0 + it.q_len > p.total_q ||
+  const bool prefix = p.part_o != nullptr;  // every row sees all n keys
+  if (it.q0 < 0 || it.q_len < 0 || (!prefix && it.q_len > it.n) || (int64_t)it.q0 + it.q_len > p.total_q ||
       (int64_t)it.n > (int64_t)p.max_blocks * p.block_size ||
       it.q_len > p.num_q_pairs * kPfTiles * tq) {
     if (report && qp == p.num_q_pairs - 1 && it.kvh == 0) atomicCAS(p.err, 0, KV_ERR_BOUNDS);
@@ -251,12 +263,12 @@ __device__ __forceinline__ bool item_at(const PrefillParams& p, int64_t v, bool 
   // Key tiles start at kb: 0, or with a sliding window the 16-key chunk
   // holding the first position any row of the item sees (no block before
   // it is read: it may already be released).
-  it.kb = p.window > 0 ? max(0, it.n - it.q_len + it.t0 - p.window + 1) / 16 * 16 : 0;
+  it.kb = p.window > 0 && !prefix ? max(0, it.n - it.q_len + it.t0 - p.window + 1) / 16 * 16 : 0;
 #pragma unroll
   for (int x = 0; x < kPfTiles; ++x) {
     const int tx = it.t0 + x * tq;
     it.ntok[x] = tx < it.q_len ? min(tq, it.q_len - tx) : 0;
-    it.kendx[x] = it.ntok[x] ? it.n - it.q_len + tx + it.ntok[x] : 0;  // keys .. kend - 1
+    it.kendx[x] = it.ntok[x] ? (prefix ? it.n : it.n - it.q_len + tx + it.ntok[x]) : 0;  // keys .. kend - 1
     it.ntx[x] = it.ntok[x] ? (it.kendx[x] - it.kb + kPfKeys - 1) / kPfKeys : 0;
   }
   it.kend = max(it.kendx[0], it.kendx[1]);
@@ -611,7 +623,9 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       continue;
     }
     const bool valid = r < qrows && tok < (x ? it.ntok[1] : it.ntok[0]);
-    const int prow = valid ? it.n - it.q_len + it.t0 + x * tq + tok : (x ? it.kendx[1] : it.kendx[0]) - 1;
+    const bool prefix = p.part_o != nullptr;
+    const int prow = valid && !prefix ? it.n - it.q_len + it.t0 + x * tq + tok
+                                      : (x ? it.kendx[1] : it.kendx[0]) - 1;
     float m_ref = -INFINITY, l = 0.f;
     for (int j = 0; j < nt; ++j) {
       ok = __all_sync(0xffffffffu, pf::wait(SF(x), (sc + j) & 1, abort_flag, p.err));
@@ -768,13 +782,26 @@ paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap 
       const float inv = 1.f / l;
       const int64_t orow =
           ((int64_t)(it.q0 + it.t0 + x * tq + tok) * p.num_q_heads + it.kvh * g + head) * D;
+      // shared-prefix mode: partition 0 of the row's sequence, unnormalised
+      int64_t prow_part = -1;
+      if (prefix && valid) {
+        const int64_t sq = p.prefix_rows[it.q0 + it.t0 + x * tq + tok];
+        prow_part = (sq * p.num_q_heads + it.kvh * g + head) * p.num_parts;
+        *reinterpret_cast<float4*>(p.part_ml + prow_part * 4) = make_float4(m_ref, l, m_ref, 0.f);
+      }
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tc::ld32(tO + 32 * c, o);
         tc::wait_ld();
         tc::pin(o);
-        if (valid) {
+        if (prow_part >= 0) {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + prow_part * D + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+        } else if (valid && !prefix) {
           if (p.out_kind == PF_OUT_F32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + 32 * c);
 #pragma unroll

@@ -26,7 +26,8 @@ from __future__ import annotations
 import numpy as np
 
 from . import (KV_F32, block_copy, kv_sched_outputs, kv_sched_step, kv_sched_swap_outputs, kv_swap_in,
-               kv_swap_out, paged_attention_decode, paged_attention_prefill,
+               kv_swap_out, paged_attention_decode, paged_attention_decode_shared_prefix,
+               paged_attention_prefill, paged_attention_shared_prefix_workspace_bytes,
                paged_attention_workspace_bytes, paged_kv_write)
 
 
@@ -53,6 +54,32 @@ def schedule_order(context_lens, policy="long_first"):
     return np.concatenate([long, rest]).astype(np.int32)
 
 
+def find_shared_prefix(block_tables, context_lens, block_size, min_sharers=2, min_tokens=1):
+    """The largest group of running sequences whose block tables start with
+    the same physical blocks (forked sequences, a common prompt cached once):
+    (batch indices of the group, the common leading block ids), cut to whole
+    blocks inside every member's context; (None, None) when no group of at
+    least min_sharers shares at least min_tokens tokens.  Only the first
+    column is grouped: one shared prefix per step."""
+    lens = np.asarray(context_lens)
+    b = lens.shape[0]
+    if b < min_sharers:
+        return None, None
+    tables = np.asarray(block_tables)[:b]
+    first = tables[:, 0]
+    vals, counts = np.unique(first[first >= 0], return_counts=True)
+    if counts.size == 0 or counts.max() < min_sharers:
+        return None, None
+    rows = np.nonzero(first == vals[np.argmax(counts)])[0]
+    sub = tables[rows]
+    same = np.all(sub == sub[0], axis=0) & (sub[0] >= 0)
+    k = sub.shape[1] if same.all() else int(np.argmin(same))
+    k = min(k, int(lens[rows].min()) // block_size)
+    if k * block_size < max(min_tokens, 1):
+        return None, None
+    return rows.astype(np.int32), sub[0, :k].astype(np.int32)
+
+
 class DecodeLoop:
     """Runs the iteration above on one device.  The step's metadata (slots,
     block tables, context lengths, scheduling order, copy pairs) is packed
@@ -63,7 +90,8 @@ class DecodeLoop:
 
     def __init__(self, pool, sched, *, num_q_heads, kv_heads, head_dim, block_size, q_dtype,
                  scale, max_batch, max_blocks, max_tokens, max_context, device="cuda",
-                 order_policy="batch", host_swap=None, swap_slots=0):
+                 order_policy="batch", host_swap=None, swap_slots=0, shared_prefix=False,
+                 min_sharers=8, min_prefix_tokens=256):
         import torch
         self.torch = torch
         self.pool, self.sched = pool, sched
@@ -72,7 +100,14 @@ class DecodeLoop:
         self.max_batch, self.max_blocks, self.max_tokens = max_batch, max_blocks, max_tokens
         self.order_policy = order_policy
         self.host_swap, self.swap_slots = host_swap, swap_slots
+        # shared-prefix decode (paged_attention_decode_shared_prefix) when a
+        # group of at least min_sharers sequences shares min_prefix_tokens
+        self.shared_prefix = shared_prefix
+        self.min_sharers, self.min_prefix_tokens = min_sharers, min_prefix_tokens
+        self.last_prefix = (None, None)
         cap = 8 * max_tokens + 4 * (max_batch * max_blocks + 6 * max_batch + 1) + 256
+        if shared_prefix:
+            cap += 4 * (2 * max_batch + max_blocks) + 64
         if swap_slots:
             cap += 16 * swap_slots + 64
         self.cap = (cap + 255) // 256 * 256
@@ -86,6 +121,9 @@ class DecodeLoop:
         # the scratch is sized for the largest need over every batch size
         ws = max(paged_attention_workspace_bytes(pool, b, num_q_heads, max_context)
                  for b in range(1, max_batch + 1))
+        if shared_prefix:
+            ws = max(ws, max(paged_attention_shared_prefix_workspace_bytes(pool, b, num_q_heads, max_context, b)
+                             for b in range(1, max_batch + 1)))
         self.ws_cap = max(ws, 16)
         self.d_ws = torch.empty(self.ws_cap, dtype=torch.uint8, device=device)
 
@@ -100,11 +138,12 @@ class DecodeLoop:
         return out
 
     @staticmethod
-    def _layout(b, t, c, width, a=0, so=0, si=0):
+    def _layout(b, t, c, width, a=0, so=0, si=0, sh=0, shb=0):
         off, lay = 0, {}
         for name, n, size in (("slots", t, 8), ("tables", b * width, 4), ("lens", b, 4),
                               ("order", b, 4), ("cow", 2 * c, 4), ("cu", a + 1 if a else 0, 4),
-                              ("pf_lens", a, 4), ("swo", 2 * so, 4), ("swi", 2 * si, 4)):
+                              ("pf_lens", a, 4), ("swo", 2 * so, 4), ("swi", 2 * si, 4),
+                              ("sh_seqs", sh, 4), ("sh_blocks", shb, 4), ("skip", b if sh else 0, 4)):
             lay[name] = (off, n)
             off += (n * size + 15) // 16 * 16
         return lay, off
@@ -137,7 +176,13 @@ class DecodeLoop:
             raise RuntimeError("the step swaps but the loop has no host swap space")
         k = self.it % 2
         self.it += 1
-        lay, nbytes = self._layout(b, t, c, w, a, so, si)
+        sh_rows = sh_blocks = None
+        if self.shared_prefix and b:
+            sh_rows, sh_blocks = find_shared_prefix(plan["block_tables"], plan["context_lens"], self.bs,
+                                                    self.min_sharers, self.min_prefix_tokens)
+        self.last_prefix = (sh_rows, sh_blocks)
+        nsh, nshb = (len(sh_rows), len(sh_blocks)) if sh_rows is not None else (0, 0)
+        lay, nbytes = self._layout(b, t, c, w, a, so, si, nsh, nshb)
         if nbytes > self.cap:
             raise RuntimeError("step metadata exceeds the loop's buffers")
         if self.copy_ev[k] is not None:  # the pinned buffer is reused: its last upload must be done
@@ -158,6 +203,12 @@ class DecodeLoop:
             put("swo", plan["swap_out"], np.int32)
         if si:
             put("swi", plan["swap_in"], np.int32)
+        if nsh:
+            put("sh_seqs", sh_rows, np.int32)
+            put("sh_blocks", sh_blocks, np.int32)
+            skip = np.zeros(b, np.int32)
+            skip[sh_rows] = nshb * self.bs
+            put("skip", skip, np.int32)
         if a:
             put("cu", np.concatenate([[0], np.cumsum(new)]), np.int32)
             put("pf_lens", np.asarray(plan["context_lens"][-a:], np.int64) - 1, np.int32)
@@ -191,7 +242,19 @@ class DecodeLoop:
                                     int(new.sum()), int(new.max()), tables, w, dview("pf_lens", torch.int32),
                                     a, self.scale, prefill_out, KV_F32 if out_dtype is None else out_dtype,
                                     main)
-        if b:
+        if b and nsh:
+            need = paged_attention_shared_prefix_workspace_bytes(self.pool, b, self.hq, max_ctx, nsh)
+            if need > self.ws_cap:
+                raise RuntimeError("decode workspace too small")
+            if before_decode is not None:
+                before_decode(main)
+            paged_attention_decode_shared_prefix(
+                self.pool, layer, q, self.q_dtype, self.hq, dview("tables", torch.int32), w,
+                dview("lens", torch.int32), b, max_ctx, dview("sh_seqs", torch.int32), nsh,
+                dview("sh_blocks", torch.int32), nshb * self.bs, dview("skip", torch.int32), self.scale, out,
+                KV_F32 if out_dtype is None else out_dtype, self.d_ws, need, main,
+                seq_order=dview("order", torch.int32))
+        elif b:
             need = paged_attention_workspace_bytes(self.pool, b, self.hq, max_ctx)
             if need > self.ws_cap:
                 raise RuntimeError("decode workspace too small")

@@ -63,16 +63,21 @@ def test_pool_bytes_and_workspace_sizes():
     pool = pk.kv_pool_create(16, 100, 8, 128, pk.KV_BF16, 2)
     kvb, sb = pk.kv_pool_bytes(pool)
     assert kvb == 100 * 8 * 16 * 128 * 2 and sb == 0
+    # split partials (head_dim + 4 floats per partition and query head) plus
+    # one int merge counter per (sequence, kv head), padded to 16 bytes
+    def ws(b, parts):
+        return b * 64 * parts * 132 * 4 + (b * 8 * 4 + 15) // 16 * 16
+
     # automatic policy: partitions of at most 4096 tokens ...
     assert pk.paged_attention_workspace_bytes(pool, 512, 64, 4096) == 0
-    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 8192) == 512 * 64 * 2 * 132 * 4
+    assert pk.paged_attention_workspace_bytes(pool, 512, 64, 8192) == ws(512, 2)
     # ... and more, down to 512 tokens, when there are few (sequence, kv head) units
-    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 1024) == 4 * 64 * 2 * 132 * 4
+    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 1024) == ws(4, 2)
     assert pk.paged_attention_workspace_bytes(pool, 4, 64, 512) == 0
     pk.kv_pool_set_decode_config(pool, 4096, 0, 0)
     assert pk.paged_attention_workspace_bytes(pool, 4, 64, 4096) == 0
     pk.kv_pool_set_decode_config(pool, 256, 2, 4)
-    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 513) == 4 * 64 * 3 * 132 * 4
+    assert pk.paged_attention_workspace_bytes(pool, 4, 64, 513) == ws(4, 3)
     for bad in ((8, 0, 0), (16400, 0, 0), (100, 0, 0), (0, 5, 0), (0, 1, 0), (0, 7, 0), (0, 0, 6), (0, 4, 8)):
         with pytest.raises(pk.KVError):
             pk.kv_pool_set_decode_config(pool, *bad)

@@ -54,9 +54,10 @@ def mirror_initial(tr, w, plan):
     return bm, sched, kh, vh, init_slots
 
 
-def run_trace(w, iters, check_pool_at, sample_every=1):
+def run_trace(w, iters, check_pool_at, sample_every=1, shared_prefix=False):
     plan = gqa_trace_plan(w)
-    tr = GqaTrace(w, plan)
+    tr = GqaTrace(w, plan, shared_prefix=shared_prefix)
+    used_prefix = 0
     bm, sched, kh, vh, init_slots = mirror_initial(tr, w, plan)
     assert np.array_equal(init_slots, tr.init_slots)
     bs = w.block_size
@@ -88,13 +89,20 @@ def run_trace(w, iters, check_pool_at, sample_every=1):
             assert np.array_equal(host16(tr.v), vh), f"V pool differs after iteration {it}"
         if it % sample_every == 0 and info.batch:
             B = info.batch
-            picks = sorted({0, B // 2, B - 1} | ({want["running"].index(want["admitted"][0])} if want["admitted"] else set()))
+            picks = {0, B // 2, B - 1} | ({want["running"].index(want["admitted"][0])} if want["admitted"] else set())
+            rows, _ = tr.loop.last_prefix
+            if rows is not None:  # the shared-prefix decode ran: check sharers too
+                used_prefix += 1
+                picks |= {int(rows[0]), int(rows[len(rows) // 2]), int(rows[-1])}
+            picks = sorted(picks)
             tables = np.full((len(picks), max(len(want["block_tables"][i]) for i in picks)), -1, np.int32)
             for j, i in enumerate(picks):
                 tables[j, :len(want["block_tables"][i])] = want["block_tables"][i]
             lens = np.array([want["context_lens"][i] for i in picks], np.int32)
             ref = oracle.paged_decode(kh, vh, BF16, host16(q)[picks], BF16, tables, lens, w.scale, bs)
             assert max_abs(out[picks].cpu().numpy(), ref) <= TOL[BF16], f"iteration {it}"
+    if shared_prefix:
+        assert used_prefix > 0
     return tr, cow_total
 
 
@@ -103,6 +111,15 @@ def test_gqa_trace_full_size_matches_oracle():
     tr, cow_total = run_trace(w, w.extra["iters"], check_pool_at={0, 1, 50, w.extra["iters"] - 1})
     # every sharer but the last copied the shared partly filled block
     assert cow_total >= len(tr.sharers) - 1
+
+
+def test_gqa_trace_with_shared_prefix_decode_matches_oracle():
+    """The same trace with the serving loop's shared-prefix decode: the
+    sharers' common blocks are attended once per kv head on the tensor cores
+    and merged with each sequence's own tokens; outputs (sharers sampled
+    every iteration) still match the oracle."""
+    w = WORKLOADS["gqa_trace"]
+    run_trace(w, 40, check_pool_at={39}, shared_prefix=True)
 
 
 def test_trace_with_block_aligned_prefix_needs_no_copy():

@@ -41,3 +41,28 @@ def test_metadata_layout_is_16_byte_aligned_with_prefill_fields():
         assert off % 16 == 0, name
     assert lay["cu"][1] == 3 and lay["pf_lens"][1] == 2
     assert total >= lay["pf_lens"][0] + 8
+
+
+def test_find_shared_prefix_groups_the_largest_common_leading_run():
+    from paged_kv_cache_451_b200.serving import find_shared_prefix
+    bs = 16
+    tables = np.array([
+        [7, 8, 9, 30, -1],   # sharer: prefix 7 8 9
+        [1, 2, -1, -1, -1],  # own blocks
+        [7, 8, 9, 31, 32],   # sharer
+        [7, 8, 9, 33, -1],   # sharer
+        [7, 8, 5, -1, -1],   # shares only 7 8
+    ], np.int32)
+    lens = np.array([60, 20, 70, 49, 40], np.int32)
+    rows, blocks = find_shared_prefix(tables, lens, bs, min_sharers=2)
+    assert rows.tolist() == [0, 2, 3, 4] and blocks.tolist() == [7, 8]  # the fourth diverges at block 2
+    rows, blocks = find_shared_prefix(tables[:4], lens[:4], bs, min_sharers=2)
+    assert rows.tolist() == [0, 2, 3] and blocks.tolist() == [7, 8, 9]
+    # cut to whole blocks inside every member's context: 33 tokens -> 2 blocks
+    lens2 = np.array([60, 20, 70, 33], np.int32)
+    rows, blocks = find_shared_prefix(tables[:4], lens2, bs, min_sharers=2)
+    assert blocks.tolist() == [7, 8]
+    # thresholds
+    assert find_shared_prefix(tables[:4], lens[:4], bs, min_sharers=4) == (None, None)
+    assert find_shared_prefix(tables[:4], lens[:4], bs, min_sharers=2, min_tokens=64) == (None, None)
+    assert find_shared_prefix(tables[[1]], lens[[1]], bs) == (None, None)

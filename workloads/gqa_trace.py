@@ -35,7 +35,8 @@ FIRST_ARRIVAL = 10_000
 
 
 class GqaTrace:
-    def __init__(self, w, plan, device="cuda", seed=0, decode_config=None, order_policy="batch"):
+    def __init__(self, w, plan, device="cuda", seed=0, decode_config=None, order_policy="batch",
+                 shared_prefix=False):
         import torch
 
         self.torch, self.w, self.plan, self.seed = torch, w, plan, seed
@@ -87,7 +88,7 @@ class GqaTrace:
                                head_dim=w.head_dim, block_size=bs, q_dtype=w.q_fmt, scale=w.scale,
                                max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
                                max_tokens=max_tokens, max_context=e["cap"] + e["iters"] + bs,
-                               device=device, order_policy=order_policy)
+                               device=device, order_policy=order_policy, shared_prefix=shared_prefix)
 
     def _seed(self, it, kind):
         return (self.w.seed * 1_000_003 + (it + 2) * 7919 + kind * 104_729 + self.seed) % (2 ** 62)

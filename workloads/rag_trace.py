@@ -37,7 +37,7 @@ def rag_plan(w):
 
 
 class RagTrace:
-    def __init__(self, w, plan, caching=True, device="cuda", seed=0):
+    def __init__(self, w, plan, caching=True, device="cuda", seed=0, shared_prefix=False):
         import torch
 
         self.torch, self.w, self.plan, self.seed, self.device = torch, w, plan, seed, device
@@ -66,7 +66,7 @@ class RagTrace:
                                head_dim=w.head_dim, block_size=bs, q_dtype=w.q_fmt, scale=w.scale,
                                max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
                                max_tokens=max_prompt_tokens + e["max_num_seqs"], max_context=max_ctx,
-                               device=device)
+                               device=device, shared_prefix=shared_prefix)
 
     def _seed(self, it, kind):
         return (self.w.seed * 1_000_003 + (it + 2) * 7919 + kind * 104_729 + self.seed) % (2 ** 62)
