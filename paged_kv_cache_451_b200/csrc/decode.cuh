@@ -26,7 +26,7 @@
 //   rounding residual (~16 significant bits together) and transposed into B
 //   fragments with movmatrix
 //   O^T[D x 8] += V^T[D x 16 tokens] . P^T, once for the value and once for the
-//   residual.
+//   residual (FP8 pools: P as one f16 value, one pass).
 // FP8 (E4M3) pools are decoded to f16 in registers (exact); the queries are
 // scaled by a power of two per head so they fit f16 without losing bits; the
 // K scale of each (block, head) multiplies its logits.  The V scale enters
@@ -566,13 +566,22 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
         }
       }
 
-      // P^T as B fragments: P (tokens x heads) in 16-bit value + residual
-      // halves, transposed so lane (g, c) holds tokens 2c, 2c+1 of head g
-      uint32_t h0, l0, h1, l1;
-      split2<kBf16Mma>(pr[0], pr[1], h0, l0);  // token gq, heads a, b
-      split2<kBf16Mma>(pr[2], pr[3], h1, l1);  // token gq + 8
+      // P^T as B fragments, transposed so lane (g, c) holds tokens 2c, 2c+1
+      // of head g.  16-bit caches: P as 16-bit value + rounding residual
+      // (P.V runs once per half; 16 (bf16) to 22 (f16) significant bits
+      // together), for the 2e-3 bound.  FP8 caches: P as one f16 value; its relative
+      // rounding error 2^-11 moves the output by at most 2^-11 max |v|, far
+      // inside the FP8 bound of 1e-2, and the second P.V pass is saved.
+      uint32_t h0, l0 = 0u, h1, l1 = 0u;
+      if constexpr (kFp8) {
+        h0 = pack2<false>(pr[0], pr[1]);  // token gq, heads a, b
+        h1 = pack2<false>(pr[2], pr[3]);  // token gq + 8
+      } else {
+        split2<kBf16Mma>(pr[0], pr[1], h0, l0);
+        split2<kBf16Mma>(pr[2], pr[3], h1, l1);
+      }
       const uint32_t bh0 = movmatrix_t(h0), bh1 = movmatrix_t(h1);
-      const uint32_t bl0 = movmatrix_t(l0), bl1 = movmatrix_t(l1);
+      const uint32_t bl0 = kFp8 ? 0u : movmatrix_t(l0), bl1 = kFp8 ? 0u : movmatrix_t(l1);
 
       // O^T += V^T . P^T.  The last chunk of a context zeroes the V values of
       // its tokens >= vt (stale slots may hold any bits, and 0 * NaN is NaN);
@@ -616,7 +625,6 @@ paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap km
               e4m3x4_to_f16x4(__byte_perm(lo, hi, 0x6420), a0, a2);
               e4m3x4_to_f16x4(__byte_perm(lo, hi, 0x7531), a1, a3);
               mma_16816<false>(o[2 * cp + h], a0, a1, a2, a3, bh0, bh1);
-              mma_16816<false>(o[2 * cp + h], a0, a1, a2, a3, bl0, bl1);
             }
           }
         }

@@ -252,8 +252,9 @@ def test_every_layer_decodes_its_own_pool(kv_fmt, q_fmt):
 
 @pytest.mark.parametrize("q_fmt", [BF16, F16])
 def test_fp8_queries_spanning_many_binades(q_fmt):
-    """FP8 caches take the query as a sum of E4M3 terms (exact for bf16
-    queries, and for f16 ones up to components far below the head's largest):
+    """FP8 caches take the query scaled by a power of two per head into f16
+    (exact for bf16 queries, and for f16 ones up to components far below the
+    head's largest, which leave the f16 range):
     queries whose components span 2^-24 .. 2^6 in magnitude, with a few huge
     and many tiny values per head, still match the oracle."""
     rng = np.random.default_rng(31)
