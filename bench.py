@@ -77,6 +77,47 @@ def tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def stream_rooflines(torch, stream):
+    """Two plain streams timed on this GPU as extra, context-only
+    denominators beside the official peak: a read-only stream over 4 GiB
+    (the faster of a bf16 vector-matrix product, which reads the matrix once,
+    and a float32 sum of the same bytes), as the decode only reads its K/V,
+    and a copy (1 Gi bf16 elements, counting read + write bytes, the method
+    of the measured-peak file).  Best of 10 CUDA-event-timed passes after 3
+    warm-ups; the inputs are far larger than L2."""
+    def best(fn, nbytes):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return nbytes / (min(ts) * 1e-3) / 1e9
+    with torch.cuda.stream(stream):
+        x = torch.ones(1 << 31, dtype=torch.bfloat16, device="cuda")
+        w = torch.ones(1 << 15, dtype=torch.bfloat16, device="cuda")
+        mat = x.view(1 << 15, 1 << 16)
+        gemv = best(lambda: w @ mat, x.numel() * 2)
+        x32 = x.view(torch.float32)
+        fsum = best(lambda: x32.sum(), x.numel() * 2)
+        del x, w, mat, x32
+        src = torch.ones(1 << 30, dtype=torch.bfloat16, device="cuda")
+        dst = torch.empty_like(src)
+        copy = best(lambda: dst.copy_(src), 2 * src.numel() * 2)
+        del src, dst
+    torch.cuda.empty_cache()
+    return {"read_gbs": round(max(gemv, fsum), 1), "read_gemv_gbs": round(gemv, 1), "read_sum_gbs": round(fsum, 1),
+            "copy_gbs": round(copy, 1),
+            "method": "read: bf16 vector x [32768 x 65536] matrix (torch / cuBLAS) and a float32 sum of the same "
+                      "4 GiB, the faster; copy: 1 Gi bf16 elements, read + write bytes (torch copy_); best of 10 "
+                      "CUDA-event-timed passes; context only, the official peak stays MEASURED_PEAKS.json or "
+                      "the fallback"}
+
+
 def source_hash(files):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_451_b200", "csrc")
@@ -459,6 +500,11 @@ def run_ours(args, rank, world, local_rank):
     case.destroy()
     del case
     torch.cuda.empty_cache()
+    if not args.no_extras:
+        sr = stream_rooflines(torch, stream)
+        sr["decode_frac_of_read"] = round(m["roofline"]["achieved"] / sr["read_gbs"], 4)
+        sr["decode_frac_of_copy"] = round(m["roofline"]["achieved"] / sr["copy_gbs"], 4)
+        line["stream_rooflines"] = sr
     if world == 1 and not args.no_extras and args.workload == "kv_example":
         line["per_config"] = per_config(args, torch, pk, stream, flush, clk)
     if dist:
