@@ -129,6 +129,39 @@ def test_prefill_large_logits_move_the_reference_max(fmt, d, scale):
     assert max_abs(got, ref) <= TOL[fmt]
 
 
+def test_prefill_bf16_values_beyond_the_f16_range():
+    """bf16 V values far beyond the f16 range (around 2^17, keys 130..140 of
+    the first sequence: its second 128-key tile) and far below its normal
+    range (around 2^-20, keys 300..319) in one prompt: P.V must keep bf16's
+    range and precision.  Outputs are then large, so the bound is relative to
+    the largest V; rows that never see the large values keep the plain
+    bound."""
+    rng = np.random.default_rng(41)
+    lens, q_lens, d, hq, hkv, bs = [700, 300], [700, 120], 128, 16, 2, 16
+    kh, vh, tables = make_pool(rng, BF16, d, bs, hkv, lens)
+    vf = (vh.astype(np.uint32) << 16).view(np.float32)
+    for t in range(130, 141):
+        vf[tables[0][t // bs], :, t % bs, :] *= 2.0 ** 17
+    for t in range(300, 320):
+        vf[tables[0][t // bs], :, t % bs, :] *= 2.0 ** -20
+    vh = (vf.view(np.uint32) >> 16).astype(np.uint16)  # the scalings are exact in bf16
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q = normal_bits(rng, (int(cu[-1]), hq, d), BF16)
+    pool = DevicePool(kh.shape[0], hkv, d, bs, BF16, k=[dev(kh)], v=[dev(vh)])
+    scale = 1.0 / math.sqrt(d)
+    lens_a = np.asarray(lens, np.int32)
+    out = prefill(pool, dev(q), BF16, hq, dev(cu), int(cu[-1]), max(q_lens), dev(tables), dev(lens_a), scale)
+    torch.cuda.synchronize()
+    assert pk.kv_get_device_error() == pk.KV_OK
+    ref = oracle.paged_prefill(kh, vh, BF16, q, BF16, cu, tables, lens_a, scale, bs)
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    vmax = float(np.abs(vf[np.isfinite(vf)]).max())
+    assert max_abs(got, ref) <= TOL[BF16] + 1e-4 * vmax
+    # rows whose keys never reach the large values stay within the plain bound
+    assert max_abs(got[:130], ref[:130]) <= TOL[BF16]
+
+
 def test_write_then_prefill_end_to_end():
     """paged_kv_write the new tokens of a chunk, then prefill over the pool:
     the pool equals the oracle's write mirror bit for bit and the output the
