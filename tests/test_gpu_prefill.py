@@ -162,6 +162,40 @@ def test_prefill_bf16_values_beyond_the_f16_range():
     assert max_abs(got[:130], ref[:130]) <= TOL[BF16]
 
 
+@pytest.mark.parametrize("fmt,boost", [(BF16, 6), (F16, 3)])
+def test_prefill_logit_jumps_inside_a_tile(fmt, boost):
+    """Keys 300 and 301 of a 700-token prompt (the third 128-key tile, its
+    third 16-key chunk) have K scaled by 2^boost, so the rows that see them
+    find logits tens of binades above everything before, in the middle of a
+    tile: the probabilities already computed for that tile, the sums and O
+    must all move to the new reference."""
+    rng = np.random.default_rng(43 + boost)
+    lens, q_lens, d, hq, hkv, bs = [700, 260], [700, 260], 128, 8, 2, 16
+    kh, vh, tables = make_pool(rng, fmt, d, bs, hkv, lens)
+    if fmt == BF16:
+        kf = (kh.astype(np.uint32) << 16).view(np.float32)
+    else:
+        kf = kh.view(np.float16).astype(np.float32)
+    for t in (300, 301):
+        kf[tables[0][t // bs], :, t % bs, :] *= 2.0 ** boost
+    if fmt == BF16:
+        kh = (kf.view(np.uint32) >> 16).astype(np.uint16)
+    else:
+        kh = kf.astype(np.float16).view(np.uint16)
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q = normal_bits(rng, (int(cu[-1]), hq, d), fmt)
+    pool = DevicePool(kh.shape[0], hkv, d, bs, fmt, k=[dev(kh)], v=[dev(vh)])
+    scale = 1.0 / math.sqrt(d)
+    lens_a = np.asarray(lens, np.int32)
+    out = prefill(pool, dev(q), fmt, hq, dev(cu), int(cu[-1]), max(q_lens), dev(tables), dev(lens_a), scale)
+    torch.cuda.synchronize()
+    assert pk.kv_get_device_error() == pk.KV_OK
+    ref = oracle.paged_prefill(kh, vh, fmt, q, fmt, cu, tables, lens_a, scale, bs)
+    got = out.cpu().numpy()
+    assert not np.isnan(got).any()
+    assert max_abs(got, ref) <= TOL[fmt]
+
+
 def test_write_then_prefill_end_to_end():
     """paged_kv_write the new tokens of a chunk, then prefill over the pool:
     the pool equals the oracle's write mirror bit for bit and the output the
