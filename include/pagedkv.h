@@ -108,12 +108,14 @@ int kv_pool_bind(kv_pool* pool, int layer, void* k_base, void* v_base, float* k_
  * merged by a log-sum-exp reduce (see paged_attention_decode).  0 chooses
  * automatically: partitions of at most 4096 tokens; if batch * kv_heads is
  * under three waves of resident CTAs, enough partitions (of at least 512
- * tokens) for four waves.  A context that fits one partition is written
- * directly and skips the reduce.  stages: shared-memory pipeline
+ * tokens) for four waves, raised (up to twice) until the last wave of
+ * equal partitions is at least 85% full.  A context that fits one partition
+ * is written directly and skips the reduce.  stages: shared-memory pipeline
  * depth per warp, 0 for automatic, else 2, 3, 4, 6 or 8; warps: warps per
  * CTA, 0 for automatic, else 4 or 8.  Automatic: 4 warps x 3 stages for
- * 8 KB and 4 KB stages (16-bit or FP8 with head_dim 128, 16-bit with 64),
- * 4 x 6 for 2 KB stages.  A shape whose shared memory exceeds 227 KB per CTA is rejected
+ * 8 KB and 4 KB stages (16-bit or FP8 with head_dim 128, 16-bit with 64;
+ * 2 stages for 8 KB stages with GQA groups of 4 or more), 4 x 6 for 2 KB
+ * stages.  A shape whose shared memory exceeds 227 KB per CTA is rejected
  * with KV_ERR_ARG.  Host only. */
 int kv_pool_set_decode_config(kv_pool* pool, int partition_tokens, int stages, int warps);
 
