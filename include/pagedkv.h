@@ -189,8 +189,13 @@ size_t paged_attention_workspace_bytes(const kv_pool* pool, int batch, int num_q
  *                 may be NULL when that is 0.  Contexts longer than one
  *                 partition are split: each partition writes its unnormalised
  *                 output and its running maxima and sum there
- *                 (head_dim + 4 floats per (sequence, head, partition)), and
- *                 a second kernel merges them by log-sum-exp.
+ *                 (head_dim + 4 floats per (sequence, head, partition)),
+ *                 followed by one int merge counter per (sequence, kv head),
+ *                 and the partials are merged by log-sum-exp: by the last
+ *                 partition CTA of each (sequence, kv head) to finish when a
+ *                 16-bit pool's contexts split into at most 4 partitions,
+ *                 else by a second kernel.  The call zeroes the counters on
+ *                 the stream itself; the workspace needs no initialisation.
  *   seq_order     NULL, or device int32 [batch]: a permutation of 0..batch-1
  *                 giving the order in which sequences are scheduled onto the
  *                 GPU; outputs are unaffected.  Longest context first keeps
