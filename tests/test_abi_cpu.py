@@ -7,6 +7,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import paged_kv_cache_451_b200 as pk
 
@@ -84,6 +85,24 @@ def test_pool_bytes_and_workspace_sizes():
     pk.kv_pool_destroy(pool)
     fp8 = pk.kv_pool_create(32, 10, 4, 64, pk.KV_FP8_E4M3, 1)
     assert pk.kv_pool_bytes(fp8) == (10 * 4 * 32 * 64, 10 * 4 * 4)
+    pk.kv_pool_destroy(fp8)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="on a GPU the policy sees the device's real occupancy")
+def test_partition_count_fills_the_last_wave():
+    """Without a device the policy counts one resident CTA per SM on 148
+    SMs.  2 x 16K-token FP8 contexts with 32 kv heads are 64 units: four
+    waves need 10 partitions (640 CTAs, 4.3 waves, the last one 32% full);
+    the count is raised to 16 (1024 CTAs, 6.9 waves, the last 92% full) of
+    1024 tokens each.  A forced partition length is kept as it is."""
+    fp8 = pk.kv_pool_create(16, 4096, 32, 128, pk.KV_FP8_E4M3, 1)
+    per = 132 * 4  # head_dim + 4 floats per (sequence, head, partition)
+    counters = (2 * 32 * 4 + 15) // 16 * 16
+    assert pk.paged_attention_workspace_bytes(fp8, 2, 32, 16384) == 2 * 32 * 16 * per + counters
+    # 8 sequences: 256 units, 4 partitions already fill 92% of their last wave
+    assert pk.paged_attention_workspace_bytes(fp8, 8, 32, 16384) == 8 * 32 * 4 * per + (8 * 32 * 4 + 15) // 16 * 16
+    pk.kv_pool_set_decode_config(fp8, 512, 0, 0)
+    assert pk.paged_attention_workspace_bytes(fp8, 2, 32, 16384) == 2 * 32 * 32 * per + counters
     pk.kv_pool_destroy(fp8)
 
 
