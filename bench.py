@@ -715,7 +715,7 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
     cur = {"k": 0}
 
     def inputs(T, B):
-        k, main = cur["k"], torch.cuda.current_stream()
+        k, main = cur["k"], stream  # the loop's stream: the current one
         views = []
         with torch.cuda.stream(up):
             if kern_done[k] is not None:  # the kernels that read this set two iterations ago
@@ -734,8 +734,8 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
 
     def one(it):
         k = cur["k"] = it % 2
-        main = torch.cuda.current_stream()
-        fin, arr, pl, *_r = tr.iteration(it, out_dtype=w.q_fmt, inputs=inputs, out=outs[k])
+        main = stream
+        fin, arr, pl, *_r = tr.iteration(it, out_dtype=w.q_fmt, inputs=inputs, out=outs[k], stream=stream)
         ev = torch.cuda.Event()
         ev.record(main)
         kern_done[k] = ev

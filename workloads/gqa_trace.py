@@ -79,9 +79,13 @@ class GqaTrace:
         d_slots = torch.from_numpy(self.init_slots).to(device)
         paged_kv_write(self.pool, 0, self.init_k, self.init_v, w.kv_fmt, d_slots, T)
 
-        self.remaining = {s: int(plan["remaining"][s]) for s in range(w.batch)}
+        # output tokens still to generate, indexed by sequence id (arrivals
+        # take ids from FIRST_ARRIVAL on), and the running set's ids
+        n_arr = sum(len(a) for a in plan["arrivals"])
+        self.remaining = np.zeros(FIRST_ARRIVAL + n_arr + 1, np.int64)
+        self.remaining[:w.batch] = np.asarray(plan["remaining"][:w.batch], np.int64)
         self.next_id = FIRST_ARRIVAL
-        self.running = list(range(w.batch))
+        self.running = np.arange(w.batch, dtype=np.int64)
         self.max_blocks = int(math.ceil((e["cap"] + e["iters"] + 2 * bs) / bs))
         max_tokens = 256 + 16 * e["prompt_hi"]
         self.loop = DecodeLoop(self.pool, self.sched, num_q_heads=w.num_q_heads, kv_heads=w.kv_heads,
@@ -100,7 +104,7 @@ class GqaTrace:
         return table[t // bs].astype(np.int64) * bs + t % bs
 
     def finished(self):
-        return [s for s in self.running if self.remaining[s] <= 0]
+        return self.running[self.remaining[self.running] <= 0].tolist()
 
     def arrivals(self, it):
         """Queue this iteration's arrivals; returns [(id, prompt_len)]."""
@@ -114,14 +118,15 @@ class GqaTrace:
         return out
 
     def iteration(self, it, out_dtype=None, out=None, before_launch=None, after_launch=None,
-                  before_decode=None, inputs=None):
+                  before_decode=None, inputs=None, stream=None):
         """One trace iteration: returns (finished, arrivals, plan, q, k_new,
         v_new, out) with device tensors of this step's inputs and output.
         before_launch / after_launch are called right around the library
         calls (after the inputs are drawn), e.g. to record timing events.
         ``inputs(T, B)``, if given, supplies (q, k_new, v_new) instead of the
         seeded draws (e.g. views of buffers it uploads from host memory); it
-        is called after before_launch."""
+        is called after before_launch.  ``stream``: the stream the kernels run
+        on (default: the current one)."""
         torch, w = self.torch, self.w
         import time
         fin = self.finished()
@@ -130,7 +135,7 @@ class GqaTrace:
         plan = self.loop.schedule(fin)
         self.last_schedule_s = time.perf_counter() - t0
         info = plan["info"]
-        self.running = [int(x) for x in plan["running"]]
+        self.running = np.asarray(plan["running"], np.int64)
         T, B = info.num_tokens, info.batch
         if inputs is None:
             k_new = self.draw((max(T, 1), w.kv_heads, w.head_dim), w.kv_fmt, self.device, self._seed(it, 0))
@@ -143,11 +148,11 @@ class GqaTrace:
             before_launch()
         if inputs is not None:
             q, k_new, v_new = inputs(max(T, 1), max(B, 1))
-        self.loop.launch(plan, k_new, v_new, q, out, out_dtype=out_dtype, before_decode=before_decode)
+        self.loop.launch(plan, k_new, v_new, q, out, out_dtype=out_dtype, before_decode=before_decode,
+                         stream=stream)
         if after_launch is not None:
             after_launch()
-        for s in self.running:
-            self.remaining[s] -= 1
+        self.remaining[self.running] -= 1
         return fin, arr, plan, q, k_new, v_new, out
 
     def free_blocks(self):
