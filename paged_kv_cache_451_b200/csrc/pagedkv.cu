@@ -169,7 +169,11 @@ int decode_slots(const kv_pool* pool, int group) {
 // partitions for 8 x 16K-token FP8 contexts (256 units); a 4K-token window
 // over 8 x 16K-token bf16 contexts runs the same with 0.5K to 1.4K-token
 // partitions.
-constexpr int kFusedMergeMaxParts = 4;  // measured: GQA trace (3) +3%, FP8 16K contexts (10, 32) -1%, -6%
+// The decode merges its own split partials up to this many partitions per
+// context (measured in-kernel against the separate reduce: GQA trace, 3
+// partitions, +3%; FP8 16K contexts, 16 and 32, -3% and -9%; a 4K-token
+// window, 8, -3%).
+constexpr int kFusedMergeMaxParts = 4;
 constexpr int kWavesKeep = 3;
 constexpr int kWavesSplit = 4;
 constexpr int kAutoPartition = 4096;
