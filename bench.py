@@ -690,62 +690,64 @@ def trace_measure(args, rank, world, local_rank, dist, clk, flush, stream, min_s
 
 def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, dist, world, shared_prefix):
     """The trace end to end from host buffers, run back to back as a serving
-    loop runs it (no device-side gate): each iteration uploads its queries
-    and new K/V rows from pinned host memory on an upload stream into one of
-    two device buffer sets (so the upload overlaps the previous iteration's
-    kernels), and its output is read back on a read-back stream (overlapping
-    the next iteration); the K iterations are timed as one region, host
-    scheduling included.  Bytes per step are the device-timed run's."""
+    loop runs it (no device-side gate): each iteration takes the library's
+    serving step (kv_serve_schedule: scheduler step, metadata packed into a
+    pinned buffer and uploaded; kv_serve_launch: copy-on-write, cache write,
+    decode), uploads its queries and new K/V rows from one pinned host
+    staging buffer with one copy on an upload stream into one of two device
+    buffer sets (so the upload overlaps the previous iteration's kernels),
+    and its output is read back on a read-back stream (overlapping the next
+    iteration); the K iterations are timed as one region, host scheduling
+    included.  Bytes per step are the device-timed run's."""
     import torch
     from workloads.gqa_trace import GqaTrace
     e = w.extra
     hq, hkv, d = w.num_q_heads, w.kv_heads, w.head_dim
+    native = not shared_prefix  # the library's serving step has no shared-prefix decode
     tr = GqaTrace(w, plan, seed=rank, decode_config=(args.partition, args.stages, args.warps),
-                  order_policy=args.order or "batch", shared_prefix=shared_prefix)
+                  order_policy=args.order or "batch", shared_prefix=shared_prefix, native=native)
     max_b, max_t = e["max_num_seqs"], tr.loop.max_tokens
     g = torch.Generator().manual_seed(w.seed * 31 + rank)
-    host = {n: torch.randn(m, generator=g).to(torch.bfloat16).view(torch.int16).pin_memory()
-            for n, m in (("q", max_b * hq * d), ("k", max_t * hkv * d), ("v", max_t * hkv * d))}
-    devb = [{n: torch.empty_like(t, device="cuda") for n, t in host.items()} for _ in range(2)]
+    # one staging buffer per step: q rows, then new K rows, then new V rows
+    n_max = (max_b * hq + 2 * max_t * hkv) * d
+    host = torch.randn(n_max, generator=g).to(torch.bfloat16).view(torch.int16).pin_memory()
+    devb = [torch.empty_like(host, device="cuda") for _ in range(2)]
     outs = [torch.empty((max_b, hq, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     hout = torch.empty(max_b * hq * d, dtype=torch.bfloat16).pin_memory()
     up, rb = torch.cuda.Stream(), torch.cuda.Stream()
-    kern_done, rb_done = [None, None], [None, None]  # kernels / read-back of buffer set k finished
+    up_done = [torch.cuda.Event(), torch.cuda.Event()]    # inputs of buffer set k uploaded
+    kern_done = [torch.cuda.Event(), torch.cuda.Event()]  # kernels reading buffer set k finished
+    rb_done = [torch.cuda.Event(), torch.cuda.Event()]    # read-back of output k finished
+    used = [False, False]
     moved = {"h2d": 0, "d2h": 0}
     cur = {"k": 0}
 
     def inputs(T, B):
         k, main = cur["k"], stream  # the loop's stream: the current one
-        views = []
+        nq, nk = B * hq * d, T * hkv * d
+        if used[k]:  # the kernels that read this set two iterations ago
+            up.wait_event(kern_done[k])
         with torch.cuda.stream(up):
-            if kern_done[k] is not None:  # the kernels that read this set two iterations ago
-                up.wait_event(kern_done[k])
-            for n, rows, heads in (("q", B, hq), ("k", T, hkv), ("v", T, hkv)):
-                m = rows * heads * d
-                devb[k][n][:m].copy_(host[n][:m], non_blocking=True)
-                moved["h2d"] += 2 * m
-                views.append(devb[k][n][:m].view(rows, heads, d))
-            ev = torch.cuda.Event()
-            ev.record(up)
-        main.wait_event(ev)
-        if rb_done[k] is not None:  # this set's output was read back
+            devb[k][:nq + 2 * nk].copy_(host[:nq + 2 * nk], non_blocking=True)
+        up_done[k].record(up)
+        moved["h2d"] += 2 * (nq + 2 * nk)
+        main.wait_event(up_done[k])
+        if used[k]:  # this set's output was read back
             main.wait_event(rb_done[k])
-        return views[0], views[1], views[2]
+        buf = devb[k]
+        return (buf[:nq].view(B, hq, d), buf[nq:nq + nk].view(T, hkv, d),
+                buf[nq + nk:nq + 2 * nk].view(T, hkv, d))
 
     def one(it):
         k = cur["k"] = it % 2
-        main = stream
         fin, arr, pl, *_r = tr.iteration(it, out_dtype=w.q_fmt, inputs=inputs, out=outs[k], stream=stream)
-        ev = torch.cuda.Event()
-        ev.record(main)
-        kern_done[k] = ev
+        kern_done[k].record(stream)
         n = max(pl["info"].batch, 1) * hq * d
+        rb.wait_event(kern_done[k])
         with torch.cuda.stream(rb):
-            rb.wait_event(ev)
             hout[:n].copy_(outs[k].view(-1)[:n], non_blocking=True)
-            done = torch.cuda.Event()
-            done.record(rb)
-            rb_done[k] = done
+        rb_done[k].record(rb)
+        used[k] = True
         moved["d2h"] += 2 * n
 
     for it in range(W):
@@ -762,15 +764,20 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
     torch.cuda.synchronize()
     span = (t0, time.perf_counter())
     ms = max_over_ranks(a.elapsed_time(b), dist, "cuda") / K
+    if native:
+        tr.loop.close()
     del tr
     return {"value": round(world * (uniq_b + other_b) / steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 5), "steps": K, "h2d_bytes_per_step": int(moved["h2d"] / K),
             "d2h_bytes_per_step": int(moved["d2h"] / K),
-            "mode": "serving loop from host memory, pipelined: per iteration the native scheduler step, the "
-                    "packed metadata upload, the upload of the step's q and new K/V rows from pinned host "
-                    "memory on an upload stream (two device buffer sets), the kernels, and the output read "
-                    "back on a read-back stream; K iterations timed as one region (host scheduling and "
-                    "Python sequencing included)",
+            "mode": "serving loop from host memory, pipelined: per iteration the library's serving step "
+                    + ("(kv_serve_schedule: native scheduler step, metadata packed in a pinned buffer and "
+                       "uploaded; kv_serve_launch: copy-on-write, cache write, decode), " if native else
+                       "(Python sequencing with the shared-prefix decode), ")
+                    + "one upload of the step's q and new K/V rows from a pinned staging buffer on an upload "
+                    "stream (two device buffer sets), and the output read back on a read-back stream; K "
+                    "iterations timed as one region (host scheduling included)",
+            "serving_step": "native" if native else "python",
             "clocks": clk.summary(*span)}
 
 

@@ -68,6 +68,7 @@ typedef enum { KV_PREEMPT_NONE = 0, KV_PREEMPT_SWAP = 1, KV_PREEMPT_RECOMPUTE = 
 typedef struct kv_pool kv_pool;
 typedef struct kv_alloc kv_alloc;
 typedef struct kv_sched kv_sched;
+typedef struct kv_serve kv_serve;
 
 /* Message for the calling thread's most recent failure ("" if none). */
 const char* kv_last_error(void);
@@ -568,6 +569,113 @@ int kv_sched_admitted_cached(const kv_sched* s, int32_t* cached_tokens);
 int kv_sched_stats(const kv_sched* s, int* running, int* waiting, int* used_blocks,
                    int* total_blocks);
 int kv_sched_destroy(kv_sched* s);
+
+/* ---------------------------------------------------------- serving step */
+
+/* One continuous-batching iteration sequenced by the library ([CB]: free the
+ * finished, admit first come first served, append one slot per running
+ * sequence, then the step's kernels), so a serving loop makes two calls per
+ * step instead of one per array and kernel. */
+
+/* Order in which the decode places the batch's sequences on the GPU (the
+ * seq_order argument of paged_attention_decode; outputs do not depend on it).
+ * BATCH: batch order (no permutation).  LONGEST: decreasing context length,
+ * ties in batch order.  LONG_FIRST: the sequences longer than the batch mean,
+ * longest first, then the rest in batch order. */
+typedef enum { KV_ORDER_BATCH = 0, KV_ORDER_LONGEST = 1, KV_ORDER_LONG_FIRST = 2 } kv_order_policy;
+
+/* Where a packed step's arrays sit in its buffer: byte offsets, each a
+ * multiple of 16, or -1 for an array the step does not have. */
+typedef struct {
+  kv_step_info info;
+  int table_width;      /* row stride of block_tables: max(info.max_blocks, 1) */
+  int max_context_len;  /* longest context after the append (0: empty batch) */
+  int num_swap_out;     /* swap-out pairs (kv_sched_swap_outputs) */
+  int num_swap_in;      /* swap-in pairs */
+  int prefill_tokens;   /* admitted prompts' uncached tokens, cu_seqlens[num_admitted] */
+  int max_prefill_len;  /* most uncached tokens of one admitted prompt */
+  int64_t bytes;        /* bytes of the buffer the step uses */
+  int64_t slot_mapping;          /* int64[num_tokens] */
+  int64_t block_tables;          /* int32[batch][table_width], padded with -1 */
+  int64_t context_lens;          /* int32[batch] */
+  int64_t seq_order;             /* int32[batch]; -1 under KV_ORDER_BATCH */
+  int64_t cow_pairs;             /* int32[num_cow][2] */
+  int64_t swap_out_pairs;        /* int32[num_swap_out][2] */
+  int64_t swap_in_pairs;         /* int32[num_swap_in][2] */
+  int64_t cu_seqlens;            /* int32[num_admitted + 1]: prefix sums of uncached prompt tokens */
+  int64_t prefill_context_lens;  /* int32[num_admitted]: prompt lengths (context minus the appended token) */
+} kv_step_layout;
+
+/* Bytes a packed step can need with at most max_batch running sequences,
+ * max_tokens written slots, tables of at most max_table_width blocks and
+ * max_swap_pairs swap pairs each way (0 on a negative argument). */
+size_t kv_step_packed_bytes(int max_batch, int max_tokens, int max_table_width, int max_swap_pairs);
+
+/* kv_sched_step, then the step's device metadata written into buf (host
+ * memory, 16-byte aligned, buf_bytes long) at the offsets returned in
+ * *layout: the same arrays kv_sched_outputs / kv_sched_swap_outputs give,
+ * the block tables at the step's own width, the scheduling order of
+ * order_policy, and for the admitted prompts (the last num_admitted rows of
+ * the running set) the cu_seqlens / context lengths paged_attention_prefill
+ * takes.  running_ids (may be NULL) receives int64[batch].  Errors of
+ * kv_sched_step are returned as they are (nothing changes for KV_ERR_STATE);
+ * KV_ERR_ARG for a step whose tables are wider than max_table_width or whose
+ * arrays do not fit buf: the scheduler step has then been taken and its
+ * outputs stay readable with kv_sched_outputs. */
+int kv_sched_step_packed(kv_sched* s, const int64_t* finished_ids, int n_finished, int order_policy,
+                         int max_table_width, void* buf, size_t buf_bytes, int64_t* running_ids,
+                         kv_step_layout* layout);
+
+/* Decode scratch a serving loop needs for every batch of 1..max_batch
+ * sequences with contexts up to max_context_len (the split policy divides
+ * more finely when fewer sequences run). */
+size_t kv_serve_workspace_bytes(const kv_pool* pool, int num_q_heads, int max_batch, int max_context_len);
+
+/* A serving loop over pool and sched (both must outlive it).  The caller owns
+ * every buffer: two pinned host and two device metadata buffers of
+ * meta_bytes each (>= kv_step_packed_bytes(max_batch, max_tokens,
+ * max_table_width, swap_slots), 16-byte aligned), the decode workspace
+ * (>= kv_serve_workspace_bytes), and for swap preemption the mapped pinned
+ * host swap space of swap_slots slots (kv_swap_out).  Consecutive steps
+ * alternate between the two buffer pairs; the loop creates four CUDA events
+ * on the current device, which must stay current for its calls.
+ * num_q_heads, q_dtype (also the type of the new K/V rows) and scale are
+ * those of the decode.  KV_ERR_ARG on bad arguments; KV_ERR_CUDA if an event
+ * cannot be created. */
+int kv_serve_create(kv_pool* pool, kv_sched* sched, int num_q_heads, kv_dtype q_dtype, float scale,
+                    int order_policy, int max_batch, int max_tokens, int max_table_width, void* host_swap,
+                    int swap_slots, void* const host_meta[2], void* const dev_meta[2], size_t meta_bytes,
+                    void* workspace, size_t workspace_bytes, kv_serve** out);
+
+/* The step's host half: waits (host) until the other pinned buffer's last
+ * upload is done, runs kv_sched_step_packed into it, and enqueues on
+ * upload_stream, after the kernels that last read the matching device buffer,
+ * one copy of the packed bytes to that device buffer.  running_ids
+ * (int64[max_batch], written only for a batch that fits) and layout may be
+ * NULL.  KV_ERR_STATE if the previous step was never launched
+ * (checked first: nothing changes); otherwise as kv_sched_step_packed, plus
+ * KV_ERR_ARG when the step exceeds max_batch / max_tokens and KV_ERR_STATE
+ * when it swaps without swap space (the scheduler step is then taken). */
+int kv_serve_schedule(kv_serve* s, const int64_t* finished_ids, int n_finished, kv_stream_t upload_stream,
+                      int64_t* running_ids, kv_step_layout* layout);
+
+/* The step's kernels for one layer, on stream, after the step's metadata
+ * upload: on the first call of a step kv_swap_out, kv_swap_in and block_copy
+ * for all layers; then paged_kv_write of the step's num_tokens new rows
+ * (k_new / v_new [num_tokens][kv_heads][head_dim] of q_dtype, FP8 pools'
+ * inverse scales as in paged_kv_write), paged_attention_prefill of the
+ * admitted prompts' uncached tokens when prefill_q / prefill_out are given
+ * ([prefill_tokens][num_q_heads][head_dim], rows prompt by prompt), and
+ * paged_attention_decode of the running set (q, out [batch][num_q_heads]
+ * [head_dim]) in the loop's scheduling order.  Call once per layer after
+ * each kv_serve_schedule.  KV_ERR_STATE with no step scheduled; otherwise the
+ * first error of the entry points above (later ones are not enqueued). */
+int kv_serve_launch(kv_serve* s, int layer, const void* q, const void* k_new, const void* v_new,
+                    const float* k_inv_scale, const float* v_inv_scale, void* out, kv_dtype out_dtype,
+                    const void* prefill_q, void* prefill_out, kv_stream_t stream);
+
+/* Waits for the loop's uploads and kernels (host), then frees it. */
+int kv_serve_destroy(kv_serve* s);
 
 #ifdef __cplusplus
 }

@@ -16,6 +16,7 @@ from . import build as _build
 
 KV_F16, KV_BF16, KV_FP8_E4M3, KV_F32 = 0, 1, 2, 3
 KV_PREEMPT_NONE, KV_PREEMPT_SWAP, KV_PREEMPT_RECOMPUTE = 0, 1, 2
+KV_ORDER_BATCH, KV_ORDER_LONGEST, KV_ORDER_LONG_FIRST = 0, 1, 2
 KV_OK, KV_ERR_ARG, KV_ERR_OOM, KV_ERR_STATE, KV_ERR_BOUNDS, KV_ERR_CUDA, KV_ERR_TIMEOUT = (
     0, -1, -2, -3, -4, -5, -6)
 ERROR_NAMES = {0: "KV_OK", -1: "KV_ERR_ARG", -2: "KV_ERR_OOM", -3: "KV_ERR_STATE",
@@ -52,6 +53,15 @@ P = ctypes.POINTER
 class kv_step_info(ctypes.Structure):
     _fields_ = [("batch", c_int), ("num_tokens", c_int), ("num_cow", c_int),
                 ("num_admitted", c_int), ("max_blocks", c_int)]
+
+
+class kv_step_layout(ctypes.Structure):
+    _fields_ = [("info", kv_step_info), ("table_width", c_int), ("max_context_len", c_int),
+                ("num_swap_out", c_int), ("num_swap_in", c_int), ("prefill_tokens", c_int),
+                ("max_prefill_len", c_int), ("bytes", c_int64), ("slot_mapping", c_int64),
+                ("block_tables", c_int64), ("context_lens", c_int64), ("seq_order", c_int64),
+                ("cow_pairs", c_int64), ("swap_out_pairs", c_int64), ("swap_in_pairs", c_int64),
+                ("cu_seqlens", c_int64), ("prefill_context_lens", c_int64)]
 
 
 _SIGS = {
@@ -122,6 +132,16 @@ _SIGS = {
                                  c_void_p, c_void_p]),
     "kv_sched_stats": (c_int, [c_void_p, P(c_int), P(c_int), P(c_int), P(c_int)]),
     "kv_sched_destroy": (c_int, [c_void_p]),
+    "kv_step_packed_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "kv_sched_step_packed": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p,
+                                     P(kv_step_layout)]),
+    "kv_serve_workspace_bytes": (c_size_t, [c_void_p, c_int, c_int, c_int]),
+    "kv_serve_create": (c_int, [c_void_p, c_void_p, c_int, c_int, c_float, c_int, c_int, c_int, c_int, c_void_p,
+                                c_int, P(c_void_p), P(c_void_p), c_size_t, c_void_p, c_size_t, P(c_void_p)]),
+    "kv_serve_schedule": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, P(kv_step_layout)]),
+    "kv_serve_launch": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                c_int, c_void_p, c_void_p, c_void_p]),
+    "kv_serve_destroy": (c_int, [c_void_p]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -492,3 +512,59 @@ def kv_sched_stats(s):
 
 def kv_sched_destroy(s):
     _check(_lib.kv_sched_destroy(s))
+
+
+# ------------------------------------------------------------ serving step
+
+def kv_step_packed_bytes(max_batch, max_tokens, max_table_width, max_swap_pairs=0) -> int:
+    return int(_lib.kv_step_packed_bytes(max_batch, max_tokens, max_table_width, max_swap_pairs))
+
+
+def kv_sched_step_packed(s, finished_ids, order_policy, max_table_width, buf, buf_bytes, running_ids=None):
+    """Scheduler step packed into ``buf`` (host, 16-byte aligned); returns
+    the kv_step_layout."""
+    import numpy as np
+    fin = np.ascontiguousarray(finished_ids, np.int64)
+    lay = kv_step_layout()
+    _check(_lib.kv_sched_step_packed(s, _ptr(fin) if fin.size else None, int(fin.size), order_policy,
+                                     max_table_width, _ptr(buf), buf_bytes, _ptr(running_ids),
+                                     ctypes.byref(lay)))
+    return lay
+
+
+def kv_serve_workspace_bytes(pool, num_q_heads, max_batch, max_context_len) -> int:
+    return int(_lib.kv_serve_workspace_bytes(pool, num_q_heads, max_batch, max_context_len))
+
+
+def kv_serve_create(pool, sched, num_q_heads, q_dtype, scale, order_policy, max_batch, max_tokens,
+                    max_table_width, host_swap, swap_slots, host_meta, dev_meta, meta_bytes, workspace,
+                    workspace_bytes):
+    h = c_void_p()
+    hm = (c_void_p * 2)(*[_ptr(x) for x in host_meta])
+    dm = (c_void_p * 2)(*[_ptr(x) for x in dev_meta])
+    _check(_lib.kv_serve_create(pool, sched, num_q_heads, q_dtype, float(scale), order_policy, max_batch,
+                                max_tokens, max_table_width, _ptr(host_swap), swap_slots, hm, dm, meta_bytes,
+                                _ptr(workspace), workspace_bytes, ctypes.byref(h)))
+    return h
+
+
+def kv_serve_schedule(sv, finished_ids, upload_stream=None, running_ids=None, layout=None):
+    """Returns the step's kv_step_layout (``layout``, if given, is filled and
+    returned)."""
+    import numpy as np
+    fin = np.ascontiguousarray(finished_ids, np.int64)
+    lay = kv_step_layout() if layout is None else layout
+    _check(_lib.kv_serve_schedule(sv, _ptr(fin) if fin.size else None, int(fin.size), _stream(upload_stream),
+                                  _ptr(running_ids), ctypes.byref(lay)))
+    return lay
+
+
+def kv_serve_launch(sv, layer, q, k_new, v_new, out, out_dtype, k_inv_scale=None, v_inv_scale=None,
+                    prefill_q=None, prefill_out=None, stream=None):
+    _check(_lib.kv_serve_launch(sv, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_inv_scale),
+                                _ptr(v_inv_scale), _ptr(out), out_dtype, _ptr(prefill_q), _ptr(prefill_out),
+                                _stream(stream)))
+
+
+def kv_serve_destroy(sv):
+    _check(_lib.kv_serve_destroy(sv))

@@ -12,7 +12,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpagedkv.so")
 SOURCES = [os.path.join(CSRC, "pagedkv.cu"), os.path.join(CSRC, "prefill.cu"),
-           os.path.join(CSRC, "alloc.cpp")]
+           os.path.join(CSRC, "alloc.cpp"), os.path.join(CSRC, "serve.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [
     os.path.join(ROOT, "include", "pagedkv.h")]
 

@@ -579,7 +579,8 @@ struct kv_sched {
   std::vector<int64_t> running;
   // outputs of the last step
   std::vector<int64_t> out_running;
-  std::vector<std::vector<int32_t>> out_tables;
+  std::vector<int32_t> out_table_flat;  // the running sequences' tables, back to back
+  std::vector<int64_t> out_table_off{0};  // row i is [off[i], off[i + 1]) of out_table_flat
   std::vector<int32_t> out_lens;
   std::vector<int64_t> out_slots;
   std::vector<int32_t> out_cow;
@@ -640,7 +641,8 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   kv_alloc* a = s->a;
   // validate before changing anything
   std::unordered_set<int64_t> fin;
-  std::unordered_set<int64_t> run(s->running.begin(), s->running.end());
+  std::unordered_set<int64_t> run;
+  if (n_finished > 0) run.insert(s->running.begin(), s->running.end());
   for (int i = 0; i < n_finished; ++i) {
     if (!run.count(finished_ids[i]))
       return fail(KV_ERR_STATE, "finished sequence %lld is not running", (long long)finished_ids[i]);
@@ -648,7 +650,8 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
       return fail(KV_ERR_STATE, "sequence %lld finished twice", (long long)finished_ids[i]);
   }
   s->out_running.clear();
-  s->out_tables.clear();
+  s->out_table_flat.clear();
+  s->out_table_off.assign(1, 0);
   s->out_lens.clear();
   s->out_slots.clear();
   s->out_cow.clear();
@@ -760,7 +763,8 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   }
   s->out_slots = prompt_slots;
   int max_blocks = 0;
-  std::unordered_set<int64_t> admitted(s->out_admitted.begin(), s->out_admitted.end());
+  std::unordered_set<int64_t> admitted;
+  if (s->window > 0) admitted.insert(s->out_admitted.begin(), s->out_admitted.end());
   for (int64_t r : s->running) {
     SeqState& st = a->seqs[r];
     int64_t slot;
@@ -778,7 +782,8 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
       kv_alloc_release_before(a, r, st.tokens - s->window, nullptr);
     }
     s->out_running.push_back(r);
-    s->out_tables.push_back(st.blocks);
+    s->out_table_flat.insert(s->out_table_flat.end(), st.blocks.begin(), st.blocks.end());
+    s->out_table_off.push_back((int64_t)s->out_table_flat.size());
     s->out_lens.push_back((int32_t)st.tokens);
     if ((int)st.blocks.size() > max_blocks) max_blocks = (int)st.blocks.size();
   }
@@ -795,13 +800,16 @@ int kv_sched_outputs(const kv_sched* s, int64_t* running_ids, int32_t* block_tab
                      int32_t* cow_pairs, int64_t* admitted_ids) {
   if (!s) return fail(KV_ERR_ARG, "NULL scheduler");
   if (block_tables) {
-    for (const auto& t : s->out_tables)
-      if ((int)t.size() > table_width)
-        return fail(KV_ERR_ARG, "table_width %d < longest table %zu", table_width, t.size());
-    for (size_t i = 0; i < s->out_tables.size(); ++i) {
+    const size_t n = s->out_table_off.size() - 1;
+    for (size_t i = 0; i < n; ++i)
+      if (s->out_table_off[i + 1] - s->out_table_off[i] > table_width)
+        return fail(KV_ERR_ARG, "table_width %d < longest table %lld", table_width,
+                    (long long)(s->out_table_off[i + 1] - s->out_table_off[i]));
+    for (size_t i = 0; i < n; ++i) {
       int32_t* row = block_tables + i * (size_t)table_width;
-      const auto& t = s->out_tables[i];
-      for (int j = 0; j < table_width; ++j) row[j] = j < (int)t.size() ? t[j] : -1;
+      const int len = (int)(s->out_table_off[i + 1] - s->out_table_off[i]);
+      if (len) std::memcpy(row, s->out_table_flat.data() + s->out_table_off[i], sizeof(int32_t) * len);
+      for (int j = len; j < table_width; ++j) row[j] = -1;
     }
   }
   if (running_ids) std::memcpy(running_ids, s->out_running.data(), sizeof(int64_t) * s->out_running.size());

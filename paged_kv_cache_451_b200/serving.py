@@ -25,10 +25,14 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import (KV_F32, block_copy, kv_sched_outputs, kv_sched_step, kv_sched_swap_outputs, kv_swap_in,
+from . import (KV_F32, KV_ORDER_BATCH, KV_ORDER_LONG_FIRST, KV_ORDER_LONGEST, block_copy, kv_sched_outputs,
+               kv_sched_step, kv_sched_swap_outputs, kv_serve_create, kv_serve_destroy, kv_serve_launch,
+               kv_serve_schedule, kv_serve_workspace_bytes, kv_step_layout, kv_step_packed_bytes, kv_swap_in,
                kv_swap_out, paged_attention_decode, paged_attention_decode_shared_prefix,
                paged_attention_prefill, paged_attention_shared_prefix_workspace_bytes,
                paged_attention_workspace_bytes, paged_kv_write)
+
+ORDER_POLICIES = {"batch": KV_ORDER_BATCH, "longest": KV_ORDER_LONGEST, "long_first": KV_ORDER_LONG_FIRST}
 
 
 def schedule_order(context_lens, policy="long_first"):
@@ -268,3 +272,71 @@ class DecodeLoop:
         done.record(main)
         self.done_ev[k] = done
         return max_ctx
+
+
+class NativeDecodeLoop:
+    """The iteration of :class:`DecodeLoop` sequenced inside the library
+    (``kv_serve_schedule`` / ``kv_serve_launch``): the scheduler step packs
+    the step's metadata straight into one of two pinned buffers and queues
+    its upload on the loop's upload stream; one launch call then enqueues
+    the swaps, copy-on-write, cache write, optional prefill and decode.  No
+    shared-prefix decode (use :class:`DecodeLoop` for that).  This class only
+    owns the buffers and passes pointers.  With ``full_plan`` set, schedule()
+    also returns every array of the step (kv_sched_outputs and the swap
+    outputs), for callers that check or mirror it."""
+
+    def __init__(self, pool, sched, *, num_q_heads, kv_heads, head_dim, block_size, q_dtype,
+                 scale, max_batch, max_blocks, max_tokens, max_context, device="cuda",
+                 order_policy="batch", host_swap=None, swap_slots=0):
+        import torch
+        self.torch = torch
+        self.pool, self.sched = pool, sched
+        self.hq, self.hkv, self.d, self.bs = num_q_heads, kv_heads, head_dim, block_size
+        self.max_batch, self.max_blocks, self.max_tokens = max_batch, max_blocks, max_tokens
+        self.meta_bytes = kv_step_packed_bytes(max_batch, max_tokens, max_blocks, swap_slots)
+        self.h_buf = [torch.empty(self.meta_bytes, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        self.d_buf = [torch.empty(self.meta_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.ws_cap = max(kv_serve_workspace_bytes(pool, num_q_heads, max_batch, max_context), 16)
+        self.d_ws = torch.empty(self.ws_cap, dtype=torch.uint8, device=device)
+        self.up = torch.cuda.Stream(device=device)
+        self.host_swap = host_swap
+        self.handle = kv_serve_create(pool, sched, num_q_heads, q_dtype, scale, ORDER_POLICIES[order_policy],
+                                      max_batch, max_tokens, max_blocks, host_swap, swap_slots, self.h_buf,
+                                      self.d_buf, self.meta_bytes, self.d_ws, self.ws_cap)
+        self.running_buf = np.empty(max_batch, np.int64)
+        self.layout = kv_step_layout()
+        self.last_prefix = (None, None)
+        self.full_plan = False
+
+    def schedule(self, finished_ids):
+        """Native scheduler step + packed upload; returns {"info", "layout",
+        "running"} (``running`` is a view valid until the next step)."""
+        lay = kv_serve_schedule(self.handle, finished_ids, self.up, self.running_buf, self.layout)
+        if not self.full_plan:
+            return {"info": lay.info, "layout": lay, "running": self.running_buf[:lay.info.batch]}
+        out = kv_sched_outputs(self.sched, lay.info, lay.table_width)
+        out.update(kv_sched_swap_outputs(self.sched))
+        out.update(info=lay.info, layout=lay)
+        return out
+
+    def launch(self, plan, k_new, v_new, q, out, k_inv=None, v_inv=None, out_dtype=None,
+               layer=0, stream=None, prefill_q=None, prefill_out=None, before_decode=None):
+        """Enqueue the step's kernels for one layer (``before_decode`` is
+        called before the single launch call, which holds the decode)."""
+        main = self.torch.cuda.current_stream() if stream is None else stream
+        if before_decode is not None:
+            before_decode(main)
+        kv_serve_launch(self.handle, layer, q, k_new, v_new, out, KV_F32 if out_dtype is None else out_dtype,
+                        k_inv, v_inv, prefill_q, prefill_out, main)
+        return self.layout.max_context_len
+
+    def close(self):
+        if self.handle is not None:
+            kv_serve_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001  (interpreter shutdown)
+            pass

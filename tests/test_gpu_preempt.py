@@ -24,13 +24,15 @@ def host16(t):
     return t.cpu().numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("mode", ["swap", "recompute"])
-def test_preempt_trace_matches_oracle(mode):
+@pytest.mark.parametrize("mode,native", [("swap", False), ("recompute", False), ("swap", True)])
+def test_preempt_trace_matches_oracle(mode, native):
+    """native: the same trace through the library's serving step
+    (kv_serve_schedule / kv_serve_launch)."""
     w0 = WORKLOADS["preempt_trace"]
     w = dataclasses.replace(w0, extra=dict(w0.extra, out_lo=30, out_hi=80, num_blocks=2400, iters=45,
                                            arrival_rate=2.0))
     plan = preempt_plan(w)
-    tr = PreemptTrace(w, plan, mode=mode)
+    tr = PreemptTrace(w, plan, mode=mode, native=native)
     bs, nb = w.block_size, tr.num_blocks
     bm = BlockManager(nb, bs, tr.order)
     bm.set_swap_space(tr.swap_slots)

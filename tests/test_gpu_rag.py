@@ -23,11 +23,13 @@ def host16(t):
     return t.cpu().numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("caching", [True, False])
-def test_rag_trace_matches_oracle(caching):
+@pytest.mark.parametrize("caching,native", [(True, False), (False, False), (True, True)])
+def test_rag_trace_matches_oracle(caching, native):
+    """native: the same trace through the library's serving step, its
+    prefill arrays packed by the library."""
     w = WORKLOADS["rag_trace"]
     plan = rag_plan(w)
-    tr = RagTrace(w, plan, caching=caching)
+    tr = RagTrace(w, plan, caching=caching, native=native)
     bs = w.block_size
     bm = (PrefixCachingBlockManager if caching else BlockManager)(tr.num_blocks, bs, tr.order)
     sched = Scheduler(bm, w.extra["max_num_seqs"])

@@ -54,9 +54,11 @@ def mirror_initial(tr, w, plan):
     return bm, sched, kh, vh, init_slots
 
 
-def run_trace(w, iters, check_pool_at, sample_every=1, shared_prefix=False):
+def run_trace(w, iters, check_pool_at, sample_every=1, shared_prefix=False, native=False, order_policy="batch"):
     plan = gqa_trace_plan(w)
-    tr = GqaTrace(w, plan, shared_prefix=shared_prefix)
+    tr = GqaTrace(w, plan, shared_prefix=shared_prefix, native=native, order_policy=order_policy)
+    if native:
+        tr.loop.full_plan = True  # the step's arrays, to compare with the oracle scheduler
     used_prefix = 0
     bm, sched, kh, vh, init_slots = mirror_initial(tr, w, plan)
     assert np.array_equal(init_slots, tr.init_slots)
@@ -111,6 +113,18 @@ def test_gqa_trace_full_size_matches_oracle():
     tr, cow_total = run_trace(w, w.extra["iters"], check_pool_at={0, 1, 50, w.extra["iters"] - 1})
     # every sharer but the last copied the shared partly filled block
     assert cow_total >= len(tr.sharers) - 1
+
+
+@pytest.mark.parametrize("order_policy,iters", [("batch", 30), ("long_first", 12)])
+def test_gqa_trace_through_the_native_serving_step(order_policy, iters):
+    """The trace sequenced by the library (kv_serve_schedule packs the step
+    into a pinned buffer and uploads it; kv_serve_launch enqueues copy,
+    write and decode in the packed scheduling order): pool and sampled
+    outputs still equal the oracle mirror's."""
+    w = WORKLOADS["gqa_trace"]
+    tr, cow_total = run_trace(w, iters, check_pool_at={0, iters - 1}, native=True, order_policy=order_policy)
+    assert cow_total >= len(tr.sharers) - 1
+    tr.loop.close()
 
 
 def test_gqa_trace_with_shared_prefix_decode_matches_oracle():

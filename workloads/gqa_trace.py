@@ -26,7 +26,7 @@ from paged_kv_cache_451_b200 import (kv_alloc_allocate, kv_alloc_block_table, kv
                                      kv_alloc_fork, kv_alloc_free, kv_alloc_num_free, kv_pool_bind,
                                      kv_pool_create, kv_sched_adopt, kv_sched_add_request,
                                      kv_sched_create, kv_pool_set_decode_config, paged_kv_write)
-from paged_kv_cache_451_b200.serving import DecodeLoop
+from paged_kv_cache_451_b200.serving import DecodeLoop, NativeDecodeLoop
 
 from . import blocks_needed, device_normal_bits
 
@@ -36,7 +36,7 @@ FIRST_ARRIVAL = 10_000
 
 class GqaTrace:
     def __init__(self, w, plan, device="cuda", seed=0, decode_config=None, order_policy="batch",
-                 shared_prefix=False):
+                 shared_prefix=False, native=False):
         import torch
 
         self.torch, self.w, self.plan, self.seed = torch, w, plan, seed
@@ -88,11 +88,15 @@ class GqaTrace:
         self.running = np.arange(w.batch, dtype=np.int64)
         self.max_blocks = int(math.ceil((e["cap"] + e["iters"] + 2 * bs) / bs))
         max_tokens = 256 + 16 * e["prompt_hi"]
-        self.loop = DecodeLoop(self.pool, self.sched, num_q_heads=w.num_q_heads, kv_heads=w.kv_heads,
-                               head_dim=w.head_dim, block_size=bs, q_dtype=w.q_fmt, scale=w.scale,
-                               max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
-                               max_tokens=max_tokens, max_context=e["cap"] + e["iters"] + bs,
-                               device=device, order_policy=order_policy, shared_prefix=shared_prefix)
+        # native: the iteration sequenced inside the library (kv_serve_*)
+        if native and shared_prefix:
+            raise ValueError("the native serving step has no shared-prefix decode")
+        kw = dict(num_q_heads=w.num_q_heads, kv_heads=w.kv_heads, head_dim=w.head_dim, block_size=bs,
+                  q_dtype=w.q_fmt, scale=w.scale, max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
+                  max_tokens=max_tokens, max_context=e["cap"] + e["iters"] + bs, device=device,
+                  order_policy=order_policy)
+        self.loop = (NativeDecodeLoop(self.pool, self.sched, **kw) if native else
+                     DecodeLoop(self.pool, self.sched, shared_prefix=shared_prefix, **kw))
 
     def _seed(self, it, kind):
         return (self.w.seed * 1_000_003 + (it + 2) * 7919 + kind * 104_729 + self.seed) % (2 ** 62)
@@ -135,7 +139,7 @@ class GqaTrace:
         plan = self.loop.schedule(fin)
         self.last_schedule_s = time.perf_counter() - t0
         info = plan["info"]
-        self.running = np.asarray(plan["running"], np.int64)
+        self.running = np.array(plan["running"], np.int64)
         T, B = info.num_tokens, info.batch
         if inputs is None:
             k_new = self.draw((max(T, 1), w.kv_heads, w.head_dim), w.kv_fmt, self.device, self._seed(it, 0))

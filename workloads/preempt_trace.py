@@ -19,7 +19,7 @@ from paged_kv_cache_451_b200 import (KV_PREEMPT_RECOMPUTE, KV_PREEMPT_SWAP, kv_a
                                      kv_alloc_set_swap_space, kv_pool_bind, kv_pool_create,
                                      kv_sched_add_request, kv_sched_create, kv_sched_set_preemption,
                                      kv_swap_block_bytes)
-from paged_kv_cache_451_b200.serving import DecodeLoop
+from paged_kv_cache_451_b200.serving import DecodeLoop, NativeDecodeLoop
 
 from . import device_normal_bits, rng_for
 
@@ -35,7 +35,7 @@ def preempt_plan(w):
 
 
 class PreemptTrace:
-    def __init__(self, w, plan, mode="swap", device="cuda", seed=0):
+    def __init__(self, w, plan, mode="swap", device="cuda", seed=0, native=False):
         import torch
 
         self.torch, self.w, self.plan, self.seed, self.device = torch, w, plan, seed, device
@@ -64,11 +64,14 @@ class PreemptTrace:
             self._add(plen, olen)
         max_ctx = e["prompt_hi"] + e["out_hi"] + 2 * bs
         self.max_blocks = -(-max_ctx // bs)
-        self.loop = DecodeLoop(self.pool, self.sched, num_q_heads=w.num_q_heads, kv_heads=w.kv_heads,
-                               head_dim=w.head_dim, block_size=bs, q_dtype=w.q_fmt, scale=w.scale,
-                               max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
-                               max_tokens=e["max_num_seqs"] * (max_ctx + 1), max_context=max_ctx,
-                               device=device, host_swap=self.host, swap_slots=self.swap_slots)
+        # native: the iteration sequenced inside the library (kv_serve_*)
+        self.loop = (NativeDecodeLoop if native else DecodeLoop)(
+            self.pool, self.sched, num_q_heads=w.num_q_heads, kv_heads=w.kv_heads, head_dim=w.head_dim,
+            block_size=bs, q_dtype=w.q_fmt, scale=w.scale, max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
+            max_tokens=e["max_num_seqs"] * (max_ctx + 1), max_context=max_ctx, device=device, host_swap=self.host,
+            swap_slots=self.swap_slots)
+        if native:
+            self.loop.full_plan = True  # callers mirror the swap pairs
 
     def _add(self, plen, olen):
         sid = self.next_id

@@ -16,7 +16,7 @@ import numpy as np
 
 from paged_kv_cache_451_b200 import (kv_alloc_create, kv_alloc_enable_prefix_caching, kv_pool_bind,
                                      kv_pool_create, kv_sched_add_request_tokens, kv_sched_create)
-from paged_kv_cache_451_b200.serving import DecodeLoop
+from paged_kv_cache_451_b200.serving import DecodeLoop, NativeDecodeLoop
 
 from . import device_normal_bits, rng_for
 
@@ -37,7 +37,7 @@ def rag_plan(w):
 
 
 class RagTrace:
-    def __init__(self, w, plan, caching=True, device="cuda", seed=0, shared_prefix=False):
+    def __init__(self, w, plan, caching=True, device="cuda", seed=0, shared_prefix=False, native=False):
         import torch
 
         self.torch, self.w, self.plan, self.seed, self.device = torch, w, plan, seed, device
@@ -62,11 +62,17 @@ class RagTrace:
         max_ctx = e["doc_len"] + e["question_hi"] + e["out_hi"] + e["iters"] + 2 * bs
         self.max_blocks = -(-max_ctx // bs)
         max_prompt_tokens = 16 * (e["doc_len"] + e["question_hi"])
-        self.loop = DecodeLoop(self.pool, self.sched, num_q_heads=w.num_q_heads, kv_heads=w.kv_heads,
-                               head_dim=w.head_dim, block_size=bs, q_dtype=w.q_fmt, scale=w.scale,
-                               max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
-                               max_tokens=max_prompt_tokens + e["max_num_seqs"], max_context=max_ctx,
-                               device=device, shared_prefix=shared_prefix)
+        # native: the iteration sequenced inside the library (kv_serve_*)
+        if native and shared_prefix:
+            raise ValueError("the native serving step has no shared-prefix decode")
+        kw = dict(num_q_heads=w.num_q_heads, kv_heads=w.kv_heads, head_dim=w.head_dim, block_size=bs,
+                  q_dtype=w.q_fmt, scale=w.scale, max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
+                  max_tokens=max_prompt_tokens + e["max_num_seqs"], max_context=max_ctx, device=device)
+        if native:
+            self.loop = NativeDecodeLoop(self.pool, self.sched, **kw)
+            self.loop.full_plan = True  # the prefill sizes come from the step's arrays
+        else:
+            self.loop = DecodeLoop(self.pool, self.sched, shared_prefix=shared_prefix, **kw)
 
     def _seed(self, it, kind):
         return (self.w.seed * 1_000_003 + (it + 2) * 7919 + kind * 104_729 + self.seed) % (2 ** 62)
