@@ -750,6 +750,29 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
         used[k] = True
         moved["d2h"] += 2 * n
 
+    if native:
+        # the library orders the staging copies: kv_serve_upload on the
+        # loop's upload stream into buffer set layout.buffer (the step's
+        # parity), kv_serve_readback on the read-back stream
+        loop = tr.loop
+        hb, hob = host.data_ptr(), hout.data_ptr()
+        dbase, obase = [t.data_ptr() for t in devb], [t.data_ptr() for t in outs]
+
+        def inputs(T, B):  # noqa: F811
+            k = loop.layout.buffer
+            nq, nk = B * hq * d, T * hkv * d
+            loop.upload(dbase[k], hb, 2 * (nq + 2 * nk))
+            moved["h2d"] += 2 * (nq + 2 * nk) + loop.layout.bytes
+            return dbase[k], dbase[k] + 2 * nq, dbase[k] + 2 * (nq + nk)
+
+        def one(it):  # noqa: F811
+            k = it % 2
+            fin, arr, pl, *_r = tr.iteration(it, out_dtype=w.q_fmt, inputs=inputs, out=obase[k], stream=stream)
+            assert pl["layout"].buffer == k
+            n = max(pl["info"].batch, 1) * hq * d
+            loop.readback(hob, obase[k], 2 * n, rb)
+            moved["d2h"] += 2 * n
+
     for it in range(W):
         one(it)
     torch.cuda.synchronize()
@@ -759,7 +782,9 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
     a.record(stream)
     for i in range(K):
         one(W + i)
-    stream.wait_event(rb_done[(W + K - 1) % 2])  # the last read-back is inside the region
+    last = torch.cuda.Event()
+    last.record(rb)  # every read-back ran on rb: the last one is inside the region
+    stream.wait_event(last)
     b.record(stream)
     torch.cuda.synchronize()
     span = (t0, time.perf_counter())
@@ -775,8 +800,9 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
                        "uploaded; kv_serve_launch: copy-on-write, cache write, decode), " if native else
                        "(Python sequencing with the shared-prefix decode), ")
                     + "one upload of the step's q and new K/V rows from a pinned staging buffer on an upload "
-                    "stream (two device buffer sets), and the output read back on a read-back stream; K "
-                    "iterations timed as one region (host scheduling included)",
+                    "stream (two device buffer sets; kv_serve_upload), and the output read back on a read-back "
+                    "stream (kv_serve_readback); K iterations timed as one region (host scheduling included); "
+                    "h2d counts the packed metadata too",
             "serving_step": "native" if native else "python",
             "clocks": clk.summary(*span)}
 

@@ -594,6 +594,7 @@ typedef struct {
   int num_swap_in;      /* swap-in pairs */
   int prefill_tokens;   /* admitted prompts' uncached tokens, cu_seqlens[num_admitted] */
   int max_prefill_len;  /* most uncached tokens of one admitted prompt */
+  int buffer;           /* kv_serve_schedule: the step's buffer set, 0 or 1 (alternating); else 0 */
   int64_t bytes;        /* bytes of the buffer the step uses */
   int64_t slot_mapping;          /* int64[num_tokens] */
   int64_t block_tables;          /* int32[batch][table_width], padded with -1 */
@@ -637,7 +638,7 @@ size_t kv_serve_workspace_bytes(const kv_pool* pool, int num_q_heads, int max_ba
  * max_table_width, swap_slots), 16-byte aligned), the decode workspace
  * (>= kv_serve_workspace_bytes), and for swap preemption the mapped pinned
  * host swap space of swap_slots slots (kv_swap_out).  Consecutive steps
- * alternate between the two buffer pairs; the loop creates four CUDA events
+ * alternate between the two buffer pairs; the loop creates six CUDA events
  * on the current device, which must stay current for its calls.
  * num_q_heads, q_dtype (also the type of the new K/V rows) and scale are
  * those of the decode.  KV_ERR_ARG on bad arguments; KV_ERR_CUDA if an event
@@ -674,7 +675,21 @@ int kv_serve_launch(kv_serve* s, int layer, const void* q, const void* k_new, co
                     const float* k_inv_scale, const float* v_inv_scale, void* out, kv_dtype out_dtype,
                     const void* prefill_q, void* prefill_out, kv_stream_t stream);
 
-/* Waits for the loop's uploads and kernels (host), then frees it. */
+/* Host input and output staging for a loop whose inputs come from host
+ * memory.  The caller keeps two sets of device input and output buffers and
+ * uses set layout.buffer for a step.  kv_serve_upload (after
+ * kv_serve_schedule, before the step's first launch) copies bytes from
+ * pinned host memory to dev_dst on the step's upload stream, after the
+ * kernels that last read that set (the step before the previous one); the
+ * step's launches wait for it.  kv_serve_readback (after a launch) copies
+ * bytes from dev_src to pinned host memory on readback_stream once the
+ * step's kernels so far are done; the first launch of the step after next,
+ * which reuses the set, waits for it.  KV_ERR_STATE when called out of that
+ * order, KV_ERR_ARG on NULL pointers with bytes > 0. */
+int kv_serve_upload(kv_serve* s, void* dev_dst, const void* host_src, size_t bytes);
+int kv_serve_readback(kv_serve* s, void* host_dst, const void* dev_src, size_t bytes, kv_stream_t readback_stream);
+
+/* Waits for the loop's uploads, kernels and read-backs (host), then frees it. */
 int kv_serve_destroy(kv_serve* s);
 
 #ifdef __cplusplus

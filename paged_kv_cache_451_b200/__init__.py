@@ -58,7 +58,7 @@ class kv_step_info(ctypes.Structure):
 class kv_step_layout(ctypes.Structure):
     _fields_ = [("info", kv_step_info), ("table_width", c_int), ("max_context_len", c_int),
                 ("num_swap_out", c_int), ("num_swap_in", c_int), ("prefill_tokens", c_int),
-                ("max_prefill_len", c_int), ("bytes", c_int64), ("slot_mapping", c_int64),
+                ("max_prefill_len", c_int), ("buffer", c_int), ("bytes", c_int64), ("slot_mapping", c_int64),
                 ("block_tables", c_int64), ("context_lens", c_int64), ("seq_order", c_int64),
                 ("cow_pairs", c_int64), ("swap_out_pairs", c_int64), ("swap_in_pairs", c_int64),
                 ("cu_seqlens", c_int64), ("prefill_context_lens", c_int64)]
@@ -141,6 +141,8 @@ _SIGS = {
     "kv_serve_schedule": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, P(kv_step_layout)]),
     "kv_serve_launch": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_int, c_void_p, c_void_p, c_void_p]),
+    "kv_serve_upload": (c_int, [c_void_p, c_void_p, c_void_p, c_size_t]),
+    "kv_serve_readback": (c_int, [c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "kv_serve_destroy": (c_int, [c_void_p]),
 }
 
@@ -564,6 +566,14 @@ def kv_serve_launch(sv, layer, q, k_new, v_new, out, out_dtype, k_inv_scale=None
     _check(_lib.kv_serve_launch(sv, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_inv_scale),
                                 _ptr(v_inv_scale), _ptr(out), out_dtype, _ptr(prefill_q), _ptr(prefill_out),
                                 _stream(stream)))
+
+
+def kv_serve_upload(sv, dev_dst, host_src, nbytes):
+    _check(_lib.kv_serve_upload(sv, _ptr(dev_dst), _ptr(host_src), int(nbytes)))
+
+
+def kv_serve_readback(sv, host_dst, dev_src, nbytes, readback_stream=None):
+    _check(_lib.kv_serve_readback(sv, _ptr(host_dst), _ptr(dev_src), int(nbytes), _stream(readback_stream)))
 
 
 def kv_serve_destroy(sv):

@@ -74,9 +74,11 @@ struct kv_serve {
   size_t meta_bytes = 0;
   void* ws = nullptr;
   size_t ws_bytes = 0;
-  cudaEvent_t copy_ev[2] = {nullptr, nullptr};  // upload into buffer k done
-  cudaEvent_t done_ev[2] = {nullptr, nullptr};  // kernels reading buffer k done
-  bool copy_rec[2] = {false, false}, done_rec[2] = {false, false};
+  cudaEvent_t copy_ev[2] = {nullptr, nullptr};  // uploads into buffer set k done
+  cudaEvent_t done_ev[2] = {nullptr, nullptr};  // kernels reading buffer set k done
+  cudaEvent_t rb_ev[2] = {nullptr, nullptr};    // read-back of output set k done
+  bool copy_rec[2] = {false, false}, done_rec[2] = {false, false}, rb_rec[2] = {false, false};
+  cudaStream_t up = nullptr;  // the current step's upload stream
   int k = 1;               // buffer of the current step
   bool scheduled = false;  // a step is scheduled and not launched yet
   int launches = 0;        // launch calls for the current step
@@ -225,7 +227,8 @@ int kv_serve_create(kv_pool* pool, kv_sched* sched, int num_q_heads, kv_dtype q_
   s->ws_bytes = workspace ? workspace_bytes : 0;
   for (int i = 0; i < 2; ++i) {
     if (cudaEventCreateWithFlags(&s->copy_ev[i], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&s->done_ev[i], cudaEventDisableTiming) != cudaSuccess) {
+        cudaEventCreateWithFlags(&s->done_ev[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s->rb_ev[i], cudaEventDisableTiming) != cudaSuccess) {
       const cudaError_t e = cudaGetLastError();
       kv_serve_destroy(s);
       return fail(KV_ERR_CUDA, "cudaEventCreate: %s", cudaGetErrorString(e));
@@ -268,6 +271,8 @@ int kv_serve_schedule(kv_serve* s, const int64_t* finished_ids, int n_finished, 
     return fail(KV_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(cudaGetLastError()));
   s->copy_rec[k] = true;
   s->k = k;
+  s->up = up;
+  L.buffer = k;
   s->lay = L;
   s->scheduled = true;
   s->launches = 0;
@@ -294,6 +299,9 @@ int kv_serve_launch(kv_serve* s, int layer, const void* q, const void* k_new, co
   auto i32 = [&](int64_t o) { return o < 0 ? nullptr : reinterpret_cast<const int32_t*>(d + o); };
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamWaitEvent(st, s->copy_ev[k], 0) != cudaSuccess)
+    return fail(KV_ERR_CUDA, "cudaStreamWaitEvent: %s", cudaGetErrorString(cudaGetLastError()));
+  // outputs of set k are overwritten only after their last read-back
+  if (s->launches == 0 && s->rb_rec[k] && cudaStreamWaitEvent(st, s->rb_ev[k], 0) != cudaSuccess)
     return fail(KV_ERR_CUDA, "cudaStreamWaitEvent: %s", cudaGetErrorString(cudaGetLastError()));
   int rc = KV_OK;
   if (s->launches == 0) {
@@ -326,9 +334,40 @@ int kv_serve_launch(kv_serve* s, int layer, const void* q, const void* k_new, co
   return rc;
 }
 
+int kv_serve_upload(kv_serve* s, void* dev_dst, const void* host_src, size_t bytes) {
+  if (!s || (bytes && (!dev_dst || !host_src))) return fail(KV_ERR_ARG, "bad argument");
+  if (!s->scheduled || s->launches) return fail(KV_ERR_STATE, "uploads go between kv_serve_schedule and the step's launch");
+  if (!bytes) return ok();
+  const int k = s->k;
+  if (cudaMemcpyAsync(dev_dst, host_src, bytes, cudaMemcpyHostToDevice, s->up) != cudaSuccess)
+    return fail(KV_ERR_CUDA, "upload: %s", cudaGetErrorString(cudaGetLastError()));
+  if (cudaEventRecord(s->copy_ev[k], s->up) != cudaSuccess)
+    return fail(KV_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(cudaGetLastError()));
+  return ok();
+}
+
+int kv_serve_readback(kv_serve* s, void* host_dst, const void* dev_src, size_t bytes, kv_stream_t readback_stream) {
+  if (!s || (bytes && (!host_dst || !dev_src))) return fail(KV_ERR_ARG, "bad argument");
+  if (!s->scheduled || !s->launches) return fail(KV_ERR_STATE, "read-back goes after the step's launch");
+  const int k = s->k;
+  cudaStream_t rb = reinterpret_cast<cudaStream_t>(readback_stream);
+  if (cudaStreamWaitEvent(rb, s->done_ev[k], 0) != cudaSuccess)
+    return fail(KV_ERR_CUDA, "cudaStreamWaitEvent: %s", cudaGetErrorString(cudaGetLastError()));
+  if (bytes && cudaMemcpyAsync(host_dst, dev_src, bytes, cudaMemcpyDeviceToHost, rb) != cudaSuccess)
+    return fail(KV_ERR_CUDA, "read-back: %s", cudaGetErrorString(cudaGetLastError()));
+  if (cudaEventRecord(s->rb_ev[k], rb) != cudaSuccess)
+    return fail(KV_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(cudaGetLastError()));
+  s->rb_rec[k] = true;
+  return ok();
+}
+
 int kv_serve_destroy(kv_serve* s) {
   if (!s) return ok();
   for (int i = 0; i < 2; ++i) {
+    if (s->rb_ev[i]) {
+      cudaEventSynchronize(s->rb_ev[i]);
+      cudaEventDestroy(s->rb_ev[i]);
+    }
     if (s->copy_ev[i]) {
       cudaEventSynchronize(s->copy_ev[i]);
       cudaEventDestroy(s->copy_ev[i]);

@@ -27,10 +27,10 @@ import numpy as np
 
 from . import (KV_F32, KV_ORDER_BATCH, KV_ORDER_LONG_FIRST, KV_ORDER_LONGEST, block_copy, kv_sched_outputs,
                kv_sched_step, kv_sched_swap_outputs, kv_serve_create, kv_serve_destroy, kv_serve_launch,
-               kv_serve_schedule, kv_serve_workspace_bytes, kv_step_layout, kv_step_packed_bytes, kv_swap_in,
-               kv_swap_out, paged_attention_decode, paged_attention_decode_shared_prefix,
-               paged_attention_prefill, paged_attention_shared_prefix_workspace_bytes,
-               paged_attention_workspace_bytes, paged_kv_write)
+               kv_serve_readback, kv_serve_schedule, kv_serve_upload, kv_serve_workspace_bytes, kv_step_layout,
+               kv_step_packed_bytes, kv_swap_in, kv_swap_out, paged_attention_decode,
+               paged_attention_decode_shared_prefix, paged_attention_prefill,
+               paged_attention_shared_prefix_workspace_bytes, paged_attention_workspace_bytes, paged_kv_write)
 
 ORDER_POLICIES = {"batch": KV_ORDER_BATCH, "longest": KV_ORDER_LONGEST, "long_first": KV_ORDER_LONG_FIRST}
 
@@ -329,6 +329,16 @@ class NativeDecodeLoop:
         kv_serve_launch(self.handle, layer, q, k_new, v_new, out, KV_F32 if out_dtype is None else out_dtype,
                         k_inv, v_inv, prefill_q, prefill_out, main)
         return self.layout.max_context_len
+
+    def upload(self, dev_dst, host_src, nbytes):
+        """Copy the step's inputs from pinned host memory into buffer set
+        ``plan["layout"].buffer`` (between schedule and launch)."""
+        kv_serve_upload(self.handle, dev_dst, host_src, nbytes)
+
+    def readback(self, host_dst, dev_src, nbytes, stream):
+        """Copy the step's outputs to pinned host memory on ``stream``
+        (after launch)."""
+        kv_serve_readback(self.handle, host_dst, dev_src, nbytes, stream)
 
     def close(self):
         if self.handle is not None:

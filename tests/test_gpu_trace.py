@@ -54,18 +54,60 @@ def mirror_initial(tr, w, plan):
     return bm, sched, kh, vh, init_slots
 
 
-def run_trace(w, iters, check_pool_at, sample_every=1, shared_prefix=False, native=False, order_policy="batch"):
+class HostStaging:
+    """Inputs drawn into pinned host memory and uploaded by the serving
+    loop (kv_serve_upload) into the step's buffer set; outputs read back by
+    it (kv_serve_readback) into pinned host memory."""
+
+    def __init__(self, tr, w):
+        e = w.extra
+        self.loop, self.w = tr.loop, w
+        hq, hkv, d = w.num_q_heads, w.kv_heads, w.head_dim
+        n = (e["max_num_seqs"] * hq + 2 * tr.loop.max_tokens * hkv) * d
+        self.host = torch.empty(n, dtype=torch.int16).pin_memory()
+        self.dev = [torch.empty(n, dtype=torch.int16, device="cuda") for _ in range(2)]
+        self.outs = [torch.empty((e["max_num_seqs"], hq, d), dtype=torch.float32, device="cuda") for _ in range(2)]
+        self.hout = [torch.empty((e["max_num_seqs"], hq, d), dtype=torch.float32).pin_memory() for _ in range(2)]
+        self.rb = torch.cuda.Stream()
+        self.rng = np.random.default_rng(99)
+
+    def inputs(self, T, B):
+        w, k = self.w, self.loop.layout.buffer
+        nq, nk = B * w.num_q_heads * w.head_dim, T * w.kv_heads * w.head_dim
+        torch.cuda.current_stream().synchronize()  # the host buffer is rewritten: earlier uploads must be done
+        self.loop.up.synchronize()
+        bits = self.rng.standard_normal(nq + 2 * nk).astype(np.float32)
+        self.host[:nq + 2 * nk].copy_(torch.from_numpy(bits).to(torch.bfloat16).view(torch.int16))
+        self.loop.upload(self.dev[k], self.host, 2 * (nq + 2 * nk))
+        buf = self.dev[k]
+        return (buf[:nq].view(B, w.num_q_heads, w.head_dim), buf[nq:nq + nk].view(T, w.kv_heads, w.head_dim),
+                buf[nq + nk:nq + 2 * nk].view(T, w.kv_heads, w.head_dim))
+
+
+def run_trace(w, iters, check_pool_at, sample_every=1, shared_prefix=False, native=False, order_policy="batch",
+              staging=False):
     plan = gqa_trace_plan(w)
     tr = GqaTrace(w, plan, shared_prefix=shared_prefix, native=native, order_policy=order_policy)
     if native:
         tr.loop.full_plan = True  # the step's arrays, to compare with the oracle scheduler
+    st = HostStaging(tr, w) if staging else None
     used_prefix = 0
     bm, sched, kh, vh, init_slots = mirror_initial(tr, w, plan)
     assert np.array_equal(init_slots, tr.init_slots)
     bs = w.block_size
     cow_total = 0
     for it in range(iters):
-        fin, arr, gplan, q, kn, vn, out = tr.iteration(it)
+        if st is None:
+            fin, arr, gplan, q, kn, vn, out = tr.iteration(it)
+        else:
+            k = it % 2
+            fin, arr, gplan, q, kn, vn, out = tr.iteration(it, inputs=st.inputs, out=st.outs[k])
+            assert gplan["layout"].buffer == k
+            nout = gplan["info"].batch * w.num_q_heads * w.head_dim
+            tr.loop.readback(st.hout[k], out, 4 * nout, st.rb)
+            st.rb.synchronize()
+            # the read-back waited for this step's decode
+            assert torch.equal(st.hout[k].view(-1)[:nout], out.view(-1)[:nout].cpu())
         for sid, plen in arr:
             sched.add_request(sid, plen)
         want = sched.step(fin)
@@ -124,6 +166,15 @@ def test_gqa_trace_through_the_native_serving_step(order_policy, iters):
     w = WORKLOADS["gqa_trace"]
     tr, cow_total = run_trace(w, iters, check_pool_at={0, iters - 1}, native=True, order_policy=order_policy)
     assert cow_total >= len(tr.sharers) - 1
+    tr.loop.close()
+
+
+def test_gqa_trace_with_host_staging_through_the_serving_loop():
+    """Inputs uploaded from pinned host memory by kv_serve_upload into
+    alternating buffer sets, outputs read back by kv_serve_readback: the
+    pool, the sampled outputs and the read-back bytes all check."""
+    w = WORKLOADS["gqa_trace"]
+    tr, _ = run_trace(w, 10, check_pool_at={0, 9}, native=True, staging=True)
     tr.loop.close()
 
 

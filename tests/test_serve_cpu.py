@@ -221,7 +221,8 @@ def test_serve_create_checks_arguments_before_any_cuda_call():
                                b.get("max_width", 16), None, b.get("swap_slots", 0), b.get("host", h), d,
                                b.get("meta_bytes", need), ws, 16)
         assert e.value.code == pk.KV_ERR_ARG
-    for f in (lambda: pk.kv_serve_schedule(None, []), lambda: pk.kv_serve_launch(None, 0, 0, 0, 0, 0, pk.KV_F32)):
+    for f in (lambda: pk.kv_serve_schedule(None, []), lambda: pk.kv_serve_launch(None, 0, 0, 0, 0, 0, pk.KV_F32),
+              lambda: pk.kv_serve_upload(None, 0, 0, 0), lambda: pk.kv_serve_readback(None, 0, 0, 0, 0)):
         with pytest.raises(pk.KVError) as e:
             f()
         assert e.value.code == pk.KV_ERR_ARG
