@@ -640,14 +640,22 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
     return fail(KV_ERR_ARG, "bad argument");
   kv_alloc* a = s->a;
   // validate before changing anything
-  std::unordered_set<int64_t> fin;
-  std::unordered_set<int64_t> run;
-  if (n_finished > 0) run.insert(s->running.begin(), s->running.end());
-  for (int i = 0; i < n_finished; ++i) {
-    if (!run.count(finished_ids[i]))
-      return fail(KV_ERR_STATE, "finished sequence %lld is not running", (long long)finished_ids[i]);
-    if (!fin.insert(finished_ids[i]).second)
-      return fail(KV_ERR_STATE, "sequence %lld finished twice", (long long)finished_ids[i]);
+  // the finished ids, sorted (a few per step): each must be running, once
+  std::vector<int64_t> fin(finished_ids, finished_ids + n_finished);
+  std::sort(fin.begin(), fin.end());
+  for (size_t i = 1; i < fin.size(); ++i)
+    if (fin[i] == fin[i - 1]) return fail(KV_ERR_STATE, "sequence %lld finished twice", (long long)fin[i]);
+  auto finished = [&](int64_t r) { return std::binary_search(fin.begin(), fin.end(), r); };
+  if (n_finished > 0) {
+    size_t found = 0;
+    for (int64_t r : s->running) found += finished(r);
+    if (found != fin.size()) {
+      std::vector<int64_t> run(s->running);
+      std::sort(run.begin(), run.end());
+      for (int64_t f : fin)
+        if (!std::binary_search(run.begin(), run.end(), f))
+          return fail(KV_ERR_STATE, "finished sequence %lld is not running", (long long)f);
+    }
   }
   s->out_running.clear();
   s->out_table_flat.clear();
@@ -667,7 +675,7 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   std::vector<int64_t> keep;
   keep.reserve(s->running.size());
   for (int64_t r : s->running)
-    if (!fin.count(r)) keep.push_back(r);
+    if (!finished(r)) keep.push_back(r);
   s->running.swap(keep);
   for (int i = 0; i < n_finished; ++i) kv_alloc_free(a, finished_ids[i]);
 

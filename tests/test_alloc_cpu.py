@@ -165,10 +165,11 @@ def test_native_scheduler_rejects_bad_finished_ids_without_changes():
     pk.kv_sched_add_request(s, 1, 3)
     pk.kv_sched_step(s, [])
     before = pk.kv_alloc_snapshot(a, 8)
-    for bad in ([7], [1, 1]):
+    for bad, msg in (([7], "7 is not running"), ([1, 1], "1 finished twice"), ([1, 7], "7 is not running"),
+                     ([7, 1], "7 is not running")):
         with pytest.raises(pk.KVError) as e:
             pk.kv_sched_step(s, bad)
-        assert e.value.code == pk.KV_ERR_STATE
+        assert e.value.code == pk.KV_ERR_STATE and msg in pk.kv_last_error()
     after = pk.kv_alloc_snapshot(a, 8)
     assert all(np.array_equal(x, y) for x, y in zip(before, after))
     pk.kv_sched_destroy(s)
