@@ -248,7 +248,9 @@ def kv_write(k_pool, v_pool, kv_fmt, k_new, v_new, src_fmt, slot_mapping, block_
         rows = np.asarray(new)[keep]  # [n][hkv][d] raw source storage
         if kv_fmt == E4M3:
             x = decode(rows, src_fmt).astype(np.float32)  # exact: 16-bit values fit fp32
-            y = (x * np.asarray(inv, np.float32)[blk][:, :, None]).astype(np.float32)
+            # the fp32 product may overflow to +-inf, which the encoder saturates
+            with np.errstate(over="ignore"):
+                y = (x * np.asarray(inv, np.float32)[blk][:, :, None]).astype(np.float32)
             pool[blk, :, off, :] = e4m3_encode(y)
         else:
             assert src_fmt == kv_fmt
