@@ -255,7 +255,11 @@ int kv_pool_set_sliding_window(kv_pool* pool, int window);
  *   out           device [total_q][num_q_heads][head_dim] of out_dtype (the
  *                 pool dtype or KV_F32), 16-byte aligned.
  * batch, total_q or max_q_len == 0 enqueues nothing.  No workspace.  Errors:
- * KV_ERR_ARG, KV_ERR_STATE (layer not bound), KV_ERR_CUDA. */
+ * KV_ERR_ARG, KV_ERR_STATE (layer not bound), KV_ERR_CUDA.
+ * The first call on a device (this one or paged_attention_decode_shared_prefix)
+ * looks up the device address of the library's error word and keeps it until
+ * the process exits; after cudaDeviceReset that address is stale, so a process
+ * that resets a device must not call these two entry points on it again. */
 int paged_attention_prefill(const kv_pool* pool, int layer, const void* q, kv_dtype q_dtype,
                             int num_q_heads, const int32_t* cu_seqlens_q, int total_q,
                             int max_q_len, const int32_t* block_tables, int max_blocks_per_seq,
