@@ -231,3 +231,28 @@ def test_serve_create_checks_arguments_before_any_cuda_call():
     pk.kv_pool_destroy(pool)
     pk.kv_sched_destroy(s)
     pk.kv_alloc_destroy(a)
+
+
+@pytest.mark.parametrize("lens,policy,want", [
+    ([9, 19, 29], pk.KV_ORDER_LONG_FIRST, [2, 0, 1]),           # 20 equals the mean: not long
+    ([9, 19, 29], pk.KV_ORDER_LONGEST, [2, 1, 0]),
+    ([4, 4, 4, 4], pk.KV_ORDER_LONG_FIRST, [0, 1, 2, 3]),       # nothing above the mean
+    ([4, 4, 4, 4], pk.KV_ORDER_LONGEST, [0, 1, 2, 3]),          # ties keep batch order
+    ([1, 50, 3, 50, 2], pk.KV_ORDER_LONG_FIRST, [1, 3, 0, 2, 4]),
+    ([1, 50, 3, 50, 2], pk.KV_ORDER_LONGEST, [1, 3, 2, 4, 0]),
+])
+def test_packed_orders_on_chosen_lengths(lens, policy, want):
+    """Contexts of chosen lengths (each step appends one token): the packed
+    scheduling order against the policy worked by hand."""
+    a = pk.kv_alloc_create(64, 16)
+    s = pk.kv_sched_create(a, 8)
+    for i, n in enumerate(lens):
+        pk.kv_alloc_allocate(a, i, n)
+        pk.kv_sched_adopt(s, i)
+    cap = pk.kv_step_packed_bytes(8, 8, 8, 0)
+    buf = aligned(cap)
+    lay = pk.kv_sched_step_packed(s, [], policy, 8, buf, cap)
+    assert section(buf, lay.context_lens, np.int32, len(lens)).tolist() == [n + 1 for n in lens]
+    assert section(buf, lay.seq_order, np.int32, len(lens)).tolist() == want
+    pk.kv_sched_destroy(s)
+    pk.kv_alloc_destroy(a)
