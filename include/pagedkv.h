@@ -645,8 +645,9 @@ size_t kv_serve_workspace_bytes(const kv_pool* pool, int num_q_heads, int max_ba
  * alternate between the two buffer pairs; the loop creates six CUDA events
  * on the current device, which must stay current for its calls.
  * num_q_heads, q_dtype (also the type of the new K/V rows) and scale are
- * those of the decode.  KV_ERR_ARG on bad arguments; KV_ERR_CUDA if an event
- * cannot be created. */
+ * those of the decode.  A loop holds per-step state: one host thread at a
+ * time drives it (and its scheduler).  KV_ERR_ARG on bad arguments;
+ * KV_ERR_CUDA if an event cannot be created. */
 int kv_serve_create(kv_pool* pool, kv_sched* sched, int num_q_heads, kv_dtype q_dtype, float scale,
                     int order_policy, int max_batch, int max_tokens, int max_table_width, void* host_swap,
                     int swap_slots, void* const host_meta[2], void* const dev_meta[2], size_t meta_bytes,
