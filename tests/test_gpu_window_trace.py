@@ -15,7 +15,7 @@ import oracle
 import paged_kv_cache_451_b200 as pk
 from gpu_util import TOL, max_abs
 from oracle.sched import BlockManager, Scheduler
-from paged_kv_cache_451_b200.serving import DecodeLoop
+from paged_kv_cache_451_b200.serving import DecodeLoop, NativeDecodeLoop
 from workloads import BF16, device_normal_bits
 
 pytestmark = pytest.mark.gpu
@@ -25,7 +25,10 @@ def host16(t):
     return t.cpu().numpy().view(np.uint16)
 
 
-def test_windowed_serving_loop_matches_oracle():
+@pytest.mark.parametrize("native", [False, True])
+def test_windowed_serving_loop_matches_oracle(native):
+    """native: the same loop through the library's serving step (tables
+    with released entries packed as they are)."""
     rng = np.random.default_rng(91)
     nb, bs, hkv, hq, d, W = 400, 16, 4, 16, 128, 200
     order = rng.permutation(nb).astype(np.int32)
@@ -39,9 +42,12 @@ def test_windowed_serving_loop_matches_oracle():
     pool = pk.kv_pool_create(bs, nb, hkv, d, BF16, 1)
     pk.kv_pool_bind(pool, 0, k, v)
     pk.kv_pool_set_sliding_window(pool, W)
-    loop = DecodeLoop(pool, sched, num_q_heads=hq, kv_heads=hkv, head_dim=d, block_size=bs, q_dtype=BF16,
-                      scale=1 / math.sqrt(d), max_batch=48, max_blocks=80, max_tokens=48 * 700,
-                      max_context=1200, order_policy="batch")
+    loop = (NativeDecodeLoop if native else DecodeLoop)(
+        pool, sched, num_q_heads=hq, kv_heads=hkv, head_dim=d, block_size=bs, q_dtype=BF16,
+        scale=1 / math.sqrt(d), max_batch=48, max_blocks=80, max_tokens=48 * 700, max_context=1200,
+        order_policy="batch")
+    if native:
+        loop.full_plan = True
     kh = np.zeros((nb, hkv, bs, d), np.uint16)
     vh = np.zeros_like(kh)
     remaining, running, nxt, released = {}, [], 0, 0
@@ -88,6 +94,8 @@ def test_windowed_serving_loop_matches_oracle():
         for r in running:
             remaining[r] -= 1
     assert released > 0
+    if native:
+        loop.close()
     pk.kv_sched_destroy(sched)
     pk.kv_alloc_destroy(alloc)
     pk.kv_pool_destroy(pool)
