@@ -694,8 +694,8 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
     serving step (kv_serve_schedule: scheduler step, metadata packed into a
     pinned buffer and uploaded; kv_serve_launch: copy-on-write, cache write,
     decode), uploads its queries and new K/V rows from one pinned host
-    staging buffer with one copy on an upload stream into one of two device
-    buffer sets (so the upload overlaps the previous iteration's kernels),
+    staging buffer with one copy on an upload stream into one of the loop's
+    three device buffer sets (so uploads overlap the earlier iterations' kernels),
     and its output is read back on a read-back stream (overlapping the next
     iteration); the K iterations are timed as one region, host scheduling
     included.  Bytes per step are the device-timed run's."""
@@ -711,8 +711,9 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
     # one staging buffer per step: q rows, then new K rows, then new V rows
     n_max = (max_b * hq + 2 * max_t * hkv) * d
     host = torch.randn(n_max, generator=g).to(torch.bfloat16).view(torch.int16).pin_memory()
-    devb = [torch.empty_like(host, device="cuda") for _ in range(2)]
-    outs = [torch.empty((max_b, hq, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    nsets = tr.loop.num_sets if native else 2  # the caller's input / output sets follow the loop's
+    devb = [torch.empty_like(host, device="cuda") for _ in range(nsets)]
+    outs = [torch.empty((max_b, hq, d), dtype=torch.bfloat16, device="cuda") for _ in range(nsets)]
     hout = torch.empty(max_b * hq * d, dtype=torch.bfloat16).pin_memory()
     up, rb = torch.cuda.Stream(), torch.cuda.Stream()
     up_done = [torch.cuda.Event(), torch.cuda.Event()]    # inputs of buffer set k uploaded
@@ -766,7 +767,7 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
             return dbase[k], dbase[k] + 2 * nq, dbase[k] + 2 * (nq + nk)
 
         def one(it):  # noqa: F811
-            k = it % 2
+            k = it % nsets
             fin, arr, pl, *_r = tr.iteration(it, out_dtype=w.q_fmt, inputs=inputs, out=obase[k], stream=stream)
             assert pl["layout"].buffer == k
             n = max(pl["info"].batch, 1) * hq * d
@@ -789,22 +790,80 @@ def trace_e2e(args, rank, w, plan, W, K, stream, clk, uniq_b, other_b, steps, di
     torch.cuda.synchronize()
     span = (t0, time.perf_counter())
     ms = max_over_ranks(a.elapsed_time(b), dist, "cuda") / K
+    timeline = serving_timeline(tr, one, W + K, 60) if native and getattr(args, "timeline", False) else None
     if native:
         tr.loop.close()
     del tr
-    return {"value": round(world * (uniq_b + other_b) / steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    return {**({"timeline": timeline} if timeline else {}),
+            "value": round(world * (uniq_b + other_b) / steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 5), "steps": K, "h2d_bytes_per_step": int(moved["h2d"] / K),
             "d2h_bytes_per_step": int(moved["d2h"] / K),
-            "mode": "serving loop from host memory, pipelined: per iteration the library's serving step "
-                    + ("(kv_serve_schedule: native scheduler step, metadata packed in a pinned buffer and "
-                       "uploaded; kv_serve_launch: copy-on-write, cache write, decode), " if native else
-                       "(Python sequencing with the shared-prefix decode), ")
-                    + "one upload of the step's q and new K/V rows from a pinned staging buffer on an upload "
-                    "stream (two device buffer sets; kv_serve_upload), and the output read back on a read-back "
-                    "stream (kv_serve_readback); K iterations timed as one region (host scheduling included); "
-                    "h2d counts the packed metadata too",
+            "mode": ("serving loop from host memory, pipelined: per iteration the library's serving step "
+                     f"(kv_serve_schedule: native scheduler step, metadata packed in a pinned buffer and uploaded; "
+                     f"kv_serve_launch: copy-on-write, cache write, decode), one upload of the step's q and new "
+                     f"K/V rows from a pinned staging buffer (kv_serve_upload) into one of {nsets} device buffer "
+                     f"sets used in turn, and the output read back on a read-back stream (kv_serve_readback); K "
+                     f"iterations timed as one region (host scheduling included); h2d counts the packed "
+                     f"metadata too" if native else
+                     "serving loop from host memory, pipelined: per iteration the Python serving loop with the "
+                     "shared-prefix decode, one upload of the step's q and new K/V rows from a pinned staging "
+                     "buffer on an upload stream into one of two device buffer sets, and the output read back "
+                     "on a read-back stream; K iterations timed as one region (host scheduling included)"),
             "serving_step": "native" if native else "python",
             "clocks": clk.summary(*span)}
+
+
+def serving_timeline(tr, one, it0, n):
+    """After the timed region (never inside it): n more iterations of the
+    end-to-end loop with timing events around each input upload on the
+    loop's upload stream, and host clocks around the library's scheduling
+    step, to show what bounds the loop (the PCIe upload or the host)."""
+    import torch
+    n = min(n, len(tr.plan["arrivals"]) - it0)  # the trace's iterations left after the timed region
+    if n < 8:
+        return {"skipped": f"only {max(n, 0)} trace iterations left after the timed region"}
+    loop = tr.loop
+    ev, host = [], {"schedule": 0.0, "total": 0.0, "bytes": 0}
+    sched, upload = loop.schedule, loop.upload
+
+    def timed_schedule(fin):
+        t0 = time.perf_counter()
+        r = sched(fin)
+        host["schedule"] += time.perf_counter() - t0
+        return r
+
+    def timed_upload(dst, src, nbytes):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(loop.up)
+        upload(dst, src, nbytes)
+        b.record(loop.up)
+        ev.append((a, b))
+        host["bytes"] += nbytes
+
+    loop.schedule, loop.upload = timed_schedule, timed_upload
+    try:
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for i in range(n):
+            one(it0 + i)
+        torch.cuda.synchronize()
+        host["total"] = time.perf_counter() - t0
+    finally:
+        del loop.schedule, loop.upload  # back to the class methods
+    start = ev[0][0]
+    u0 = [start.elapsed_time(a) for a, _ in ev]
+    u1 = [start.elapsed_time(b) for _, b in ev]
+    busy = sum(y - x for x, y in zip(u0, u1))
+    period = (u1[-1] - u1[0]) / (len(ev) - 1)
+    return {"iterations": n, "period_ms": round(period, 4),
+            "input_upload_ms": round(busy / len(ev), 4),
+            "input_upload_gbs": round(host["bytes"] / (busy * 1e-3) / 1e9, 1),
+            "input_upload_busy_frac": round(busy / (u1[-1] - u0[0]), 3),
+            "host_ms_per_iteration": round(host["total"] * 1e3 / n, 4),
+            "host_in_schedule_ms": round(host["schedule"] * 1e3 / n, 4),
+            "buffer_sets": loop.num_sets,
+            "note": "a separate pass after the timed region; the schedule call includes its wait for the "
+                    "uploads of the step that last used its buffer set"}
 
 
 def run_trace(args, rank, world, local_rank):
@@ -1583,6 +1642,9 @@ def main():
                     help="decode scheduling order (default: longest first for one decode step, "
                          "batch order for the continuous-batching trace)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--timeline", action="store_true",
+                    help="gqa_trace: after the timed region, time the end-to-end loop's input uploads and host "
+                         "scheduling per iteration (added under e2e.timeline)")
     ap.add_argument("--shared-prefix", action="store_true",
                     help="serving traces: the shared-prefix decode for the largest group of sequences "
                          "sharing leading blocks (default: the plain decode)")

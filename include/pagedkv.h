@@ -598,7 +598,7 @@ typedef struct {
   int num_swap_in;      /* swap-in pairs */
   int prefill_tokens;   /* admitted prompts' uncached tokens, cu_seqlens[num_admitted] */
   int max_prefill_len;  /* most uncached tokens of one admitted prompt */
-  int buffer;           /* kv_serve_schedule: the step's buffer set, 0 or 1 (alternating); else 0 */
+  int buffer;           /* kv_serve_schedule: the step's buffer set, 0 .. num_sets - 1 in turn; else 0 */
   int64_t bytes;        /* bytes of the buffer the step uses */
   int64_t slot_mapping;          /* int64[num_tokens] */
   int64_t block_tables;          /* int32[batch][table_width], padded with -1 */
@@ -636,26 +636,33 @@ int kv_sched_step_packed(kv_sched* s, const int64_t* finished_ids, int n_finishe
  * more finely when fewer sequences run). */
 size_t kv_serve_workspace_bytes(const kv_pool* pool, int num_q_heads, int max_batch, int max_context_len);
 
+/* Most buffer sets a serving loop cycles through. */
+#define KV_SERVE_MAX_SETS 4
+
 /* A serving loop over pool and sched (both must outlive it).  The caller owns
- * every buffer: two pinned host and two device metadata buffers of
- * meta_bytes each (>= kv_step_packed_bytes(max_batch, max_tokens,
- * max_table_width, swap_slots), 16-byte aligned), the decode workspace
- * (>= kv_serve_workspace_bytes), and for swap preemption the mapped pinned
- * host swap space of swap_slots slots (kv_swap_out).  Consecutive steps
- * alternate between the two buffer pairs; the loop creates six CUDA events
- * on the current device, which must stay current for its calls.
+ * every buffer: num_sets (2 .. KV_SERVE_MAX_SETS) pinned host and as many
+ * device metadata buffers of meta_bytes each (>= kv_step_packed_bytes(
+ * max_batch, max_tokens, max_table_width, swap_slots), 16-byte aligned), the
+ * decode workspace (>= kv_serve_workspace_bytes), and for swap preemption the
+ * mapped pinned host swap space of swap_slots slots (kv_swap_out).
+ * Consecutive steps use the sets in turn, and a step's uploads wait only for
+ * the kernels of the step num_sets before it: with 2 sets, two steps cost at
+ * least one upload plus one step's kernels; with 3 or more, uploads and
+ * kernels of neighbouring steps overlap fully.  The loop creates three CUDA
+ * events per set on the current device, which must stay current for its
+ * calls.
  * num_q_heads, q_dtype (also the type of the new K/V rows) and scale are
  * those of the decode.  A loop holds per-step state: one host thread at a
  * time drives it (and its scheduler).  KV_ERR_ARG on bad arguments;
  * KV_ERR_CUDA if an event cannot be created. */
 int kv_serve_create(kv_pool* pool, kv_sched* sched, int num_q_heads, kv_dtype q_dtype, float scale,
                     int order_policy, int max_batch, int max_tokens, int max_table_width, void* host_swap,
-                    int swap_slots, void* const host_meta[2], void* const dev_meta[2], size_t meta_bytes,
-                    void* workspace, size_t workspace_bytes, kv_serve** out);
+                    int swap_slots, int num_sets, void* const* host_meta, void* const* dev_meta,
+                    size_t meta_bytes, void* workspace, size_t workspace_bytes, kv_serve** out);
 
-/* The step's host half: waits (host) until the other pinned buffer's last
- * upload is done, runs kv_sched_step_packed into it, and enqueues on
- * upload_stream, after the kernels that last read the matching device buffer,
+/* The step's host half: waits (host) until the next set's pinned buffer's
+ * last upload is done, runs kv_sched_step_packed into it, and enqueues on
+ * upload_stream, after the kernels that last read the set's device buffer,
  * one copy of the packed bytes to that device buffer.  running_ids
  * (int64[max_batch], written only for a batch that fits) and layout may be
  * NULL.  KV_ERR_STATE if the previous step was never launched
@@ -681,15 +688,15 @@ int kv_serve_launch(kv_serve* s, int layer, const void* q, const void* k_new, co
                     const void* prefill_q, void* prefill_out, kv_stream_t stream);
 
 /* Host input and output staging for a loop whose inputs come from host
- * memory.  The caller keeps two sets of device input and output buffers and
- * uses set layout.buffer for a step.  kv_serve_upload (after
+ * memory.  The caller keeps num_sets sets of device input and output
+ * buffers and uses set layout.buffer for a step.  kv_serve_upload (after
  * kv_serve_schedule, before the step's first launch) copies bytes from
  * pinned host memory to dev_dst on the step's upload stream, after the
- * kernels that last read that set (the step before the previous one); the
- * step's launches wait for it.  kv_serve_readback (after a launch) copies
- * bytes from dev_src to pinned host memory on readback_stream once the
- * step's kernels so far are done; the first launch of the step after next,
- * which reuses the set, waits for it.  KV_ERR_STATE when called out of that
+ * kernels that last read that set (the step num_sets before); the step's
+ * launches wait for it.  kv_serve_readback (after a launch) copies bytes from
+ * dev_src to pinned host memory on readback_stream once the step's kernels
+ * so far are done; the first launch of the next step that reuses the set
+ * waits for it.  KV_ERR_STATE when called out of that
  * order, KV_ERR_ARG on NULL pointers with bytes > 0. */
 int kv_serve_upload(kv_serve* s, void* dev_dst, const void* host_src, size_t bytes);
 int kv_serve_readback(kv_serve* s, void* host_dst, const void* dev_src, size_t bytes, kv_stream_t readback_stream);

@@ -17,6 +17,7 @@ from . import build as _build
 KV_F16, KV_BF16, KV_FP8_E4M3, KV_F32 = 0, 1, 2, 3
 KV_PREEMPT_NONE, KV_PREEMPT_SWAP, KV_PREEMPT_RECOMPUTE = 0, 1, 2
 KV_ORDER_BATCH, KV_ORDER_LONGEST, KV_ORDER_LONG_FIRST = 0, 1, 2
+KV_SERVE_MAX_SETS = 4
 KV_OK, KV_ERR_ARG, KV_ERR_OOM, KV_ERR_STATE, KV_ERR_BOUNDS, KV_ERR_CUDA, KV_ERR_TIMEOUT = (
     0, -1, -2, -3, -4, -5, -6)
 ERROR_NAMES = {0: "KV_OK", -1: "KV_ERR_ARG", -2: "KV_ERR_OOM", -3: "KV_ERR_STATE",
@@ -137,7 +138,8 @@ _SIGS = {
                                      P(kv_step_layout)]),
     "kv_serve_workspace_bytes": (c_size_t, [c_void_p, c_int, c_int, c_int]),
     "kv_serve_create": (c_int, [c_void_p, c_void_p, c_int, c_int, c_float, c_int, c_int, c_int, c_int, c_void_p,
-                                c_int, P(c_void_p), P(c_void_p), c_size_t, c_void_p, c_size_t, P(c_void_p)]),
+                                c_int, c_int, P(c_void_p), P(c_void_p), c_size_t, c_void_p, c_size_t,
+                                P(c_void_p)]),
     "kv_serve_schedule": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, P(kv_step_layout)]),
     "kv_serve_launch": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_int, c_void_p, c_void_p, c_void_p]),
@@ -541,11 +543,15 @@ def kv_serve_workspace_bytes(pool, num_q_heads, max_batch, max_context_len) -> i
 def kv_serve_create(pool, sched, num_q_heads, q_dtype, scale, order_policy, max_batch, max_tokens,
                     max_table_width, host_swap, swap_slots, host_meta, dev_meta, meta_bytes, workspace,
                     workspace_bytes):
+    """host_meta / dev_meta: one buffer per set (their count is num_sets)."""
     h = c_void_p()
-    hm = (c_void_p * 2)(*[_ptr(x) for x in host_meta])
-    dm = (c_void_p * 2)(*[_ptr(x) for x in dev_meta])
+    n = len(host_meta)
+    if len(dev_meta) != n:
+        raise ValueError("host_meta and dev_meta need the same number of sets")
+    hm = (c_void_p * max(n, 1))(*[_ptr(x) for x in host_meta])
+    dm = (c_void_p * max(n, 1))(*[_ptr(x) for x in dev_meta])
     _check(_lib.kv_serve_create(pool, sched, num_q_heads, q_dtype, float(scale), order_policy, max_batch,
-                                max_tokens, max_table_width, _ptr(host_swap), swap_slots, hm, dm, meta_bytes,
+                                max_tokens, max_table_width, _ptr(host_swap), swap_slots, n, hm, dm, meta_bytes,
                                 _ptr(workspace), workspace_bytes, ctypes.byref(h)))
     return h
 

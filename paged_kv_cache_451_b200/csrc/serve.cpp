@@ -5,9 +5,9 @@
 //
 // kv_sched_step_packed runs the scheduler step and writes all of the step's
 // device metadata into one caller buffer (pinned host memory), so a single
-// copy uploads it.  kv_serve_* keep two such buffers and two device buffers:
-// the upload of step i + 1 runs on an upload stream while the kernels of
-// step i read the other device buffer, with events ordering reuse.  Only
+// copy uploads it.  kv_serve_* cycle through 2 to 4 sets of such buffers and
+// device buffers: the upload of step i + 1 runs on an upload stream while the
+// kernels of step i read another set, with events ordering reuse.  Only
 // host code here; every kernel is enqueued through the library's own entry
 // points (block_copy, kv_swap_out / kv_swap_in, paged_kv_write,
 // paged_attention_prefill, paged_attention_decode).
@@ -69,17 +69,18 @@ struct kv_serve {
   int max_batch = 0, max_tokens = 0, max_width = 0;
   void* host_swap = nullptr;
   int swap_slots = 0;
-  uint8_t* h[2] = {nullptr, nullptr};
-  uint8_t* d[2] = {nullptr, nullptr};
+  int sets = 2;  // buffer sets, used in turn by consecutive steps
+  uint8_t* h[KV_SERVE_MAX_SETS] = {};
+  uint8_t* d[KV_SERVE_MAX_SETS] = {};
   size_t meta_bytes = 0;
   void* ws = nullptr;
   size_t ws_bytes = 0;
-  cudaEvent_t copy_ev[2] = {nullptr, nullptr};  // uploads into buffer set k done
-  cudaEvent_t done_ev[2] = {nullptr, nullptr};  // kernels reading buffer set k done
-  cudaEvent_t rb_ev[2] = {nullptr, nullptr};    // read-back of output set k done
-  bool copy_rec[2] = {false, false}, done_rec[2] = {false, false}, rb_rec[2] = {false, false};
+  cudaEvent_t copy_ev[KV_SERVE_MAX_SETS] = {};  // uploads into buffer set k done
+  cudaEvent_t done_ev[KV_SERVE_MAX_SETS] = {};  // kernels reading buffer set k done
+  cudaEvent_t rb_ev[KV_SERVE_MAX_SETS] = {};    // read-back of output set k done
+  bool copy_rec[KV_SERVE_MAX_SETS] = {}, done_rec[KV_SERVE_MAX_SETS] = {}, rb_rec[KV_SERVE_MAX_SETS] = {};
   cudaStream_t up = nullptr;  // the current step's upload stream
-  int k = 1;               // buffer of the current step
+  int k = -1;              // buffer set of the current step
   bool scheduled = false;  // a step is scheduled and not launched yet
   int launches = 0;        // launch calls for the current step
   kv_step_layout lay{};
@@ -191,13 +192,14 @@ size_t kv_serve_workspace_bytes(const kv_pool* pool, int num_q_heads, int max_ba
 
 int kv_serve_create(kv_pool* pool, kv_sched* sched, int num_q_heads, kv_dtype q_dtype, float scale,
                     int order_policy, int max_batch, int max_tokens, int max_table_width, void* host_swap,
-                    int swap_slots, void* const host_meta[2], void* const dev_meta[2], size_t meta_bytes,
-                    void* workspace, size_t workspace_bytes, kv_serve** out) {
+                    int swap_slots, int num_sets, void* const* host_meta, void* const* dev_meta,
+                    size_t meta_bytes, void* workspace, size_t workspace_bytes, kv_serve** out) {
   if (!pool || !sched || !out || !host_meta || !dev_meta || num_q_heads <= 0 || max_batch <= 0 ||
+      num_sets < 2 || num_sets > KV_SERVE_MAX_SETS ||
       max_tokens < 0 || max_table_width < 1 || swap_slots < 0 || (swap_slots > 0 && !host_swap) ||
       (order_policy != KV_ORDER_BATCH && order_policy != KV_ORDER_LONGEST && order_policy != KV_ORDER_LONG_FIRST))
     return fail(KV_ERR_ARG, "bad argument");
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < num_sets; ++i) {
     if (!host_meta[i] || !dev_meta[i]) return fail(KV_ERR_ARG, "NULL metadata buffer");
     if (reinterpret_cast<uintptr_t>(host_meta[i]) % kAlign || reinterpret_cast<uintptr_t>(dev_meta[i]) % kAlign)
       return fail(KV_ERR_ARG, "metadata buffers must be 16-byte aligned");
@@ -218,14 +220,16 @@ int kv_serve_create(kv_pool* pool, kv_sched* sched, int num_q_heads, kv_dtype q_
   s->max_width = max_table_width;
   s->host_swap = host_swap;
   s->swap_slots = swap_slots;
-  for (int i = 0; i < 2; ++i) {
+  s->sets = num_sets;
+  s->k = num_sets - 1;
+  for (int i = 0; i < num_sets; ++i) {
     s->h[i] = static_cast<uint8_t*>(host_meta[i]);
     s->d[i] = static_cast<uint8_t*>(dev_meta[i]);
   }
   s->meta_bytes = meta_bytes;
   s->ws = workspace;
   s->ws_bytes = workspace ? workspace_bytes : 0;
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < num_sets; ++i) {
     if (cudaEventCreateWithFlags(&s->copy_ev[i], cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&s->done_ev[i], cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&s->rb_ev[i], cudaEventDisableTiming) != cudaSuccess) {
@@ -243,7 +247,7 @@ int kv_serve_schedule(kv_serve* s, const int64_t* finished_ids, int n_finished, 
   if (!s) return fail(KV_ERR_ARG, "NULL serving loop");
   if (s->scheduled && s->launches == 0)
     return fail(KV_ERR_STATE, "the previous step was scheduled but never launched");
-  const int k = 1 - s->k;
+  const int k = (s->k + 1) % s->sets;
   // the pinned buffer is rewritten: its last upload must have finished
   if (s->copy_rec[k] && cudaEventSynchronize(s->copy_ev[k]) != cudaSuccess)
     return fail(KV_ERR_CUDA, "cudaEventSynchronize: %s", cudaGetErrorString(cudaGetLastError()));
@@ -363,7 +367,7 @@ int kv_serve_readback(kv_serve* s, void* host_dst, const void* dev_src, size_t b
 
 int kv_serve_destroy(kv_serve* s) {
   if (!s) return ok();
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < KV_SERVE_MAX_SETS; ++i) {
     if (s->rb_ev[i]) {
       cudaEventSynchronize(s->rb_ev[i]);
       cudaEventDestroy(s->rb_ev[i]);

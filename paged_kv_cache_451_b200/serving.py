@@ -287,15 +287,18 @@ class NativeDecodeLoop:
 
     def __init__(self, pool, sched, *, num_q_heads, kv_heads, head_dim, block_size, q_dtype,
                  scale, max_batch, max_blocks, max_tokens, max_context, device="cuda",
-                 order_policy="batch", host_swap=None, swap_slots=0):
+                 order_policy="batch", host_swap=None, swap_slots=0, num_sets=3):
         import torch
         self.torch = torch
         self.pool, self.sched = pool, sched
         self.hq, self.hkv, self.d, self.bs = num_q_heads, kv_heads, head_dim, block_size
         self.max_batch, self.max_blocks, self.max_tokens = max_batch, max_blocks, max_tokens
+        # buffer sets used in turn: a step's uploads wait for the kernels of
+        # the step num_sets before it (3 lets uploads and kernels overlap fully)
+        self.num_sets = num_sets
         self.meta_bytes = kv_step_packed_bytes(max_batch, max_tokens, max_blocks, swap_slots)
-        self.h_buf = [torch.empty(self.meta_bytes, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
-        self.d_buf = [torch.empty(self.meta_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.h_buf = [torch.empty(self.meta_bytes, dtype=torch.uint8, pin_memory=True) for _ in range(num_sets)]
+        self.d_buf = [torch.empty(self.meta_bytes, dtype=torch.uint8, device=device) for _ in range(num_sets)]
         self.ws_cap = max(kv_serve_workspace_bytes(pool, num_q_heads, max_batch, max_context), 16)
         self.d_ws = torch.empty(self.ws_cap, dtype=torch.uint8, device=device)
         self.up = torch.cuda.Stream(device=device)
@@ -331,8 +334,8 @@ class NativeDecodeLoop:
         return self.layout.max_context_len
 
     def upload(self, dev_dst, host_src, nbytes):
-        """Copy the step's inputs from pinned host memory into buffer set
-        ``plan["layout"].buffer`` (between schedule and launch)."""
+        """Copy the step's inputs from pinned host memory into the caller's
+        buffer set ``plan["layout"].buffer`` (between schedule and launch)."""
         kv_serve_upload(self.handle, dev_dst, host_src, nbytes)
 
     def readback(self, host_dst, dev_src, nbytes, stream):

@@ -24,8 +24,8 @@ def host16(t):
     return t.cpu().numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("order_policy", ["batch", "longest"])
-def test_serving_step_on_a_multi_layer_pool(order_policy):
+@pytest.mark.parametrize("order_policy,num_sets", [("batch", 3), ("longest", 2), ("batch", 4)])
+def test_serving_step_on_a_multi_layer_pool(order_policy, num_sets):
     rng = np.random.default_rng(5 if order_policy == "batch" else 6)
     nb, bs, hkv, hq, d, L, max_seqs = 160, 16, 2, 8, 128, 3, 12
     scale = 1.0 / np.sqrt(d)
@@ -58,7 +58,7 @@ def test_serving_step_on_a_multi_layer_pool(order_policy):
 
     loop = NativeDecodeLoop(pool.h, s, num_q_heads=hq, kv_heads=hkv, head_dim=d, block_size=bs, q_dtype=BF16,
                             scale=scale, max_batch=max_seqs, max_blocks=32, max_tokens=max_seqs * 200,
-                            max_context=500, order_policy=order_policy)
+                            max_context=500, order_policy=order_policy, num_sets=num_sets)
     loop.full_plan = True
     remaining = {100: 30, 101: 12, 102: 45}
     nxt, cow_total, admitted = 200, 0, 0

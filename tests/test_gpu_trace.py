@@ -65,9 +65,10 @@ class HostStaging:
         hq, hkv, d = w.num_q_heads, w.kv_heads, w.head_dim
         n = (e["max_num_seqs"] * hq + 2 * tr.loop.max_tokens * hkv) * d
         self.host = torch.empty(n, dtype=torch.int16).pin_memory()
-        self.dev = [torch.empty(n, dtype=torch.int16, device="cuda") for _ in range(2)]
-        self.outs = [torch.empty((e["max_num_seqs"], hq, d), dtype=torch.float32, device="cuda") for _ in range(2)]
-        self.hout = [torch.empty((e["max_num_seqs"], hq, d), dtype=torch.float32).pin_memory() for _ in range(2)]
+        sets = tr.loop.num_sets  # one input / output set per buffer set of the loop
+        self.dev = [torch.empty(n, dtype=torch.int16, device="cuda") for _ in range(sets)]
+        self.outs = [torch.empty((e["max_num_seqs"], hq, d), dtype=torch.float32, device="cuda") for _ in range(sets)]
+        self.hout = [torch.empty((e["max_num_seqs"], hq, d), dtype=torch.float32).pin_memory() for _ in range(sets)]
         self.rb = torch.cuda.Stream()
         self.rng = np.random.default_rng(99)
 
@@ -85,9 +86,10 @@ class HostStaging:
 
 
 def run_trace(w, iters, check_pool_at, sample_every=1, shared_prefix=False, native=False, order_policy="batch",
-              staging=False):
+              staging=False, serve_sets=3):
     plan = gqa_trace_plan(w)
-    tr = GqaTrace(w, plan, shared_prefix=shared_prefix, native=native, order_policy=order_policy)
+    tr = GqaTrace(w, plan, shared_prefix=shared_prefix, native=native, order_policy=order_policy,
+                  serve_sets=serve_sets)
     if native:
         tr.loop.full_plan = True  # the step's arrays, to compare with the oracle scheduler
     st = HostStaging(tr, w) if staging else None
@@ -100,7 +102,7 @@ def run_trace(w, iters, check_pool_at, sample_every=1, shared_prefix=False, nati
         if st is None:
             fin, arr, gplan, q, kn, vn, out = tr.iteration(it)
         else:
-            k = it % 2
+            k = it % tr.loop.num_sets
             fin, arr, gplan, q, kn, vn, out = tr.iteration(it, inputs=st.inputs, out=st.outs[k])
             assert gplan["layout"].buffer == k
             nout = gplan["info"].batch * w.num_q_heads * w.head_dim
@@ -169,12 +171,13 @@ def test_gqa_trace_through_the_native_serving_step(order_policy, iters):
     tr.loop.close()
 
 
-def test_gqa_trace_with_host_staging_through_the_serving_loop():
-    """Inputs uploaded from pinned host memory by kv_serve_upload into
-    alternating buffer sets, outputs read back by kv_serve_readback: the
+@pytest.mark.parametrize("serve_sets", [2, 3])
+def test_gqa_trace_with_host_staging_through_the_serving_loop(serve_sets):
+    """Inputs uploaded from pinned host memory by kv_serve_upload into the
+    loop's buffer sets in turn, outputs read back by kv_serve_readback: the
     pool, the sampled outputs and the read-back bytes all check."""
     w = WORKLOADS["gqa_trace"]
-    tr, _ = run_trace(w, 10, check_pool_at={0, 9}, native=True, staging=True)
+    tr, _ = run_trace(w, 10, check_pool_at={0, 9}, native=True, staging=True, serve_sets=serve_sets)
     tr.loop.close()
 
 

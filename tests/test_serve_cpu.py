@@ -214,11 +214,13 @@ def test_serve_create_checks_arguments_before_any_cuda_call():
         dict(order=5),                                    # unknown policy
         dict(swap_slots=4),                               # swap slots without swap space
         dict(max_width=0),
+        dict(host=[h[0]], dev=[d[0]]),                    # one buffer set
+        dict(host=h * 3, dev=d * 3),                      # six sets, above KV_SERVE_MAX_SETS
     ]
     for b in bad:
         with pytest.raises(pk.KVError) as e:
             pk.kv_serve_create(pool, s, 8, pk.KV_BF16, 0.1, b.get("order", pk.KV_ORDER_BATCH), 8, 64,
-                               b.get("max_width", 16), None, b.get("swap_slots", 0), b.get("host", h), d,
+                               b.get("max_width", 16), None, b.get("swap_slots", 0), b.get("host", h), b.get("dev", d),
                                b.get("meta_bytes", need), ws, 16)
         assert e.value.code == pk.KV_ERR_ARG
     for f in (lambda: pk.kv_serve_schedule(None, []), lambda: pk.kv_serve_launch(None, 0, 0, 0, 0, 0, pk.KV_F32),

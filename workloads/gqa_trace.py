@@ -36,7 +36,7 @@ FIRST_ARRIVAL = 10_000
 
 class GqaTrace:
     def __init__(self, w, plan, device="cuda", seed=0, decode_config=None, order_policy="batch",
-                 shared_prefix=False, native=False):
+                 shared_prefix=False, native=False, serve_sets=3):
         import torch
 
         self.torch, self.w, self.plan, self.seed = torch, w, plan, seed
@@ -95,7 +95,7 @@ class GqaTrace:
                   q_dtype=w.q_fmt, scale=w.scale, max_batch=e["max_num_seqs"], max_blocks=self.max_blocks,
                   max_tokens=max_tokens, max_context=e["cap"] + e["iters"] + bs, device=device,
                   order_policy=order_policy)
-        self.loop = (NativeDecodeLoop(self.pool, self.sched, **kw) if native else
+        self.loop = (NativeDecodeLoop(self.pool, self.sched, num_sets=serve_sets, **kw) if native else
                      DecodeLoop(self.pool, self.sched, shared_prefix=shared_prefix, **kw))
 
     def _seed(self, it, kind):
