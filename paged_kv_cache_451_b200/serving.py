@@ -277,8 +277,9 @@ class DecodeLoop:
 class NativeDecodeLoop:
     """The iteration of :class:`DecodeLoop` sequenced inside the library
     (``kv_serve_schedule`` / ``kv_serve_launch``): the scheduler step packs
-    the step's metadata straight into one of two pinned buffers and queues
-    its upload on the loop's upload stream; one launch call then enqueues
+    the step's metadata straight into one of ``num_sets`` pinned buffers
+    (used in turn) and queues its upload on the loop's upload stream; one
+    launch call per layer then enqueues
     the swaps, copy-on-write, cache write, optional prefill and decode.  No
     shared-prefix decode (use :class:`DecodeLoop` for that).  This class only
     owns the buffers and passes pointers.  With ``full_plan`` set, schedule()
