@@ -76,16 +76,20 @@ def check_step(buf, lay, want, policy, cached):
 @pytest.mark.parametrize("mode,policy,seed", [
     ("none", pk.KV_ORDER_BATCH, 0), ("none", pk.KV_ORDER_LONGEST, 1), ("none", pk.KV_ORDER_LONG_FIRST, 2),
     ("swap", pk.KV_ORDER_LONG_FIRST, 3), ("recompute", pk.KV_ORDER_BATCH, 4), ("swap", pk.KV_ORDER_LONGEST, 5),
+    ("window", pk.KV_ORDER_LONG_FIRST, 6),
 ])
 def test_packed_step_equals_the_oracle_scheduler(mode, policy, seed):
     rng = np.random.default_rng(700 + seed)
-    nb, bs, max_seqs, slots = (48, 8, 16, 24) if mode != "none" else (400, 16, 24, 0)
+    nb, bs, max_seqs, slots = (48, 8, 16, 24) if mode in ("swap", "recompute") else (400, 16, 24, 0)
     order = rng.permutation(nb)
     bm = BlockManager(nb, bs, order)
-    sch = Scheduler(bm, max_seqs)
+    window = 40 if mode == "window" else 0  # blocks that left a sequence's last 40 positions are released
+    sch = Scheduler(bm, max_seqs, window=window)
     a = pk.kv_alloc_create(nb, bs, order.astype(np.int32))
     s = pk.kv_sched_create(a, max_seqs)
-    if mode != "none":
+    if window:
+        pk.kv_sched_set_window(s, window)
+    elif mode != "none":
         bm.set_swap_space(slots)
         sch.preemption = mode
         pk.kv_alloc_set_swap_space(a, slots)
@@ -109,12 +113,16 @@ def test_packed_step_equals_the_oracle_scheduler(mode, policy, seed):
         check_step(buf, lay, want, policy, [0] * len(want["admitted"]))
         assert lay.bytes <= cap
         seen |= {k for k in ("cow_pairs", "swap_out", "swap_in", "admitted") if want.get(k)}
+        if any(b == -1 for t in want["block_tables"] for b in t):
+            seen.add("released")
         running = want["running"]
         for r in running:
             remaining[r] -= 1
     assert "admitted" in seen
     if mode == "swap":
         assert {"swap_out", "swap_in"} <= seen
+    if mode == "window":
+        assert "released" in seen
     pk.kv_sched_destroy(s)
     pk.kv_alloc_destroy(a)
 
