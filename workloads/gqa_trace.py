@@ -8,7 +8,9 @@ freed, so the prefix blocks and the partly filled last block are held by
 every sharer); the other half hold their own lognormal-length contexts.  In
 the first iteration every sharer appends its first own token into the
 shared partly filled block, so all but the last of them copy it on write.
-Each iteration then follows :class:`serving.DecodeLoop`: finished sequences
+Each iteration then follows :class:`serving.DecodeLoop` (or, with ``native``,
+the library's own serving step through :class:`serving.NativeDecodeLoop`):
+finished sequences
 leave, Poisson arrivals are admitted while blocks allow, every running
 sequence writes one token and is decoded.
 
