@@ -10,9 +10,8 @@ the first iteration every sharer appends its first own token into the
 shared partly filled block, so all but the last of them copy it on write.
 Each iteration then follows :class:`serving.DecodeLoop` (or, with ``native``,
 the library's own serving step through :class:`serving.NativeDecodeLoop`):
-finished sequences
-leave, Poisson arrivals are admitted while blocks allow, every running
-sequence writes one token and is decoded.
+finished sequences leave, Poisson arrivals are admitted while blocks allow,
+every running sequence writes one token and is decoded.
 
 Values (q, K, V of new tokens) are drawn on the device from seeded torch
 generators; the caller may copy them back to mirror the run on the host.
