@@ -266,3 +266,51 @@ def test_packed_orders_on_chosen_lengths(lens, policy, want):
     assert section(buf, lay.seq_order, np.int32, len(lens)).tolist() == want
     pk.kv_sched_destroy(s)
     pk.kv_alloc_destroy(a)
+
+
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+
+@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(seed=st.integers(0, 2 ** 31 - 1), window=st.sampled_from([0, 0, 24, 64]),
+       policy=st.sampled_from([pk.KV_ORDER_BATCH, pk.KV_ORDER_LONGEST, pk.KV_ORDER_LONG_FIRST]),
+       max_seqs=st.integers(1, 6), nb=st.integers(8, 40))
+def test_packed_step_random_operations(seed, window, policy, max_seqs, nb):
+    """Random arrivals (1 to 70 tokens), random finishes (all at once
+    included), empty steps, small pools that hold admissions back: every
+    packed array equals the oracle scheduler's step."""
+    rng = np.random.default_rng(seed)
+    bs = 8
+    order = rng.permutation(nb)
+    bm = BlockManager(nb, bs, order)
+    sch = Scheduler(bm, max_seqs, window=window)
+    a = pk.kv_alloc_create(nb, bs, order.astype(np.int32))
+    s = pk.kv_sched_create(a, max_seqs)
+    if window:
+        pk.kv_sched_set_window(s, window)
+    width = nb
+    cap = pk.kv_step_packed_bytes(max_seqs, 80 * max_seqs + max_seqs, width, 0)
+    buf = aligned(cap)
+    nxt = 0
+    try:
+        for _ in range(25):
+            for _ in range(int(rng.integers(0, 3))):
+                plen = int(rng.integers(1, 71))
+                sch.add_request(nxt, plen)
+                pk.kv_sched_add_request(s, nxt, plen)
+                nxt += 1
+            run = list(sch.running)
+            fin = run if rng.random() < 0.1 else [r for r in run if rng.random() < 0.25]
+            try:
+                want = sch.step(fin)
+            except Exception:  # the oracle ran out of blocks for the appends: the native step must too
+                with pytest.raises(pk.KVError) as e:
+                    pk.kv_sched_step_packed(s, fin, policy, width, buf, cap)
+                assert e.value.code == pk.KV_ERR_OOM
+                break
+            lay = pk.kv_sched_step_packed(s, fin, policy, width, buf, cap)
+            check_step(buf, lay, want, policy, [0] * len(want["admitted"]))
+    finally:
+        pk.kv_sched_destroy(s)
+        pk.kv_alloc_destroy(a)
