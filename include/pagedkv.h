@@ -512,8 +512,10 @@ typedef struct {
  * stays at the head and admission stops); (4) one slot is appended for every
  * running sequence.  Outputs are kept until the next step; read them with
  * kv_sched_outputs.  KV_ERR_STATE (bad finished id) changes nothing;
- * KV_ERR_OOM means the appends of (4) would run out of blocks: (1)-(3) are
- * applied, no slot is appended. */
+ * KV_ERR_OOM means the appends of (4), run in batch order (with a window,
+ * each followed by its sequence's release, whose blocks later appends may
+ * take), would run out of blocks: (1)-(3) are applied, no slot is
+ * appended. */
 int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_step_info* info);
 /* Copy the last step's outputs to host arrays sized from kv_step_info (any
  * may be NULL): running_ids[batch]; block_tables[batch][table_width]

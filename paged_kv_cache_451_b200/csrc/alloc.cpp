@@ -230,6 +230,56 @@ struct kv_alloc {
     }
   }
 
+  // Whether the appends of `ids`, run in that order and each followed (for
+  // a sequence not in `admitted`, with window > 0) by the release of the
+  // blocks wholly before its last `window` positions, always find a free
+  // block when they need one: a block boundary or a copy of a shared partly
+  // filled last block takes one, a release whose block loses its last
+  // reference returns one.  Changes nothing.
+  bool appends_fit(const std::vector<int64_t>& ids, const std::unordered_set<int64_t>& admitted, int window) {
+    int64_t f = n_free;
+    std::unordered_map<int32_t, int32_t> rc;  // refcounts of shared blocks as the simulation changes them
+    auto ref = [&](int32_t b) -> int32_t& {
+      auto it = rc.find(b);
+      if (it == rc.end()) it = rc.emplace(b, refcount[b]).first;
+      return it->second;
+    };
+    for (int64_t r : ids) {
+      const SeqState& st = seqs[r];
+      const int64_t pos = st.tokens;
+      if (pos % block_size == 0) {
+        if (f == 0) return false;
+        --f;
+      } else {
+        const int32_t last = st.blocks.back();
+        if (refcount[last] > 1 || rc.count(last)) {  // refcounts only fall: an exclusive block stays so
+          int32_t& c = ref(last);
+          if (c > 1) {
+            if (f == 0) return false;
+            --f;
+            --c;
+          }
+        }
+      }
+      if (window > 0 && !admitted.count(r)) {
+        // the append's own block (index pos / block_size) is never released here
+        const int64_t token = pos + 1 - window;
+        const int64_t upto = std::min<int64_t>(token < 0 ? 0 : token / block_size, (int64_t)st.blocks.size());
+        for (int64_t i = 0; i < upto; ++i) {
+          const int32_t b = st.blocks[i];
+          if (b < 0) continue;
+          if (refcount[b] == 1 && !rc.count(b)) {
+            ++f;
+            rc.emplace(b, 0);
+          } else if (--ref(b) == 0) {
+            ++f;
+          }
+        }
+      }
+    }
+    return true;
+  }
+
   // Fresh blocks the appends of `seqs` take: one per sequence at a block
   // boundary, plus the copies of shared partly filled last blocks (at most
   // refcount - 1 per block).
@@ -757,10 +807,13 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
     free_blocks = a->n_free;
   }
 
-  // (4) one slot per running sequence; check the whole batch fits first
+  // (4) one slot per running sequence; check the whole batch fits first, in
+  // the loop's own order (a window's releases free blocks for later appends)
+  std::unordered_set<int64_t> admitted;
+  if (s->window > 0) admitted.insert(s->out_admitted.begin(), s->out_admitted.end());
   {
     const int64_t need = a->append_need(s->running);
-    if (need > a->n_free) {
+    if (need > a->n_free && !(s->window > 0 && a->appends_fit(s->running, admitted, s->window))) {
       info->batch = (int)s->running.size();
       info->num_tokens = info->num_cow = 0;
       info->num_admitted = (int)s->out_admitted.size();
@@ -771,8 +824,6 @@ int kv_sched_step(kv_sched* s, const int64_t* finished_ids, int n_finished, kv_s
   }
   s->out_slots = prompt_slots;
   int max_blocks = 0;
-  std::unordered_set<int64_t> admitted;
-  if (s->window > 0) admitted.insert(s->out_admitted.begin(), s->out_admitted.end());
   for (int64_t r : s->running) {
     SeqState& st = a->seqs[r];
     int64_t slot;
