@@ -272,42 +272,62 @@ from hypothesis import HealthCheck, example, given, settings
 from hypothesis import strategies as st
 
 
-@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
 # a window's releases free blocks that later appends of the same step take:
 # the step must not report running out of blocks when the appends, run in
 # order, fit (found by this test)
-@example(seed=23, window=24, policy=pk.KV_ORDER_BATCH, max_seqs=6, nb=23, reserve=0)
+@example(seed=23, window=24, policy=pk.KV_ORDER_BATCH, max_seqs=6, nb=23, reserve=0, mode="none")
 @given(seed=st.integers(0, 2 ** 31 - 1), window=st.sampled_from([0, 0, 24, 64]),
        policy=st.sampled_from([pk.KV_ORDER_BATCH, pk.KV_ORDER_LONGEST, pk.KV_ORDER_LONG_FIRST]),
-       max_seqs=st.integers(1, 6), nb=st.integers(8, 40), reserve=st.sampled_from([-1, -1, 0]))
-def test_packed_step_random_operations(seed, window, policy, max_seqs, nb, reserve):
-    """Random arrivals (1 to 70 tokens), random finishes (all at once
-    included), empty steps, small pools that hold admissions back, and with
-    no admission reserve the appends running out of blocks (the step where
-    that happens must agree): every packed array equals the oracle
-    scheduler's step."""
+       max_seqs=st.integers(1, 6), nb=st.integers(8, 40), reserve=st.sampled_from([-1, -1, 0]),
+       mode=st.sampled_from(["none", "swap", "recompute", "caching"]))
+def test_packed_step_random_operations(seed, window, policy, max_seqs, nb, reserve, mode):
+    """Random arrivals (1 to 70 tokens; with prefix caching, token prompts
+    sharing a system prefix), random finishes (all at once included), empty
+    steps, small pools that hold admissions back, swap or recompute
+    preemption, and with no admission reserve the appends running out of
+    blocks (the step where that happens must agree): every packed array, the
+    swap outputs and the allocator's free list and refcounts equal the
+    oracle scheduler's."""
     rng = np.random.default_rng(seed)
     bs = 8
     order = rng.permutation(nb)
-    bm = BlockManager(nb, bs, order)
+    caching = mode == "caching"
+    bm = (PrefixCachingBlockManager if caching else BlockManager)(nb, bs, order)
     sch = Scheduler(bm, max_seqs, min_blocks=None if reserve < 0 else reserve, window=window)
     a = pk.kv_alloc_create(nb, bs, order.astype(np.int32))
+    slots = int(rng.integers(0, 30)) if mode == "swap" else 0
+    if caching:
+        pk.kv_alloc_enable_prefix_caching(a)
+    if mode in ("swap", "recompute"):
+        bm.set_swap_space(slots)
+        sch.preemption = mode
+        pk.kv_alloc_set_swap_space(a, slots)
     s = pk.kv_sched_create(a, max_seqs, reserve)
+    if mode in ("swap", "recompute"):
+        pk.kv_sched_set_preemption(s, pk.KV_PREEMPT_SWAP if mode == "swap" else pk.KV_PREEMPT_RECOMPUTE)
     if window:
         pk.kv_sched_set_window(s, window)
-    width = nb + 16  # windowed tables keep their released entries (-1): rows may outgrow the pool
-    cap = pk.kv_step_packed_bytes(max_seqs, 80 * max_seqs + max_seqs, width, 0)
+    width = nb + 32  # windowed tables keep their released entries (-1): rows may outgrow the pool
+    cap = pk.kv_step_packed_bytes(max_seqs, 200 * max_seqs, width, slots)
     buf = aligned(cap)
-    nxt = 0
+    system = [int(x) for x in rng.integers(0, 50, size=60)]
+    remaining, nxt = {}, 0
     try:
         for _ in range(25):
             for _ in range(int(rng.integers(0, 3))):
-                plen = int(rng.integers(1, 71))
-                sch.add_request(nxt, plen)
-                pk.kv_sched_add_request(s, nxt, plen)
+                if caching:
+                    toks = system[:int(rng.integers(0, 60))] + [int(x) for x in rng.integers(0, 50, size=int(rng.integers(1, 30)))]
+                    sch.add_request_tokens(nxt, toks)
+                    pk.kv_sched_add_request_tokens(s, nxt, toks)
+                else:
+                    plen = int(rng.integers(1, 71))
+                    sch.add_request(nxt, plen)
+                    pk.kv_sched_add_request(s, nxt, plen)
+                remaining[nxt] = int(rng.integers(2, 40))
                 nxt += 1
             run = list(sch.running)
-            fin = run if rng.random() < 0.1 else [r for r in run if rng.random() < 0.25]
+            fin = run if rng.random() < 0.05 else [r for r in run if remaining[r] <= 0 or rng.random() < 0.1]
             try:
                 want = sch.step(fin)
             except OracleOOM:  # the oracle ran out of blocks for the appends: the native step must too
@@ -316,7 +336,14 @@ def test_packed_step_random_operations(seed, window, policy, max_seqs, nb, reser
                 assert e.value.code == pk.KV_ERR_OOM
                 break
             lay = pk.kv_sched_step_packed(s, fin, policy, width, buf, cap)
-            check_step(buf, lay, want, policy, [0] * len(want["admitted"]))
+            check_step(buf, lay, want, policy, want["cached"] if caching else [0] * len(want["admitted"]))
+            sw = pk.kv_sched_swap_outputs(s)
+            assert list(sw["preempted"]) == want["preempted"] and list(sw["recomputed"]) == want["recomputed"]
+            assert list(sw["swapped_in"]) == want["swapped_in"]
+            free, rc = pk.kv_alloc_snapshot(a, nb)
+            assert list(free) == list(bm.free_list) and list(rc) == bm.refcount
+            for r in want["running"]:
+                remaining[r] -= 1
     finally:
         pk.kv_sched_destroy(s)
         pk.kv_alloc_destroy(a)
