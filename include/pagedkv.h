@@ -463,9 +463,11 @@ int kv_alloc_commit(kv_alloc* a, int64_t seq_id, int* num_registered);
 int kv_alloc_set_swap_space(kv_alloc* a, int num_slots);
 
 /* Sliding window: release every block of seq_id wholly before position
- * `token` (blocks 0 .. token / block_size - 1 not yet released); their table
- * entries become -1 so logical block indices stay put.  Shared blocks only
- * lose this sequence's reference.  num_released may be NULL. */
+ * min(token, n), n the sequence's token count (blocks 0 .. min(token, n) /
+ * block_size - 1 not yet released), so the block that receives the next
+ * token is never released; their table entries become -1 so logical block
+ * indices stay put.  Shared blocks only lose this sequence's reference.
+ * num_released may be NULL. */
 int kv_alloc_release_before(kv_alloc* a, int64_t seq_id, int64_t token, int* num_released);
 
 /* Cumulative hit blocks and evictions, and the number of registered blocks

@@ -156,12 +156,14 @@ class BlockManager:
 
     def release_before(self, seq_id: int, token: int) -> int:
         """Sliding window: release every block wholly before position
-        `token` (its table entry becomes -1; the table keeps its length so
-        logical block indices stay put).  Returns the number released."""
+        min(token, n), n the sequence's token count (its table entry becomes
+        -1; the table keeps its length so logical block indices stay put).
+        Only positions the sequence holds count, so the block that receives
+        its next token is never released.  Returns the number released."""
         if seq_id not in self.tables:
             raise OracleStateError(f"sequence {seq_id} is unknown")
         table = self.tables[seq_id]
-        upto = min(max(token, 0) // self.block_size, len(table))
+        upto = min(min(max(token, 0), self.tokens[seq_id]) // self.block_size, len(table))
         n = 0
         for i in range(upto):
             b = table[i]

@@ -585,7 +585,10 @@ int kv_alloc_release_before(kv_alloc* a, int64_t seq_id, int64_t token, int* num
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return fail(KV_ERR_STATE, "sequence %lld is unknown", (long long)seq_id);
   SeqState& st = it->second;
-  const int64_t upto = std::min<int64_t>(token < 0 ? 0 : token / a->block_size, (int64_t)st.blocks.size());
+  // only positions the sequence holds: the block that receives its next
+  // token is never released
+  const int64_t held = std::min<int64_t>(token < 0 ? 0 : token, st.tokens);
+  const int64_t upto = std::min<int64_t>(held / a->block_size, (int64_t)st.blocks.size());
   int released = 0;
   for (int64_t i = 0; i < upto; ++i) {
     if (st.blocks[i] < 0) continue;

@@ -92,3 +92,34 @@ def test_native_release_before_matches_oracle():
     free, rc = pk.kv_alloc_snapshot(a, 20)
     assert list(free) == list(bm.free_list) and sorted(free) == list(range(20))
     pk.kv_alloc_destroy(a)
+
+
+def test_release_covers_only_positions_the_sequence_holds():
+    """Traced by hand: a window release past the sequence's length keeps the
+    block that receives the next token.  9 tokens in blocks of 4: blocks 0
+    and 1 (positions 0..7) go, block 2 (position 8, next token 9) stays and
+    the append lands in it at offset 1.  16 tokens: all four full blocks go
+    and the append takes a fresh block."""
+    for native in (False, True):
+        if native:
+            a = pk.kv_alloc_create(8, 4)
+            pk.kv_alloc_allocate(a, 1, 9)
+            pk.kv_alloc_allocate(a, 2, 16)
+            t1, t2 = list(pk.kv_alloc_block_table(a, 1)), list(pk.kv_alloc_block_table(a, 2))
+            n1, n2 = pk.kv_alloc_release_before(a, 1, 100), pk.kv_alloc_release_before(a, 2, 100)
+            slot1, _, _ = pk.kv_alloc_append_slot(a, 1)
+            slot2, _, _ = pk.kv_alloc_append_slot(a, 2)
+            tab1, tab2 = list(pk.kv_alloc_block_table(a, 1)), list(pk.kv_alloc_block_table(a, 2))
+            pk.kv_alloc_destroy(a)
+        else:
+            bm = BlockManager(8, 4)
+            bm.allocate(1, 9)
+            bm.allocate(2, 16)
+            t1, t2 = list(bm.tables[1]), list(bm.tables[2])
+            n1, n2 = bm.release_before(1, 100), bm.release_before(2, 100)
+            slot1, _, _ = bm.append_slot(1)
+            slot2, _, _ = bm.append_slot(2)
+            tab1, tab2 = list(bm.tables[1]), list(bm.tables[2])
+        assert (n1, n2) == (2, 4)
+        assert tab1 == [-1, -1, t1[2]] and slot1 == t1[2] * 4 + 1
+        assert tab2[:4] == [-1, -1, -1, -1] and len(tab2) == 5 and tab2[4] >= 0 and slot2 == tab2[4] * 4
