@@ -8,7 +8,7 @@ import os
 
 import numpy as np
 import pytest
-from hypothesis import given, settings, strategies as st
+from hypothesis import HealthCheck, given, settings, strategies as st
 
 import paged_kv_cache_451_b200 as pk
 from oracle.sched import BlockManager, OracleOOM, OracleStateError, Scheduler
@@ -187,3 +187,56 @@ def test_native_scheduler_reports_append_oom_with_explicit_small_reserve():
     assert pk.kv_sched_stats(s)[:2] == (2, 0)
     pk.kv_sched_destroy(s)
     pk.kv_alloc_destroy(a)
+
+
+@settings(max_examples=80, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(seed=st.integers(0, 2 ** 31 - 1), nb=st.integers(2, 30), bs=st.sampled_from([4, 8, 16]))
+def test_native_allocator_random_operations_match_oracle(seed, nb, bs):
+    """Random allocate / append / fork / free / window release sequences
+    (release tokens below, at and past a sequence's length, exhaustion
+    included): every result, error and the full allocator state (free list
+    order, refcounts, every live table) equal the oracle's after each
+    operation."""
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(nb)
+    bm = BlockManager(nb, bs, order)
+    a = pk.kv_alloc_create(nb, bs, order.astype(np.int32))
+    live, nxt = [], 0
+    try:
+        for _ in range(60):
+            kind = str(rng.choice(["alloc", "append", "append", "fork", "free", "release"]))
+            if kind != "alloc" and not live:
+                continue
+            sid = int(rng.choice(live)) if kind != "alloc" else None
+            n = int(rng.integers(0, 40))
+            tok = int(rng.integers(-5, bm.tokens[sid] + 6)) if kind == "release" else 0
+            ops = {
+                "alloc": (lambda: bm.allocate(nxt, n), lambda: pk.kv_alloc_allocate(a, nxt, n)),
+                "append": (lambda: bm.append_slot(sid), lambda: pk.kv_alloc_append_slot(a, sid)),
+                "fork": (lambda: bm.fork(sid, nxt), lambda: pk.kv_alloc_fork(a, sid, nxt)),
+                "free": (lambda: bm.free(sid), lambda: pk.kv_alloc_free(a, sid)),
+                "release": (lambda: bm.release_before(sid, tok), lambda: pk.kv_alloc_release_before(a, sid, tok)),
+            }[kind]
+            try:
+                want, oerr = ops[0](), None
+            except (OracleOOM, OracleStateError) as e:
+                want, oerr = None, e
+            if oerr is not None:
+                with pytest.raises(pk.KVError) as e:
+                    ops[1]()
+                assert e.value.code == (pk.KV_ERR_OOM if isinstance(oerr, OracleOOM) else pk.KV_ERR_STATE)
+                continue
+            got = ops[1]()
+            if kind in ("append", "release"):
+                assert tuple(np.atleast_1d(got)) == tuple(np.atleast_1d(want)), kind
+            if kind in ("alloc", "fork"):
+                live.append(nxt)
+                nxt += 1
+            elif kind == "free":
+                live.remove(sid)
+            free, rc = pk.kv_alloc_snapshot(a, nb)
+            assert list(free) == list(bm.free_list) and list(rc) == bm.refcount
+            for x in live:
+                assert list(pk.kv_alloc_block_table(a, x)) == bm.block_table(x)
+    finally:
+        pk.kv_alloc_destroy(a)
