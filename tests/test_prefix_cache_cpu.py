@@ -13,8 +13,8 @@ from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 
 import paged_kv_cache_451_b200 as pk
-from oracle.sched import (BlockManager, OracleOOM, PrefixCachingBlockManager, Scheduler, block_key,
-                          fnv1a64)
+from oracle.sched import (BlockManager, OracleOOM, OracleStateError, PrefixCachingBlockManager, Scheduler,
+                          block_key, fnv1a64)
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -242,3 +242,59 @@ def test_native_scheduler_with_prompt_tokens_matches_oracle(seed):
     assert hits > 0
     pk.kv_sched_destroy(s)
     pk.kv_alloc_destroy(a)
+
+
+@settings(max_examples=60, deadline=None)
+@given(seed=st.integers(0, 2 ** 31 - 1), nb=st.integers(3, 30), bs=st.sampled_from([4, 8]))
+def test_native_prefix_caching_random_operations_match_oracle(seed, nb, bs):
+    """Random prompts sharing a system prefix (cache hits, evictions),
+    token appends and plain appends, commits, frees, forks and window
+    releases: results, errors, the free list, refcounts and every live table
+    equal the oracle's after each operation."""
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(nb)
+    bm = PrefixCachingBlockManager(nb, bs, order)
+    a = pk.kv_alloc_create(nb, bs, order.astype(np.int32))
+    pk.kv_alloc_enable_prefix_caching(a)
+    system = [int(x) for x in rng.integers(0, 6, size=40)]
+    live, nxt = [], 0
+    try:
+        for _ in range(60):
+            kind = str(rng.choice(["prompt", "prompt", "append_tok", "append", "commit", "free", "fork", "release"]))
+            if kind != "prompt" and not live:
+                continue
+            sid = int(rng.choice(live)) if kind != "prompt" else None
+            toks = system[:int(rng.integers(0, 40))] + [int(x) for x in rng.integers(0, 6, size=int(rng.integers(1, 12)))]
+            tk = int(rng.integers(0, 6))
+            tok = int(rng.integers(-3, (bm.tokens[sid] if sid is not None else 0) + 5))
+            ops = {
+                "prompt": (lambda: bm.allocate_prompt(nxt, toks), lambda: pk.kv_alloc_allocate_prompt(a, nxt, toks)),
+                "append_tok": (lambda: bm.append_token(sid, tk), lambda: pk.kv_alloc_append_token(a, sid, tk)),
+                "append": (lambda: bm.append_slot(sid), lambda: pk.kv_alloc_append_slot(a, sid)),
+                "commit": (lambda: bm.commit(sid), lambda: pk.kv_alloc_commit(a, sid)),
+                "free": (lambda: bm.free(sid), lambda: pk.kv_alloc_free(a, sid)),
+                "fork": (lambda: bm.fork(sid, nxt), lambda: pk.kv_alloc_fork(a, sid, nxt)),
+                "release": (lambda: bm.release_before(sid, tok), lambda: pk.kv_alloc_release_before(a, sid, tok)),
+            }[kind]
+            try:
+                want, oerr = ops[0](), None
+            except (OracleOOM, OracleStateError) as e:
+                want, oerr = None, e
+            if oerr is not None:
+                with pytest.raises(pk.KVError) as e:
+                    ops[1]()
+                assert e.value.code == (pk.KV_ERR_OOM if isinstance(oerr, OracleOOM) else pk.KV_ERR_STATE)
+                continue
+            got = ops[1]()
+            if kind not in ("free", "fork"):
+                assert tuple(np.atleast_1d(got)) == tuple(np.atleast_1d(want)), kind
+            if kind in ("prompt", "fork"):
+                live.append(nxt)
+                nxt += 1
+            elif kind == "free":
+                live.remove(sid)
+            assert native_state(a, nb) == (list(bm.free_list), bm.refcount)
+            for x in live:
+                assert list(pk.kv_alloc_block_table(a, x)) == bm.block_table(x)
+    finally:
+        pk.kv_alloc_destroy(a)
