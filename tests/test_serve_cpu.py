@@ -283,9 +283,9 @@ from hypothesis import strategies as st
        mode=st.sampled_from(["none", "swap", "recompute", "caching"]))
 def test_packed_step_random_operations(seed, window, policy, max_seqs, nb, reserve, mode):
     """Random arrivals (1 to 70 tokens; with prefix caching, token prompts
-    sharing a system prefix), random finishes (all at once included), empty
-    steps, small pools that hold admissions back, swap or recompute
-    preemption, and with no admission reserve the appends running out of
+    sharing a system prefix), a forked group sharing its blocks, random
+    finishes (all at once included), empty steps, small pools that hold
+    admissions back, swap or recompute preemption, and with no admission reserve the appends running out of
     blocks (the step where that happens must agree): every packed array, the
     swap outputs and the allocator's free list and refcounts equal the
     oracle scheduler's."""
@@ -313,6 +313,18 @@ def test_packed_step_random_operations(seed, window, policy, max_seqs, nb, reser
     buf = aligned(cap)
     system = [int(x) for x in rng.integers(0, 50, size=60)]
     remaining, nxt = {}, 0
+    # a forked group sharing its blocks (the partly filled last one included)
+    plen, forks = int(rng.integers(1, 3 * bs)), int(rng.integers(0, 3))
+    if not caching and bm.can_allocate(plen):
+        bm.allocate(10_000, plen)
+        pk.kv_alloc_allocate(a, 10_000, plen)
+        for c in range(forks):
+            bm.fork(10_000, 10_001 + c)
+            pk.kv_alloc_fork(a, 10_000, 10_001 + c)
+        for sid in ([10_000] + [10_001 + c for c in range(forks)])[:max_seqs]:
+            sch.adopt(sid)
+            pk.kv_sched_adopt(s, sid)
+            remaining[sid] = int(rng.integers(2, 40))
     try:
         for _ in range(25):
             for _ in range(int(rng.integers(0, 3))):
