@@ -359,3 +359,24 @@ def test_packed_step_random_operations(seed, window, policy, max_seqs, nb, reser
     finally:
         pk.kv_sched_destroy(s)
         pk.kv_alloc_destroy(a)
+
+
+@pytest.mark.parametrize("hkv,hq,fmt,max_b,max_ctx", [
+    (8, 64, pk.KV_BF16, 256, 8324),      # the GQA serving trace
+    (40, 40, pk.KV_F16, 64, 2048),       # the Llama layer
+    (32, 32, pk.KV_FP8_E4M3, 8, 16384),  # long FP8 contexts
+])
+def test_serve_workspace_bounds_every_batch_and_shorter_context(hkv, hq, fmt, max_b, max_ctx):
+    """kv_serve_workspace_bytes takes the largest need over the batch sizes
+    at the longest context; no step with fewer sequences or shorter contexts
+    may need more (the split policy divides short contexts too)."""
+    pool = pk.kv_pool_create(16, 4096, hkv, 128, fmt, 1)
+    try:
+        cap = pk.kv_serve_workspace_bytes(pool, hq, max_b, max_ctx)
+        for b in list(range(1, 41)) + list(range(41, max_b + 1, 9)) + [max_b]:
+            if b > max_b:
+                continue
+            for c in list(range(1, 400, 13)) + list(range(400, max_ctx + 1, 97)) + [max_ctx]:
+                assert pk.paged_attention_workspace_bytes(pool, b, hq, c) <= cap, (b, c)
+    finally:
+        pk.kv_pool_destroy(pool)
