@@ -266,7 +266,8 @@ int kv_serve_schedule(kv_serve* s, const int64_t* finished_ids, int n_finished, 
   if ((L.num_swap_out || L.num_swap_in) && !s->host_swap)
     return fail(KV_ERR_STATE, "the step swaps but the loop has no host swap space; the scheduler step is taken");
   cudaStream_t up = reinterpret_cast<cudaStream_t>(upload_stream);
-  // the device buffer is rewritten: the kernels that read it two steps ago must be done
+  // the device buffer is rewritten: the kernels that last read it (the step
+  // num_sets before this one) must be done
   if (s->done_rec[k] && cudaStreamWaitEvent(up, s->done_ev[k], 0) != cudaSuccess)
     return fail(KV_ERR_CUDA, "cudaStreamWaitEvent: %s", cudaGetErrorString(cudaGetLastError()));
   if (L.bytes > 0 && cudaMemcpyAsync(s->d[k], s->h[k], (size_t)L.bytes, cudaMemcpyHostToDevice, up) != cudaSuccess)
