@@ -13,8 +13,7 @@ from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 
 import paged_kv_cache_451_b200 as pk
-from oracle.sched import (BlockManager, OracleOOM, OracleStateError, PrefixCachingBlockManager, Scheduler,
-                          block_key, fnv1a64)
+from oracle.sched import OracleOOM, OracleStateError, PrefixCachingBlockManager, Scheduler, block_key, fnv1a64
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 
