@@ -583,7 +583,7 @@ int kv_sched_destroy(kv_sched* s);
 /* One continuous-batching iteration sequenced by the library ([CB]: free the
  * finished, admit first come first served, append one slot per running
  * sequence, then the step's kernels), so a serving loop makes two calls per
- * step instead of one per array and kernel. */
+ * step (four with host staging) instead of one per array and kernel. */
 
 /* Order in which the decode places the batch's sequences on the GPU (the
  * seq_order argument of paged_attention_decode; outputs do not depend on it).
@@ -685,7 +685,10 @@ int kv_serve_schedule(kv_serve* s, const int64_t* finished_ids, int n_finished, 
  * ([prefill_tokens][num_q_heads][head_dim], rows prompt by prompt), and
  * paged_attention_decode of the running set (q, out [batch][num_q_heads]
  * [head_dim]) in the loop's scheduling order.  Call once per layer after
- * each kv_serve_schedule.  KV_ERR_STATE with no step scheduled; otherwise the
+ * each kv_serve_schedule.  KV_ERR_STATE with no step scheduled; KV_ERR_ARG
+ * for a missing q / out (batch > 0) or k_new / v_new (tokens > 0), one of
+ * prefill_q / prefill_out without the other, or a workspace smaller than the
+ * step's decode needs (checked before anything is enqueued); otherwise the
  * first error of the entry points above (later ones are not enqueued). */
 int kv_serve_launch(kv_serve* s, int layer, const void* q, const void* k_new, const void* v_new,
                     const float* k_inv_scale, const float* v_inv_scale, void* out, kv_dtype out_dtype,
