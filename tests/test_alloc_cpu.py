@@ -189,7 +189,7 @@ def test_native_scheduler_reports_append_oom_with_explicit_small_reserve():
     pk.kv_alloc_destroy(a)
 
 
-@settings(max_examples=80, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@settings(max_examples=80, deadline=None, derandomize=True, suppress_health_check=[HealthCheck.too_slow])
 @given(seed=st.integers(0, 2 ** 31 - 1), nb=st.integers(2, 30), bs=st.sampled_from([4, 8, 16]))
 def test_native_allocator_random_operations_match_oracle(seed, nb, bs):
     """Random allocate / append / fork / free / window release sequences

@@ -243,7 +243,7 @@ def test_native_scheduler_with_prompt_tokens_matches_oracle(seed):
     pk.kv_alloc_destroy(a)
 
 
-@settings(max_examples=60, deadline=None)
+@settings(max_examples=60, deadline=None, derandomize=True)
 @given(seed=st.integers(0, 2 ** 31 - 1), nb=st.integers(3, 30), bs=st.sampled_from([4, 8]))
 def test_native_prefix_caching_random_operations_match_oracle(seed, nb, bs):
     """Random prompts sharing a system prefix (cache hits, evictions),

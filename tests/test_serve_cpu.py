@@ -272,7 +272,7 @@ from hypothesis import HealthCheck, example, given, settings
 from hypothesis import strategies as st
 
 
-@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@settings(max_examples=60, deadline=None, derandomize=True, suppress_health_check=[HealthCheck.too_slow])
 # a window's releases free blocks that later appends of the same step take:
 # the step must not report running out of blocks when the appends, run in
 # order, fit (found by this test)
