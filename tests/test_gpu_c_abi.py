@@ -59,11 +59,7 @@ def test_write_and_decode_from_c(tmp_path):
         f.write(lens.tobytes())
         f.write(slots.tobytes())
     exe = str(tmp_path / "decode_from_c")
-    libdir = os.path.dirname(pk.LIB_PATH)
-    subprocess.run(["gcc", "-std=gnu11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
-                    "-I", os.path.join(CUDA, "include"), SRC, "-L", libdir, "-lpagedkv",
-                    "-L", os.path.join(CUDA, "lib64"), "-lcudart", f"-Wl,-rpath,{libdir}",
-                    f"-Wl,-rpath,{os.path.join(CUDA, 'lib64')}", "-o", exe], check=True, capture_output=True)
+    compile_c(SRC, exe)
     out_path = tmp_path / "out.bin"
     run = subprocess.run([exe, str(inp), str(out_path)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
